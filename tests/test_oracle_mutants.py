@@ -1,0 +1,74 @@
+"""Plant plausible mistakes in copies of the oracle (CPU only) and check that the pins catch each.
+
+Every mutant is a textual edit of ``oracle/rra_oracle.c`` compiled to a temporary library; the
+real oracle source is never modified.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle_pins
+from oracle import oracle as O
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "rra_oracle.c")
+
+MUTANTS = {
+    "drop_scale": ("s[j] = acc * scale;", "s[j] = acc;"),
+    "max_sign": ("s[j] = exp(s[j] - m);", "s[j] = exp(m - s[j]);"),
+    "no_max_shift": ("s[j] = exp(s[j] - m);", "s[j] = exp(s[j]);"),
+    "no_denominator": ("out[c] = acc / denom;", "out[c] = acc;"),
+    "key_wrong_head": ("load_elem(k, dtype, ((seq_start + j) * H + h) * (int64_t)d + c)",
+                       "load_elem(k, dtype, ((seq_start + j) * H + 0) * (int64_t)d + c)"),
+    "qk_transposed": ("load_elem(q, dtype, (t * H + h) * (int64_t)d + c) *",
+                      "load_elem(q, dtype, ((seq_start + j) * H + h) * (int64_t)d + c) *"),
+    "value_from_query_row": ("acc += s[j] * load_elem(v, dtype, ((seq_start + j) * H + h) * (int64_t)d + c);",
+                             "acc += s[j] * load_elem(v, dtype, (t * H + h) * (int64_t)d + c);"),
+    "causal": ("for (int64_t j = 0; j < L; ++j) {\n        double acc = 0.0;",
+               "for (int64_t j = 0; j < L; ++j) {\n        if (seq_start + j > t) { s[j] = -INFINITY; continue; }\n        double acc = 0.0;"),
+    "last_key_dropped": ("for (int64_t j = 0; j < L; ++j) {\n        s[j] = exp(s[j] - m);",
+                         "for (int64_t j = 0; j < L; ++j) {\n        s[j] = (j == L - 1) ? 0.0 : exp(s[j] - m);"),
+    "rank_off_by_one": ("rank[(int64_t)b * N + n] = r++;", "rank[(int64_t)b * N + n] = ++r;"),
+    "cu_not_cumulative": ("cu[b + 1] = (int32_t)run;", "cu[b + 1] = (int32_t)run; run = 0;"),
+    "pack_reverse_order": ("int64_t out_row = (int64_t)cu[b] + r;",
+                           "int64_t out_row = (int64_t)cu[b + 1] - 1 - r;"),
+    "pack_ignores_capacity": ("if (out_row >= capacity)\n                continue;", ""),
+    "unpack_no_fill": ("memset(out, 0, (size_t)row_bytes);", ";"),
+    "unpack_wrong_row": ("int64_t src_row = (int64_t)cu[b] + r;", "int64_t src_row = (int64_t)b * N + n;"),
+    "f16_bias": ("v = ldexp((double)(1024 + m), e - 25);", "v = ldexp((double)(1024 + m), e - 24);"),
+    "f16_subnormal": ("v = ldexp((double)m, -24);", "v = ldexp((double)m, -25);"),
+    "bf16_truncated": ("uint32_t u = ((uint32_t)b) << 16;", "uint32_t u = ((uint32_t)(b & 0xFFF0)) << 16;"),
+    "mask_byte_is_bool": ("if (mask[(int64_t)b * N + n] != 0)\n                run += 1;",
+                          "if (mask[(int64_t)b * N + n] == 1)\n                run += 1;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    text = open(SRC).read()
+    assert text.count(old) >= 1, f"mutation site for {name} not found"
+    src = tmp_path / "mutant.c"
+    src.write_text(text.replace(old, new))
+    lib_path = str(tmp_path / "libmutant.so")
+    O.build(src=str(src), out=lib_path, extra_flags=("-w",))
+    # Run the pins in a child process: a mutant that writes out of bounds may crash, which
+    # also counts as caught.
+    tests_dir = os.path.dirname(os.path.abspath(__file__))
+    code = (
+        "import sys; sys.path[:0] = [%r, %r]\n"
+        "import oracle_pins\n"
+        "from oracle import oracle as O\n"
+        "lib = O.load(%r)\n"
+        "bad = []\n"
+        "for pin in oracle_pins.ALL_PINS:\n"
+        "    try:\n"
+        "        pin(lib)\n"
+        "    except Exception:\n"
+        "        bad.append(pin.__name__)\n"
+        "print('FAILED_PINS', bad)\n"
+        "sys.exit(3 if bad else 0)\n"
+    ) % (tests_dir, os.path.dirname(tests_dir), lib_path)
+    proc = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600)
+    assert proc.returncode != 0, f"mutant {name} passed every pin: {proc.stdout[-500:]}"
