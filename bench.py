@@ -1,0 +1,497 @@
+#!/usr/bin/env python
+"""Benchmark of the pack -> attend -> unpack call on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2] [--impl ours|reference]
+
+One step = one whole call (rra_pack, rra_attend, rra_unpack for every pruning stage of the
+workload) replayed from a CUDA graph over inputs resident in HBM.  L2 is flushed (a 256 MiB
+write, untimed) before every timed step, and each step is bracketed by CUDA events on the
+launching stream; per-kernel events recorded inside the graph give the per-kernel times.
+
+Prints ONE JSON line on rank 0: packed tokens/s (whole job), us per call, the roofline of the
+dominant kernel, end-to-end throughput through the public API with pinned host buffers,
+the float64 CPU oracle on a bounded sample, clocks sampled during the timed region, and how
+many of this library's kernels ran in the timed region.
+
+With torchrun (N > 1) every rank runs an independent replica of the workload on its own GPU
+(images are independent, so the path shards with no exchange): weak scaling, timings reduced
+as the max over ranks.
+
+--impl reference times the float64 CPU oracle itself (rank 0 only) on the same workload,
+metric and unit, one bounded sample of images per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from ragged_varlen_attention_rra_b200 import rra, workloads  # noqa: E402
+
+METRIC = "packed tokens/s & us per pack-attend-unpack call (1 B200, graph); % roofline"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+KERNELS = ("pack", "attend", "unpack")
+KERNEL_SOURCES = {
+    "pack": "ragged_varlen_attention_rra_b200/csrc/pack_unpack.cu",
+    "unpack": "ragged_varlen_attention_rra_b200/csrc/pack_unpack.cu",
+    "attend": "ragged_varlen_attention_rra_b200/csrc/attend.cu",
+}
+
+
+# ------------------------------------------------------------------------------------ helpers
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash(rel):
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source still matches."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("source_sha") != source_hash(KERNEL_SOURCES[kernel]):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def algorithmic_bytes(w, lengths, row_bytes, out_row_bytes):
+    """Per-stage algorithmic HBM bytes of each kernel (the minimal reads + writes)."""
+    B, N = w.B, w.N
+    T = int(lengths.sum())
+    return {
+        "pack": B * N + 2 * 3 * T * row_bytes + 4 * (B + 1),
+        "attend": 3 * T * row_bytes + T * out_row_bytes + 4 * (B + 1),
+        "unpack": T * out_row_bytes + B * N * out_row_bytes + B * N + 4 * (B + 1),
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            self.fh = os.fdopen(fd, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------ CPU oracle
+
+def oracle_call(w, stage_masks, images):
+    """One oracle pack-attend-unpack over the given images of every stage; returns tokens done."""
+    sys.path.insert(0, ROOT)
+    from oracle import oracle as O
+    sel = torch.as_tensor(images, dtype=torch.long)
+    q, k, v = w.q[sel], w.k[sel], w.v[sel]
+    tokens = 0
+    for m in stage_masks:
+        ms = m[sel]
+        qp, cu = O.pack(ms, q)
+        kp, _ = O.pack(ms, k)
+        vp, _ = O.pack(ms, v)
+        o = O.attend(qp, kp, vp, cu, w.H, 64, dtype=w.dtype)
+        O.unpack(o, cu, ms)
+        tokens += int(cu[-1])
+    return tokens
+
+
+def cpu_baseline(w, budget_s=10.0):
+    """The oracle, as it stands, on whole calls of the workload until about `budget_s` of CPU time."""
+    from oracle import oracle as O
+    O.load()
+    imgs = list(range(w.B))
+    t0 = time.perf_counter()
+    tokens, calls = 0, 0
+    while True:
+        tokens += oracle_call(w, w.masks, imgs)
+        calls += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": tokens / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{calls} whole call(s) of {w.name} (all {w.B} images, {len(w.masks)} stage(s)), "
+                      f"single-threaded float64 C, {dt:.1f} s"}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = workloads.by_name(args.workload)
+    from oracle import oracle as O
+    O.load()
+    per_step = max(1, min(w.B, args.ref_images))
+    order = list(range(w.B))
+    step_tokens, step_times = [], []
+    for i in range(args.warmup + args.steps):
+        imgs = [order[(i * per_step + j) % w.B] for j in range(per_step)]
+        t0 = time.perf_counter()
+        tok = oracle_call(w, w.masks, imgs)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            step_tokens.append(tok)
+            step_times.append(dt)
+    total_t = sum(step_times)
+    value = sum(step_tokens) / total_t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d": 64, "stages": len(w.masks),
+                   "seed": w.seed, "recipe": w.recipe, "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{per_step} image(s) of {w.name} per step, every stage, single-threaded"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------ GPU arm
+
+class Pipeline:
+    """Device buffers + one CUDA graph of the whole call (all stages), with timing events."""
+
+    def __init__(self, w, out_dtype, stream):
+        self.w = w
+        dev = "cuda"
+        self.masks = [m.to(dev) for m in w.masks]
+        self.q, self.k, self.v = (t.to(dev) for t in (w.q, w.k, w.v))
+        self.bufs = rra.Buffers(w.B, w.N, w.H, w.q.dtype, out_dtype=out_dtype)
+        self.ys = [torch.empty(w.B, w.N, w.H, 64, dtype=self.bufs.y.dtype, device=dev) for _ in self.masks]
+        self.stream = stream
+        self.graph = None
+        self.events = None
+
+    def enqueue(self, events=None):
+        b = self.bufs
+        s = self.stream
+        for i, m in enumerate(self.masks):
+            if events:
+                events[3 * i].record(s)
+            rra.rra_pack(m, [self.q, self.k, self.v], b.packed, b.cu, dev_error=b.err, stream=s)
+            if events:
+                events[3 * i + 1].record(s)
+            rra.rra_attend(b.packed[0], b.packed[1], b.packed[2], b.o, b.cu, max_seqlen=self.w.N,
+                           dev_error=b.err, stream=s)
+            if events:
+                events[3 * i + 2].record(s)
+            rra.rra_unpack(b.o, b.cu, m, self.ys[i], fill_mode=0, dev_error=b.err, stream=s)
+        if events:
+            events[3 * len(self.masks)].record(s)
+
+    def capture(self):
+        with torch.cuda.stream(self.stream):
+            self.enqueue()
+        torch.cuda.synchronize()
+        n_ev = 3 * len(self.masks) + 1
+        events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
+        g = torch.cuda.CUDAGraph()
+        try:
+            with torch.cuda.graph(g, stream=self.stream):
+                self.enqueue(events)
+            self.graph, self.events = g, events
+        except Exception:  # event-record nodes unavailable: graph without per-kernel events
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream):
+                self.enqueue()
+            self.graph, self.events = g, None
+        torch.cuda.synchronize()
+
+
+def main_gpu(args):
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev_index = torch.cuda.current_device()
+    w = workloads.by_name(args.workload)
+    stream = torch.cuda.Stream()
+    out_dtype = torch.float32 if args.out == "f32" else None
+    pipe = Pipeline(w, out_dtype, stream)
+    pipe.capture()
+    stages = len(w.masks)
+    lengths = w.lengths
+    T_call = int(sum(int(l.sum()) for l in lengths))
+    row_bytes = w.H * 64 * w.q.element_size()
+    out_row_bytes = w.H * 64 * pipe.bufs.o.element_size()
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def step(record_kernels):
+        with torch.cuda.stream(stream):
+            flush.fill_(step.counter & 0xFF)
+            step.counter += 1
+            start.record(stream)
+            pipe.graph.replay()
+            end.record(stream)
+    step.counter = 0
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+    step_ms = []
+    kern_ms = {k: [] for k in KERNELS}
+    with ClockSampler(dev_index) as clk:
+        for _ in range(args.steps):
+            step(True)
+            stream.synchronize()
+            step_ms.append(start.elapsed_time(end))
+            if pipe.events is not None:
+                ev = pipe.events
+                for s in range(stages):
+                    kern_ms["pack"].append(ev[3 * s].elapsed_time(ev[3 * s + 1]))
+                    kern_ms["attend"].append(ev[3 * s + 1].elapsed_time(ev[3 * s + 2]))
+                    kern_ms["unpack"].append(ev[3 * s + 2].elapsed_time(ev[3 * s + 3] if s + 1 == stages
+                                                                        else ev[3 * (s + 1)]))
+    torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    err = rra.rra_get_device_error(pipe.bufs.err, stream)
+    if err != 0:
+        raise RuntimeError(f"device error {rra.rra_status_string(err)} in the timed region")
+
+    total_ms = float(sum(step_ms))
+    if ws > 1:
+        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = ws * args.steps * T_call / (total_ms * 1e-3)
+
+    # dispatch floor: host time to enqueue one graph replay, and one eager call through the API
+    torch.cuda.synchronize()
+    n_disp = 200
+    with torch.cuda.stream(stream):
+        t0 = time.perf_counter()
+        for _ in range(n_disp):
+            pipe.graph.replay()
+        host_graph_us = (time.perf_counter() - t0) / n_disp * 1e6
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(n_disp):
+            pipe.enqueue()
+        host_eager_us = (time.perf_counter() - t0) / n_disp * 1e6
+        torch.cuda.synchronize()
+    # back-to-back replays (warm L2): device time per call including graph launch gaps
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(n_disp):
+            pipe.graph.replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    warm_us = start.elapsed_time(end) / n_disp * 1e3
+
+    # ---- roofline of the dominant kernel
+    hbm_peak, peak_kind = peaks()
+    alg = {k: 0 for k in KERNELS}
+    for l in lengths:
+        a = algorithmic_bytes(w, l, row_bytes, out_row_bytes)
+        for k in KERNELS:
+            alg[k] += a[k]
+    kern_us = {k: (1e3 * statistics.mean(v) * stages if v else None) for k, v in kern_ms.items()}  # per call
+    roofline = None
+    per_kernel = {}
+    if all(v is not None for v in kern_us.values()):
+        for k in KERNELS:
+            per_launch_bytes = alg[k] / stages
+            per_launch_us = kern_us[k] / stages
+            per_kernel[k] = {"us_per_launch": per_launch_us, "gbs": per_launch_bytes / (per_launch_us * 1e3),
+                             "alg_bytes_per_launch": per_launch_bytes,
+                             "frac_of_hbm": per_launch_bytes / (per_launch_us * 1e3) / hbm_peak}
+        dom = max(KERNELS, key=lambda k: kern_us[k])
+        ach = per_kernel[dom]["gbs"]
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": ach / hbm_peak, "peak_source": peak_kind,
+                    "traffic": ncu_traffic(dom, w.name)}
+    flops = sum(4 * 64 * w.H * int((l.astype(np.int64) ** 2).sum()) for l in lengths)
+    attn_tflops = flops / (kern_us["attend"] * 1e-6) / 1e12 if kern_us["attend"] else None
+
+    # ---- end to end through the public API: pinned host inputs in, padded result out
+    e2e = None
+    if not args.no_e2e:
+        host_in = [t.pin_memory() for t in (w.q, w.k, w.v)]
+        host_masks = [m.pin_memory() for m in w.masks]
+        host_out = [torch.empty(pipe.ys[0].shape, dtype=pipe.ys[0].dtype).pin_memory() for _ in w.masks]
+        dq, dk, dv = (torch.empty(w.q.shape, dtype=w.q.dtype, device="cuda") for _ in range(3))
+        dmasks = [torch.empty(m.shape, dtype=m.dtype, device="cuda") for m in w.masks]
+        bufs = rra.Buffers(w.B, w.N, w.H, w.q.dtype, out_dtype=out_dtype)
+        e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                for d, h in zip((dq, dk, dv), host_in):
+                    d.copy_(h, non_blocking=True)
+                for d, h in zip(dmasks, host_masks):
+                    d.copy_(h, non_blocking=True)
+                for i, m in enumerate(dmasks):
+                    y = rra.forward(m, dq, dk, dv, bufs, stream=stream)
+                    host_out[i].copy_(y, non_blocking=True)
+        for _ in range(max(3, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        e2e_ms = []
+        for _ in range(args.steps):
+            with torch.cuda.stream(stream):
+                flush.fill_(1)
+                e_start.record(stream)
+            e2e_step()
+            with torch.cuda.stream(stream):
+                e_end.record(stream)
+            stream.synchronize()
+            e2e_ms.append(e_start.elapsed_time(e_end))
+        tot = float(sum(e2e_ms))
+        if ws > 1:
+            t = torch.tensor([tot], device="cuda", dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            tot = float(t.item())
+        h2d = 3 * w.q.numel() * w.q.element_size() + sum(m.numel() for m in w.masks)
+        d2h = sum(t.numel() * t.element_size() for t in host_out)
+        e2e = {"value": ws * args.steps * T_call / (tot * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": tot / args.steps, "api": "rra.forward (eager)"}
+        if err == 0:
+            err2 = rra.rra_get_device_error(bufs.err, stream)
+            if err2 != 0:
+                raise RuntimeError(f"device error {rra.rra_status_string(err2)} in the e2e region")
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": {torch.bfloat16: "bf16", torch.float16: "f16"}[w.q.dtype],
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d": 64, "stages": stages,
+                       "tokens_per_call": T_call, "seed": w.seed, "recipe": w.recipe,
+                       "out_dtype": str(pipe.bufs.o.dtype).replace("torch.", ""),
+                       "l2": "flushed before every timed step (256 MiB write, untimed)",
+                       "parallelism": f"replicas x{ws}"},
+            "us_per_call": ms_per_step * 1e3,
+            "us_per_call_warm_back_to_back": warm_us,
+            "host_dispatch_us": {"graph_replay": host_graph_us, "eager_three_calls": host_eager_us},
+            "kernels": per_kernel,
+            "attention_tflops": attn_tflops,
+            "roofline": roofline,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "clocks": clk.summary(),
+            "gpu_launches": args.steps * 3 * stages,
+        }
+        print(json.dumps(line), flush=True)
+    del pipe
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c2", help="c1 | c2 | c3:B | c4 | c5:r:B | c5s:B")
+    ap.add_argument("--out", choices=["native", "f32"], default="native")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-images", type=int, default=16, help="images per step of the reference arm")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return main_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

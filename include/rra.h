@@ -1,0 +1,165 @@
+/*
+ * rra.h -- C ABI of the ragged varlen attention library (librra.so) for token-pruned ViTs.
+ *
+ * The library implements the pack -> attend -> unpack pipeline of "Dispatch-Aware Ragged
+ * Attention for Pruned Vision Transformers" (sota2.com paper card, Abstract; aissential.tech
+ * summary, Method) as hand-written CUDA kernels for sm_100a (B200):
+ *
+ *   rra_pack    keep mask -> per-image kept counts -> cu_seqlens, and a gather of the kept
+ *               token rows of up to three padded tensors into a packed, padding-free layout
+ *               (the summary's "two-phase token packer": index computation, then gather);
+ *   rra_attend  bidirectional (non-causal) softmax(Q K^T * scale) V, independently per image
+ *               and head, over the variable-length sequences described by cu_seqlens
+ *               (the card's "lightweight bidirectional ... attention kernel");
+ *   rra_unpack  scatter of packed rows back to the padded layout, pruned rows zero-filled
+ *               (the card's "pack-attend-unpack pipeline").
+ *
+ * Layouts (all row-major, C-contiguous):
+ *   keep_mask   uint8  [B, N]        nonzero = the token survives pruning
+ *   padded      dtype  [B, N, H, d]  one row = H*d elements
+ *   packed      dtype  [capacity, H, d]; image b occupies rows cu_seqlens[b] .. cu_seqlens[b+1)-1,
+ *               its kept tokens in ascending original index order
+ *   cu_seqlens  int32  [B+1]         cu[0] = 0, cu[b+1] = cu[b] + L_b (the varlen convention)
+ *
+ * Conventions shared by every call:
+ *   - All pointers except the host arrays `src`/`dst` of rra_pack and `host_out` are DEVICE
+ *     pointers owned by the caller.  No call allocates, frees or synchronises: each only
+ *     enqueues kernels on `stream` (NULL = the legacy default stream), so the whole sequence
+ *     can be captured into a CUDA graph and replayed with new data in the same buffers.
+ *   - Synchronous errors (bad arguments, unsupported shapes, launch failures) are returned
+ *     before anything is enqueued, except RRA_ERR_CUDA from a failed launch.
+ *   - Data-dependent errors found by a kernel (more kept tokens than `capacity`, malformed
+ *     cu_seqlens, a bounded wait that ran out) are written to `dev_error`, an int32 device
+ *     word the caller zeroes before use: the first error code wins, later ones are dropped.
+ *     `dev_error` may be NULL, in which case those errors are not reported -- the kernels
+ *     still never read or write outside the buffers described here.
+ *   - Device pointers must be 16-byte aligned (the kernels move 16-byte vectors).
+ */
+#ifndef RRA_H
+#define RRA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *rra_stream_t;
+
+typedef enum {
+    RRA_OK = 0,
+    RRA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, misaligned pointer           */
+    RRA_ERR_UNSUPPORTED = 2,   /* shape or dtype outside what the kernels implement          */
+    RRA_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed                */
+    RRA_ERR_CAPACITY = 4,      /* device: more kept tokens than the packed buffer's capacity */
+    RRA_ERR_TIMEOUT = 5,       /* device: a bounded wait inside a kernel ran out             */
+    RRA_ERR_BAD_SEQLENS = 6    /* device: cu_seqlens decreasing, past capacity, or not
+                                  matching the keep mask                                     */
+} rra_status;
+
+typedef enum { RRA_F16 = 0, RRA_BF16 = 1, RRA_F32 = 2 } rra_dtype;
+
+/*
+ * rra_pack -- the token packer (aissential.tech summary, Method: "two-phase fused token packer";
+ * sota2.com card, Abstract: pruning drops uninformative patches before attention).
+ *
+ * Phase 1: L_b = number of nonzero bytes of keep_mask[b, :]; cu_seqlens[b+1] = sum_{b'<=b} L_b'.
+ * Phase 2: for every kept (b, n) and every tensor i < n_tensors,
+ *          dst[i][cu_seqlens[b] + rank(b, n)] = src[i][b, n]   (a byte copy of one row),
+ *          rank(b, n) = number of kept n' < n of image b.
+ * Rows of dst at or beyond T = cu_seqlens[B] are not written.
+ *
+ *   keep_mask   device uint8 [B, N]
+ *   B, N        images and padded tokens per image (B >= 0, N >= 1)
+ *   H, d        heads and head dim; one row is H*d elements of `dt` and must be a multiple
+ *               of 16 bytes
+ *   dt          element type of src/dst (any of rra_dtype; the copy is bitwise)
+ *   n_tensors   1..3 (typically Q, K, V)
+ *   src         HOST array of n_tensors device pointers, each [B, N, H, d]
+ *   dst         HOST array of n_tensors device pointers, each [capacity, H, d]
+ *   capacity    rows available in each dst (B*N always suffices); if T > capacity, rows at or
+ *               beyond capacity are not written and RRA_ERR_CAPACITY is raised on dev_error;
+ *               cu_seqlens still receives the true counts
+ *   cu_seqlens  device int32 [B+1], written
+ *   dev_error   device int32 or NULL
+ *   stream      CUDA stream
+ */
+rra_status rra_pack(const uint8_t *keep_mask, int B, int N, int H, int d, rra_dtype dt,
+                    int n_tensors, const void *const *src, void *const *dst, int64_t capacity,
+                    int32_t *cu_seqlens, int32_t *dev_error, rra_stream_t stream);
+
+/*
+ * rra_attend -- bidirectional ragged attention (sota2.com card, Abstract: a bidirectional
+ * attention kernel over the variable-length post-pruning sequences; aissential.tech summary,
+ * Method: the "specialized bidirectional ... attention kernel" fed by the packer).
+ *
+ * For every image b with L_b = cu_seqlens[b+1] - cu_seqlens[b], head h and i < L_b:
+ *     o[cu_seqlens[b]+i, h, :] = sum_j softmax_j(scale * q_i . k_j) v_j,   j over all L_b tokens.
+ * Inputs are fp16 or bf16, products and sums are accumulated in fp32, the output is written
+ * in out_dt (in_dt or RRA_F32).  Rows of o outside [0, T) are not written.
+ *
+ *   q, k, v        device [capacity, H, d] in in_dt (RRA_F16 or RRA_BF16)
+ *   o              device [capacity, H, d] in out_dt
+ *   cu_seqlens     device int32 [B+1], non-decreasing, cu_seqlens[B] <= capacity; an image
+ *                  that breaks this is skipped and RRA_ERR_BAD_SEQLENS raised on dev_error
+ *   B, H, d        images, heads, head dim (d must be 64)
+ *   max_seqlen     host upper bound on any L_b, used only to size the launch (longer
+ *                  sequences are still computed correctly); pass N if unsure
+ *   capacity       rows of q/k/v/o
+ *   softmax_scale  <= 0 selects 1/sqrt(d)
+ *   workspace      reserved (may be NULL); ws_bytes must be >= rra_attend_workspace_size()
+ *   dev_error      device int32 or NULL
+ */
+rra_status rra_attend(const void *q, const void *k, const void *v, void *o,
+                      const int32_t *cu_seqlens, int B, int H, int d, int max_seqlen,
+                      int64_t capacity, float softmax_scale, rra_dtype in_dt, rra_dtype out_dt,
+                      void *workspace, size_t ws_bytes, int32_t *dev_error, rra_stream_t stream);
+
+/* Bytes of device workspace rra_attend needs for these sizes (currently always 0). */
+size_t rra_attend_workspace_size(int B, int H, int max_seqlen);
+
+/*
+ * rra_unpack -- scatter back to the padded layout (sota2.com card, Abstract: the
+ * "pack-attend-unpack pipeline").
+ *
+ * For every (b, n): if keep_mask[b, n] != 0, dst[b, n] = packed[cu_seqlens[b] + rank(b, n)]
+ * (a byte copy of one row); otherwise the row is set to zero bytes (fill_mode 0) or left
+ * untouched (fill_mode 1).  A kept row whose source row is at or beyond `capacity`, or beyond
+ * cu_seqlens[b+1], is left untouched and RRA_ERR_BAD_SEQLENS / RRA_ERR_CAPACITY is raised.
+ *
+ *   packed      device [capacity, H, d] in dt
+ *   cu_seqlens  device int32 [B+1] (as written by rra_pack for the same mask)
+ *   keep_mask   device uint8 [B, N]
+ *   dst         device [B, N, H, d] in dt
+ */
+rra_status rra_unpack(const void *packed, const int32_t *cu_seqlens, const uint8_t *keep_mask,
+                      int B, int N, int H, int d, rra_dtype dt, int fill_mode, int64_t capacity,
+                      void *dst, int32_t *dev_error, rra_stream_t stream);
+
+/*
+ * rra_get_device_error -- copy the device error word to *host_out.  This SYNCHRONISES `stream`
+ * (it is the only call that does) and so must not be used inside stream capture.
+ */
+rra_status rra_get_device_error(const int32_t *dev_error, rra_stream_t stream, int32_t *host_out);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *rra_status_string(rra_status status);
+
+/*
+ * Debugging knob for the bounded waits inside rra_attend: the time, in nanoseconds of the
+ * GPU global timer, after which a wait for an asynchronous copy or tensor-core operation gives
+ * up, raises RRA_ERR_TIMEOUT and ends its block after draining the work it issued.  The default
+ * is 2e9 (two seconds); 0 makes every wait that is not already complete give up at once.
+ * Applies to launches enqueued after the call, process-wide.
+ */
+void rra_set_wait_timeout_ns(uint64_t timeout_ns);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int rra_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RRA_H */

@@ -1,0 +1,189 @@
+// api.cu -- the extern "C" boundary of librra.so (declared in include/rra.h): argument
+// validation, per-device attributes and kernel launches.  No call allocates or synchronises,
+// except rra_get_device_error, which reads the device error word back.
+#include <atomic>
+#include <mutex>
+
+#include "../../include/rra.h"
+#include "rra_internal.h"
+
+namespace {
+
+std::atomic<uint64_t> g_wait_ns{2000000000ull};
+
+int num_sms_of_current_device(int *out)
+{
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return -1;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 64 && cache[dev] > 0) {
+        *out = cache[dev];
+        return 0;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return -1;
+    if (dev < 64)
+        cache[dev] = n;
+    *out = n;
+    return 0;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int elem_size(rra_dtype dt)
+{
+    switch (dt) {
+    case RRA_F16:
+    case RRA_BF16: return 2;
+    case RRA_F32: return 4;
+    default: return 0;
+    }
+}
+
+constexpr int64_t kMaxRows = 0x7fffffffLL;
+
+}  // namespace
+
+extern "C" {
+
+rra_status rra_pack(const uint8_t *keep_mask, int B, int N, int H, int d, rra_dtype dt, int n_tensors,
+                    const void *const *src, void *const *dst, int64_t capacity, int32_t *cu_seqlens,
+                    int32_t *dev_error, rra_stream_t stream)
+{
+    if (keep_mask == nullptr || src == nullptr || dst == nullptr || cu_seqlens == nullptr)
+        return RRA_ERR_INVALID_ARG;
+    if (B < 0 || N < 1 || H < 1 || d < 1 || capacity < 1 || n_tensors < 1 || n_tensors > 3)
+        return RRA_ERR_INVALID_ARG;
+    const int es = elem_size(dt);
+    if (es == 0)
+        return RRA_ERR_UNSUPPORTED;
+    const int64_t row_bytes = static_cast<int64_t>(H) * d * es;
+    if (row_bytes % 16 != 0 || row_bytes > 8192)
+        return RRA_ERR_UNSUPPORTED;
+    if (B > 65535 || static_cast<int64_t>(B) * N > kMaxRows || capacity > kMaxRows)
+        return RRA_ERR_UNSUPPORTED;
+    for (int i = 0; i < n_tensors; ++i) {
+        if (src[i] == nullptr || dst[i] == nullptr)
+            return RRA_ERR_INVALID_ARG;
+        if (!aligned16(src[i]) || !aligned16(dst[i]))
+            return RRA_ERR_INVALID_ARG;
+    }
+    int sms = 0;
+    if (num_sms_of_current_device(&sms) != 0)
+        return RRA_ERR_CUDA;
+    const cudaError_t e = rra::launch_pack(keep_mask, B, N, row_bytes, n_tensors, src, dst, capacity, cu_seqlens,
+                                           dev_error, sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RRA_OK : RRA_ERR_CUDA;
+}
+
+rra_status rra_attend(const void *q, const void *k, const void *v, void *o, const int32_t *cu_seqlens, int B, int H,
+                      int d, int max_seqlen, int64_t capacity, float softmax_scale, rra_dtype in_dt,
+                      rra_dtype out_dt, void *workspace, size_t ws_bytes, int32_t *dev_error,
+                      rra_stream_t stream)
+{
+    (void)workspace;
+    if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || cu_seqlens == nullptr)
+        return RRA_ERR_INVALID_ARG;
+    if (B < 0 || H < 1 || capacity < 1 || max_seqlen < 0)
+        return RRA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return RRA_ERR_INVALID_ARG;
+    if (d != 64 || (in_dt != RRA_F16 && in_dt != RRA_BF16) || (out_dt != in_dt && out_dt != RRA_F32))
+        return RRA_ERR_UNSUPPORTED;
+    if (B > rra::kAttendMaxBatch || H > 65535 || capacity > kMaxRows)
+        return RRA_ERR_UNSUPPORTED;
+    if (ws_bytes < rra_attend_workspace_size(B, H, max_seqlen))
+        return RRA_ERR_INVALID_ARG;
+    if (!(softmax_scale == softmax_scale))
+        return RRA_ERR_INVALID_ARG;
+    int sms = 0;
+    if (num_sms_of_current_device(&sms) != 0)
+        return RRA_ERR_CUDA;
+    rra::AttendArgs a;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.o = o;
+    a.cu = cu_seqlens;
+    a.B = B;
+    a.H = H;
+    a.max_seqlen = max_seqlen;
+    a.capacity = capacity;
+    a.scale = softmax_scale > 0.f ? softmax_scale : 0.125f;  // 1/sqrt(64)
+    a.in_bf16 = in_dt == RRA_BF16;
+    a.out_dt = static_cast<int>(out_dt);
+    a.err = dev_error;
+    a.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+    const cudaError_t e = rra::launch_attend(a, sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RRA_OK : RRA_ERR_CUDA;
+}
+
+size_t rra_attend_workspace_size(int B, int H, int max_seqlen)
+{
+    (void)B;
+    (void)H;
+    (void)max_seqlen;
+    return 0;
+}
+
+rra_status rra_unpack(const void *packed, const int32_t *cu_seqlens, const uint8_t *keep_mask, int B, int N, int H,
+                      int d, rra_dtype dt, int fill_mode, int64_t capacity, void *dst, int32_t *dev_error,
+                      rra_stream_t stream)
+{
+    if (packed == nullptr || cu_seqlens == nullptr || keep_mask == nullptr || dst == nullptr)
+        return RRA_ERR_INVALID_ARG;
+    if (B < 0 || N < 1 || H < 1 || d < 1 || capacity < 1 || (fill_mode != 0 && fill_mode != 1))
+        return RRA_ERR_INVALID_ARG;
+    if (!aligned16(packed) || !aligned16(dst))
+        return RRA_ERR_INVALID_ARG;
+    const int es = elem_size(dt);
+    if (es == 0)
+        return RRA_ERR_UNSUPPORTED;
+    const int64_t row_bytes = static_cast<int64_t>(H) * d * es;
+    if (row_bytes % 16 != 0 || row_bytes > 8192)
+        return RRA_ERR_UNSUPPORTED;
+    if (B > 65535 || static_cast<int64_t>(B) * N > kMaxRows || capacity > kMaxRows)
+        return RRA_ERR_UNSUPPORTED;
+    int sms = 0;
+    if (num_sms_of_current_device(&sms) != 0)
+        return RRA_ERR_CUDA;
+    const cudaError_t e = rra::launch_unpack(packed, cu_seqlens, keep_mask, B, N, row_bytes, fill_mode, capacity,
+                                             dst, dev_error, sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RRA_OK : RRA_ERR_CUDA;
+}
+
+rra_status rra_get_device_error(const int32_t *dev_error, rra_stream_t stream, int32_t *host_out)
+{
+    if (dev_error == nullptr || host_out == nullptr)
+        return RRA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(host_out, dev_error, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return RRA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess)
+        return RRA_ERR_CUDA;
+    return RRA_OK;
+}
+
+const char *rra_status_string(rra_status status)
+{
+    switch (status) {
+    case RRA_OK: return "RRA_OK";
+    case RRA_ERR_INVALID_ARG: return "RRA_ERR_INVALID_ARG";
+    case RRA_ERR_UNSUPPORTED: return "RRA_ERR_UNSUPPORTED";
+    case RRA_ERR_CUDA: return "RRA_ERR_CUDA";
+    case RRA_ERR_CAPACITY: return "RRA_ERR_CAPACITY";
+    case RRA_ERR_TIMEOUT: return "RRA_ERR_TIMEOUT";
+    case RRA_ERR_BAD_SEQLENS: return "RRA_ERR_BAD_SEQLENS";
+    default: return "RRA_ERR_UNKNOWN";
+    }
+}
+
+void rra_set_wait_timeout_ns(uint64_t timeout_ns) { g_wait_ns.store(timeout_ns, std::memory_order_relaxed); }
+
+int rra_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,38 @@
+// rra_internal.h -- launchers shared between the kernel files and the C-ABI layer.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace rra {
+
+// Padded rows handled by one pack/unpack block (bounded by the block's shared rank table).
+constexpr int kMaxRowsPerSplit = 1024;
+
+cudaError_t launch_pack(const uint8_t *mask, int B, int N, int64_t row_bytes, int n_tensors,
+                        const void *const *src, void *const *dst, int64_t capacity, int32_t *cu, int32_t *err,
+                        int num_sms, cudaStream_t stream);
+
+cudaError_t launch_unpack(const void *packed, const int32_t *cu, const uint8_t *mask, int B, int N,
+                          int64_t row_bytes, int fill_mode, int64_t capacity, void *dst, int32_t *err, int num_sms,
+                          cudaStream_t stream);
+
+struct AttendArgs {
+    const void *q, *k, *v;
+    void *o;
+    const int32_t *cu;
+    int B, H, max_seqlen;
+    int64_t capacity;
+    float scale;
+    bool in_bf16;
+    int out_dt;  // rra_dtype of o
+    int32_t *err;
+    uint64_t wait_ns;
+};
+
+// Largest B rra_attend accepts (its per-block tile table lives in shared memory).
+constexpr int kAttendMaxBatch = 16384;
+
+cudaError_t launch_attend(const AttendArgs &a, int num_sms, cudaStream_t stream);
+
+}  // namespace rra

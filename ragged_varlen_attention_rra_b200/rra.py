@@ -1,0 +1,192 @@
+"""Thin Python binding of librra.so (the C ABI in include/rra.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA kernels.  PyTorch
+supplies device memory and the current stream.  If librra.so is missing or cannot be loaded,
+every function here raises -- there is no fallback.
+
+Names follow the C ABI: :func:`rra_pack`, :func:`rra_attend`, :func:`rra_unpack`,
+:func:`rra_get_device_error`, :func:`rra_status_string`, :func:`rra_attend_workspace_size`,
+:func:`rra_set_wait_timeout_ns`.  :func:`forward` chains the three calls (the whole
+pack-attend-unpack call of one pruning stage).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.environ.get("RRA_LIBRARY", os.path.join(_HERE, "librra.so"))
+
+RRA_OK, RRA_ERR_INVALID_ARG, RRA_ERR_UNSUPPORTED, RRA_ERR_CUDA = 0, 1, 2, 3
+RRA_ERR_CAPACITY, RRA_ERR_TIMEOUT, RRA_ERR_BAD_SEQLENS = 4, 5, 6
+RRA_F16, RRA_BF16, RRA_F32 = 0, 1, 2
+
+_DT = {torch.float16: RRA_F16, torch.bfloat16: RRA_BF16, torch.float32: RRA_F32}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class RRAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what} failed: {rra_status_string(status)} ({status})")
+
+
+def _declare(lib):
+    c = ctypes
+    vp, i32p = c.c_void_p, c.c_void_p
+    lib.rra_pack.argtypes = [vp, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int,
+                             c.POINTER(c.c_void_p), c.POINTER(c.c_void_p), c.c_int64, i32p, i32p, vp]
+    lib.rra_pack.restype = c.c_int
+    lib.rra_attend.argtypes = [vp, vp, vp, vp, i32p, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int64,
+                               c.c_float, c.c_int, c.c_int, vp, c.c_size_t, i32p, vp]
+    lib.rra_attend.restype = c.c_int
+    lib.rra_attend_workspace_size.argtypes = [c.c_int, c.c_int, c.c_int]
+    lib.rra_attend_workspace_size.restype = c.c_size_t
+    lib.rra_unpack.argtypes = [vp, i32p, vp, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int,
+                               c.c_int64, vp, i32p, vp]
+    lib.rra_unpack.restype = c.c_int
+    lib.rra_get_device_error.argtypes = [i32p, vp, c.POINTER(c.c_int32)]
+    lib.rra_get_device_error.restype = c.c_int
+    lib.rra_status_string.argtypes = [c.c_int]
+    lib.rra_status_string.restype = c.c_char_p
+    lib.rra_set_wait_timeout_ns.argtypes = [c.c_uint64]
+    lib.rra_set_wait_timeout_ns.restype = None
+    lib.rra_version.argtypes = []
+    lib.rra_version.restype = c.c_int
+    return lib
+
+
+def lib():
+    """The loaded librra.so (ctypes handle).  Raises if the library is missing."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise ImportError(
+                        f"librra.so not found at {LIB_PATH}; build it with "
+                        "`python -m ragged_varlen_attention_rra_b200.build` (no CPU fallback exists)")
+                _lib = _declare(ctypes.CDLL(LIB_PATH))
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(status: int, what: str):
+    if status != RRA_OK:
+        raise RRAError(status, what)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("rra calls take contiguous CUDA tensors")
+
+
+# ------------------------------------------------------------------------------------ calls
+
+def rra_status_string(status: int) -> str:
+    return lib().rra_status_string(int(status)).decode()
+
+
+def rra_attend_workspace_size(B: int, H: int, max_seqlen: int) -> int:
+    return int(lib().rra_attend_workspace_size(B, H, max_seqlen))
+
+
+def rra_set_wait_timeout_ns(ns: int) -> None:
+    lib().rra_set_wait_timeout_ns(int(ns))
+
+
+def rra_get_device_error(dev_error: torch.Tensor, stream=None) -> int:
+    """Read the device error word (synchronises the stream)."""
+    out = ctypes.c_int32(0)
+    _check(lib().rra_get_device_error(_ptr(dev_error), _stream(stream), ctypes.byref(out)), "rra_get_device_error")
+    return int(out.value)
+
+
+def rra_pack(mask: torch.Tensor, srcs: Sequence[torch.Tensor], dsts: Sequence[torch.Tensor],
+             cu_seqlens: torch.Tensor, capacity: Optional[int] = None,
+             dev_error: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Keep mask [B, N] + padded srcs [B, N, H, d] -> packed dsts [capacity, H, d] and cu_seqlens [B+1]."""
+    _require_cuda(mask, cu_seqlens, dev_error, *srcs, *dsts)
+    B, N = mask.shape
+    H, d = srcs[0].shape[2], srcs[0].shape[3]
+    cap = dsts[0].shape[0] if capacity is None else capacity
+    n = len(srcs)
+    src_arr = (ctypes.c_void_p * n)(*[s.data_ptr() for s in srcs])
+    dst_arr = (ctypes.c_void_p * n)(*[t.data_ptr() for t in dsts])
+    st = lib().rra_pack(_ptr(mask), B, N, H, d, _DT[srcs[0].dtype], n, src_arr, dst_arr, cap,
+                        _ptr(cu_seqlens), _ptr(dev_error), _stream(stream))
+    _check(st, "rra_pack")
+
+
+def rra_attend(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, cu_seqlens: torch.Tensor,
+               max_seqlen: int, softmax_scale: float = 0.0, dev_error: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Packed q/k/v [capacity, H, 64] + cu_seqlens [B+1] -> packed o (o's dtype selects the output type)."""
+    _require_cuda(q, k, v, o, cu_seqlens, dev_error, workspace)
+    B = cu_seqlens.shape[0] - 1
+    cap, H, d = q.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().rra_attend(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cu_seqlens), B, H, d, int(max_seqlen), cap,
+                          float(softmax_scale), _DT[q.dtype], _DT[o.dtype], _ptr(workspace), ws_bytes,
+                          _ptr(dev_error), _stream(stream))
+    _check(st, "rra_attend")
+
+
+def rra_unpack(packed: torch.Tensor, cu_seqlens: torch.Tensor, mask: torch.Tensor, dst: torch.Tensor,
+               fill_mode: int = 0, capacity: Optional[int] = None, dev_error: Optional[torch.Tensor] = None,
+               stream=None) -> None:
+    """Packed [capacity, H, d] -> padded dst [B, N, H, d]; pruned rows zero (fill_mode 0) or untouched (1)."""
+    _require_cuda(packed, cu_seqlens, mask, dst, dev_error)
+    B, N = mask.shape
+    cap, H, d = packed.shape if capacity is None else (capacity,) + tuple(packed.shape[1:])
+    st = lib().rra_unpack(_ptr(packed), _ptr(cu_seqlens), _ptr(mask), B, N, H, d, _DT[packed.dtype],
+                          int(fill_mode), cap, _ptr(dst), _ptr(dev_error), _stream(stream))
+    _check(st, "rra_unpack")
+
+
+# ------------------------------------------------------------------------------------ whole call
+
+class Buffers:
+    """Device buffers for one pack-attend-unpack call at capacity B*N (reused across calls)."""
+
+    def __init__(self, B: int, N: int, H: int, dtype: torch.dtype, out_dtype: Optional[torch.dtype] = None,
+                 device="cuda"):
+        cap = max(1, B * N)
+        self.B, self.N, self.H, self.capacity = B, N, H, cap
+        self.packed = [torch.empty(cap, H, 64, dtype=dtype, device=device) for _ in range(3)]
+        od = out_dtype or dtype
+        self.o = torch.empty(cap, H, 64, dtype=od, device=device)
+        self.y = torch.empty(B, N, H, 64, dtype=od, device=device)
+        self.cu = torch.empty(B + 1, dtype=torch.int32, device=device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def forward(mask: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bufs: Buffers,
+            softmax_scale: float = 0.0, stream=None) -> torch.Tensor:
+    """One pruning stage: pack the kept tokens of q/k/v, attend per image and head, unpack to padded.
+
+    All three calls are enqueued on `stream` without any host synchronisation; the padded
+    result is bufs.y (pruned rows zero)."""
+    rra_pack(mask, [q, k, v], bufs.packed, bufs.cu, dev_error=bufs.err, stream=stream)
+    rra_attend(bufs.packed[0], bufs.packed[1], bufs.packed[2], bufs.o, bufs.cu, max_seqlen=mask.shape[1],
+               softmax_scale=softmax_scale, dev_error=bufs.err, stream=stream)
+    rra_unpack(bufs.o, bufs.cu, mask, bufs.y, fill_mode=0, dev_error=bufs.err, stream=stream)
+    return bufs.y
