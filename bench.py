@@ -348,26 +348,28 @@ def main_gpu(args):
 
     # dispatch floor: host time to enqueue one graph replay, and one eager call through the API
     torch.cuda.synchronize()
-    n_disp = 200
+    n_disp = 0 if args.profile else 200
     with torch.cuda.stream(stream):
         t0 = time.perf_counter()
         for _ in range(n_disp):
             pipe.graph.replay()
-        host_graph_us = (time.perf_counter() - t0) / n_disp * 1e6
+        host_graph_us = (time.perf_counter() - t0) / max(n_disp, 1) * 1e6
         torch.cuda.synchronize()
         t0 = time.perf_counter()
         for _ in range(n_disp):
             pipe.enqueue()
-        host_eager_us = (time.perf_counter() - t0) / n_disp * 1e6
+        host_eager_us = (time.perf_counter() - t0) / max(n_disp, 1) * 1e6
         torch.cuda.synchronize()
     # back-to-back replays (warm L2): device time per call including graph launch gaps
-    with torch.cuda.stream(stream):
-        start.record(stream)
-        for _ in range(n_disp):
-            pipe.graph.replay()
-        end.record(stream)
-    torch.cuda.synchronize()
-    warm_us = start.elapsed_time(end) / n_disp * 1e3
+    warm_us = None
+    if n_disp:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(n_disp):
+                pipe.graph.replay()
+            end.record(stream)
+        torch.cuda.synchronize()
+        warm_us = start.elapsed_time(end) / n_disp * 1e3
 
     # ---- roofline of the dominant kernel
     hbm_peak, peak_kind = peaks()
@@ -396,7 +398,7 @@ def main_gpu(args):
 
     # ---- end to end through the public API: pinned host inputs in, padded result out
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.profile:
         host_in = [t.pin_memory() for t in (w.q, w.k, w.v)]
         host_masks = [m.pin_memory() for m in w.masks]
         host_out = [torch.empty(pipe.ys[0].shape, dtype=pipe.ys[0].dtype).pin_memory() for _ in w.masks]
@@ -442,7 +444,7 @@ def main_gpu(args):
                 raise RuntimeError(f"device error {rra.rra_status_string(err2)} in the e2e region")
 
     cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline and not args.profile:
         cpu = cpu_baseline(w, args.cpu_seconds)
 
     if rank == 0:
@@ -483,6 +485,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="c2", help="c1 | c2 | c3:B | c4 | c5:r:B | c5s:B")
     ap.add_argument("--out", choices=["native", "f32"], default="native")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="timed steps only (no dispatch loops, e2e or CPU leg): the command ncu captures")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-images", type=int, default=16, help="images per step of the reference arm")

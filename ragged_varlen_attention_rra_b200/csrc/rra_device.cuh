@@ -65,10 +65,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return done != 0;
 }
 
+// Non-blocking probe of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 // Wait until the phase with the given parity of `bar` completes, or until `limit_ns` of GPU
-// global time has passed.  Returns false on timeout.  Never spins unboundedly.
+// global time has passed.  Returns false on timeout.  Never spins unboundedly.  A zero limit
+// is a single non-blocking probe (try_wait may suspend the thread in hardware for a while).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
 {
+    if (limit_ns == 0)
+        return mbar_test_wait(bar, parity);
     if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = global_timer_ns();
