@@ -3,13 +3,16 @@
 // Method -- a two-phase packer, index computation then gather; sota2.com card, Abstract -- the
 // pack-attend-unpack pipeline back to the padded layout).
 //
-// Both kernels are HBM-bound byte movers.  A block owns a range of padded rows of one image
-// (grid = splits x images).  It derives everything it needs from the keep mask itself:
-//   * the packed start of its image, cu[b] = number of nonzero mask bytes of images < b
-//     (pack only; a block-wide count with 16-byte loads, so no second launch and no
-//     inter-block wait is needed), and
-//   * the rank of each kept row inside the image (warp ballots + a block prefix),
-// then moves rows as 16-byte vectors, eight independent loads in flight per thread.
+// Both kernels are HBM-bound row movers.  A block owns up to 256 padded rows of one image
+// (grid = splits x images) and derives everything it needs from the keep mask in one pass:
+//   * pack: the packed start of its image (nonzero mask bytes of images < b), the rank of its
+//     first row inside the image, and the image length, counted together from 16-byte mask
+//     chunks and reduced once -- so no second launch and no inter-block wait is needed;
+//   * both: the slot of every kept row of its range (warp ballots + one block prefix).
+// Rows then move as 16-byte vectors, one warp per row, every load of a row (all tensors) in
+// flight before its stores.
+#include <type_traits>
+
 #include "rra_device.cuh"
 #include "rra_internal.h"
 
@@ -19,7 +22,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBatch = 8;  // 16-byte vectors in flight per thread
+constexpr int kChunkBatch = 4;  // 16-byte mask chunks in flight per thread
 
 struct SrcPtrs { const uint8_t *p[3]; };
 struct DstPtrs { uint8_t *p[3]; };
@@ -33,212 +36,223 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *p)
     return v;
 }
 
-__device__ __forceinline__ int block_sum(int v, int *red)
+// Bit k of the result is set iff byte k of the 16-byte chunk is nonzero.
+__device__ __forceinline__ uint32_t kept_bits16(uint4 c)
 {
-    v = __reduce_add_sync(0xffffffffu, v);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __syncthreads();  // red[] may still be read by a previous call
-    if (lane == 0)
-        red[warp] = v;
-    __syncthreads();
-    int total = 0;
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    uint32_t m = 0;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w)
-        total += red[w];
-    return total;
-}
-
-// Number of nonzero bytes in p[0, n), computed by the whole block.
-__device__ int block_count_nonzero(const uint8_t *p, int64_t n, int *red)
-{
-    int local = 0;
-    if (n > 0) {
-        const uintptr_t addr = reinterpret_cast<uintptr_t>(p);
-        const int64_t align_gap = static_cast<int64_t>((16u - (addr & 15u)) & 15u);
-        const int64_t head = n < align_gap ? n : align_gap;
-        if (threadIdx.x < head)
-            local += p[threadIdx.x] != 0;
-        const uint4 *body = reinterpret_cast<const uint4 *>(p + head);
-        const int64_t nvec = (n - head) >> 4;
-        for (int64_t i0 = threadIdx.x; i0 < nvec; i0 += static_cast<int64_t>(kThreads) * kBatch) {
-            uint4 v[kBatch];
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                const int64_t i = i0 + static_cast<int64_t>(u) * kThreads;
-                v[u] = (i < nvec) ? __ldg(body + i) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u)
-                local += nonzero_bytes(v[u].x) + nonzero_bytes(v[u].y) + nonzero_bytes(v[u].z) +
-                         nonzero_bytes(v[u].w);
-        }
-        const int64_t tail0 = head + (nvec << 4);
-        if (tail0 + threadIdx.x < n)
-            local += p[tail0 + threadIdx.x] != 0;
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t t = (((w[i] & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w[i]) & 0x80808080u;
+        const uint32_t nib = ((t >> 7) & 1u) | ((t >> 14) & 2u) | ((t >> 21) & 4u) | ((t >> 28) & 8u);
+        m |= nib << (4 * i);
     }
-    return block_sum(local, red);
+    return m;
 }
 
-// Scan mask row bytes [n0, n1): for every kept position write its local rank slot into
-// `slot_of` (indexed n - n0; -1 when pruned).  Returns the number of kept positions.
-__device__ int block_scan_row(const uint8_t *row, int n0, int n1, int16_t *slot_of, int *warp_tot)
+// Bits k (0..15) with lo <= s + k < hi.
+__device__ __forceinline__ uint32_t range_bits16(int64_t s, int64_t lo, int64_t hi)
+{
+    const int64_t a = lo - s, b = hi - s;
+    const int l = a < 0 ? 0 : (a > 16 ? 16 : static_cast<int>(a));
+    const int h = b < 0 ? 0 : (b > 16 ? 16 : static_cast<int>(b));
+    return h > l ? (((1u << h) - 1u) & ~((1u << l) - 1u)) : 0u;
+}
+
+// Per-thread counts of nonzero mask bytes (byte indices relative to `mask`) in [0, r0),
+// [r0, r1) and [r0, r2), r0 <= r1 <= r2, read as 16-byte-aligned chunks.  Bytes outside
+// [0, r2) are ignored; an aligned 16-byte chunk never crosses a page, so reading the whole
+// chunk around either end of the range cannot fault.
+struct Counts { int before, upto, total; };
+
+__device__ __forceinline__ Counts count_ranges(const uint8_t *mask, int64_t r0, int64_t r1, int64_t r2)
+{
+    const uintptr_t addr = reinterpret_cast<uintptr_t>(mask);
+    const int off = static_cast<int>(addr & 15u);
+    const uint4 *base = reinterpret_cast<const uint4 *>(addr - off);
+    const int64_t nchunks = (off + r2 + 15) >> 4;
+    Counts c{0, 0, 0};
+    for (int64_t j0 = threadIdx.x; j0 < nchunks; j0 += static_cast<int64_t>(kThreads) * kChunkBatch) {
+        uint4 v[kChunkBatch];
+#pragma unroll
+        for (int u = 0; u < kChunkBatch; ++u) {
+            const int64_t j = j0 + static_cast<int64_t>(u) * kThreads;
+            v[u] = j < nchunks ? __ldg(base + j) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kChunkBatch; ++u) {
+            const int64_t s = (j0 + static_cast<int64_t>(u) * kThreads) * 16 - off;
+            const uint32_t m = kept_bits16(v[u]) & range_bits16(s, 0, r2);
+            c.before += __popc(m & range_bits16(s, 0, r0));
+            c.upto += __popc(m & range_bits16(s, r0, r1));
+            c.total += __popc(m & range_bits16(s, r0, r2));
+        }
+    }
+    return c;
+}
+
+struct BlockScan {
+    int before, upto, total;  // block-wide sums of Counts
+    int nk;                   // kept rows in the block's range
+};
+
+// One barrier round: reduces the three counts and prefixes the kept flags of rows [n0, n1)
+// (one row per thread).  slot_of[i] = slot of row n0+i among the kept rows of the range, or
+// -1; n_of_slot[slot] = i.
+__device__ __forceinline__ BlockScan block_scan(Counts c, const uint8_t *row, int n0, int n1, int16_t *slot_of,
+                                                int16_t *n_of_slot, int (*part)[4])
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int running = 0;
-    for (int c0 = n0; c0 < n1; c0 += kThreads) {
-        const int n = c0 + threadIdx.x;
-        const bool keep = (n < n1) && row[n] != 0;
-        const unsigned bal = __ballot_sync(0xffffffffu, keep);
-        __syncthreads();
-        if (lane == 0)
-            warp_tot[warp] = __popc(bal);
-        __syncthreads();
-        int before = 0, chunk = 0;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const int t = warp_tot[w];
-            before += (w < warp) ? t : 0;
-            chunk += t;
-        }
-        if (n < n1)
-            slot_of[n - n0] = keep ? static_cast<int16_t>(running + before + __popc(bal & ((1u << lane) - 1u)))
-                                   : static_cast<int16_t>(-1);
-        running += chunk;
+    const int n = n0 + static_cast<int>(threadIdx.x);
+    const bool keep = n < n1 && row[n] != 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    c.before = __reduce_add_sync(0xffffffffu, c.before);
+    c.upto = __reduce_add_sync(0xffffffffu, c.upto);
+    c.total = __reduce_add_sync(0xffffffffu, c.total);
+    if (lane == 0) {
+        part[warp][0] = c.before;
+        part[warp][1] = c.upto;
+        part[warp][2] = c.total;
+        part[warp][3] = __popc(bal);
     }
     __syncthreads();
-    return running;
+    BlockScan r{0, 0, 0, 0};
+    int warp_base = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        r.before += part[w][0];
+        r.upto += part[w][1];
+        r.total += part[w][2];
+        warp_base += (w < warp) ? part[w][3] : 0;
+        r.nk += part[w][3];
+    }
+    if (n < n1) {
+        const int slot = keep ? warp_base + __popc(bal & ((1u << lane) - 1u)) : -1;
+        slot_of[threadIdx.x] = static_cast<int16_t>(slot);
+        if (keep)
+            n_of_slot[slot] = static_cast<int16_t>(threadIdx.x);
+    }
+    __syncthreads();
+    return r;
 }
 
-__global__ void __launch_bounds__(kThreads) pack_kernel(const uint8_t *__restrict__ mask, int B, int N,
-                                                        int rows_per_split, int vec_per_row, int n_tensors,
-                                                        SrcPtrs src, DstPtrs dst, int64_t capacity,
-                                                        int32_t *__restrict__ cu, int32_t *err)
+template <int VPL>
+__global__ void __launch_bounds__(kThreads) pack_kernel(const uint8_t *__restrict__ mask, int N, int rows_per_split,
+                                                        int V, int n_tensors, SrcPtrs src, DstPtrs dst,
+                                                        int64_t capacity, int32_t *__restrict__ cu, int32_t *err)
 {
-    __shared__ int red[kWarps];
-    __shared__ int warp_tot[kWarps];
-    __shared__ int16_t slot_of[kMaxRowsPerSplit];
-    __shared__ int16_t n_of_slot[kMaxRowsPerSplit];
+    __shared__ int part[kWarps][4];
+    __shared__ int16_t slot_of[kThreads];
+    __shared__ int16_t n_of_slot[kThreads];
 
     const int b = blockIdx.y;
     const int n0 = blockIdx.x * rows_per_split;
     if (n0 >= N)
         return;
     const int n1 = min(N, n0 + rows_per_split);
-    const uint8_t *row = mask + static_cast<int64_t>(b) * N;
+    const int64_t img0 = static_cast<int64_t>(b) * N;
 
-    // Phase 1: where this image starts in the packed layout, and where this split starts in it.
-    const int64_t image_start = block_count_nonzero(mask, static_cast<int64_t>(b) * N, red);
-    const int rank0 = block_count_nonzero(row, n0, red);
-    if (blockIdx.x == 0) {
-        const int Lb = block_count_nonzero(row, N, red);
-        if (threadIdx.x == 0) {
-            if (b == 0)
-                cu[0] = 0;
-            cu[b + 1] = static_cast<int32_t>(image_start + Lb);
-            if (image_start + Lb > capacity)
-                raise_error(err, RRA_ERR_CAPACITY);
-        }
+    // Phase 1: image start, rank of row n0 inside the image, image length -- one pass.
+    const Counts c = count_ranges(mask, img0, img0 + n0, img0 + N);
+    const BlockScan s = block_scan(c, mask + img0, n0, n1, slot_of, n_of_slot, part);
+    const int64_t image_start = s.before;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        if (b == 0)
+            cu[0] = 0;
+        cu[b + 1] = static_cast<int32_t>(image_start + s.total);
+        if (image_start + s.total > capacity)
+            raise_error(err, RRA_ERR_CAPACITY);
     }
-    const int nk = block_scan_row(row, n0, n1, slot_of, warp_tot);
-    for (int i = threadIdx.x; i < n1 - n0; i += kThreads)
-        if (slot_of[i] >= 0)
-            n_of_slot[slot_of[i]] = static_cast<int16_t>(i);
-    __syncthreads();
 
-    // Phase 2: gather, 16-byte vectors; work index = ((slot * n_tensors) + tensor) * V + vec.
-    const int64_t out_row0 = image_start + rank0;
-    const int V = vec_per_row;
-    const int total = nk * n_tensors * V;
-    for (int i0 = threadIdx.x; i0 < total; i0 += kThreads * kBatch) {
-        uint4 val[kBatch];
-        uint4 *dptr[kBatch];
+    // Phase 2: one warp per kept row, all tensors' vectors loaded before any store.
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t out0 = image_start + s.upto;
+    for (int slot = warp; slot < s.nk; slot += kWarps) {
+        const int64_t out_row = out0 + slot;
+        if (out_row >= capacity)
+            break;
+        const int64_t in_row = img0 + n0 + n_of_slot[slot];
+        uint4 buf[3][VPL];
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int i = i0 + u * kThreads;
-            dptr[u] = nullptr;
-            if (i < total) {
-                const int pair = i / V;
-                const int vec = i - pair * V;
-                const int slot = pair / n_tensors;
-                const int t = pair - slot * n_tensors;
-                const int64_t out_row = out_row0 + slot;
-                if (out_row < capacity) {
-                    const int64_t in_row = static_cast<int64_t>(b) * N + n0 + n_of_slot[slot];
-                    const uint8_t *sp = t == 0 ? src.p[0] : (t == 1 ? src.p[1] : src.p[2]);
-                    uint8_t *dp = t == 0 ? dst.p[0] : (t == 1 ? dst.p[1] : dst.p[2]);
-                    val[u] = ld_stream(reinterpret_cast<const uint4 *>(sp) + in_row * V + vec);
-                    dptr[u] = reinterpret_cast<uint4 *>(dp) + out_row * V + vec;
-                }
+        for (int t = 0; t < 3; ++t) {
+            if (t < n_tensors) {
+                const uint4 *sp =
+                    reinterpret_cast<const uint4 *>(t == 0 ? src.p[0] : (t == 1 ? src.p[1] : src.p[2])) + in_row * V;
+#pragma unroll
+                for (int k = 0; k < VPL; ++k)
+                    if (lane + 32 * k < V)
+                        buf[t][k] = ld_stream(sp + lane + 32 * k);
             }
         }
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u)
-            if (dptr[u] != nullptr)
-                *dptr[u] = val[u];
+        for (int t = 0; t < 3; ++t) {
+            if (t < n_tensors) {
+                uint4 *dp = reinterpret_cast<uint4 *>(t == 0 ? dst.p[0] : (t == 1 ? dst.p[1] : dst.p[2])) + out_row * V;
+#pragma unroll
+                for (int k = 0; k < VPL; ++k)
+                    if (lane + 32 * k < V)
+                        dp[lane + 32 * k] = buf[t][k];
+            }
+        }
     }
 }
 
+template <int VPL>
 __global__ void __launch_bounds__(kThreads) unpack_kernel(const uint8_t *__restrict__ packed,
                                                           const int32_t *__restrict__ cu,
-                                                          const uint8_t *__restrict__ mask, int B, int N,
-                                                          int rows_per_split, int vec_per_row, int fill_mode,
-                                                          int64_t capacity, uint8_t *__restrict__ dst, int32_t *err)
+                                                          const uint8_t *__restrict__ mask, int N, int rows_per_split,
+                                                          int V, int fill_mode, int64_t capacity,
+                                                          uint8_t *__restrict__ dst, int32_t *err)
 {
-    __shared__ int red[kWarps];
-    __shared__ int warp_tot[kWarps];
-    __shared__ int16_t slot_of[kMaxRowsPerSplit];
+    __shared__ int part[kWarps][4];
+    __shared__ int16_t slot_of[kThreads];
+    __shared__ int16_t n_of_slot[kThreads];
 
     const int b = blockIdx.y;
     const int n0 = blockIdx.x * rows_per_split;
     if (n0 >= N)
         return;
     const int n1 = min(N, n0 + rows_per_split);
-    const uint8_t *row = mask + static_cast<int64_t>(b) * N;
+    const int64_t img0 = static_cast<int64_t>(b) * N;
     const int64_t start = cu[b];
     const int64_t end = cu[b + 1];
 
-    const int rank0 = block_count_nonzero(row, n0, red);
-    const int nk = block_scan_row(row, n0, n1, slot_of, warp_tot);
+    const Counts c = count_ranges(mask + img0, 0, n0, N);
+    const BlockScan s = block_scan(c, mask + img0, n0, n1, slot_of, n_of_slot, part);
     const bool image_ok = start >= 0 && end >= start;
-    if (threadIdx.x == 0) {
-        if (!image_ok || (n1 == N && rank0 + nk != end - start))
+    if (threadIdx.x == 0 && blockIdx.x == 0) {
+        if (!image_ok || s.total != end - start)
             raise_error(err, RRA_ERR_BAD_SEQLENS);
-        else if (start + rank0 + nk > capacity)
+        else if (end > capacity)
             raise_error(err, RRA_ERR_CAPACITY);
     }
     // kept rows read packed rows [start, lim) only; a malformed image reads nothing
     const int64_t lim = image_ok ? min(end, capacity) : start;
 
-    const int V = vec_per_row;
-    const int total = (n1 - n0) * V;
-    for (int i0 = threadIdx.x; i0 < total; i0 += kThreads * kBatch) {
-        uint4 val[kBatch];
-        uint4 *dptr[kBatch];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = warp; i < n1 - n0; i += kWarps) {
+        const int slot = slot_of[i];
+        uint4 *dp = reinterpret_cast<uint4 *>(dst) + (img0 + n0 + i) * V;
+        if (slot >= 0) {
+            const int64_t in_row = start + s.upto + slot;
+            if (in_row < start || in_row >= lim)
+                continue;
+            const uint4 *sp = reinterpret_cast<const uint4 *>(packed) + in_row * V;
+            uint4 buf[VPL];
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int i = i0 + u * kThreads;
-            dptr[u] = nullptr;
-            if (i < total) {
-                const int r = i / V;
-                const int vec = i - r * V;
-                const int slot = slot_of[r];
-                const int64_t out_row = static_cast<int64_t>(b) * N + n0 + r;
-                if (slot >= 0) {
-                    const int64_t in_row = start + rank0 + slot;
-                    if (in_row >= start && in_row < lim) {
-                        val[u] = ld_stream(reinterpret_cast<const uint4 *>(packed) + in_row * V + vec);
-                        dptr[u] = reinterpret_cast<uint4 *>(dst) + out_row * V + vec;
-                    }
-                } else if (fill_mode == 0) {
-                    val[u] = make_uint4(0, 0, 0, 0);
-                    dptr[u] = reinterpret_cast<uint4 *>(dst) + out_row * V + vec;
-                }
-            }
+            for (int k = 0; k < VPL; ++k)
+                if (lane + 32 * k < V)
+                    buf[k] = ld_stream(sp + lane + 32 * k);
+#pragma unroll
+            for (int k = 0; k < VPL; ++k)
+                if (lane + 32 * k < V)
+                    dp[lane + 32 * k] = buf[k];
+        } else if (fill_mode == 0) {
+#pragma unroll
+            for (int k = 0; k < VPL; ++k)
+                if (lane + 32 * k < V)
+                    dp[lane + 32 * k] = make_uint4(0, 0, 0, 0);
         }
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u)
-            if (dptr[u] != nullptr)
-                *dptr[u] = val[u];
     }
 }
 
@@ -249,10 +263,30 @@ int choose_splits(int B, int N, int num_sms)
     const int max_splits = (N + 15) / 16;  // at least 16 padded rows per block
     if (splits > max_splits)
         splits = max_splits;
-    const int min_splits = (N + kMaxRowsPerSplit - 1) / kMaxRowsPerSplit;
+    const int min_splits = (N + kThreads - 1) / kThreads;  // at most one row per thread
     if (splits < min_splits)
         splits = min_splits;
     return splits < 1 ? 1 : splits;
+}
+
+template <typename F>
+cudaError_t dispatch_vpl(int V, F &&launch)
+{
+    switch ((V + 31) / 32) {
+    case 1: return launch(std::integral_constant<int, 1>{});
+    case 2: return launch(std::integral_constant<int, 2>{});
+    case 3: return launch(std::integral_constant<int, 3>{});
+    case 4: return launch(std::integral_constant<int, 4>{});
+    case 5:
+    case 6: return launch(std::integral_constant<int, 6>{});
+    case 7:
+    case 8: return launch(std::integral_constant<int, 8>{});
+    case 9:
+    case 10:
+    case 11:
+    case 12: return launch(std::integral_constant<int, 12>{});
+    default: return launch(std::integral_constant<int, 16>{});
+    }
 }
 
 }  // namespace
@@ -267,16 +301,17 @@ cudaError_t launch_pack(const uint8_t *mask, int B, int N, int64_t row_bytes, in
         s.p[i] = static_cast<const uint8_t *>(src[i]);
         d.p[i] = static_cast<uint8_t *>(dst[i]);
     }
-    if (B == 0) {
-        // Nothing to gather; cu_seqlens = {0}.
-        return cudaMemsetAsync(cu, 0, sizeof(int32_t), stream);
-    }
+    if (B == 0)
+        return cudaMemsetAsync(cu, 0, sizeof(int32_t), stream);  // cu_seqlens = {0}
     const int splits = choose_splits(B, N, num_sms);
     const int rows = (N + splits - 1) / splits;
-    dim3 grid(splits, B);
-    pack_kernel<<<grid, kThreads, 0, stream>>>(mask, B, N, rows, static_cast<int>(row_bytes / 16), n_tensors, s, d,
-                                               capacity, cu, err);
-    return cudaGetLastError();
+    const int V = static_cast<int>(row_bytes / 16);
+    const dim3 grid(splits, B);
+    return dispatch_vpl(V, [&](auto vpl) {
+        pack_kernel<decltype(vpl)::value><<<grid, kThreads, 0, stream>>>(mask, N, rows, V, n_tensors, s, d,
+                                                                         capacity, cu, err);
+        return cudaGetLastError();
+    });
 }
 
 cudaError_t launch_unpack(const void *packed, const int32_t *cu, const uint8_t *mask, int B, int N,
@@ -287,11 +322,14 @@ cudaError_t launch_unpack(const void *packed, const int32_t *cu, const uint8_t *
         return cudaSuccess;
     const int splits = choose_splits(B, N, num_sms);
     const int rows = (N + splits - 1) / splits;
-    dim3 grid(splits, B);
-    unpack_kernel<<<grid, kThreads, 0, stream>>>(static_cast<const uint8_t *>(packed), cu, mask, B, N, rows,
-                                                 static_cast<int>(row_bytes / 16), fill_mode, capacity,
-                                                 static_cast<uint8_t *>(dst), err);
-    return cudaGetLastError();
+    const int V = static_cast<int>(row_bytes / 16);
+    const dim3 grid(splits, B);
+    return dispatch_vpl(V, [&](auto vpl) {
+        unpack_kernel<decltype(vpl)::value><<<grid, kThreads, 0, stream>>>(
+            static_cast<const uint8_t *>(packed), cu, mask, N, rows, V, fill_mode, capacity,
+            static_cast<uint8_t *>(dst), err);
+        return cudaGetLastError();
+    });
 }
 
 }  // namespace rra

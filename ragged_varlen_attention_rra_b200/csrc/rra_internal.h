@@ -6,8 +6,6 @@
 
 namespace rra {
 
-// Padded rows handled by one pack/unpack block (bounded by the block's shared rank table).
-constexpr int kMaxRowsPerSplit = 1024;
 
 cudaError_t launch_pack(const uint8_t *mask, int B, int N, int64_t row_bytes, int n_tensors,
                         const void *const *src, void *const *dst, int64_t capacity, int32_t *cu, int32_t *err,
