@@ -6,22 +6,27 @@
 //     o_i = sum_j softmax_j(scale * q_i . k_j) v_j,   j over all L_b kept tokens of image b.
 //
 // How (B200-specific design, not the pages' Triton kernel):
-//   * one persistent launch; each block walks a list of (image, q-tile, head) work items that
-//     it derives from cu_seqlens on the device, so the host never learns T;
-//   * Q, K, V tiles [128 tokens x 64] of one head are fetched by TMA straight from the packed
-//     [T, H, 64] layout (a 3-D tensor map; the head is a coordinate), 128-byte swizzled;
-//   * S = Q K^T and O_chunk = P V run as tcgen05.mma with fp32 accumulators in TMEM; P goes
-//     from registers back to TMEM and feeds the PV MMA as its A operand;
-//   * thread r of the 128-thread block owns row r of S and O (TMEM lane r), so the softmax
-//     row max / row sum are thread-local; keys are processed in chunks of 128 with an online
-//     (running max, rescaled sum) merge of O in registers;
+//   * one persistent launch of two blocks per SM; each block walks a list of
+//     (image, 128-row q-tile, head) work items that it derives from cu_seqlens on the device,
+//     so the host never learns T;
+//   * inside a block, warps specialise:
+//       warp 0      TMA producer: Q tile and 128-key K/V chunks of one head, fetched straight
+//                   from the packed [T, H, 64] layout (3-D tensor map, head = coordinate,
+//                   128-byte swizzle) into two-slot rings, so the next item's loads overlap
+//                   the current item's math;
+//       warp 1      tensor-core issuer: S = Q K^T and O_chunk = P V as tcgen05.mma with fp32
+//                   accumulators in TMEM (P comes from TMEM as the A operand);
+//       warps 2..5  softmax: thread r owns row r of S and O (TMEM lane r), so the row max
+//                   and row sum are thread-local; keys are taken in chunks of 128 with an
+//                   online (running max, rescaled sum) merge of O in registers, then the
+//                   row is normalised and stored;
 //   * for bf16 inputs P is split into a bf16 head and a bf16 remainder (two PV MMAs), which
 //     keeps P at ~16 significant bits; fp16 P (11 bits) is used as is;
-//   * key rows past the sequence end are masked to probability 0 and the matching V rows are
-//     zeroed in shared memory, so whatever bytes lie there (the next image, or uninitialised
-//     capacity rows) never reach the output;
-//   * every wait on an asynchronous copy or MMA is bounded in time; on expiry the block
-//     records RRA_ERR_TIMEOUT, waits for its own outstanding work and leaves.
+//   * key rows past the sequence end get probability 0 and the matching V rows are zeroed
+//     in shared memory, so whatever bytes lie there (the next image, or uninitialised capacity
+//     rows) never reach the output;
+//   * every wait is bounded in time; on expiry the block records RRA_ERR_TIMEOUT, raises a
+//     block-wide abort flag, drains the copies and MMAs it issued, frees TMEM and leaves.
 #include <cuda.h>
 
 #include <mutex>
@@ -36,14 +41,22 @@ namespace {
 constexpr int BM = 128;                 // query rows per tile (TMEM lanes)
 constexpr int BN = 128;                 // keys per chunk
 constexpr int kD = 64;                  // head dim
-constexpr int kThreads = 128;
+constexpr int kThreads = 192;           // 6 warps: producer, MMA, 4 x softmax
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0;           // S chunk, fp32 [128 x 128]; P (head part) reuses its first 64 columns
 constexpr uint32_t kColPlo = 128;       // P remainder part (bf16 only), 64 columns
 constexpr uint32_t kColO = 192;         // O chunk, fp32 [128 x 64]
 constexpr uint32_t kTileBytes = 128 * 128;
-constexpr int kSmemFixed = 1024 /*align*/ + 3 * kTileBytes + 64;
-constexpr int kSmemFloor = 90 * 1024;   // keeps at most two blocks (2 x 256 TMEM columns) per SM
+constexpr int kStages = 2;              // ring depth of the Q slots and of the K/V chunk slots
+
+// shared-memory map (offsets from a 1024-byte aligned base)
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kOffQ + kStages * kTileBytes;
+constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
+constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
+constexpr uint32_t kOffTile = kOffBar + 256;
+constexpr int kSmemFixed = 1024 /*align slack*/ + kOffTile;
+constexpr int kSmemFloor = 80 * 1024;   // keeps at most two blocks (2 x 256 TMEM columns) per SM
 
 struct Params {
     const int32_t *cu;
@@ -58,26 +71,83 @@ struct Params {
 
 constexpr uint64_t kDrainNs = 2000000000ull;
 
-__device__ __forceinline__ uint32_t pack_pair(float a, float b, bool bf16, float &ra, float &rb)
-{
-    if (bf16) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-        const float2 f = __bfloat1622float2(h);
-        ra = a - f.x;
-        rb = b - f.y;
-        return *reinterpret_cast<const uint32_t *>(&h);
-    } else {
-        const __half2 h = __floats2half2_rn(a, b);
-        ra = 0.f;
-        rb = 0.f;
-        return *reinterpret_cast<const uint32_t *>(&h);
-    }
-}
+struct Bars {
+    uint64_t q_full[kStages], q_empty[kStages];
+    uint64_t kv_full[kStages], kv_empty[kStages];
+    uint64_t s_full, p_full, o_full, o_free, drain;
+    uint32_t tmem_slot;
+    int abort;
+    int warp_sums[kThreads / 32];
+};
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 {
     const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float a, float b)
+{
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// One decoded work item.
+struct Item {
+    int b, h, qt, seq0, L;
+};
+
+__device__ __forceinline__ Item decode_item(int64_t item, int H, int B, const int32_t *tile_pre, const int32_t *cu)
+{
+    Item it;
+    const int g = static_cast<int>(item / H);
+    it.h = static_cast<int>(item - static_cast<int64_t>(g) * H);
+    int lo = 0, hi = B;  // tile_pre[lo] <= g < tile_pre[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tile_pre[mid] <= g)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    it.b = lo;
+    it.qt = g - tile_pre[lo];
+    it.seq0 = cu[lo];
+    it.L = cu[lo + 1] - it.seq0;
+    return it;
+}
+
+// Bounded wait used by every role: returns false when the block is aborting or the wait ran
+// out (which itself raises the abort flag and the timeout error).
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Bars *bars, const Params &p)
+{
+    if (mbar_test_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (*reinterpret_cast<volatile int *>(&bars->abort))
+            return false;
+        if (p.wait_ns == 0 ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity))
+            return true;
+        if (global_timer_ns() - t0 >= p.wait_ns) {
+            *reinterpret_cast<volatile int *>(&bars->abort) = 1;
+            raise_error(p.err, RRA_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Warp-uniform version: every lane waits, and the warp proceeds only if all lanes saw the
+// phase complete (so no lane can leave a loop that its warp-mates stay in).
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, Bars *bars, const Params &p)
+{
+    const bool ok = wait_or_abort(bar, parity, bars, p);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 template <bool kBF16>
@@ -87,14 +157,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sQ = base;
-    uint8_t *sK = base + kTileBytes;
-    uint8_t *sV = base + 2 * kTileBytes;
-    uint64_t *bar_load = reinterpret_cast<uint64_t *>(base + 3 * kTileBytes);
-    uint64_t *bar_mma = bar_load + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_load + 2);
-    int *warp_sums = reinterpret_cast<int *>(bar_load + 4);        // 4 ints
-    int32_t *tile_pre = reinterpret_cast<int32_t *>(base + 3 * kTileBytes + 64);  // [B+1]
+    Bars *bars = reinterpret_cast<Bars *>(base + kOffBar);
+    int32_t *tile_pre = reinterpret_cast<int32_t *>(base + kOffTile);  // [B+1]
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -105,12 +169,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
-        mbar_init(bar_load, 1);
-        mbar_init(bar_mma, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bars->q_full[s], 1);
+            mbar_init(&bars->q_empty[s], 1);
+            mbar_init(&bars->kv_full[s], 1);
+            mbar_init(&bars->kv_empty[s], 1);
+        }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->p_full, 4);   // one arrival per softmax warp
+        mbar_init(&bars->o_full, 1);
+        mbar_init(&bars->o_free, 4);
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
         fence_mbarrier_init();
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_alloc(&bars->tmem_slot, kTmemCols);
         tmem_relinquish();
     }
 
@@ -138,14 +212,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 incl += t;
         }
         if (lane == 31)
-            warp_sums[warp] = incl;
+            bars->warp_sums[warp] = incl;
         __syncthreads();
         int before = carry;
         int chunk = 0;
 #pragma unroll
         for (int w = 0; w < kThreads / 32; ++w) {
-            before += (w < warp) ? warp_sums[w] : 0;
-            chunk += warp_sums[w];
+            before += (w < warp) ? bars->warp_sums[w] : 0;
+            chunk += bars->warp_sums[w];
         }
         if (b < B)
             tile_pre[b + 1] = before + incl;
@@ -156,225 +230,287 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem = bars->tmem_slot;
     const int64_t total_items = static_cast<int64_t>(tile_pre[B]) * H;
 
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const uint32_t sQa = smem_addr(sQ), sKa = smem_addr(sK), sVa = smem_addr(sV);
-    uint32_t ld_phase = 0, mma_phase = 0;
-    bool failed = false;
-
-    for (int64_t item = blockIdx.x; item < total_items && !failed; item += gridDim.x) {
-        const int g = static_cast<int>(item / H);
-        const int h = static_cast<int>(item - static_cast<int64_t>(g) * H);
-        int lo = 0, hi = B;  // tile_pre[lo] <= g < tile_pre[hi]
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (tile_pre[mid] <= g)
-                lo = mid;
-            else
-                hi = mid;
+    if (warp == 0) {
+        // ================================================================ TMA producer
+        // Empty-slot waits use the usual parity idiom: on a fresh barrier the phase "before"
+        // phase 0 counts as complete, so waiting on parity (phase ^ 1) passes at once for the
+        // first fill of each slot, then tracks the consumer's releases.
+        uint32_t q_phase[kStages] = {0, 0}, kv_phase[kStages] = {0, 0};
+        uint32_t q_issued = 0, kv_issued = 0;  // how many Q / KV slot fills were issued
+        int qs = 0, ks = 0;
+        bool ok = true;
+        for (int64_t item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+            const Item it = decode_item(item, H, B, tile_pre, p.cu);
+            const int nkc = (it.L + BN - 1) / BN;
+            // Q slot: free once the previous user of the slot has finished its last PV MMA
+            ok = warp_wait(&bars->q_empty[qs], q_phase[qs] ^ 1u, bars, p);
+            if (!ok)
+                break;
+            q_phase[qs] ^= 1u;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&bars->q_full[qs], kTileBytes);
+                tma_load_3d(base + kOffQ + qs * kTileBytes, &tm_q, &bars->q_full[qs], 0, it.h, it.seq0 + it.qt * BM);
+            }
+            __syncwarp();
+            ++q_issued;
+            qs ^= 1;
+            for (int kc = 0; kc < nkc; ++kc) {
+                ok = warp_wait(&bars->kv_empty[ks], kv_phase[ks] ^ 1u, bars, p);
+                if (!ok)
+                    break;
+                kv_phase[ks] ^= 1u;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&bars->kv_full[ks], 2 * kTileBytes);
+                    tma_load_3d(base + kOffK + ks * kTileBytes, &tm_k, &bars->kv_full[ks], 0, it.h, it.seq0 + kc * BN);
+                    tma_load_3d(base + kOffV + ks * kTileBytes, &tm_v, &bars->kv_full[ks], 0, it.h, it.seq0 + kc * BN);
+                }
+                __syncwarp();
+                ++kv_issued;
+                ks ^= 1;
+            }
         }
-        const int b = lo;
-        const int qt = g - tile_pre[b];
-        const int seq0 = p.cu[b];
-        const int L = p.cu[b + 1] - seq0;
-        const int q0 = qt * BM;
-        const int qrows = min(BM, L - q0);
-        const int nkc = (L + BN - 1) / BN;
-        const bool warp_active = warp * 32 < qrows;
-
-        float m_run = -INFINITY, l_run = 0.f;
-        float o[kD];
-#pragma unroll
-        for (int j = 0; j < kD; ++j)
-            o[j] = 0.f;
-
-        for (int kc = 0; kc < nkc; ++kc) {
-            const int k0 = kc * BN;
-            const int nk = min(BN, L - k0);
-            const int nk16 = (nk + 15) & ~15;
-
-            // ---- TMA: (Q on the first chunk) + K + V chunk of this head
-            if (tid == 0) {
-                mbar_arrive_expect_tx(bar_load, (kc == 0 ? 3u : 2u) * kTileBytes);
-                if (kc == 0)
-                    tma_load_3d(sQ, &tm_q, bar_load, 0, h, seq0 + q0);
-                tma_load_3d(sK, &tm_k, bar_load, 0, h, seq0 + k0);
-                tma_load_3d(sV, &tm_v, bar_load, 0, h, seq0 + k0);
-            }
-            bool ok = mbar_wait_bounded(bar_load, ld_phase, p.wait_ns);
-            if (__syncthreads_or(!ok)) {
-                if (tid == 0) {
-                    raise_error(p.err, RRA_ERR_TIMEOUT);
-                    mbar_wait_bounded(bar_load, ld_phase, kDrainNs);
-                }
-                failed = true;
+        // drain: every issued fill has landed before the block may leave
+        for (int s = 0; s < kStages; ++s) {
+            const uint32_t nq = q_issued / kStages + (static_cast<uint32_t>(s) < q_issued % kStages ? 1u : 0u);
+            if (nq > 0)
+                mbar_wait_bounded(&bars->q_full[s], (nq - 1) & 1u, kDrainNs);
+            const uint32_t nk = kv_issued / kStages + (static_cast<uint32_t>(s) < kv_issued % kStages ? 1u : 0u);
+            if (nk > 0)
+                mbar_wait_bounded(&bars->kv_full[s], (nk - 1) & 1u, kDrainNs);
+        }
+    } else if (warp == 1) {
+        // ================================================================ tcgen05 issuer
+        uint32_t q_ph[kStages] = {0, 0}, kv_ph[kStages] = {0, 0};
+        uint32_t p_ph = 0, ofree_ph = 0, pv_ph = 0;
+        uint32_t n_pv = 0;  // PV commits issued (each completes a phase of o_full)
+        int qs = 0, ks = 0;
+        const uint32_t idPV = idesc_f16(BM, kD, kBF16 ? 1u : 0u, 1u);
+        bool ok = true;
+        for (int64_t item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+            const Item it = decode_item(item, H, B, tile_pre, p.cu);
+            const int nkc = (it.L + BN - 1) / BN;
+            ok = warp_wait(&bars->q_full[qs], q_ph[qs], bars, p);
+            if (!ok)
                 break;
-            }
-            ld_phase ^= 1;
-
-            // ---- zero V rows [nk, nk16): they enter the PV MMA with probability 0
-            if (nk < nk16) {
-                const int nz = (nk16 - nk) * 8;
-                for (int i = tid; i < nz; i += kThreads) {
-                    const int r = nk + (i >> 3);
-                    *reinterpret_cast<uint4 *>(sV + r * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+            q_ph[qs] ^= 1u;
+            const uint32_t sQa = smem_addr(base + kOffQ + qs * kTileBytes);
+            for (int kc = 0; kc < nkc; ++kc) {
+                const int nk = min(BN, it.L - kc * BN);
+                const int nk16 = (nk + 15) & ~15;
+                ok = warp_wait(&bars->kv_full[ks], kv_ph[ks], bars, p);
+                if (!ok)
+                    break;
+                kv_ph[ks] ^= 1u;
+                uint8_t *sV = base + kOffV + ks * kTileBytes;
+                // zero V rows [nk, nk16): they enter the PV MMA with probability 0
+                if (nk < nk16) {
+                    for (int i = lane; i < (nk16 - nk) * 8; i += 32)
+                        *reinterpret_cast<uint4 *>(sV + (nk + (i >> 3)) * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+                    fence_proxy_async_smem();
                 }
-                fence_proxy_async_smem();
+                __syncwarp();
+                // S region (which holds the previous chunk's P) is free once that PV completed
+                if (n_pv > 0) {
+                    ok = warp_wait(&bars->o_full, pv_ph, bars, p);
+                    if (!ok)
+                        break;
+                    pv_ph ^= 1u;
+                }
+                const uint32_t sKa = smem_addr(base + kOffK + ks * kTileBytes);
+                const uint32_t sVa = smem_addr(sV);
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint32_t idS = idesc_f16(BM, nk16, kBF16 ? 1u : 0u, 0u);
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk)
+                        mma_ss(tmem + kColS, smem_desc_sw128(sQa + kk * 32, 16, 1024),
+                               smem_desc_sw128(sKa + kk * 32, 16, 1024), idS, kk > 0 ? 1u : 0u);
+                    mma_commit(&bars->s_full);
+                }
+                __syncwarp();
+                // P written by the softmax warps, previous O chunk consumed
+                ok = warp_wait(&bars->p_full, p_ph, bars, p);
+                if (!ok)
+                    break;
+                p_ph ^= 1u;
+                if (n_pv > 0) {
+                    ok = warp_wait(&bars->o_free, ofree_ph, bars, p);
+                    if (!ok)
+                        break;
+                    ofree_ph ^= 1u;
+                }
+                if (lane == 0) {
+                    tc_fence_after();
+                    for (int j = 0; j < nk16 / 16; ++j)
+                        mma_ts(tmem + kColO, tmem + kColS + j * 8, smem_desc_sw128(sVa + j * 2048, 16, 1024), idPV,
+                               j > 0 ? 1u : 0u);
+                    if (kBF16)
+                        for (int j = 0; j < nk16 / 16; ++j)
+                            mma_ts(tmem + kColO, tmem + kColPlo + j * 8, smem_desc_sw128(sVa + j * 2048, 16, 1024),
+                                   idPV, 1u);
+                    mma_commit(&bars->o_full);
+                    mma_commit(&bars->kv_empty[ks]);
+                    if (kc == nkc - 1)
+                        mma_commit(&bars->q_empty[qs]);
+                }
+                __syncwarp();
+                ++n_pv;
+                ks ^= 1;
             }
-            __syncthreads();
-
-            // ---- S = Q K^T  (M = 128, N = nk16, K = 64 in four steps of 16)
-            if (tid == 0) {
+            qs ^= 1;
+        }
+        // drain: every MMA this thread issued has completed
+        if (lane == 0) {
+            mma_commit(&bars->drain);
+            mbar_wait_bounded(&bars->drain, 0, kDrainNs);
+        }
+        __syncwarp();
+    } else {
+        // ================================================================ softmax + epilogue
+        const int q4 = warp & 3;                     // TMEM lane quarter of this warp
+        const int row = q4 * 32 + lane;              // row of S / O owned by this thread
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+        uint32_t s_ph = 0, o_ph = 0;
+        bool ok = true;
+        for (int64_t item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+            const Item it = decode_item(item, H, B, tile_pre, p.cu);
+            const int nkc = (it.L + BN - 1) / BN;
+            const int q0 = it.qt * BM;
+            const int qrows = min(BM, it.L - q0);
+            const bool warp_active = q4 * 32 < qrows;
+            float m_run = -INFINITY, l_run = 0.f;
+            float o[kD];
+#pragma unroll
+            for (int j = 0; j < kD; ++j)
+                o[j] = 0.f;
+            for (int kc = 0; kc < nkc; ++kc) {
+                const int nk = min(BN, it.L - kc * BN);
+                const int nk16 = (nk + 15) & ~15;
+                ok = warp_wait(&bars->s_full, s_ph, bars, p);
+                if (!ok)
+                    break;
+                s_ph ^= 1u;
                 tc_fence_after();
-                const uint32_t idS = idesc_f16(BM, nk16, kBF16 ? 1u : 0u, 0u);
+                float m_new = m_run, l_add = 0.f;
+                if (warp_active) {
+                    // pass 1: row max over the valid keys of this chunk
+                    float mx = -INFINITY;
+                    for (int c = 0; c < nk16; c += 32) {
+                        uint32_t r[32];
+                        tmem_ld32(lane_base + kColS + c, r);
+                        tmem_wait_ld();
+                        if (c + 32 <= nk) {
 #pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                    const uint64_t ad = smem_desc_sw128(sQa + ks * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(sKa + ks * 32, 16, 1024);
-                    mma_ss(tmem + kColS, ad, bd, idS, ks > 0 ? 1u : 0u);
+                            for (int j = 0; j < 32; ++j)
+                                mx = fmaxf(mx, __uint_as_float(r[j]));
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (c + j < nk)
+                                    mx = fmaxf(mx, __uint_as_float(r[j]));
+                        }
+                    }
+                    m_new = fmaxf(m_run, mx);
+                    const float neg_m = -m_new * p.scale_log2;
+                    // pass 2: P = exp2(scale*log2e*s - scale*log2e*m), row sum, P -> TMEM
+                    for (int c = 0; c < nk16; c += 32) {
+                        uint32_t r[32];
+                        tmem_ld32(lane_base + kColS + c, r);
+                        tmem_wait_ld();
+                        float pv[32];
+                        if (c + 32 <= nk) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                pv[j] = ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, neg_m));
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                pv[j] = (c + j < nk) ? ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, neg_m)) : 0.f;
+                        }
+                        uint32_t phi[16], plo[16];
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj) {
+                            const float a = pv[2 * jj], b = pv[2 * jj + 1];
+                            l_add += a + b;
+                            if (kBF16) {
+                                phi[jj] = pack_bf16(a, b);
+                                const float ha = __uint_as_float(phi[jj] << 16);
+                                const float hb = __uint_as_float(phi[jj] & 0xFFFF0000u);
+                                plo[jj] = pack_bf16(a - ha, b - hb);
+                            } else {
+                                phi[jj] = pack_f16(a, b);
+                            }
+                        }
+                        tmem_st16(lane_base + kColS + c / 2, phi);
+                        if (kBF16)
+                            tmem_st16(lane_base + kColPlo + c / 2, plo);
+                    }
+                    tmem_wait_st();
                 }
-                mma_commit(bar_mma);
-            }
-            ok = mbar_wait_bounded(bar_mma, mma_phase, p.wait_ns);
-            if (__syncthreads_or(!ok)) {
-                if (tid == 0) {
-                    raise_error(p.err, RRA_ERR_TIMEOUT);
-                    mbar_wait_bounded(bar_mma, mma_phase, kDrainNs);
-                }
-                failed = true;
-                break;
-            }
-            mma_phase ^= 1;
-            tc_fence_after();
-
-            // ---- softmax of this chunk: row max, P = exp2(scale*log2e*(s - m)), row sum
-            float m_new = m_run, l_add = 0.f;
-            if (warp_active) {
-                float mx = -INFINITY;
-                for (int c = 0; c < nk16; c += 32) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bars->p_full);
+                // O chunk = P V; merge with a running max rescale
+                ok = warp_wait(&bars->o_full, o_ph, bars, p);
+                if (!ok)
+                    break;
+                o_ph ^= 1u;
+                tc_fence_after();
+                if (warp_active) {
+                    const float alpha = ex2_approx((m_run - m_new) * p.scale_log2);
                     uint32_t r[32];
-                    tmem_ld32(lane_base + kColS + c, r);
+                    tmem_ld32(lane_base + kColO, r);
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if (c + j < nk)
-                            mx = fmaxf(mx, __uint_as_float(r[j]));
-                }
-                m_new = fmaxf(m_run, mx);
-                const float neg_m = -m_new * p.scale_log2;
-                for (int c = 0; c < nk16; c += 32) {
-                    uint32_t r[32];
-                    tmem_ld32(lane_base + kColS + c, r);
+                        o[j] = fmaf(o[j], alpha, __uint_as_float(r[j]));
+                    tmem_ld32(lane_base + kColO + 32, r);
                     tmem_wait_ld();
-                    uint32_t phi[16], plo[16];
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        const int j0 = c + 2 * jj;
-                        const float p0 = (j0 < nk) ? ex2_approx(fmaf(__uint_as_float(r[2 * jj]), p.scale_log2, neg_m)) : 0.f;
-                        const float p1 = (j0 + 1 < nk) ? ex2_approx(fmaf(__uint_as_float(r[2 * jj + 1]), p.scale_log2, neg_m)) : 0.f;
-                        l_add += p0 + p1;
-                        float r0, r1;
-                        phi[jj] = pack_pair(p0, p1, kBF16, r0, r1);
-                        plo[jj] = kBF16 ? pack_bf16(r0, r1) : 0u;
-                    }
-                    tmem_st16(lane_base + kColS + c / 2, phi);
-                    if (kBF16)
-                        tmem_st16(lane_base + kColPlo + c / 2, plo);
+                    for (int j = 0; j < 32; ++j)
+                        o[32 + j] = fmaf(o[32 + j], alpha, __uint_as_float(r[j]));
+                    l_run = fmaf(l_run, alpha, l_add);
+                    m_run = m_new;
                 }
-                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bars->o_free);
             }
-            tc_fence_before();
-            __syncthreads();
-
-            // ---- O_chunk = P V  (M = 128, N = 64, K = nk16; P from TMEM, V MN-major in smem)
-            if (tid == 0) {
-                tc_fence_after();
-                const uint32_t idPV = idesc_f16(BM, kD, kBF16 ? 1u : 0u, 1u);
-                for (int j = 0; j < nk16 / 16; ++j) {
-                    const uint64_t bd = smem_desc_sw128(sVa + j * 2048, 16, 1024);
-                    mma_ts(tmem + kColO, tmem + kColS + j * 8, bd, idPV, j > 0 ? 1u : 0u);
-                }
-                if (kBF16) {
-                    for (int j = 0; j < nk16 / 16; ++j) {
-                        const uint64_t bd = smem_desc_sw128(sVa + j * 2048, 16, 1024);
-                        mma_ts(tmem + kColO, tmem + kColPlo + j * 8, bd, idPV, 1u);
-                    }
-                }
-                mma_commit(bar_mma);
-            }
-            ok = mbar_wait_bounded(bar_mma, mma_phase, p.wait_ns);
-            if (__syncthreads_or(!ok)) {
-                if (tid == 0) {
-                    raise_error(p.err, RRA_ERR_TIMEOUT);
-                    mbar_wait_bounded(bar_mma, mma_phase, kDrainNs);
-                }
-                failed = true;
+            if (!ok)
                 break;
-            }
-            mma_phase ^= 1;
-            tc_fence_after();
-
-            // ---- online merge: O = O * exp2(c (m_old - m_new)) + O_chunk
-            if (warp_active) {
-                const float alpha = ex2_approx((m_run - m_new) * p.scale_log2);
-                uint32_t r[32];
-                tmem_ld32(lane_base + kColO, r);
-                tmem_wait_ld();
+            // epilogue: normalise and store this thread's row
+            if (row < qrows) {
+                const float inv = 1.f / l_run;
+                const int64_t t = static_cast<int64_t>(it.seq0) + q0 + row;
+                const int64_t off = (t * H + it.h) * kD;
+                if (p.out_dt == RRA_F32) {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    o[j] = fmaf(o[j], alpha, __uint_as_float(r[j]));
-                tmem_ld32(lane_base + kColO + 32, r);
-                tmem_wait_ld();
+                    for (int j = 0; j < kD / 4; ++j)
+                        dst[j] = make_float4(o[4 * j] * inv, o[4 * j + 1] * inv, o[4 * j + 2] * inv, o[4 * j + 3] * inv);
+                } else {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + off);
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    o[32 + j] = fmaf(o[32 + j], alpha, __uint_as_float(r[j]));
-                l_run = fmaf(l_run, alpha, l_add);
-                m_run = m_new;
-            }
-            tc_fence_before();
-            __syncthreads();
-        }
-        if (failed)
-            break;
-
-        // ---- epilogue: normalise and store this thread's row
-        if (tid < qrows) {
-            const float inv = 1.f / l_run;
-            const int64_t row = static_cast<int64_t>(seq0) + q0 + tid;
-            const int64_t off = (row * H + h) * kD;
-            if (p.out_dt == RRA_F32) {
-                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
-#pragma unroll
-                for (int j = 0; j < kD / 4; ++j)
-                    dst[j] = make_float4(o[4 * j] * inv, o[4 * j + 1] * inv, o[4 * j + 2] * inv, o[4 * j + 3] * inv);
-            } else if (p.out_dt == RRA_BF16) {
-                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + off);
-#pragma unroll
-                for (int j = 0; j < kD / 8; ++j) {
-                    uint4 w;
-                    w.x = pack_bf16(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
-                    w.y = pack_bf16(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
-                    w.z = pack_bf16(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
-                    w.w = pack_bf16(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
-                    dst[j] = w;
-                }
-            } else {
-                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__half *>(p.out) + off);
-#pragma unroll
-                for (int j = 0; j < kD / 8; ++j) {
-                    uint4 w;
-                    __half2 t;
-                    t = __floats2half2_rn(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
-                    w.x = *reinterpret_cast<uint32_t *>(&t);
-                    t = __floats2half2_rn(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
-                    w.y = *reinterpret_cast<uint32_t *>(&t);
-                    t = __floats2half2_rn(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
-                    w.z = *reinterpret_cast<uint32_t *>(&t);
-                    t = __floats2half2_rn(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
-                    w.w = *reinterpret_cast<uint32_t *>(&t);
-                    dst[j] = w;
+                    for (int j = 0; j < kD / 8; ++j) {
+                        uint4 w;
+                        if (p.out_dt == RRA_BF16) {
+                            w.x = pack_bf16(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
+                            w.y = pack_bf16(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
+                            w.z = pack_bf16(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
+                            w.w = pack_bf16(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
+                        } else {
+                            w.x = pack_f16(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
+                            w.y = pack_f16(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
+                            w.z = pack_f16(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
+                            w.w = pack_f16(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
+                        }
+                        dst[j] = w;
+                    }
                 }
             }
         }
