@@ -16,10 +16,12 @@
 //                   the current item's math;
 //       warp 1      tensor-core issuer: S = Q K^T and O_chunk = P V as tcgen05.mma with fp32
 //                   accumulators in TMEM (P comes from TMEM as the A operand);
-//       warps 2..5  softmax: thread r owns row r of S and O (TMEM lane r), so the row max
-//                   and row sum are thread-local; keys are taken in chunks of 128 with an
-//                   online (running max, rescaled sum) merge of O in registers, then the
-//                   row is normalised and stored;
+//       warps 2..9  softmax: a pair of warps owns each quarter of the rows (TMEM lanes);
+//                   within a 128-key chunk the two warps take alternate 32-key slices, so
+//                   row max / row sum are thread-local plus one exchange per chunk between
+//                   the two warps of a pair; keys are taken in chunks of 128 with an online
+//                   (running max, rescaled sum) merge of O in registers (each warp of a pair
+//                   keeps 32 of the 64 output columns), then rows are normalised and stored;
 //   * for bf16 inputs P is split into a bf16 head and a bf16 remainder (two PV MMAs), which
 //     keeps P at ~16 significant bits; fp16 P (11 bits) is used as is;
 //   * key rows past the sequence end get probability 0 and the matching V rows are zeroed
@@ -41,11 +43,13 @@ namespace {
 constexpr int BM = 128;                 // query rows per tile (TMEM lanes)
 constexpr int BN = 128;                 // keys per chunk
 constexpr int kD = 64;                  // head dim
-constexpr int kThreads = 192;           // 6 warps: producer, MMA, 4 x softmax
+constexpr int kThreads = 320;           // 10 warps: producer, MMA, 8 x softmax
+constexpr int kSoftmaxWarps = 8;
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0;           // S chunk, fp32 [128 x 128]; P (head part) reuses its first 64 columns
-constexpr uint32_t kColPlo = 128;       // P remainder part (bf16 only), 64 columns
-constexpr uint32_t kColO = 192;         // O chunk, fp32 [128 x 64]
+// S chunk, fp32 [128 x 128].  The P of each 32-key slice is written back over that slice's own
+// S columns: bf16/fp16 head part in its first 16 columns, bf16 remainder in the next 16.
+constexpr uint32_t kColS = 0;
+constexpr uint32_t kColO = 128;         // O chunk, fp32 [128 x 64]
 constexpr uint32_t kTileBytes = 128 * 128;
 constexpr int kStages = 2;              // ring depth of the Q slots and of the K/V chunk slots
 
@@ -54,7 +58,8 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kStages * kTileBytes;
 constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
 constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
-constexpr uint32_t kOffTile = kOffBar + 256;
+constexpr uint32_t kOffRed = kOffBar + 256;             // row max / row sum exchange, 2 x 128 floats
+constexpr uint32_t kOffTile = kOffRed + 2 * 128 * 4;    // tile_pre[B+1], then cu[B+1]
 constexpr int kSmemFixed = 1024 /*align slack*/ + kOffTile;
 constexpr int kSmemFloor = 80 * 1024;   // keeps at most two blocks (2 x 256 TMEM columns) per SM
 
@@ -79,6 +84,7 @@ struct Bars {
     int abort;
     int warp_sums[kThreads / 32];
 };
+static_assert(sizeof(Bars) <= 256, "barrier block overflows its slot");
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 {
@@ -97,11 +103,11 @@ struct Item {
     int b, h, qt, seq0, L;
 };
 
-__device__ __forceinline__ Item decode_item(int64_t item, int H, int B, const int32_t *tile_pre, const int32_t *cu)
+__device__ __forceinline__ Item decode_item(int item, int H, int B, const int32_t *tile_pre, const int32_t *cu)
 {
     Item it;
-    const int g = static_cast<int>(item / H);
-    it.h = static_cast<int>(item - static_cast<int64_t>(g) * H);
+    const int g = item / H;
+    it.h = item - g * H;
     int lo = 0, hi = B;  // tile_pre[lo] <= g < tile_pre[hi]
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -150,6 +156,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// Barrier between the two softmax warps that share a quarter of the rows (64 threads).
+__device__ __forceinline__ void pair_sync(int quarter)
+{
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
+}
+
 template <bool kBF16>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -159,6 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars *bars = reinterpret_cast<Bars *>(base + kOffBar);
     int32_t *tile_pre = reinterpret_cast<int32_t *>(base + kOffTile);  // [B+1]
+    int32_t *cu_s = tile_pre + (p.B + 1);                               // [B+1]
+    float *red = reinterpret_cast<float *>(base + kOffRed);            // [2][128]
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -176,9 +190,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->kv_empty[s], 1);
         }
         mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_full, 4);   // one arrival per softmax warp
+        mbar_init(&bars->p_full, kSoftmaxWarps);   // one arrival per softmax warp
         mbar_init(&bars->o_full, 1);
-        mbar_init(&bars->o_free, 4);
+        mbar_init(&bars->o_free, kSoftmaxWarps);
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
         fence_mbarrier_init();
@@ -197,6 +211,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         int tiles = 0;
         if (b < B) {
             const int64_t s0 = p.cu[b], s1 = p.cu[b + 1];
+            cu_s[b] = static_cast<int32_t>(s0);
+            if (b == B - 1)
+                cu_s[B] = static_cast<int32_t>(s1);
             if (s0 < 0 || s1 < s0 || s1 > p.capacity) {
                 if (blockIdx.x == 0)
                     raise_error(p.err, RRA_ERR_BAD_SEQLENS);
@@ -231,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_slot;
-    const int64_t total_items = static_cast<int64_t>(tile_pre[B]) * H;
+    const int total_items = tile_pre[B] * H;
 
     if (warp == 0) {
         // ================================================================ TMA producer
@@ -242,8 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t q_issued = 0, kv_issued = 0;  // how many Q / KV slot fills were issued
         int qs = 0, ks = 0;
         bool ok = true;
-        for (int64_t item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-            const Item it = decode_item(item, H, B, tile_pre, p.cu);
+        for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+            const Item it = decode_item(item, H, B, tile_pre, cu_s);
             const int nkc = (it.L + BN - 1) / BN;
             // Q slot: free once the previous user of the slot has finished its last PV MMA
             ok = warp_wait(&bars->q_empty[qs], q_phase[qs] ^ 1u, bars, p);
@@ -289,8 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int qs = 0, ks = 0;
         const uint32_t idPV = idesc_f16(BM, kD, kBF16 ? 1u : 0u, 1u);
         bool ok = true;
-        for (int64_t item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-            const Item it = decode_item(item, H, B, tile_pre, p.cu);
+        for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+            const Item it = decode_item(item, H, B, tile_pre, cu_s);
             const int nkc = (it.L + BN - 1) / BN;
             ok = warp_wait(&bars->q_full[qs], q_ph[qs], bars, p);
             if (!ok)
@@ -344,13 +361,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (lane == 0) {
                     tc_fence_after();
+                    // keys 16j..16j+15 live in slice j/2: head part at column 32(j/2) + 8(j%2),
+                    // remainder 16 columns further
                     for (int j = 0; j < nk16 / 16; ++j)
-                        mma_ts(tmem + kColO, tmem + kColS + j * 8, smem_desc_sw128(sVa + j * 2048, 16, 1024), idPV,
-                               j > 0 ? 1u : 0u);
+                        mma_ts(tmem + kColO, tmem + kColS + 32 * (j >> 1) + 8 * (j & 1),
+                               smem_desc_sw128(sVa + j * 2048, 16, 1024), idPV, j > 0 ? 1u : 0u);
                     if (kBF16)
                         for (int j = 0; j < nk16 / 16; ++j)
-                            mma_ts(tmem + kColO, tmem + kColPlo + j * 8, smem_desc_sw128(sVa + j * 2048, 16, 1024),
-                                   idPV, 1u);
+                            mma_ts(tmem + kColO, tmem + kColS + 32 * (j >> 1) + 8 * (j & 1) + 16,
+                                   smem_desc_sw128(sVa + j * 2048, 16, 1024), idPV, 1u);
                     mma_commit(&bars->o_full);
                     mma_commit(&bars->kv_empty[ks]);
                     if (kc == nkc - 1)
@@ -371,20 +390,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ================================================================ softmax + epilogue
         const int q4 = warp & 3;                     // TMEM lane quarter of this warp
+        const int hf = (warp - 2) >> 2;              // which of the pair: slices hf, hf+2, ...; O columns 32hf..
         const int row = q4 * 32 + lane;              // row of S / O owned by this thread
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+        float *red_max = red;                        // [128]
+        float *red_sum = red + 128;                  // [128]
         uint32_t s_ph = 0, o_ph = 0;
         bool ok = true;
-        for (int64_t item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-            const Item it = decode_item(item, H, B, tile_pre, p.cu);
+        for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+            const Item it = decode_item(item, H, B, tile_pre, cu_s);
             const int nkc = (it.L + BN - 1) / BN;
             const int q0 = it.qt * BM;
             const int qrows = min(BM, it.L - q0);
             const bool warp_active = q4 * 32 < qrows;
             float m_run = -INFINITY, l_run = 0.f;
-            float o[kD];
+            float o[32];
 #pragma unroll
-            for (int j = 0; j < kD; ++j)
+            for (int j = 0; j < 32; ++j)
                 o[j] = 0.f;
             for (int kc = 0; kc < nkc; ++kc) {
                 const int nk = min(BN, it.L - kc * BN);
@@ -396,9 +418,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 float m_new = m_run, l_add = 0.f;
                 if (warp_active) {
-                    // pass 1: row max over the valid keys of this chunk
+                    // pass 1: row max over this warp's valid keys, combined with the pair
                     float mx = -INFINITY;
-                    for (int c = 0; c < nk16; c += 32) {
+                    for (int c = 32 * hf; c < nk16; c += 64) {
                         uint32_t r[32];
                         tmem_ld32(lane_base + kColS + c, r);
                         tmem_wait_ld();
@@ -413,10 +435,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     mx = fmaxf(mx, __uint_as_float(r[j]));
                         }
                     }
+                    if (hf == 1)
+                        red_max[row] = mx;
+                    pair_sync(q4);
+                    if (hf == 0)
+                        red_max[row] = fmaxf(mx, red_max[row]);
+                    pair_sync(q4);
+                    mx = red_max[row];
                     m_new = fmaxf(m_run, mx);
                     const float neg_m = -m_new * p.scale_log2;
-                    // pass 2: P = exp2(scale*log2e*s - scale*log2e*m), row sum, P -> TMEM
-                    for (int c = 0; c < nk16; c += 32) {
+                    // pass 2: P = exp2(scale*log2e*(s - m)), row sum, P back over this slice's S
+                    for (int c = 32 * hf; c < nk16; c += 64) {
                         uint32_t r[32];
                         tmem_ld32(lane_base + kColS + c, r);
                         tmem_wait_ld();
@@ -430,23 +459,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int j = 0; j < 32; ++j)
                                 pv[j] = (c + j < nk) ? ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, neg_m)) : 0.f;
                         }
-                        uint32_t phi[16], plo[16];
+                        uint32_t pp[32];
 #pragma unroll
                         for (int jj = 0; jj < 16; ++jj) {
                             const float a = pv[2 * jj], b = pv[2 * jj + 1];
                             l_add += a + b;
                             if (kBF16) {
-                                phi[jj] = pack_bf16(a, b);
-                                const float ha = __uint_as_float(phi[jj] << 16);
-                                const float hb = __uint_as_float(phi[jj] & 0xFFFF0000u);
-                                plo[jj] = pack_bf16(a - ha, b - hb);
+                                pp[jj] = pack_bf16(a, b);
+                                const float ha = __uint_as_float(pp[jj] << 16);
+                                const float hb = __uint_as_float(pp[jj] & 0xFFFF0000u);
+                                pp[16 + jj] = pack_bf16(a - ha, b - hb);
                             } else {
-                                phi[jj] = pack_f16(a, b);
+                                pp[jj] = pack_f16(a, b);
+                                pp[16 + jj] = 0u;
                             }
                         }
-                        tmem_st16(lane_base + kColS + c / 2, phi);
-                        if (kBF16)
-                            tmem_st16(lane_base + kColPlo + c / 2, plo);
+                        tmem_st32(lane_base + kColS + c, pp);
                     }
                     tmem_wait_st();
                 }
@@ -454,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&bars->p_full);
-                // O chunk = P V; merge with a running max rescale
+                // O chunk = P V; merge this warp's 32 output columns with a running max rescale
                 ok = warp_wait(&bars->o_full, o_ph, bars, p);
                 if (!ok)
                     break;
@@ -463,16 +491,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (warp_active) {
                     const float alpha = ex2_approx((m_run - m_new) * p.scale_log2);
                     uint32_t r[32];
-                    tmem_ld32(lane_base + kColO, r);
+                    tmem_ld32(lane_base + kColO + 32 * hf, r);
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         o[j] = fmaf(o[j], alpha, __uint_as_float(r[j]));
-                    tmem_ld32(lane_base + kColO + 32, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        o[32 + j] = fmaf(o[32 + j], alpha, __uint_as_float(r[j]));
                     l_run = fmaf(l_run, alpha, l_add);
                     m_run = m_new;
                 }
@@ -483,33 +506,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok)
                 break;
-            // epilogue: normalise and store this thread's row
-            if (row < qrows) {
-                const float inv = 1.f / l_run;
-                const int64_t t = static_cast<int64_t>(it.seq0) + q0 + row;
-                const int64_t off = (t * H + it.h) * kD;
-                if (p.out_dt == RRA_F32) {
-                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
+            // epilogue: the pair adds its partial row sums, then each warp stores its 32 columns
+            if (warp_active) {
+                if (hf == 1)
+                    red_sum[row] = l_run;
+                pair_sync(q4);
+                const float l_tot = l_run + (hf == 0 ? red_sum[row] : 0.f);
+                if (hf == 0)
+                    red_sum[row] = l_tot;
+                pair_sync(q4);
+                const float inv = 1.f / red_sum[row];
+                if (row < qrows) {
+                    const int t = it.seq0 + q0 + row;
+                    const int64_t off = (static_cast<int64_t>(t) * H + it.h) * kD + 32 * hf;
+                    if (p.out_dt == RRA_F32) {
+                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
 #pragma unroll
-                    for (int j = 0; j < kD / 4; ++j)
-                        dst[j] = make_float4(o[4 * j] * inv, o[4 * j + 1] * inv, o[4 * j + 2] * inv, o[4 * j + 3] * inv);
-                } else {
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + off);
+                        for (int j = 0; j < 8; ++j)
+                            dst[j] = make_float4(o[4 * j] * inv, o[4 * j + 1] * inv, o[4 * j + 2] * inv,
+                                                 o[4 * j + 3] * inv);
+                    } else {
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + off);
 #pragma unroll
-                    for (int j = 0; j < kD / 8; ++j) {
-                        uint4 w;
-                        if (p.out_dt == RRA_BF16) {
-                            w.x = pack_bf16(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
-                            w.y = pack_bf16(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
-                            w.z = pack_bf16(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
-                            w.w = pack_bf16(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
-                        } else {
-                            w.x = pack_f16(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
-                            w.y = pack_f16(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
-                            w.z = pack_f16(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
-                            w.w = pack_f16(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
+                        for (int j = 0; j < 4; ++j) {
+                            uint4 w;
+                            if (p.out_dt == RRA_BF16) {
+                                w.x = pack_bf16(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
+                                w.y = pack_bf16(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
+                                w.z = pack_bf16(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
+                                w.w = pack_bf16(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
+                            } else {
+                                w.x = pack_f16(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
+                                w.y = pack_f16(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
+                                w.z = pack_f16(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
+                                w.w = pack_f16(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
+                            }
+                            dst[j] = w;
                         }
-                        dst[j] = w;
                     }
                 }
             }
@@ -601,7 +634,7 @@ cudaError_t launch_attend(const AttendArgs &a, int num_sms, cudaStream_t stream)
     p.err = a.err;
     p.wait_ns = a.wait_ns;
 
-    int smem = kSmemFixed + (a.B + 1) * 4;
+    int smem = kSmemFixed + 2 * (a.B + 1) * 4;
     if (smem < kSmemFloor)
         smem = kSmemFloor;
     const int64_t max_tiles = (static_cast<int64_t>(a.max_seqlen > 0 ? a.max_seqlen : 1) + BM - 1) / BM;
