@@ -20,8 +20,10 @@
 //                   within a 128-key chunk the two warps take alternate 32-key slices, so
 //                   row max / row sum are thread-local plus one exchange per chunk between
 //                   the two warps of a pair; keys are taken in chunks of 128 with an online
-//                   (running max, rescaled sum) merge of O in registers (each warp of a pair
-//                   keeps 32 of the 64 output columns), then rows are normalised and stored;
+//                   softmax: O accumulates in TMEM across chunks, and when a row's running
+//                   max rises the warps rescale that row of O in TMEM before the next PV MMA
+//                   (each warp of a pair owns 32 of the 64 output columns), then rows are
+//                   normalised and stored;
 //   * for bf16 inputs P is split into a bf16 head and a bf16 remainder (two PV MMAs), which
 //     keeps P at ~16 significant bits; fp16 P (11 bits) is used as is;
 //   * key rows past the sequence end get probability 0 and the matching V rows are zeroed
@@ -163,7 +165,7 @@ __device__ __forceinline__ void pair_sync(int quarter)
 }
 
 template <bool kBF16>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const Params p)
 {
@@ -303,6 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t q_ph[kStages] = {0, 0}, kv_ph[kStages] = {0, 0};
         uint32_t p_ph = 0, ofree_ph = 0, pv_ph = 0;
         uint32_t n_pv = 0;  // PV commits issued (each completes a phase of o_full)
+        uint32_t n_items = 0;
         int qs = 0, ks = 0;
         const uint32_t idPV = idesc_f16(BM, kD, kBF16 ? 1u : 0u, 1u);
         bool ok = true;
@@ -348,12 +351,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_commit(&bars->s_full);
                 }
                 __syncwarp();
-                // P written by the softmax warps, previous O chunk consumed
+                // P written (and O rescaled) by the softmax warps; before the first PV of an item
+                // the previous item's O must have been read out by the epilogue
                 ok = warp_wait(&bars->p_full, p_ph, bars, p);
                 if (!ok)
                     break;
                 p_ph ^= 1u;
-                if (n_pv > 0) {
+                if (kc == 0 && n_items > 0) {
                     ok = warp_wait(&bars->o_free, ofree_ph, bars, p);
                     if (!ok)
                         break;
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // remainder 16 columns further
                     for (int j = 0; j < nk16 / 16; ++j)
                         mma_ts(tmem + kColO, tmem + kColS + 32 * (j >> 1) + 8 * (j & 1),
-                               smem_desc_sw128(sVa + j * 2048, 16, 1024), idPV, j > 0 ? 1u : 0u);
+                               smem_desc_sw128(sVa + j * 2048, 16, 1024), idPV, (kc > 0 || j > 0) ? 1u : 0u);
                     if (kBF16)
                         for (int j = 0; j < nk16 / 16; ++j)
                             mma_ts(tmem + kColO, tmem + kColS + 32 * (j >> 1) + 8 * (j & 1) + 16,
@@ -379,6 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++n_pv;
                 ks ^= 1;
             }
+            ++n_items;
             qs ^= 1;
         }
         // drain: every MMA this thread issued has completed
@@ -404,10 +409,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int qrows = min(BM, it.L - q0);
             const bool warp_active = q4 * 32 < qrows;
             float m_run = -INFINITY, l_run = 0.f;
-            float o[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                o[j] = 0.f;
             for (int kc = 0; kc < nkc; ++kc) {
                 const int nk = min(BN, it.L - kc * BN);
                 const int nk16 = (nk + 15) & ~15;
@@ -416,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 s_ph ^= 1u;
                 tc_fence_after();
-                float m_new = m_run, l_add = 0.f;
+                float m_new = m_run;
                 if (warp_active) {
                     // pass 1: row max over this warp's valid keys, combined with the pair
                     float mx = -INFINITY;
@@ -441,29 +442,52 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (hf == 0)
                         red_max[row] = fmaxf(mx, red_max[row]);
                     pair_sync(q4);
-                    mx = red_max[row];
-                    m_new = fmaxf(m_run, mx);
+                    m_new = fmaxf(m_run, red_max[row]);
+                }
+                // later chunks: the previous PV has landed in O; rescale rows whose max rose
+                if (kc > 0) {
+                    ok = warp_wait(&bars->o_full, o_ph, bars, p);
+                    if (!ok)
+                        break;
+                    o_ph ^= 1u;
+                    tc_fence_after();
+                    if (warp_active) {
+                        const float alpha = ex2_approx((m_run - m_new) * p.scale_log2);
+                        l_run *= alpha;
+                        if (__any_sync(0xffffffffu, m_new > m_run)) {
+                            uint32_t r[32];
+                            tmem_ld32(lane_base + kColO + 32 * hf, r);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
+                            tmem_st32(lane_base + kColO + 32 * hf, r);
+                        }
+                    }
+                }
+                if (warp_active) {
+                    m_run = m_new;
                     const float neg_m = -m_new * p.scale_log2;
                     // pass 2: P = exp2(scale*log2e*(s - m)), row sum, P back over this slice's S
                     for (int c = 32 * hf; c < nk16; c += 64) {
                         uint32_t r[32];
                         tmem_ld32(lane_base + kColS + c, r);
                         tmem_wait_ld();
-                        float pv[32];
                         if (c + 32 <= nk) {
 #pragma unroll
                             for (int j = 0; j < 32; ++j)
-                                pv[j] = ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, neg_m));
+                                r[j] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, neg_m)));
                         } else {
 #pragma unroll
                             for (int j = 0; j < 32; ++j)
-                                pv[j] = (c + j < nk) ? ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, neg_m)) : 0.f;
+                                r[j] = __float_as_uint(
+                                    (c + j < nk) ? ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, neg_m)) : 0.f);
                         }
                         uint32_t pp[32];
 #pragma unroll
                         for (int jj = 0; jj < 16; ++jj) {
-                            const float a = pv[2 * jj], b = pv[2 * jj + 1];
-                            l_add += a + b;
+                            const float a = __uint_as_float(r[2 * jj]), b = __uint_as_float(r[2 * jj + 1]);
+                            l_run += a + b;
                             if (kBF16) {
                                 pp[jj] = pack_bf16(a, b);
                                 const float ha = __uint_as_float(pp[jj] << 16);
@@ -476,44 +500,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         tmem_st32(lane_base + kColS + c, pp);
                     }
-                    tmem_wait_st();
                 }
+                tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&bars->p_full);
-                // O chunk = P V; merge this warp's 32 output columns with a running max rescale
-                ok = warp_wait(&bars->o_full, o_ph, bars, p);
-                if (!ok)
-                    break;
-                o_ph ^= 1u;
-                tc_fence_after();
-                if (warp_active) {
-                    const float alpha = ex2_approx((m_run - m_new) * p.scale_log2);
-                    uint32_t r[32];
-                    tmem_ld32(lane_base + kColO + 32 * hf, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        o[j] = fmaf(o[j], alpha, __uint_as_float(r[j]));
-                    l_run = fmaf(l_run, alpha, l_add);
-                    m_run = m_new;
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&bars->o_free);
             }
             if (!ok)
                 break;
-            // epilogue: the pair adds its partial row sums, then each warp stores its 32 columns
+            // epilogue: last PV landed; the pair adds its partial row sums, each warp normalises
+            // and stores its 32 output columns, then O is released for the next item
+            ok = warp_wait(&bars->o_full, o_ph, bars, p);
+            if (!ok)
+                break;
+            o_ph ^= 1u;
+            tc_fence_after();
             if (warp_active) {
+                uint32_t r[32];
+                tmem_ld32(lane_base + kColO + 32 * hf, r);
+                tmem_wait_ld();
                 if (hf == 1)
                     red_sum[row] = l_run;
                 pair_sync(q4);
-                const float l_tot = l_run + (hf == 0 ? red_sum[row] : 0.f);
                 if (hf == 0)
-                    red_sum[row] = l_tot;
+                    red_sum[row] = l_run + red_sum[row];
                 pair_sync(q4);
                 const float inv = 1.f / red_sum[row];
                 if (row < qrows) {
@@ -523,29 +534,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                         float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
 #pragma unroll
                         for (int j = 0; j < 8; ++j)
-                            dst[j] = make_float4(o[4 * j] * inv, o[4 * j + 1] * inv, o[4 * j + 2] * inv,
-                                                 o[4 * j + 3] * inv);
+                            dst[j] = make_float4(__uint_as_float(r[4 * j]) * inv, __uint_as_float(r[4 * j + 1]) * inv,
+                                                 __uint_as_float(r[4 * j + 2]) * inv,
+                                                 __uint_as_float(r[4 * j + 3]) * inv);
                     } else {
                         uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + off);
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
+                            float f[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                f[e] = __uint_as_float(r[8 * j + e]) * inv;
                             uint4 w;
                             if (p.out_dt == RRA_BF16) {
-                                w.x = pack_bf16(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
-                                w.y = pack_bf16(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
-                                w.z = pack_bf16(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
-                                w.w = pack_bf16(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
+                                w.x = pack_bf16(f[0], f[1]);
+                                w.y = pack_bf16(f[2], f[3]);
+                                w.z = pack_bf16(f[4], f[5]);
+                                w.w = pack_bf16(f[6], f[7]);
                             } else {
-                                w.x = pack_f16(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
-                                w.y = pack_f16(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
-                                w.z = pack_f16(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
-                                w.w = pack_f16(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
+                                w.x = pack_f16(f[0], f[1]);
+                                w.y = pack_f16(f[2], f[3]);
+                                w.z = pack_f16(f[4], f[5]);
+                                w.w = pack_f16(f[6], f[7]);
                             }
                             dst[j] = w;
                         }
                     }
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&bars->o_free);
         }
     }
 
