@@ -6,28 +6,28 @@
 //     o_i = sum_j softmax_j(scale * q_i . k_j) v_j,   j over all L_b kept tokens of image b.
 //
 // How (B200-specific design, not the pages' Triton kernel):
-//   * one persistent launch of two blocks per SM; each block walks a list of
-//     (image, 128-row q-tile, head) work items that it derives from cu_seqlens on the device,
-//     so the host never learns T;
-//   * inside a block, warps specialise:
-//       warp 0      TMA producer: Q tile and 128-key K/V chunks of one head, fetched straight
-//                   from the packed [T, H, 64] layout (3-D tensor map, head = coordinate,
-//                   128-byte swizzle) into two-slot rings, so the next item's loads overlap
-//                   the current item's math;
-//       warp 1      tensor-core issuer: S = Q K^T and O_chunk = P V as tcgen05.mma with fp32
-//                   accumulators in TMEM (P comes from TMEM as the A operand);
-//       warps 2..9  softmax: a pair of warps owns each quarter of the rows (TMEM lanes);
-//                   within a 128-key chunk the two warps take alternate 32-key slices, so
-//                   row max / row sum are thread-local plus one exchange per chunk between
-//                   the two warps of a pair; keys are taken in chunks of 128 with an online
-//                   softmax: O accumulates in TMEM across chunks, and when a row's running
-//                   max rises the warps rescale that row of O in TMEM before the next PV MMA
-//                   (each warp of a pair owns 32 of the 64 output columns), then rows are
-//                   normalised and stored;
+//   * one persistent block per SM walks a list of (image, 128-row q-tile, head) work items
+//     derived from cu_seqlens on the device, so the host never learns T; each item is taken
+//     in steps of 128 keys;
+//   * the block owns all 512 TMEM columns: two S buffers (fp32 [128 x 128]) and two O buffers
+//     (fp32 [128 x 64]), so the tensor core computes S of the next step while the softmax
+//     warps work on the current one, and PV of one item runs under the next item's softmax;
+//   * warps specialise:
+//       warp 0      TMA producer: Q tiles (2-slot ring) and 128-key K/V chunks (3-slot ring)
+//                   of one head, fetched straight from the packed [T, H, 64] layout (3-D tensor
+//                   map, head = coordinate, 128-byte swizzle);
+//       warp 1      tensor-core issuer: S = Q K^T (smem x smem) and O += P V (P from TMEM as the
+//                   A operand), fp32 accumulation, completion signalled through mbarriers;
+//       warps 2..9  softmax: a pair of warps owns each quarter of the rows (TMEM lanes); within
+//                   a step the two warps take alternate 32-key slices, keep them in registers
+//                   for both passes (row max, then exponentials), exchange the row max once,
+//                   write P back over their own S columns, and rescale their half of O in TMEM
+//                   when a row's running max rises; an item's normalise-and-store epilogue runs
+//                   after the next item's softmax, when its last PV has long finished;
 //   * for bf16 inputs P is split into a bf16 head and a bf16 remainder (two PV MMAs), which
 //     keeps P at ~16 significant bits; fp16 P (11 bits) is used as is;
-//   * key rows past the sequence end get probability 0 and the matching V rows are zeroed
-//     in shared memory, so whatever bytes lie there (the next image, or uninitialised capacity
+//   * key rows past the sequence end get probability 0 and the matching V rows are zeroed in
+//     shared memory, so whatever bytes lie there (the next image, or uninitialised capacity
 //     rows) never reach the output;
 //   * every wait is bounded in time; on expiry the block records RRA_ERR_TIMEOUT, raises a
 //     block-wide abort flag, drains the copies and MMAs it issued, frees TMEM and leaves.
@@ -43,27 +43,28 @@ namespace rra {
 namespace {
 
 constexpr int BM = 128;                 // query rows per tile (TMEM lanes)
-constexpr int BN = 128;                 // keys per chunk
+constexpr int BN = 128;                 // keys per step
 constexpr int kD = 64;                  // head dim
 constexpr int kThreads = 320;           // 10 warps: producer, MMA, 8 x softmax
 constexpr int kSoftmaxWarps = 8;
-constexpr uint32_t kTmemCols = 256;
-// S chunk, fp32 [128 x 128].  The P of each 32-key slice is written back over that slice's own
-// S columns: bf16/fp16 head part in its first 16 columns, bf16 remainder in the next 16.
-constexpr uint32_t kColS = 0;
-constexpr uint32_t kColO = 128;         // O chunk, fp32 [128 x 64]
+constexpr uint32_t kTmemCols = 512;
+// TMEM columns: S buffers at 0 and 128 (the P of each 32-key slice is written back over the
+// slice's own S columns: 16 columns of packed head values, then 16 of bf16 remainders), O
+// buffers at 256 and 320.
+constexpr uint32_t kColS0 = 0;
+constexpr uint32_t kColO0 = 256;
 constexpr uint32_t kTileBytes = 128 * 128;
-constexpr int kStages = 2;              // ring depth of the Q slots and of the K/V chunk slots
+constexpr int kQStages = 2;
+constexpr int kKVStages = 3;
 
 // shared-memory map (offsets from a 1024-byte aligned base)
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kStages * kTileBytes;
-constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
-constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
-constexpr uint32_t kOffRed = kOffBar + 256;             // row max / row sum exchange, 2 x 128 floats
-constexpr uint32_t kOffTile = kOffRed + 2 * 128 * 4;    // tile_pre[B+1], then cu[B+1]
+constexpr uint32_t kOffK = kOffQ + kQStages * kTileBytes;
+constexpr uint32_t kOffV = kOffK + kKVStages * kTileBytes;
+constexpr uint32_t kOffBar = kOffV + kKVStages * kTileBytes;
+constexpr uint32_t kOffRed = kOffBar + 512;             // [2 parities][2 halves][128] row max, same for row sum
+constexpr uint32_t kOffTile = kOffRed + 2 * 2 * 2 * 128 * 4;  // tile_pre[B+1], then cu[B+1]
 constexpr int kSmemFixed = 1024 /*align slack*/ + kOffTile;
-constexpr int kSmemFloor = 80 * 1024;   // keeps at most two blocks (2 x 256 TMEM columns) per SM
 
 struct Params {
     const int32_t *cu;
@@ -79,14 +80,16 @@ struct Params {
 constexpr uint64_t kDrainNs = 2000000000ull;
 
 struct Bars {
-    uint64_t q_full[kStages], q_empty[kStages];
-    uint64_t kv_full[kStages], kv_empty[kStages];
-    uint64_t s_full, p_full, o_full, o_free, drain;
+    uint64_t q_full[kQStages], q_empty[kQStages];
+    uint64_t kv_full[kKVStages], kv_empty[kKVStages];
+    uint64_t s_full[2], p_full[2], s_free[2];
+    uint64_t o_full[2], o_free[2];
+    uint64_t drain;
     uint32_t tmem_slot;
     int abort;
     int warp_sums[kThreads / 32];
 };
-static_assert(sizeof(Bars) <= 256, "barrier block overflows its slot");
+static_assert(sizeof(Bars) <= 512, "barrier block overflows its slot");
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 {
@@ -164,17 +167,74 @@ __device__ __forceinline__ void pair_sync(int quarter)
     asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
 }
 
+// Exponentials of one 32-key slice of a row (keys c .. c+31, those >= nk masked to 0), added to
+// the row sum, then written back over the slice's own TMEM columns as the PV A operand: 16
+// columns of packed head values (bf16 or fp16 pairs), then for bf16 16 columns of remainders.
 template <bool kBF16>
-__global__ void __launch_bounds__(kThreads, 2)
+__device__ __forceinline__ void softmax_slice(uint32_t (&r)[32], int c, int nk, float scale_log2, float neg_m,
+                                              float &l_sum, uint32_t taddr)
+{
+    if (c + 32 <= nk) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            r[j] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(r[j]), scale_log2, neg_m)));
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            r[j] = __float_as_uint((c + j < nk) ? ex2_approx(fmaf(__uint_as_float(r[j]), scale_log2, neg_m)) : 0.f);
+    }
+    uint32_t hi[16];
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+        const float a = __uint_as_float(r[2 * jj]), b = __uint_as_float(r[2 * jj + 1]);
+        l_sum += a + b;
+        hi[jj] = kBF16 ? pack_bf16(a, b) : pack_f16(a, b);
+    }
+    tmem_st16(taddr, hi);
+    if (kBF16) {
+        uint32_t lo[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+            const float a = __uint_as_float(r[2 * jj]) - __uint_as_float(hi[jj] << 16);
+            const float b = __uint_as_float(r[2 * jj + 1]) - __uint_as_float(hi[jj] & 0xFFFF0000u);
+            lo[jj] = pack_bf16(a, b);
+        }
+        tmem_st16(taddr + 16, lo);
+    }
+}
+
+__device__ __forceinline__ float slice_max(const uint32_t (&r)[32], int c, int nk, float mx)
+{
+    if (c + 32 <= nk) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            mx = fmaxf(mx, __uint_as_float(r[j]));
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (c + j < nk)
+                mx = fmaxf(mx, __uint_as_float(r[j]));
+    }
+    return mx;
+}
+
+// One PV step as the MMA warp sees it.
+struct PvStep {
+    int sb, ks, ob, kc, nk16;
+    bool wait_free;  // first PV of an item whose O buffer held an earlier item
+};
+
+template <bool kBF16>
+__global__ void __launch_bounds__(kThreads, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const Params p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars *bars = reinterpret_cast<Bars *>(base + kOffBar);
+    float *red = reinterpret_cast<float *>(base + kOffRed);            // max [2][2][128], sum [2][2][128]
     int32_t *tile_pre = reinterpret_cast<int32_t *>(base + kOffTile);  // [B+1]
     int32_t *cu_s = tile_pre + (p.B + 1);                               // [B+1]
-    float *red = reinterpret_cast<float *>(base + kOffRed);            // [2][128]
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -185,16 +245,21 @@ __global__ void __launch_bounds__(kThreads, 2)
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kQStages; ++s) {
             mbar_init(&bars->q_full[s], 1);
             mbar_init(&bars->q_empty[s], 1);
+        }
+        for (int s = 0; s < kKVStages; ++s) {
             mbar_init(&bars->kv_full[s], 1);
             mbar_init(&bars->kv_empty[s], 1);
         }
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_full, kSoftmaxWarps);   // one arrival per softmax warp
-        mbar_init(&bars->o_full, 1);
-        mbar_init(&bars->o_free, kSoftmaxWarps);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars->s_full[s], 1);
+            mbar_init(&bars->p_full[s], kSoftmaxWarps);  // one arrival per softmax warp
+            mbar_init(&bars->s_free[s], 1);
+            mbar_init(&bars->o_full[s], 1);
+            mbar_init(&bars->o_free[s], kSoftmaxWarps);
+        }
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
         fence_mbarrier_init();
@@ -204,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tmem_relinquish();
     }
 
-    // ---- work list: tile_pre[b] = number of 128-row query tiles of images < b.
+    // ---- work list: tile_pre[b] = number of 128-row query tiles of images < b; cu staged too.
     if (tid == 0)
         tile_pre[0] = 0;
     int carry = 0;
@@ -257,14 +322,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         // Empty-slot waits use the usual parity idiom: on a fresh barrier the phase "before"
         // phase 0 counts as complete, so waiting on parity (phase ^ 1) passes at once for the
         // first fill of each slot, then tracks the consumer's releases.
-        uint32_t q_phase[kStages] = {0, 0}, kv_phase[kStages] = {0, 0};
-        uint32_t q_issued = 0, kv_issued = 0;  // how many Q / KV slot fills were issued
+        uint32_t q_phase[kQStages] = {0, 0}, kv_phase[kKVStages] = {0, 0, 0};
+        uint32_t q_issued = 0, kv_issued = 0;
         int qs = 0, ks = 0;
         bool ok = true;
         for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
             const Item it = decode_item(item, H, B, tile_pre, cu_s);
             const int nkc = (it.L + BN - 1) / BN;
-            // Q slot: free once the previous user of the slot has finished its last PV MMA
             ok = warp_wait(&bars->q_empty[qs], q_phase[qs] ^ 1u, bars, p);
             if (!ok)
                 break;
@@ -275,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             __syncwarp();
             ++q_issued;
-            qs ^= 1;
+            qs = (qs + 1 == kQStages) ? 0 : qs + 1;
             for (int kc = 0; kc < nkc; ++kc) {
                 ok = warp_wait(&bars->kv_empty[ks], kv_phase[ks] ^ 1u, bars, p);
                 if (!ok)
@@ -288,27 +352,64 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
                 __syncwarp();
                 ++kv_issued;
-                ks ^= 1;
+                ks = (ks + 1 == kKVStages) ? 0 : ks + 1;
             }
         }
         // drain: every issued fill has landed before the block may leave
-        for (int s = 0; s < kStages; ++s) {
-            const uint32_t nq = q_issued / kStages + (static_cast<uint32_t>(s) < q_issued % kStages ? 1u : 0u);
-            if (nq > 0)
-                mbar_wait_bounded(&bars->q_full[s], (nq - 1) & 1u, kDrainNs);
-            const uint32_t nk = kv_issued / kStages + (static_cast<uint32_t>(s) < kv_issued % kStages ? 1u : 0u);
-            if (nk > 0)
-                mbar_wait_bounded(&bars->kv_full[s], (nk - 1) & 1u, kDrainNs);
+        for (int s = 0; s < kQStages; ++s) {
+            const uint32_t n = q_issued / kQStages + (static_cast<uint32_t>(s) < q_issued % kQStages ? 1u : 0u);
+            if (n > 0)
+                mbar_wait_bounded(&bars->q_full[s], (n - 1) & 1u, kDrainNs);
+        }
+        for (int s = 0; s < kKVStages; ++s) {
+            const uint32_t n = kv_issued / kKVStages + (static_cast<uint32_t>(s) < kv_issued % kKVStages ? 1u : 0u);
+            if (n > 0)
+                mbar_wait_bounded(&bars->kv_full[s], (n - 1) & 1u, kDrainNs);
         }
     } else if (warp == 1) {
         // ================================================================ tcgen05 issuer
-        uint32_t q_ph[kStages] = {0, 0}, kv_ph[kStages] = {0, 0};
-        uint32_t p_ph = 0, ofree_ph = 0, pv_ph = 0;
-        uint32_t n_pv = 0;  // PV commits issued (each completes a phase of o_full)
-        uint32_t n_items = 0;
-        int qs = 0, ks = 0;
+        // Order: S(t) then PV(t-1), so the next step's QK^T runs while the softmax warps work.
+        uint32_t q_ph[kQStages] = {0, 0}, kv_ph[kKVStages] = {0, 0, 0};
+        uint32_t p_ph[2] = {0, 0}, sfree_ph[2] = {0, 0}, ofree_ph[2] = {0, 0};
         const uint32_t idPV = idesc_f16(BM, kD, kBF16 ? 1u : 0u, 1u);
+        int qs = 0, ks = 0;
+        int t = 0, n = 0;
+        bool have_prev = false;
+        PvStep prev{0, 0, 0, 0, 0, false};
         bool ok = true;
+
+        auto issue_pv = [&](const PvStep &u) -> bool {
+            if (!warp_wait(&bars->p_full[u.sb], p_ph[u.sb], bars, p))
+                return false;
+            p_ph[u.sb] ^= 1u;
+            if (u.wait_free) {
+                // first PV of an item: the O buffer's previous item must have been read out
+                if (!warp_wait(&bars->o_free[u.ob], ofree_ph[u.ob], bars, p))
+                    return false;
+                ofree_ph[u.ob] ^= 1u;
+            }
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t sVa = smem_addr(base + kOffV + u.ks * kTileBytes);
+                const uint32_t dO = tmem + kColO0 + 64 * u.ob;
+                const uint32_t aP = tmem + kColS0 + 128 * u.sb;
+                // keys 16j..16j+15 live in slice j/2: head part at column 32(j/2) + 8(j%2),
+                // remainder 16 columns further
+                for (int j = 0; j < u.nk16 / 16; ++j)
+                    mma_ts(dO, aP + 32 * (j >> 1) + 8 * (j & 1), smem_desc_sw128(sVa + j * 2048, 16, 1024), idPV,
+                           (u.kc > 0 || j > 0) ? 1u : 0u);
+                if (kBF16)
+                    for (int j = 0; j < u.nk16 / 16; ++j)
+                        mma_ts(dO, aP + 32 * (j >> 1) + 8 * (j & 1) + 16, smem_desc_sw128(sVa + j * 2048, 16, 1024),
+                               idPV, 1u);
+                mma_commit(&bars->o_full[u.ob]);
+                mma_commit(&bars->s_free[u.sb]);
+                mma_commit(&bars->kv_empty[u.ks]);
+            }
+            __syncwarp();
+            return true;
+        };
+
         for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
             const Item it = decode_item(item, H, B, tile_pre, cu_s);
             const int nkc = (it.L + BN - 1) / BN;
@@ -320,6 +421,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int kc = 0; kc < nkc; ++kc) {
                 const int nk = min(BN, it.L - kc * BN);
                 const int nk16 = (nk + 15) & ~15;
+                const int sb = t & 1;
                 ok = warp_wait(&bars->kv_full[ks], kv_ph[ks], bars, p);
                 if (!ok)
                     break;
@@ -332,60 +434,42 @@ __global__ void __launch_bounds__(kThreads, 2)
                     fence_proxy_async_smem();
                 }
                 __syncwarp();
-                // S region (which holds the previous chunk's P) is free once that PV completed
-                if (n_pv > 0) {
-                    ok = warp_wait(&bars->o_full, pv_ph, bars, p);
+                // S buffer sb holds P of step t-2 until that PV completes
+                if (t >= 2) {
+                    ok = warp_wait(&bars->s_free[sb], sfree_ph[sb], bars, p);
                     if (!ok)
                         break;
-                    pv_ph ^= 1u;
+                    sfree_ph[sb] ^= 1u;
                 }
-                const uint32_t sKa = smem_addr(base + kOffK + ks * kTileBytes);
-                const uint32_t sVa = smem_addr(sV);
                 if (lane == 0) {
                     tc_fence_after();
+                    const uint32_t sKa = smem_addr(base + kOffK + ks * kTileBytes);
                     const uint32_t idS = idesc_f16(BM, nk16, kBF16 ? 1u : 0u, 0u);
 #pragma unroll
                     for (int kk = 0; kk < kD / 16; ++kk)
-                        mma_ss(tmem + kColS, smem_desc_sw128(sQa + kk * 32, 16, 1024),
+                        mma_ss(tmem + kColS0 + 128 * sb, smem_desc_sw128(sQa + kk * 32, 16, 1024),
                                smem_desc_sw128(sKa + kk * 32, 16, 1024), idS, kk > 0 ? 1u : 0u);
-                    mma_commit(&bars->s_full);
+                    mma_commit(&bars->s_full[sb]);
+                    if (kc == nkc - 1)
+                        mma_commit(&bars->q_empty[qs]);  // last read of this Q tile
                 }
                 __syncwarp();
-                // P written (and O rescaled) by the softmax warps; before the first PV of an item
-                // the previous item's O must have been read out by the epilogue
-                ok = warp_wait(&bars->p_full, p_ph, bars, p);
-                if (!ok)
-                    break;
-                p_ph ^= 1u;
-                if (kc == 0 && n_items > 0) {
-                    ok = warp_wait(&bars->o_free, ofree_ph, bars, p);
+                if (have_prev) {
+                    ok = issue_pv(prev);
                     if (!ok)
                         break;
-                    ofree_ph ^= 1u;
                 }
-                if (lane == 0) {
-                    tc_fence_after();
-                    // keys 16j..16j+15 live in slice j/2: head part at column 32(j/2) + 8(j%2),
-                    // remainder 16 columns further
-                    for (int j = 0; j < nk16 / 16; ++j)
-                        mma_ts(tmem + kColO, tmem + kColS + 32 * (j >> 1) + 8 * (j & 1),
-                               smem_desc_sw128(sVa + j * 2048, 16, 1024), idPV, (kc > 0 || j > 0) ? 1u : 0u);
-                    if (kBF16)
-                        for (int j = 0; j < nk16 / 16; ++j)
-                            mma_ts(tmem + kColO, tmem + kColS + 32 * (j >> 1) + 8 * (j & 1) + 16,
-                                   smem_desc_sw128(sVa + j * 2048, 16, 1024), idPV, 1u);
-                    mma_commit(&bars->o_full);
-                    mma_commit(&bars->kv_empty[ks]);
-                    if (kc == nkc - 1)
-                        mma_commit(&bars->q_empty[qs]);
-                }
-                __syncwarp();
-                ++n_pv;
-                ks ^= 1;
+                // this step's PV: O buffer n&1, released by the epilogue of item n-2
+                prev = PvStep{sb, ks, n & 1, kc, nk16, kc == 0 && n >= 2};
+                have_prev = true;
+                ++t;
+                ks = (ks + 1 == kKVStages) ? 0 : ks + 1;
             }
-            ++n_items;
-            qs ^= 1;
+            ++n;
+            qs = (qs + 1 == kQStages) ? 0 : qs + 1;
         }
+        if (ok && have_prev)
+            issue_pv(prev);
         // drain: every MMA this thread issued has completed
         if (lane == 0) {
             mma_commit(&bars->drain);
@@ -395,141 +479,34 @@ __global__ void __launch_bounds__(kThreads, 2)
     } else {
         // ================================================================ softmax + epilogue
         const int q4 = warp & 3;                     // TMEM lane quarter of this warp
-        const int hf = (warp - 2) >> 2;              // which of the pair: slices hf, hf+2, ...; O columns 32hf..
+        const int hf = (warp - 2) >> 2;              // which of the pair: slices hf, hf+2; O columns 32hf..
         const int row = q4 * 32 + lane;              // row of S / O owned by this thread
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-        float *red_max = red;                        // [128]
-        float *red_sum = red + 128;                  // [128]
-        uint32_t s_ph = 0, o_ph = 0;
+        float *red_max = red;                        // [2][2][128]
+        float *red_sum = red + 2 * 2 * 128;          // [2][2][128]
+        uint32_t s_ph[2] = {0, 0}, o_ph[2] = {0, 0};
+        int t = 0, n = 0, n_epi = 0;
         bool ok = true;
-        for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
-            const Item it = decode_item(item, H, B, tile_pre, cu_s);
-            const int nkc = (it.L + BN - 1) / BN;
-            const int q0 = it.qt * BM;
-            const int qrows = min(BM, it.L - q0);
-            const bool warp_active = q4 * 32 < qrows;
-            float m_run = -INFINITY, l_run = 0.f;
-            for (int kc = 0; kc < nkc; ++kc) {
-                const int nk = min(BN, it.L - kc * BN);
-                const int nk16 = (nk + 15) & ~15;
-                ok = warp_wait(&bars->s_full, s_ph, bars, p);
-                if (!ok)
-                    break;
-                s_ph ^= 1u;
-                tc_fence_after();
-                float m_new = m_run;
-                if (warp_active) {
-                    // pass 1: row max over this warp's valid keys, combined with the pair
-                    float mx = -INFINITY;
-                    for (int c = 32 * hf; c < nk16; c += 64) {
-                        uint32_t r[32];
-                        tmem_ld32(lane_base + kColS + c, r);
-                        tmem_wait_ld();
-                        if (c + 32 <= nk) {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                mx = fmaxf(mx, __uint_as_float(r[j]));
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (c + j < nk)
-                                    mx = fmaxf(mx, __uint_as_float(r[j]));
-                        }
-                    }
-                    if (hf == 1)
-                        red_max[row] = mx;
-                    pair_sync(q4);
-                    if (hf == 0)
-                        red_max[row] = fmaxf(mx, red_max[row]);
-                    pair_sync(q4);
-                    m_new = fmaxf(m_run, red_max[row]);
-                }
-                // later chunks: the previous PV has landed in O; rescale rows whose max rose
-                if (kc > 0) {
-                    ok = warp_wait(&bars->o_full, o_ph, bars, p);
-                    if (!ok)
-                        break;
-                    o_ph ^= 1u;
-                    tc_fence_after();
-                    if (warp_active) {
-                        const float alpha = ex2_approx((m_run - m_new) * p.scale_log2);
-                        l_run *= alpha;
-                        if (__any_sync(0xffffffffu, m_new > m_run)) {
-                            uint32_t r[32];
-                            tmem_ld32(lane_base + kColO + 32 * hf, r);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-                            tmem_st32(lane_base + kColO + 32 * hf, r);
-                        }
-                    }
-                }
-                if (warp_active) {
-                    m_run = m_new;
-                    const float neg_m = -m_new * p.scale_log2;
-                    // pass 2: P = exp2(scale*log2e*(s - m)), row sum, P back over this slice's S
-                    for (int c = 32 * hf; c < nk16; c += 64) {
-                        uint32_t r[32];
-                        tmem_ld32(lane_base + kColS + c, r);
-                        tmem_wait_ld();
-                        if (c + 32 <= nk) {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                r[j] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, neg_m)));
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                r[j] = __float_as_uint(
-                                    (c + j < nk) ? ex2_approx(fmaf(__uint_as_float(r[j]), p.scale_log2, neg_m)) : 0.f);
-                        }
-                        uint32_t pp[32];
-#pragma unroll
-                        for (int jj = 0; jj < 16; ++jj) {
-                            const float a = __uint_as_float(r[2 * jj]), b = __uint_as_float(r[2 * jj + 1]);
-                            l_run += a + b;
-                            if (kBF16) {
-                                pp[jj] = pack_bf16(a, b);
-                                const float ha = __uint_as_float(pp[jj] << 16);
-                                const float hb = __uint_as_float(pp[jj] & 0xFFFF0000u);
-                                pp[16 + jj] = pack_bf16(a - ha, b - hb);
-                            } else {
-                                pp[jj] = pack_f16(a, b);
-                                pp[16 + jj] = 0u;
-                            }
-                        }
-                        tmem_st32(lane_base + kColS + c, pp);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&bars->p_full);
-            }
-            if (!ok)
-                break;
-            // epilogue: last PV landed; the pair adds its partial row sums, each warp normalises
-            // and stores its 32 output columns, then O is released for the next item
-            ok = warp_wait(&bars->o_full, o_ph, bars, p);
-            if (!ok)
-                break;
-            o_ph ^= 1u;
+
+        // deferred epilogue of the previous item
+        bool pending = false;
+        int pend_row0 = 0, pend_h = 0, pend_qrows = 0, pend_ob = 0;
+        float pend_l = 0.f;
+        auto epilogue = [&]() -> bool {
+            if (!warp_wait(&bars->o_full[pend_ob], o_ph[pend_ob], bars, p))
+                return false;
+            o_ph[pend_ob] ^= 1u;
             tc_fence_after();
-            if (warp_active) {
+            if (q4 * 32 < pend_qrows) {
                 uint32_t r[32];
-                tmem_ld32(lane_base + kColO + 32 * hf, r);
+                tmem_ld32(lane_base + kColO0 + 64 * pend_ob + 32 * hf, r);
+                float *rs = red_sum + (n_epi & 1) * 256;
+                rs[hf * 128 + row] = pend_l;
+                pair_sync(q4);
+                const float inv = 1.f / (rs[row] + rs[128 + row]);
                 tmem_wait_ld();
-                if (hf == 1)
-                    red_sum[row] = l_run;
-                pair_sync(q4);
-                if (hf == 0)
-                    red_sum[row] = l_run + red_sum[row];
-                pair_sync(q4);
-                const float inv = 1.f / red_sum[row];
-                if (row < qrows) {
-                    const int t = it.seq0 + q0 + row;
-                    const int64_t off = (static_cast<int64_t>(t) * H + it.h) * kD + 32 * hf;
+                if (row < pend_qrows) {
+                    const int64_t off = (static_cast<int64_t>(pend_row0 + row) * H + pend_h) * kD + 32 * hf;
                     if (p.out_dt == RRA_F32) {
                         float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
 #pragma unroll
@@ -562,11 +539,108 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 }
             }
+            ++n_epi;
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&bars->o_free);
+                mbar_arrive(&bars->o_free[pend_ob]);
+            pending = false;
+            return true;
+        };
+
+        for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+            const Item it = decode_item(item, H, B, tile_pre, cu_s);
+            const int nkc = (it.L + BN - 1) / BN;
+            const int q0 = it.qt * BM;
+            const int qrows = min(BM, it.L - q0);
+            const bool warp_active = q4 * 32 < qrows;
+            const int ob = n & 1;
+            float m_run = -INFINITY, l_run = 0.f;
+            for (int kc = 0; kc < nkc; ++kc) {
+                const int nk = min(BN, it.L - kc * BN);
+                const int nk16 = (nk + 15) & ~15;
+                const int sb = t & 1;
+                const uint32_t sbase = lane_base + kColS0 + 128 * sb;
+                ok = warp_wait(&bars->s_full[sb], s_ph[sb], bars, p);
+                if (!ok)
+                    break;
+                s_ph[sb] ^= 1u;
+                tc_fence_after();
+                const int c0 = 32 * hf, c1 = c0 + 64;
+                uint32_t r0[32], r1[32];
+                float m_new = m_run;
+                if (warp_active) {
+                    // both slices of this warp in registers for both passes
+                    if (c0 < nk16)
+                        tmem_ld32(sbase + c0, r0);
+                    if (c1 < nk16)
+                        tmem_ld32(sbase + c1, r1);
+                    tmem_wait_ld();
+                    float mx = -INFINITY;
+                    if (c0 < nk16)
+                        mx = slice_max(r0, c0, nk, mx);
+                    if (c1 < nk16)
+                        mx = slice_max(r1, c1, nk, mx);
+                    float *rm = red_max + (t & 1) * 256;
+                    rm[hf * 128 + row] = mx;
+                    pair_sync(q4);
+                    m_new = fmaxf(m_run, fmaxf(rm[row], rm[128 + row]));
+                }
+                // later steps of an item: the previous PV has landed in O; rescale rows whose max rose
+                if (kc > 0) {
+                    ok = warp_wait(&bars->o_full[ob], o_ph[ob], bars, p);
+                    if (!ok)
+                        break;
+                    o_ph[ob] ^= 1u;
+                    tc_fence_after();
+                    if (warp_active) {
+                        const float alpha = ex2_approx((m_run - m_new) * p.scale_log2);
+                        l_run *= alpha;
+                        if (__any_sync(0xffffffffu, m_new > m_run)) {
+                            uint32_t r[32];
+                            const uint32_t oaddr = lane_base + kColO0 + 64 * ob + 32 * hf;
+                            tmem_ld32(oaddr, r);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
+                            tmem_st32(oaddr, r);
+                        }
+                    }
+                }
+                if (warp_active) {
+                    m_run = m_new;
+                    const float neg_m = -m_new * p.scale_log2;
+                    if (c0 < nk16)
+                        softmax_slice<kBF16>(r0, c0, nk, p.scale_log2, neg_m, l_run, sbase + c0);
+                    if (c1 < nk16)
+                        softmax_slice<kBF16>(r1, c1, nk, p.scale_log2, neg_m, l_run, sbase + c1);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bars->p_full[sb]);
+                ++t;
+            }
+            if (!ok)
+                break;
+            // the previous item's PV is long done: store it now, under this item's PV
+            if (pending) {
+                ok = epilogue();
+                if (!ok)
+                    break;
+            }
+            pending = true;
+            pend_row0 = it.seq0 + q0;
+            pend_h = it.h;
+            pend_qrows = qrows;
+            pend_ob = ob;
+            pend_l = l_run;
+            ++n;
         }
+        if (ok && pending)
+            epilogue();
     }
 
     tc_fence_before();
@@ -654,13 +728,11 @@ cudaError_t launch_attend(const AttendArgs &a, int num_sms, cudaStream_t stream)
     p.err = a.err;
     p.wait_ns = a.wait_ns;
 
-    int smem = kSmemFixed + 2 * (a.B + 1) * 4;
-    if (smem < kSmemFloor)
-        smem = kSmemFloor;
+    const int smem = kSmemFixed + 2 * (a.B + 1) * 4;
     const int64_t max_tiles = (static_cast<int64_t>(a.max_seqlen > 0 ? a.max_seqlen : 1) + BM - 1) / BM;
     int64_t grid = static_cast<int64_t>(a.B) * a.H * max_tiles;
-    if (grid > 2LL * num_sms)
-        grid = 2LL * num_sms;
+    if (grid > num_sms)
+        grid = num_sms;  // one block per SM: it owns all 512 TMEM columns
     if (grid < 1)
         grid = 1;
     cudaError_t e = a.in_bf16 ? set_smem_attr<true>(smem) : set_smem_attr<false>(smem);

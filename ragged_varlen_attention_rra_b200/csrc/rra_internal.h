@@ -28,8 +28,9 @@ struct AttendArgs {
     uint64_t wait_ns;
 };
 
-// Largest B rra_attend accepts (its per-block tile table lives in shared memory).
-constexpr int kAttendMaxBatch = 16384;
+// Largest B rra_attend accepts (its per-block tile and cu_seqlens tables live in shared memory
+// next to the 128 KiB of Q/K/V rings).
+constexpr int kAttendMaxBatch = 8192;
 
 cudaError_t launch_attend(const AttendArgs &a, int num_sms, cudaStream_t stream);
 

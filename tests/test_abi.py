@@ -90,6 +90,7 @@ def test_attend_validation(L):
     assert _attend(L, idt=2, odt=2) == rra.RRA_ERR_UNSUPPORTED   # fp32 inputs are not a tensor-core type here
     assert _attend(L, idt=0, odt=1) == rra.RRA_ERR_UNSUPPORTED   # output fp16 in or fp32 only
     assert _attend(L, B=100000) == rra.RRA_ERR_UNSUPPORTED
+    assert _attend(L, B=8193) == rra.RRA_ERR_UNSUPPORTED
     assert _attend(L, scale=float("nan")) == rra.RRA_ERR_INVALID_ARG
     assert L.rra_attend_workspace_size(64, 12, 197) == 0
 
