@@ -26,6 +26,9 @@
 //                   after the next item's softmax, when its last PV has long finished;
 //   * for bf16 inputs P is split into a bf16 head and a bf16 remainder (two PV MMAs), which
 //     keeps P at ~16 significant bits; fp16 P (11 bits) is used as is;
+//   * the PV MMA runs with N = 80: the 64 columns of V plus a constant tile whose first column
+//     is all ones, so column 64 of O accumulates the row sum of exactly the P that was used --
+//     the softmax warps never add up P themselves;
 //   * key rows past the sequence end get probability 0 and the matching V rows are zeroed in
 //     shared memory, so whatever bytes lie there (the next image, or uninitialised capacity
 //     rows) never reach the output;
@@ -50,9 +53,11 @@ constexpr int kSoftmaxWarps = 8;
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: S buffers at 0 and 128 (the P of each 32-key slice is written back over the
 // slice's own S columns: 16 columns of packed head values, then 16 of bf16 remainders), O
-// buffers at 256 and 320.
+// buffers of 80 columns (64 outputs, the row sum, 15 zeros) at 256 and 352.
 constexpr uint32_t kColS0 = 0;
 constexpr uint32_t kColO0 = 256;
+constexpr uint32_t kOCols = 96;         // stride between the two O buffers
+constexpr uint32_t kPvN = 80;
 constexpr uint32_t kTileBytes = 128 * 128;
 constexpr int kQStages = 2;
 constexpr int kKVStages = 3;
@@ -61,9 +66,10 @@ constexpr int kKVStages = 3;
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kQStages * kTileBytes;
 constexpr uint32_t kOffV = kOffK + kKVStages * kTileBytes;
-constexpr uint32_t kOffBar = kOffV + kKVStages * kTileBytes;
-constexpr uint32_t kOffRed = kOffBar + 512;             // [2 parities][2 halves][128] row max, same for row sum
-constexpr uint32_t kOffTile = kOffRed + 2 * 2 * 2 * 128 * 4;  // tile_pre[B+1], then cu[B+1]
+constexpr uint32_t kOffOnes = kOffV + kKVStages * kTileBytes;   // [128 keys x 64] MN-major, column 0 = 1
+constexpr uint32_t kOffBar = kOffOnes + kTileBytes;
+constexpr uint32_t kOffRed = kOffBar + 512;             // [2 parities][2 halves][128] row max
+constexpr uint32_t kOffTile = kOffRed + 2 * 2 * 128 * 4;  // tile_pre[B+1], then cu[B+1]
 constexpr int kSmemFixed = 1024 /*align slack*/ + kOffTile;
 
 struct Params {
@@ -167,12 +173,12 @@ __device__ __forceinline__ void pair_sync(int quarter)
     asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
 }
 
-// Exponentials of one 32-key slice of a row (keys c .. c+31, those >= nk masked to 0), added to
-// the row sum, then written back over the slice's own TMEM columns as the PV A operand: 16
-// columns of packed head values (bf16 or fp16 pairs), then for bf16 16 columns of remainders.
+// Exponentials of one 32-key slice of a row (keys c .. c+31, those >= nk masked to 0), written
+// back over the slice's own TMEM columns as the PV A operand: 16 columns of packed head values
+// (bf16 or fp16 pairs), then for bf16 16 columns of remainders.
 template <bool kBF16>
 __device__ __forceinline__ void softmax_slice(uint32_t (&r)[32], int c, int nk, float scale_log2, float neg_m,
-                                              float &l_sum, uint32_t taddr)
+                                              uint32_t taddr)
 {
     if (c + 32 <= nk) {
 #pragma unroll
@@ -186,9 +192,8 @@ __device__ __forceinline__ void softmax_slice(uint32_t (&r)[32], int c, int nk, 
     uint32_t hi[16];
 #pragma unroll
     for (int jj = 0; jj < 16; ++jj) {
-        const float a = __uint_as_float(r[2 * jj]), b = __uint_as_float(r[2 * jj + 1]);
-        l_sum += a + b;
-        hi[jj] = kBF16 ? pack_bf16(a, b) : pack_f16(a, b);
+        hi[jj] = kBF16 ? pack_bf16(__uint_as_float(r[2 * jj]), __uint_as_float(r[2 * jj + 1]))
+                       : pack_f16(__uint_as_float(r[2 * jj]), __uint_as_float(r[2 * jj + 1]));
     }
     tmem_st16(taddr, hi);
     if (kBF16) {
@@ -232,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars *bars = reinterpret_cast<Bars *>(base + kOffBar);
-    float *red = reinterpret_cast<float *>(base + kOffRed);            // max [2][2][128], sum [2][2][128]
+    float *red = reinterpret_cast<float *>(base + kOffRed);            // row max exchange [2][2][128]
     int32_t *tile_pre = reinterpret_cast<int32_t *>(base + kOffTile);  // [B+1]
     int32_t *cu_s = tile_pre + (p.B + 1);                               // [B+1]
 
@@ -267,6 +272,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         tmem_alloc(&bars->tmem_slot, kTmemCols);
         tmem_relinquish();
+    }
+
+    // ---- constant ones tile: 128 key rows of 128 bytes in the 128-byte-swizzled layout, element 0
+    // of every row = 1.0 (the 16-byte chunk c of row r sits at chunk c ^ (r % 8))
+    {
+        uint8_t *ones = base + kOffOnes;
+        const uint32_t one = kBF16 ? 0x3F80u : 0x3C00u;
+        for (int i = tid; i < 128 * 8; i += kThreads) {
+            const int r = i >> 3, c = i & 7;
+            const uint4 v = make_uint4(c == (r & 7) ? one : 0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(ones + r * 128 + c * 16) = v;
+        }
+        fence_proxy_async_smem();
     }
 
     // ---- work list: tile_pre[b] = number of 128-row query tiles of images < b; cu staged too.
@@ -322,17 +340,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Empty-slot waits use the usual parity idiom: on a fresh barrier the phase "before"
         // phase 0 counts as complete, so waiting on parity (phase ^ 1) passes at once for the
         // first fill of each slot, then tracks the consumer's releases.
-        uint32_t q_phase[kQStages] = {0, 0}, kv_phase[kKVStages] = {0, 0, 0};
+        uint32_t q_phase = 0, kv_phase = 0;  // one bit per slot
         uint32_t q_issued = 0, kv_issued = 0;
         int qs = 0, ks = 0;
         bool ok = true;
         for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
             const Item it = decode_item(item, H, B, tile_pre, cu_s);
             const int nkc = (it.L + BN - 1) / BN;
-            ok = warp_wait(&bars->q_empty[qs], q_phase[qs] ^ 1u, bars, p);
+            ok = warp_wait(&bars->q_empty[qs], ((q_phase >> qs) & 1u) ^ 1u, bars, p);
             if (!ok)
                 break;
-            q_phase[qs] ^= 1u;
+            q_phase ^= 1u << qs;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&bars->q_full[qs], kTileBytes);
                 tma_load_3d(base + kOffQ + qs * kTileBytes, &tm_q, &bars->q_full[qs], 0, it.h, it.seq0 + it.qt * BM);
@@ -341,10 +359,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++q_issued;
             qs = (qs + 1 == kQStages) ? 0 : qs + 1;
             for (int kc = 0; kc < nkc; ++kc) {
-                ok = warp_wait(&bars->kv_empty[ks], kv_phase[ks] ^ 1u, bars, p);
+                ok = warp_wait(&bars->kv_empty[ks], ((kv_phase >> ks) & 1u) ^ 1u, bars, p);
                 if (!ok)
                     break;
-                kv_phase[ks] ^= 1u;
+                kv_phase ^= 1u << ks;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&bars->kv_full[ks], 2 * kTileBytes);
                     tma_load_3d(base + kOffK + ks * kTileBytes, &tm_k, &bars->kv_full[ks], 0, it.h, it.seq0 + kc * BN);
@@ -369,9 +387,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ================================================================ tcgen05 issuer
         // Order: S(t) then PV(t-1), so the next step's QK^T runs while the softmax warps work.
-        uint32_t q_ph[kQStages] = {0, 0}, kv_ph[kKVStages] = {0, 0, 0};
-        uint32_t p_ph[2] = {0, 0}, sfree_ph[2] = {0, 0}, ofree_ph[2] = {0, 0};
-        const uint32_t idPV = idesc_f16(BM, kD, kBF16 ? 1u : 0u, 1u);
+        // phase parities, one bit per slot / buffer
+        uint32_t q_ph = 0, kv_ph = 0, p_ph = 0, sfree_ph = 0, ofree_ph = 0;
+        const uint32_t idPV = idesc_f16(BM, kPvN, kBF16 ? 1u : 0u, 1u);
+        // shared-memory descriptors of every ring slot, built once; stepping K inside a 128-byte
+        // swizzled row adds 32 bytes (2 units) to the start address, stepping 16 key rows adds
+        // 2048 bytes (128 units).  V descriptors carry, as leading offset, the distance to the
+        // ones tile that supplies PV columns 64..79.
+        // The start-address field is linear in the slot index (a tile is 1024 units of 16 bytes);
+        // for V the leading offset to the ones tile shrinks by the same amount.
+        const uint64_t qdesc0 = smem_desc_sw128(smem_addr(base + kOffQ), 16, 1024);
+        const uint64_t kdesc0 = smem_desc_sw128(smem_addr(base + kOffK), 16, 1024);
+        const uint64_t vdesc0 = smem_desc_sw128(smem_addr(base + kOffV), kOffOnes - kOffV, 1024);
+        auto slot_desc = [](uint64_t d0, int slot) { return d0 + static_cast<uint64_t>(slot) * (kTileBytes >> 4); };
+        auto v_desc = [&](int slot) {
+            return slot_desc(vdesc0, slot) - (static_cast<uint64_t>(slot) * (kTileBytes >> 4) << 16);
+        };
         int qs = 0, ks = 0;
         int t = 0, n = 0;
         bool have_prev = false;
@@ -379,29 +410,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
 
         auto issue_pv = [&](const PvStep &u) -> bool {
-            if (!warp_wait(&bars->p_full[u.sb], p_ph[u.sb], bars, p))
+            if (!warp_wait(&bars->p_full[u.sb], (p_ph >> u.sb) & 1u, bars, p))
                 return false;
-            p_ph[u.sb] ^= 1u;
+            p_ph ^= 1u << u.sb;
             if (u.wait_free) {
                 // first PV of an item: the O buffer's previous item must have been read out
-                if (!warp_wait(&bars->o_free[u.ob], ofree_ph[u.ob], bars, p))
+                if (!warp_wait(&bars->o_free[u.ob], (ofree_ph >> u.ob) & 1u, bars, p))
                     return false;
-                ofree_ph[u.ob] ^= 1u;
+                ofree_ph ^= 1u << u.ob;
             }
             if (lane == 0) {
                 tc_fence_after();
-                const uint32_t sVa = smem_addr(base + kOffV + u.ks * kTileBytes);
-                const uint32_t dO = tmem + kColO0 + 64 * u.ob;
+                const uint64_t vd = v_desc(u.ks);
+                const uint32_t dO = tmem + kColO0 + kOCols * u.ob;
                 const uint32_t aP = tmem + kColS0 + 128 * u.sb;
+                const int nj = u.nk16 >> 4;
                 // keys 16j..16j+15 live in slice j/2: head part at column 32(j/2) + 8(j%2),
                 // remainder 16 columns further
-                for (int j = 0; j < u.nk16 / 16; ++j)
-                    mma_ts(dO, aP + 32 * (j >> 1) + 8 * (j & 1), smem_desc_sw128(sVa + j * 2048, 16, 1024), idPV,
-                           (u.kc > 0 || j > 0) ? 1u : 0u);
-                if (kBF16)
-                    for (int j = 0; j < u.nk16 / 16; ++j)
-                        mma_ts(dO, aP + 32 * (j >> 1) + 8 * (j & 1) + 16, smem_desc_sw128(sVa + j * 2048, 16, 1024),
-                               idPV, 1u);
+#pragma unroll
+                for (int j = 0; j < BN / 16; ++j)
+                    if (j < nj)
+                        mma_ts(dO, aP + 32 * (j >> 1) + 8 * (j & 1), vd + 128 * j, idPV, (u.kc > 0 || j > 0) ? 1u : 0u);
+                if (kBF16) {
+#pragma unroll
+                    for (int j = 0; j < BN / 16; ++j)
+                        if (j < nj)
+                            mma_ts(dO, aP + 32 * (j >> 1) + 8 * (j & 1) + 16, vd + 128 * j, idPV, 1u);
+                }
                 mma_commit(&bars->o_full[u.ob]);
                 mma_commit(&bars->s_free[u.sb]);
                 mma_commit(&bars->kv_empty[u.ks]);
@@ -413,19 +448,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
             const Item it = decode_item(item, H, B, tile_pre, cu_s);
             const int nkc = (it.L + BN - 1) / BN;
-            ok = warp_wait(&bars->q_full[qs], q_ph[qs], bars, p);
+            ok = warp_wait(&bars->q_full[qs], (q_ph >> qs) & 1u, bars, p);
             if (!ok)
                 break;
-            q_ph[qs] ^= 1u;
-            const uint32_t sQa = smem_addr(base + kOffQ + qs * kTileBytes);
+            q_ph ^= 1u << qs;
+            const uint64_t qd = slot_desc(qdesc0, qs);
             for (int kc = 0; kc < nkc; ++kc) {
                 const int nk = min(BN, it.L - kc * BN);
                 const int nk16 = (nk + 15) & ~15;
                 const int sb = t & 1;
-                ok = warp_wait(&bars->kv_full[ks], kv_ph[ks], bars, p);
+                ok = warp_wait(&bars->kv_full[ks], (kv_ph >> ks) & 1u, bars, p);
                 if (!ok)
                     break;
-                kv_ph[ks] ^= 1u;
+                kv_ph ^= 1u << ks;
                 uint8_t *sV = base + kOffV + ks * kTileBytes;
                 // zero V rows [nk, nk16): they enter the PV MMA with probability 0
                 if (nk < nk16) {
@@ -436,19 +471,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 // S buffer sb holds P of step t-2 until that PV completes
                 if (t >= 2) {
-                    ok = warp_wait(&bars->s_free[sb], sfree_ph[sb], bars, p);
+                    ok = warp_wait(&bars->s_free[sb], (sfree_ph >> sb) & 1u, bars, p);
                     if (!ok)
                         break;
-                    sfree_ph[sb] ^= 1u;
+                    sfree_ph ^= 1u << sb;
                 }
                 if (lane == 0) {
                     tc_fence_after();
-                    const uint32_t sKa = smem_addr(base + kOffK + ks * kTileBytes);
+                    const uint64_t kd = slot_desc(kdesc0, ks);
                     const uint32_t idS = idesc_f16(BM, nk16, kBF16 ? 1u : 0u, 0u);
 #pragma unroll
                     for (int kk = 0; kk < kD / 16; ++kk)
-                        mma_ss(tmem + kColS0 + 128 * sb, smem_desc_sw128(sQa + kk * 32, 16, 1024),
-                               smem_desc_sw128(sKa + kk * 32, 16, 1024), idS, kk > 0 ? 1u : 0u);
+                        mma_ss(tmem + kColS0 + 128 * sb, qd + 2 * kk, kd + 2 * kk, idS, kk > 0 ? 1u : 0u);
                     mma_commit(&bars->s_full[sb]);
                     if (kc == nkc - 1)
                         mma_commit(&bars->q_empty[qs]);  // last read of this Q tile
@@ -483,28 +517,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = q4 * 32 + lane;              // row of S / O owned by this thread
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
         float *red_max = red;                        // [2][2][128]
-        float *red_sum = red + 2 * 2 * 128;          // [2][2][128]
-        uint32_t s_ph[2] = {0, 0}, o_ph[2] = {0, 0};
+        uint32_t s_ph = 0, o_ph = 0;  // one bit per buffer
         int t = 0, n = 0, n_epi = 0;
         bool ok = true;
 
         // deferred epilogue of the previous item
         bool pending = false;
         int pend_row0 = 0, pend_h = 0, pend_qrows = 0, pend_ob = 0;
-        float pend_l = 0.f;
         auto epilogue = [&]() -> bool {
-            if (!warp_wait(&bars->o_full[pend_ob], o_ph[pend_ob], bars, p))
+            if (!warp_wait(&bars->o_full[pend_ob], (o_ph >> pend_ob) & 1u, bars, p))
                 return false;
-            o_ph[pend_ob] ^= 1u;
+            o_ph ^= 1u << pend_ob;
             tc_fence_after();
             if (q4 * 32 < pend_qrows) {
-                uint32_t r[32];
-                tmem_ld32(lane_base + kColO0 + 64 * pend_ob + 32 * hf, r);
-                float *rs = red_sum + (n_epi & 1) * 256;
-                rs[hf * 128 + row] = pend_l;
-                pair_sync(q4);
-                const float inv = 1.f / (rs[row] + rs[128 + row]);
+                uint32_t r[32], sum[1];
+                tmem_ld32(lane_base + kColO0 + kOCols * pend_ob + 32 * hf, r);
+                tmem_ld1(lane_base + kColO0 + kOCols * pend_ob + 64, sum);
                 tmem_wait_ld();
+                const float inv = 1.f / __uint_as_float(sum[0]);
                 if (row < pend_qrows) {
                     const int64_t off = (static_cast<int64_t>(pend_row0 + row) * H + pend_h) * kD + 32 * hf;
                     if (p.out_dt == RRA_F32) {
@@ -555,16 +585,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int qrows = min(BM, it.L - q0);
             const bool warp_active = q4 * 32 < qrows;
             const int ob = n & 1;
-            float m_run = -INFINITY, l_run = 0.f;
+            float m_run = -INFINITY;
             for (int kc = 0; kc < nkc; ++kc) {
                 const int nk = min(BN, it.L - kc * BN);
                 const int nk16 = (nk + 15) & ~15;
                 const int sb = t & 1;
                 const uint32_t sbase = lane_base + kColS0 + 128 * sb;
-                ok = warp_wait(&bars->s_full[sb], s_ph[sb], bars, p);
+                ok = warp_wait(&bars->s_full[sb], (s_ph >> sb) & 1u, bars, p);
                 if (!ok)
                     break;
-                s_ph[sb] ^= 1u;
+                s_ph ^= 1u << sb;
                 tc_fence_after();
                 const int c0 = 32 * hf, c1 = c0 + 64;
                 uint32_t r0[32], r1[32];
@@ -588,23 +618,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 // later steps of an item: the previous PV has landed in O; rescale rows whose max rose
                 if (kc > 0) {
-                    ok = warp_wait(&bars->o_full[ob], o_ph[ob], bars, p);
+                    ok = warp_wait(&bars->o_full[ob], (o_ph >> ob) & 1u, bars, p);
                     if (!ok)
                         break;
-                    o_ph[ob] ^= 1u;
+                    o_ph ^= 1u << ob;
                     tc_fence_after();
-                    if (warp_active) {
+                    if (warp_active && __any_sync(0xffffffffu, m_new > m_run)) {
+                        // each warp of the pair rescales 32 output columns; the first also the sum
                         const float alpha = ex2_approx((m_run - m_new) * p.scale_log2);
-                        l_run *= alpha;
-                        if (__any_sync(0xffffffffu, m_new > m_run)) {
-                            uint32_t r[32];
-                            const uint32_t oaddr = lane_base + kColO0 + 64 * ob + 32 * hf;
-                            tmem_ld32(oaddr, r);
-                            tmem_wait_ld();
+                        const uint32_t oaddr = lane_base + kColO0 + kOCols * ob + 32 * hf;
+                        uint32_t r[32], rs[16];
+                        tmem_ld32(oaddr, r);
+                        if (hf == 0)
+                            tmem_ld16(lane_base + kColO0 + kOCols * ob + 64, rs);
+                        tmem_wait_ld();
 #pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-                            tmem_st32(oaddr, r);
+                        for (int j = 0; j < 32; ++j)
+                            r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
+                        tmem_st32(oaddr, r);
+                        if (hf == 0) {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                rs[j] = __float_as_uint(__uint_as_float(rs[j]) * alpha);
+                            tmem_st16(lane_base + kColO0 + kOCols * ob + 64, rs);
                         }
                     }
                 }
@@ -612,9 +648,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m_run = m_new;
                     const float neg_m = -m_new * p.scale_log2;
                     if (c0 < nk16)
-                        softmax_slice<kBF16>(r0, c0, nk, p.scale_log2, neg_m, l_run, sbase + c0);
+                        softmax_slice<kBF16>(r0, c0, nk, p.scale_log2, neg_m, sbase + c0);
                     if (c1 < nk16)
-                        softmax_slice<kBF16>(r1, c1, nk, p.scale_log2, neg_m, l_run, sbase + c1);
+                        softmax_slice<kBF16>(r1, c1, nk, p.scale_log2, neg_m, sbase + c1);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -636,7 +672,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             pend_h = it.h;
             pend_qrows = qrows;
             pend_ob = ob;
-            pend_l = l_run;
             ++n;
         }
         if (ok && pending)
