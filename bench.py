@@ -3,10 +3,13 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2] [--impl ours|reference]
 
-One step = one whole call (rra_pack, rra_attend, rra_unpack for every pruning stage of the
-workload) replayed from a CUDA graph over inputs resident in HBM.  L2 is flushed (a 256 MiB
-write, untimed) before every timed step, and each step is bracketed by CUDA events on the
-launching stream; per-kernel events recorded inside the graph give the per-kernel times.
+One step = one whole pack -> attend -> unpack call for every pruning stage of the workload,
+replayed from a CUDA graph over inputs resident in HBM.  The call runs either as the single
+launch rra_pack_attend_unpack (--path fused, the default: identical bytes out) or as the three
+launches rra_pack, rra_attend, rra_unpack (--path three); the other path is timed afterwards
+and reported beside it.  L2 is flushed (a 256 MiB write, untimed) before every timed step, and
+each step is bracketed by CUDA events on the launching stream; per-kernel events recorded
+inside the graph give the per-kernel times.
 
 Prints ONE JSON line on rank 0: packed tokens/s (whole job), us per call, the roofline of the
 dominant kernel, end-to-end throughput through the public API with pinned host buffers,
@@ -42,11 +45,12 @@ METRIC = "packed tokens/s & us per pack-attend-unpack call (1 B200, graph); % ro
 UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
-KERNELS = ("pack", "attend", "unpack")
+KERNELS = {"three": ("pack", "attend", "unpack"), "fused": ("pack_attend_unpack",)}
 KERNEL_SOURCES = {
     "pack": "ragged_varlen_attention_rra_b200/csrc/pack_unpack.cu",
     "unpack": "ragged_varlen_attention_rra_b200/csrc/pack_unpack.cu",
     "attend": "ragged_varlen_attention_rra_b200/csrc/attend.cu",
+    "pack_attend_unpack": "ragged_varlen_attention_rra_b200/csrc/attend.cu",
 }
 
 
@@ -94,6 +98,8 @@ def algorithmic_bytes(w, lengths, row_bytes, out_row_bytes):
         "pack": B * N + 2 * 3 * T * row_bytes + 4 * (B + 1),
         "attend": 3 * T * row_bytes + T * out_row_bytes + 4 * (B + 1),
         "unpack": T * out_row_bytes + B * N * out_row_bytes + B * N + 4 * (B + 1),
+        # single launch: mask, the kept rows of Q/K/V, the padded output, cu_seqlens
+        "pack_attend_unpack": B * N + 3 * T * row_bytes + B * N * out_row_bytes + 4 * (B + 1),
     }
 
 
@@ -231,10 +237,11 @@ def run_reference(args):
 # ------------------------------------------------------------------------------------ GPU arm
 
 class Pipeline:
-    """Device buffers + one CUDA graph of the whole call (all stages), with timing events."""
+    """Device buffers + one CUDA graph of the whole call (all stages), with per-kernel events."""
 
-    def __init__(self, w, out_dtype, stream):
+    def __init__(self, w, out_dtype, stream, path):
         self.w = w
+        self.path = path
         dev = "cuda"
         self.masks = [m.to(dev) for m in w.masks]
         self.q, self.k, self.v = (t.to(dev) for t in (w.q, w.k, w.v))
@@ -244,28 +251,36 @@ class Pipeline:
         self.graph = None
         self.events = None
 
+    @property
+    def kernels(self):
+        return KERNELS[self.path]
+
     def enqueue(self, events=None):
         b = self.bufs
         s = self.stream
+        nk = len(self.kernels)
         for i, m in enumerate(self.masks):
             if events:
-                events[3 * i].record(s)
+                events[nk * i].record(s)
+            if self.path == "fused":
+                rra.rra_pack_attend_unpack(m, self.q, self.k, self.v, self.ys[i], b.cu, dev_error=b.err, stream=s)
+                continue
             rra.rra_pack(m, [self.q, self.k, self.v], b.packed, b.cu, dev_error=b.err, stream=s)
             if events:
-                events[3 * i + 1].record(s)
+                events[nk * i + 1].record(s)
             rra.rra_attend(b.packed[0], b.packed[1], b.packed[2], b.o, b.cu, max_seqlen=self.w.N,
                            dev_error=b.err, stream=s)
             if events:
-                events[3 * i + 2].record(s)
+                events[nk * i + 2].record(s)
             rra.rra_unpack(b.o, b.cu, m, self.ys[i], fill_mode=0, dev_error=b.err, stream=s)
         if events:
-            events[3 * len(self.masks)].record(s)
+            events[nk * len(self.masks)].record(s)
 
     def capture(self):
         with torch.cuda.stream(self.stream):
             self.enqueue()
         torch.cuda.synchronize()
-        n_ev = 3 * len(self.masks) + 1
+        n_ev = len(self.kernels) * len(self.masks) + 1
         events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
         g = torch.cuda.CUDAGraph()
         try:
@@ -279,6 +294,42 @@ class Pipeline:
             self.graph, self.events = g, None
         torch.cuda.synchronize()
 
+    def kernel_times(self):
+        """Per-launch ms of each kernel of the last replay, from the in-graph events."""
+        if self.events is None:
+            return None
+        ev, nk = self.events, len(self.kernels)
+        out = {k: [] for k in self.kernels}
+        for s in range(len(self.masks)):
+            for j, k in enumerate(self.kernels):
+                out[k].append(ev[nk * s + j].elapsed_time(ev[nk * s + j + 1]))
+        return out
+
+
+def time_path(pipe, flush, steps, warmup, stream):
+    """Warm-up, then `steps` timed replays, each after an untimed L2 flush; per-step ms and
+    per-kernel per-launch ms."""
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for i in range(warmup):
+        with torch.cuda.stream(stream):
+            flush.fill_(i & 0xFF)
+            pipe.graph.replay()
+    torch.cuda.synchronize()
+    step_ms, kern = [], {k: [] for k in pipe.kernels}
+    for i in range(steps):
+        with torch.cuda.stream(stream):
+            flush.fill_((i + 7) & 0xFF)
+            start.record(stream)
+            pipe.graph.replay()
+            end.record(stream)
+        stream.synchronize()
+        step_ms.append(start.elapsed_time(end))
+        kt = pipe.kernel_times()
+        if kt:
+            for k, v in kt.items():
+                kern[k].extend(v)
+    return step_ms, kern
+
 
 def main_gpu(args):
     ws, rank, local = dist_env()
@@ -290,47 +341,22 @@ def main_gpu(args):
     w = workloads.by_name(args.workload)
     stream = torch.cuda.Stream()
     out_dtype = torch.float32 if args.out == "f32" else None
-    pipe = Pipeline(w, out_dtype, stream)
+    pipe = Pipeline(w, out_dtype, stream, args.path)
     pipe.capture()
+    other = Pipeline(w, out_dtype, stream, "three" if args.path == "fused" else "fused")
+    other.capture()
     stages = len(w.masks)
     lengths = w.lengths
     T_call = int(sum(int(l.sum()) for l in lengths))
     row_bytes = w.H * 64 * w.q.element_size()
     out_row_bytes = w.H * 64 * pipe.bufs.o.element_size()
-
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-    def step(record_kernels):
-        with torch.cuda.stream(stream):
-            flush.fill_(step.counter & 0xFF)
-            step.counter += 1
-            start.record(stream)
-            pipe.graph.replay()
-            end.record(stream)
-    step.counter = 0
-
-    for _ in range(args.warmup):
-        step(False)
-    torch.cuda.synchronize()
     if ws > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-
-    step_ms = []
-    kern_ms = {k: [] for k in KERNELS}
     with ClockSampler(dev_index) as clk:
-        for _ in range(args.steps):
-            step(True)
-            stream.synchronize()
-            step_ms.append(start.elapsed_time(end))
-            if pipe.events is not None:
-                ev = pipe.events
-                for s in range(stages):
-                    kern_ms["pack"].append(ev[3 * s].elapsed_time(ev[3 * s + 1]))
-                    kern_ms["attend"].append(ev[3 * s + 1].elapsed_time(ev[3 * s + 2]))
-                    kern_ms["unpack"].append(ev[3 * s + 2].elapsed_time(ev[3 * s + 3] if s + 1 == stages
-                                                                        else ev[3 * (s + 1)]))
+        step_ms, kern_ms = time_path(pipe, flush, args.steps, args.warmup, stream)
     torch.cuda.synchronize()
     if ws > 1:
         torch.distributed.barrier()
@@ -338,6 +364,12 @@ def main_gpu(args):
     err = rra.rra_get_device_error(pipe.bufs.err, stream)
     if err != 0:
         raise RuntimeError(f"device error {rra.rra_status_string(err)} in the timed region")
+    # the other path, same workload, same protocol (reported beside the headline)
+    o_step_ms, o_kern_ms = time_path(other, flush, args.steps, args.warmup, stream)
+    err = rra.rra_get_device_error(other.bufs.err, stream)
+    if err != 0:
+        raise RuntimeError(f"device error {rra.rra_status_string(err)} on the {other.path} path")
+    same = all(torch.equal(a.view(torch.uint8), b.view(torch.uint8)) for a, b in zip(pipe.ys, other.ys))
 
     total_ms = float(sum(step_ms))
     if ws > 1:
@@ -350,6 +382,7 @@ def main_gpu(args):
     # dispatch floor: host time to enqueue one graph replay, and one eager call through the API
     torch.cuda.synchronize()
     n_disp = 0 if args.profile else 200
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         t0 = time.perf_counter()
         for _ in range(n_disp):
@@ -374,28 +407,34 @@ def main_gpu(args):
 
     # ---- roofline of the dominant kernel
     hbm_peak, peak_kind = peaks()
-    alg = {k: 0 for k in KERNELS}
+    alg = {}
     for l in lengths:
-        a = algorithmic_bytes(w, l, row_bytes, out_row_bytes)
-        for k in KERNELS:
-            alg[k] += a[k]
-    kern_us = {k: (1e3 * statistics.mean(v) * stages if v else None) for k, v in kern_ms.items()}  # per call
-    roofline = None
-    per_kernel = {}
-    if all(v is not None for v in kern_us.values()):
-        for k in KERNELS:
+        for k, b in algorithmic_bytes(w, l, row_bytes, out_row_bytes).items():
+            alg[k] = alg.get(k, 0) + b
+
+    def kernel_table(kms):
+        table = {}
+        for k, v in kms.items():
+            if not v:
+                return None
+            per_launch_us = 1e3 * statistics.mean(v)
             per_launch_bytes = alg[k] / stages
-            per_launch_us = kern_us[k] / stages
-            per_kernel[k] = {"us_per_launch": per_launch_us, "gbs": per_launch_bytes / (per_launch_us * 1e3),
-                             "alg_bytes_per_launch": per_launch_bytes,
-                             "frac_of_hbm": per_launch_bytes / (per_launch_us * 1e3) / hbm_peak}
-        dom = max(KERNELS, key=lambda k: kern_us[k])
+            gbs = per_launch_bytes / (per_launch_us * 1e3)
+            table[k] = {"us_per_launch": per_launch_us, "gbs": gbs, "alg_bytes_per_launch": per_launch_bytes,
+                        "frac_of_hbm": gbs / hbm_peak}
+        return table
+
+    per_kernel = kernel_table(kern_ms)
+    other_kernels = kernel_table(o_kern_ms)
+    roofline = None
+    if per_kernel:
+        dom = max(per_kernel, key=lambda k: per_kernel[k]["us_per_launch"])
         ach = per_kernel[dom]["gbs"]
         roofline = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": ach / hbm_peak, "peak_source": peak_kind,
-                    "traffic": ncu_traffic(dom, w.name)}
+                    "frac": ach / hbm_peak, "peak_source": peak_kind, "traffic": ncu_traffic(dom, w.name)}
     flops = sum(4 * 64 * w.H * int((l.astype(np.int64) ** 2).sum()) for l in lengths)
-    attn_tflops = flops / (kern_us["attend"] * 1e-6) / 1e12 if kern_us["attend"] else None
+    attn_key = "pack_attend_unpack" if args.path == "fused" else "attend"
+    attn_tflops = (flops / (per_kernel[attn_key]["us_per_launch"] * stages * 1e-6) / 1e12) if per_kernel else None
 
     # ---- end to end through the public API: pinned host inputs in, padded result out
     e2e = None
@@ -415,7 +454,7 @@ def main_gpu(args):
                 for d, h in zip(dmasks, host_masks):
                     d.copy_(h, non_blocking=True)
                 for i, m in enumerate(dmasks):
-                    y = rra.forward(m, dq, dk, dv, bufs, stream=stream)
+                    y = rra.forward(m, dq, dk, dv, bufs, stream=stream, fused=args.path == "fused")
                     host_out[i].copy_(y, non_blocking=True)
         for _ in range(max(3, args.warmup)):
             e2e_step()
@@ -438,7 +477,8 @@ def main_gpu(args):
         h2d = 3 * w.q.numel() * w.q.element_size() + sum(m.numel() for m in w.masks)
         d2h = sum(t.numel() * t.element_size() for t in host_out)
         e2e = {"value": ws * args.steps * T_call / (tot * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": tot / args.steps, "api": "rra.forward (eager)"}
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": tot / args.steps,
+               "api": f"rra.forward (eager, {args.path} path)"}
         if err == 0:
             err2 = rra.rra_get_device_error(bufs.err, stream)
             if err2 != 0:
@@ -455,7 +495,7 @@ def main_gpu(args):
             "vs_baseline": None, "dtype": {torch.bfloat16: "bf16", torch.float16: "f16"}[w.q.dtype],
             "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d": 64, "stages": stages,
-                       "tokens_per_call": T_call, "seed": w.seed, "recipe": w.recipe,
+                       "tokens_per_call": T_call, "seed": w.seed, "recipe": w.recipe, "path": args.path,
                        "out_dtype": str(pipe.bufs.o.dtype).replace("torch.", ""),
                        "l2": "flushed before every timed step (256 MiB write, untimed)",
                        "parallelism": f"replicas x{ws}"},
@@ -463,15 +503,18 @@ def main_gpu(args):
             "us_per_call_warm_back_to_back": warm_us,
             "host_dispatch_us": {"graph_replay": host_graph_us, "eager_three_calls": host_eager_us},
             "kernels": per_kernel,
+            "other_path": {"path": other.path, "us_per_call": 1e3 * statistics.mean(o_step_ms),
+                           "tokens_per_s": T_call / (1e-3 * statistics.mean(o_step_ms)), "kernels": other_kernels,
+                           "identical_output": bool(same)},
             "attention_tflops": attn_tflops,
             "roofline": roofline,
             "e2e": e2e,
             "cpu_baseline": cpu,
             "clocks": clk.summary(),
-            "gpu_launches": args.steps * 3 * stages,
+            "gpu_launches": args.steps * len(pipe.kernels) * stages,
         }
         print(json.dumps(line), flush=True)
-    del pipe
+    del pipe, other
     if ws > 1:
         torch.distributed.destroy_process_group()
     return 0
@@ -485,6 +528,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c2", help="c1 | c2 | c3:B | c4 | c5:r:B | c5s:B")
     ap.add_argument("--out", choices=["native", "f32"], default="native")
+    ap.add_argument("--path", choices=["fused", "three"], default="fused",
+                    help="single launch (default) or the three calls pack, attend, unpack")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="timed steps only (no dispatch loops, e2e or CPU leg): the command ncu captures")

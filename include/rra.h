@@ -139,6 +139,29 @@ rra_status rra_unpack(const void *packed, const int32_t *cu_seqlens, const uint8
                       void *dst, int32_t *dev_error, rra_stream_t stream);
 
 /*
+ * rra_pack_attend_unpack -- the whole pack -> attend -> unpack call of one pruning stage in a
+ * single launch (sota2.com card, Abstract: the pack-attend-unpack pipeline; aissential.tech
+ * summary, Method: the "fused token packer" feeding the attention kernel).
+ *
+ * Same result as rra_pack (Q, K, V) + rra_attend + rra_unpack (fill_mode 0) with
+ * softmax_scale, byte for byte in y and cu_seqlens, but the kept rows are gathered from the
+ * padded tensors straight into the attention tiles and each output row is written straight to
+ * its padded position, so no packed buffers exist.
+ *
+ *   keep_mask   device uint8 [B, N], nonzero = keep
+ *   q, k, v     device [B, N, H, d] in in_dt (RRA_F16 or RRA_BF16), d must be 64
+ *   y           device [B, N, H, d] in out_dt (in_dt or RRA_F32): kept rows receive the attention
+ *               output, pruned rows are set to zero bytes
+ *   cu_seqlens  device int32 [B+1] written with the running kept counts, or NULL
+ *   B, N, H, d  B <= 8192, N <= 4096
+ *   softmax_scale <= 0 selects 1/sqrt(d)
+ *   dev_error   device int32 or NULL (only RRA_ERR_TIMEOUT can be raised)
+ */
+rra_status rra_pack_attend_unpack(const uint8_t *keep_mask, const void *q, const void *k, const void *v, void *y,
+                                  int32_t *cu_seqlens, int B, int N, int H, int d, float softmax_scale,
+                                  rra_dtype in_dt, rra_dtype out_dt, int32_t *dev_error, rra_stream_t stream);
+
+/*
  * rra_get_device_error -- copy the device error word to *host_out.  This SYNCHRONISES `stream`
  * (it is the only call that does) and so must not be used inside stream capture.
  */

@@ -122,6 +122,44 @@ rra_status rra_attend(const void *q, const void *k, const void *v, void *o, cons
     return e == cudaSuccess ? RRA_OK : RRA_ERR_CUDA;
 }
 
+rra_status rra_pack_attend_unpack(const uint8_t *keep_mask, const void *q, const void *k, const void *v, void *y,
+                                  int32_t *cu_seqlens, int B, int N, int H, int d, float softmax_scale,
+                                  rra_dtype in_dt, rra_dtype out_dt, int32_t *dev_error, rra_stream_t stream)
+{
+    if (keep_mask == nullptr || q == nullptr || k == nullptr || v == nullptr || y == nullptr)
+        return RRA_ERR_INVALID_ARG;
+    if (B < 0 || N < 1 || H < 1)
+        return RRA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(y))
+        return RRA_ERR_INVALID_ARG;
+    if (d != 64 || (in_dt != RRA_F16 && in_dt != RRA_BF16) || (out_dt != in_dt && out_dt != RRA_F32))
+        return RRA_ERR_UNSUPPORTED;
+    if (B > rra::kAttendMaxBatch || N > rra::kFusedMaxN || H > 65535 || static_cast<int64_t>(B) * N > kMaxRows)
+        return RRA_ERR_UNSUPPORTED;
+    if (!(softmax_scale == softmax_scale))
+        return RRA_ERR_INVALID_ARG;
+    int sms = 0;
+    if (num_sms_of_current_device(&sms) != 0)
+        return RRA_ERR_CUDA;
+    rra::FusedArgs a;
+    a.mask = keep_mask;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.y = y;
+    a.cu_out = cu_seqlens;
+    a.B = B;
+    a.N = N;
+    a.H = H;
+    a.scale = softmax_scale > 0.f ? softmax_scale : 0.125f;  // 1/sqrt(64)
+    a.in_bf16 = in_dt == RRA_BF16;
+    a.out_dt = static_cast<int>(out_dt);
+    a.err = dev_error;
+    a.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+    const cudaError_t e = rra::launch_fused(a, sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RRA_OK : RRA_ERR_CUDA;
+}
+
 size_t rra_attend_workspace_size(int B, int H, int max_seqlen)
 {
     (void)B;

@@ -34,6 +34,14 @@
 //     rows) never reach the output;
 //   * every wait is bounded in time; on expiry the block records RRA_ERR_TIMEOUT, raises a
 //     block-wide abort flag, drains the copies and MMAs it issued, frees TMEM and leaves.
+//
+// The same kernel body, instantiated with kFused, runs the whole pack -> attend -> unpack call
+// in one launch (the pages' pipeline without its two copies through HBM): the block derives
+// the kept counts of every image from the keep mask itself, the producer gathers the kept rows
+// of the padded Q/K/V straight into the swizzled tiles with TMA tile::gather4 (four rows per
+// instruction, one instruction per lane of the producer warp), zero-fills the pruned rows of
+// the padded output for its (image, head), and the epilogue writes each output row back to
+// its padded position.
 #include <cuda.h>
 
 #include <mutex>
@@ -69,13 +77,16 @@ constexpr uint32_t kOffV = kOffK + kKVStages * kTileBytes;
 constexpr uint32_t kOffOnes = kOffV + kKVStages * kTileBytes;   // [128 keys x 64] MN-major, column 0 = 1
 constexpr uint32_t kOffBar = kOffOnes + kTileBytes;
 constexpr uint32_t kOffRed = kOffBar + 512;             // [2 parities][2 halves][128] row max
-constexpr uint32_t kOffTile = kOffRed + 2 * 2 * 128 * 4;  // tile_pre[B+1], then cu[B+1]
+constexpr uint32_t kOffIdx = kOffRed + 2 * 2 * 128 * 4;  // fused: kept-row list of one image (int16)
+constexpr uint32_t kOffTile = kOffIdx + kFusedMaxN * 2;   // tile_pre[B+1], then cu[B+1]
 constexpr int kSmemFixed = 1024 /*align slack*/ + kOffTile;
 
 struct Params {
-    const int32_t *cu;
+    const int32_t *cu;      // packed path: cu_seqlens in
+    const uint8_t *mask;    // fused path: keep mask [B, N]
+    int32_t *cu_out;        // fused path: cu_seqlens out (may be null)
     void *out;
-    int B, H;
+    int B, H, N;
     int64_t capacity;
     float scale_log2;
     int out_dt;
@@ -93,7 +104,7 @@ struct Bars {
     uint64_t drain;
     uint32_t tmem_slot;
     int abort;
-    int warp_sums[kThreads / 32];
+    int warp_sums[2][kThreads / 32];
 };
 static_assert(sizeof(Bars) <= 512, "barrier block overflows its slot");
 
@@ -107,6 +118,28 @@ __device__ __forceinline__ uint32_t pack_f16(float a, float b)
 {
     const __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Bit k of the result is set iff byte k of the 16-byte chunk is nonzero.
+__device__ __forceinline__ uint32_t kept_bits16_(uint4 c)
+{
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t t = (((w[i] & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w[i]) & 0x80808080u;
+        m |= (((t >> 7) & 1u) | ((t >> 14) & 2u) | ((t >> 21) & 4u) | ((t >> 28) & 8u)) << (4 * i);
+    }
+    return m;
+}
+
+// Bits k (0..15) with lo <= s + k < hi.
+__device__ __forceinline__ uint32_t range16_(int64_t s, int64_t lo, int64_t hi)
+{
+    const int64_t a = lo - s, b = hi - s;
+    const int l = a < 0 ? 0 : (a > 16 ? 16 : static_cast<int>(a));
+    const int h = b < 0 ? 0 : (b > 16 ? 16 : static_cast<int>(b));
+    return h > l ? (((1u << h) - 1u) & ~((1u << l) - 1u)) : 0u;
 }
 
 // One decoded work item.
@@ -229,7 +262,32 @@ struct PvStep {
     bool wait_free;  // first PV of an item whose O buffer held an earlier item
 };
 
-template <bool kBF16>
+// 2-D gather of four rows (row coordinates r0..r3) of 64 elements starting at column x.
+__device__ __forceinline__ void tma_gather4(void *smem_dst, const void *tmap, uint64_t *bar, int x, int r0, int r1,
+                                            int r2, int r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_addr(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_addr(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
+
+// Fused path: the producer lane gathers rows list[base + 4*lane .. +3] of one 128-row tile
+// (entries at or past `count` repeat the tile's first row, whose result is masked later).
+__device__ __forceinline__ void gather_tile(void *tile, const void *tmap, uint64_t *bar, const int16_t *list, int base,
+                                            int count, int row_off, int x, int lane)
+{
+    int r[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int i = 4 * lane + k;
+        r[k] = row_off + list[base + (i < count ? i : 0)];
+    }
+    tma_gather4(static_cast<uint8_t *>(tile) + 512 * lane, tmap, bar, x, r[0], r[1], r[2], r[3]);
+}
+
+template <bool kBF16, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const Params p)
@@ -240,6 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *red = reinterpret_cast<float *>(base + kOffRed);            // row max exchange [2][2][128]
     int32_t *tile_pre = reinterpret_cast<int32_t *>(base + kOffTile);  // [B+1]
     int32_t *cu_s = tile_pre + (p.B + 1);                               // [B+1]
+    int16_t *idx = reinterpret_cast<int16_t *>(base + kOffIdx);         // fused: kept rows of one image
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -288,45 +347,100 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---- work list: tile_pre[b] = number of 128-row query tiles of images < b; cu staged too.
-    if (tid == 0)
-        tile_pre[0] = 0;
-    int carry = 0;
-    for (int c0 = 0; c0 < B; c0 += kThreads) {
-        const int b = c0 + tid;
-        int tiles = 0;
-        if (b < B) {
-            const int64_t s0 = p.cu[b], s1 = p.cu[b + 1];
-            cu_s[b] = static_cast<int32_t>(s0);
-            if (b == B - 1)
-                cu_s[B] = static_cast<int32_t>(s1);
-            if (s0 < 0 || s1 < s0 || s1 > p.capacity) {
-                if (blockIdx.x == 0)
-                    raise_error(p.err, RRA_ERR_BAD_SEQLENS);
-            } else {
-                tiles = static_cast<int>((s1 - s0 + BM - 1) / BM);
+    if constexpr (kFused) {
+        // kept tokens per image, counted from 16-byte chunks of the flat mask into cu_s[b+1]
+        for (int b = tid; b <= B; b += kThreads)
+            cu_s[b] = 0;
+        __syncthreads();
+        const int64_t total = static_cast<int64_t>(B) * p.N;
+        const uintptr_t addr = reinterpret_cast<uintptr_t>(p.mask);
+        const int off = static_cast<int>(addr & 15u);
+        const uint4 *m16 = reinterpret_cast<const uint4 *>(addr - off);
+        const int64_t nchunks = (off + total + 15) >> 4;
+        for (int64_t j = tid; j < nchunks; j += kThreads) {
+            const int64_t s0 = j * 16 - off;  // byte index of the chunk's first byte
+            uint32_t bits = kept_bits16_(__ldg(m16 + j)) & range16_(s0, 0, total);
+            while (bits != 0u) {
+                const int64_t first = s0 + (__ffs(bits) - 1);
+                const int b = static_cast<int>(first / p.N);
+                const uint32_t in_b = bits & range16_(s0, static_cast<int64_t>(b) * p.N, static_cast<int64_t>(b + 1) * p.N);
+                atomicAdd(&cu_s[b + 1], __popc(in_b));
+                bits &= ~in_b;
             }
         }
-        int incl = tiles;
+        __syncthreads();
+    }
+    if (tid == 0)
+        tile_pre[0] = 0;
+    int carry_t = 0, carry_l = 0;
+    for (int c0 = 0; c0 < B; c0 += kThreads) {
+        const int b = c0 + tid;
+        int tiles = 0, len = 0;
+        if (b < B) {
+            if constexpr (kFused) {
+                len = cu_s[b + 1];
+                tiles = (len + BM - 1) / BM;
+            } else {
+                const int64_t s0 = p.cu[b], s1 = p.cu[b + 1];
+                cu_s[b] = static_cast<int32_t>(s0);
+                if (b == B - 1)
+                    cu_s[B] = static_cast<int32_t>(s1);
+                if (s0 < 0 || s1 < s0 || s1 > p.capacity) {
+                    if (blockIdx.x == 0)
+                        raise_error(p.err, RRA_ERR_BAD_SEQLENS);
+                } else {
+                    tiles = static_cast<int>((s1 - s0 + BM - 1) / BM);
+                }
+            }
+        }
+        int it_incl = tiles, l_incl = len;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off)
-                incl += t;
+            const int a = __shfl_up_sync(0xffffffffu, it_incl, off);
+            const int c = __shfl_up_sync(0xffffffffu, l_incl, off);
+            if (lane >= off) {
+                it_incl += a;
+                l_incl += c;
+            }
         }
-        if (lane == 31)
-            bars->warp_sums[warp] = incl;
+        if (lane == 31) {
+            bars->warp_sums[0][warp] = it_incl;
+            bars->warp_sums[1][warp] = l_incl;
+        }
         __syncthreads();
-        int before = carry;
-        int chunk = 0;
+        int before_t = carry_t, before_l = carry_l, chunk_t = 0, chunk_l = 0;
 #pragma unroll
         for (int w = 0; w < kThreads / 32; ++w) {
-            before += (w < warp) ? bars->warp_sums[w] : 0;
-            chunk += bars->warp_sums[w];
+            before_t += (w < warp) ? bars->warp_sums[0][w] : 0;
+            before_l += (w < warp) ? bars->warp_sums[1][w] : 0;
+            chunk_t += bars->warp_sums[0][w];
+            chunk_l += bars->warp_sums[1][w];
         }
-        if (b < B)
-            tile_pre[b + 1] = before + incl;
-        carry += chunk;
+        if (b < B) {
+            tile_pre[b + 1] = before_t + it_incl;
+            if constexpr (kFused)
+                cu_s[b + 1] = before_l + l_incl;  // (reads of the count above happened before the barrier)
+        }
+        carry_t += chunk_t;
+        carry_l += chunk_l;
         __syncthreads();
+    }
+    if constexpr (kFused) {
+        if (tid == 0)
+            cu_s[0] = 0;
+        __syncthreads();
+        if (blockIdx.x == 0 && p.cu_out != nullptr)
+            for (int b = tid; b <= B; b += kThreads)
+                p.cu_out[b] = cu_s[b];
+        // images without kept tokens have no work item: their padded output rows are zeroed here
+        const int out_vecs = (p.out_dt == RRA_F32 ? 4 * kD : 2 * kD) / 16;  // 16-byte vectors per head row
+        for (int b = blockIdx.x; b < B; b += gridDim.x) {
+            if (cu_s[b + 1] != cu_s[b])
+                continue;
+            uint4 *y = reinterpret_cast<uint4 *>(p.out) + static_cast<int64_t>(b) * p.N * H * out_vecs;
+            for (int64_t i = tid; i < static_cast<int64_t>(p.N) * H * out_vecs; i += kThreads)
+                y[i] = make_uint4(0, 0, 0, 0);
+        }
     }
 
     tc_fence_before();
@@ -341,19 +455,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         // phase 0 counts as complete, so waiting on parity (phase ^ 1) passes at once for the
         // first fill of each slot, then tracks the consumer's releases.
         uint32_t q_phase = 0, kv_phase = 0;  // one bit per slot
+        int cur_b = -1;                      // fused: image whose kept-row list is in idx[]
         uint32_t q_issued = 0, kv_issued = 0;
         int qs = 0, ks = 0;
         bool ok = true;
         for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
             const Item it = decode_item(item, H, B, tile_pre, cu_s);
             const int nkc = (it.L + BN - 1) / BN;
+            const int row_off = it.b * p.N;  // fused: first padded row of this image
+            if constexpr (kFused) {
+                if (it.b != cur_b) {
+                    // kept positions of this image, in order (warp ballot scan of its mask row)
+                    int running = 0;
+                    for (int c0 = 0; c0 < p.N; c0 += 32) {
+                        const int n = c0 + lane;
+                        const bool keep = n < p.N && p.mask[row_off + n] != 0;
+                        const unsigned bal = __ballot_sync(0xffffffffu, keep);
+                        if (keep)
+                            idx[running + __popc(bal & ((1u << lane) - 1u))] = static_cast<int16_t>(n);
+                        running += __popc(bal);
+                    }
+                    __syncwarp();
+                    cur_b = it.b;
+                }
+                if (it.qt == 0) {
+                    // pruned rows of this (image, head) in the padded output become zero
+                    const int out_vecs = (p.out_dt == RRA_F32 ? 4 * kD : 2 * kD) / 16;
+                    for (int n = lane; n < p.N; n += 32) {
+                        if (p.mask[row_off + n] != 0)
+                            continue;
+                        uint4 *y = reinterpret_cast<uint4 *>(p.out) +
+                                   (static_cast<int64_t>(row_off + n) * H + it.h) * out_vecs;
+                        for (int v2 = 0; v2 < out_vecs; ++v2)
+                            y[v2] = make_uint4(0, 0, 0, 0);
+                    }
+                }
+            }
             ok = warp_wait(&bars->q_empty[qs], ((q_phase >> qs) & 1u) ^ 1u, bars, p);
             if (!ok)
                 break;
             q_phase ^= 1u << qs;
-            if (lane == 0) {
+            if (lane == 0)
                 mbar_arrive_expect_tx(&bars->q_full[qs], kTileBytes);
-                tma_load_3d(base + kOffQ + qs * kTileBytes, &tm_q, &bars->q_full[qs], 0, it.h, it.seq0 + it.qt * BM);
+            __syncwarp();
+            if constexpr (kFused) {
+                gather_tile(base + kOffQ + qs * kTileBytes, &tm_q, &bars->q_full[qs], idx, it.qt * BM,
+                            min(BM, it.L - it.qt * BM), row_off, it.h * kD, lane);
+            } else {
+                if (lane == 0)
+                    tma_load_3d(base + kOffQ + qs * kTileBytes, &tm_q, &bars->q_full[qs], 0, it.h, it.seq0 + it.qt * BM);
             }
             __syncwarp();
             ++q_issued;
@@ -363,10 +513,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok)
                     break;
                 kv_phase ^= 1u << ks;
-                if (lane == 0) {
+                if (lane == 0)
                     mbar_arrive_expect_tx(&bars->kv_full[ks], 2 * kTileBytes);
-                    tma_load_3d(base + kOffK + ks * kTileBytes, &tm_k, &bars->kv_full[ks], 0, it.h, it.seq0 + kc * BN);
-                    tma_load_3d(base + kOffV + ks * kTileBytes, &tm_v, &bars->kv_full[ks], 0, it.h, it.seq0 + kc * BN);
+                __syncwarp();
+                if constexpr (kFused) {
+                    const int cnt = min(BN, it.L - kc * BN);
+                    gather_tile(base + kOffK + ks * kTileBytes, &tm_k, &bars->kv_full[ks], idx, kc * BN, cnt, row_off,
+                                it.h * kD, lane);
+                    gather_tile(base + kOffV + ks * kTileBytes, &tm_v, &bars->kv_full[ks], idx, kc * BN, cnt, row_off,
+                                it.h * kD, lane);
+                } else {
+                    if (lane == 0) {
+                        tma_load_3d(base + kOffK + ks * kTileBytes, &tm_k, &bars->kv_full[ks], 0, it.h, it.seq0 + kc * BN);
+                        tma_load_3d(base + kOffV + ks * kTileBytes, &tm_v, &bars->kv_full[ks], 0, it.h, it.seq0 + kc * BN);
+                    }
                 }
                 __syncwarp();
                 ++kv_issued;
@@ -523,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // deferred epilogue of the previous item
         bool pending = false;
-        int pend_row0 = 0, pend_h = 0, pend_qrows = 0, pend_ob = 0;
+        int pend_row0 = 0, pend_h = 0, pend_qrows = 0, pend_ob = 0, pend_b = 0, pend_q0 = 0;
         auto epilogue = [&]() -> bool {
             if (!warp_wait(&bars->o_full[pend_ob], (o_ph >> pend_ob) & 1u, bars, p))
                 return false;
@@ -533,10 +693,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t r[32], sum[1];
                 tmem_ld32(lane_base + kColO0 + kOCols * pend_ob + 32 * hf, r);
                 tmem_ld1(lane_base + kColO0 + kOCols * pend_ob + 64, sum);
+                int64_t out_row = static_cast<int64_t>(pend_row0) + row;
+                if constexpr (kFused) {
+                    // padded position of kept token (q0 + row) of image b: warp select over its mask row
+                    const int target = pend_q0 + row;
+                    const int last = pend_q0 + q4 * 32 + 31;
+                    const uint8_t *mrow = p.mask + static_cast<int64_t>(pend_b) * p.N;
+                    int pos = 0, running = 0;
+                    for (int c0 = 0; c0 < p.N && running <= last; c0 += 32) {
+                        const bool keep = c0 + lane < p.N && mrow[c0 + lane] != 0;
+                        const unsigned bal = __ballot_sync(0xffffffffu, keep);
+                        const int cnt = __popc(bal);
+                        if (target >= running && target < running + cnt)
+                            pos = c0 + static_cast<int>(__fns(bal, 0, target - running + 1));
+                        running += cnt;
+                    }
+                    out_row = static_cast<int64_t>(pend_b) * p.N + pos;
+                }
                 tmem_wait_ld();
                 const float inv = 1.f / __uint_as_float(sum[0]);
                 if (row < pend_qrows) {
-                    const int64_t off = (static_cast<int64_t>(pend_row0 + row) * H + pend_h) * kD + 32 * hf;
+                    const int64_t off = (out_row * H + pend_h) * kD + 32 * hf;
                     if (p.out_dt == RRA_F32) {
                         float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
 #pragma unroll
@@ -669,6 +846,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             pending = true;
             pend_row0 = it.seq0 + q0;
+            pend_b = it.b;
+            pend_q0 = q0;
             pend_h = it.h;
             pend_qrows = qrows;
             pend_ob = ob;
@@ -724,7 +903,25 @@ bool make_tmap(CUtensorMap *map, const void *ptr, int64_t capacity, int H, bool 
     return r == CUDA_SUCCESS;
 }
 
-template <bool kBF16>
+// Padded [rows, H*64] 16-bit tensor seen as 2-D (element, token row) for tile::gather4: the box
+// is one row high and 64 elements (one head) wide.
+bool make_gather_tmap(CUtensorMap *map, const void *ptr, int64_t rows, int H, bool bf16)
+{
+    EncodeTiledFn enc = get_encode_fn();
+    if (enc == nullptr)
+        return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H) * kD, static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * kD * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kD), 1u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                           const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <bool kBF16, bool kFused>
 cudaError_t set_smem_attr(int bytes)
 {
     static std::mutex mu;
@@ -736,10 +933,33 @@ cudaError_t set_smem_attr(int bytes)
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 64 && done_bytes[dev] >= bytes)
         return cudaSuccess;
-    e = cudaFuncSetAttribute(attend_kernel<kBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    e = cudaFuncSetAttribute(attend_kernel<kBF16, kFused>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e == cudaSuccess && dev < 64)
         done_bytes[dev] = bytes;
     return e;
+}
+
+template <bool kFused>
+cudaError_t launch_variant(bool bf16, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                           const Params &p, int64_t grid, int smem, cudaStream_t stream)
+{
+    cudaError_t e = bf16 ? set_smem_attr<true, kFused>(smem) : set_smem_attr<false, kFused>(smem);
+    if (e != cudaSuccess)
+        return e;
+    if (bf16)
+        attend_kernel<true, kFused><<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(tq, tk, tv, p);
+    else
+        attend_kernel<false, kFused><<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+int64_t grid_for(int B, int H, int max_seqlen, int num_sms)
+{
+    const int64_t max_tiles = (static_cast<int64_t>(max_seqlen > 0 ? max_seqlen : 1) + BM - 1) / BM;
+    int64_t grid = static_cast<int64_t>(B) * H * max_tiles;
+    if (grid > num_sms)
+        grid = num_sms;  // one block per SM: it owns all 512 TMEM columns
+    return grid < 1 ? 1 : grid;
 }
 
 }  // namespace
@@ -752,7 +972,7 @@ cudaError_t launch_attend(const AttendArgs &a, int num_sms, cudaStream_t stream)
     if (!make_tmap(&tq, a.q, a.capacity, a.H, a.in_bf16) || !make_tmap(&tk, a.k, a.capacity, a.H, a.in_bf16) ||
         !make_tmap(&tv, a.v, a.capacity, a.H, a.in_bf16))
         return cudaErrorInvalidValue;
-    Params p;
+    Params p{};
     p.cu = a.cu;
     p.out = a.o;
     p.B = a.B;
@@ -762,22 +982,36 @@ cudaError_t launch_attend(const AttendArgs &a, int num_sms, cudaStream_t stream)
     p.out_dt = a.out_dt;
     p.err = a.err;
     p.wait_ns = a.wait_ns;
-
     const int smem = kSmemFixed + 2 * (a.B + 1) * 4;
-    const int64_t max_tiles = (static_cast<int64_t>(a.max_seqlen > 0 ? a.max_seqlen : 1) + BM - 1) / BM;
-    int64_t grid = static_cast<int64_t>(a.B) * a.H * max_tiles;
-    if (grid > num_sms)
-        grid = num_sms;  // one block per SM: it owns all 512 TMEM columns
-    if (grid < 1)
-        grid = 1;
-    cudaError_t e = a.in_bf16 ? set_smem_attr<true>(smem) : set_smem_attr<false>(smem);
-    if (e != cudaSuccess)
-        return e;
-    if (a.in_bf16)
-        attend_kernel<true><<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(tq, tk, tv, p);
-    else
-        attend_kernel<false><<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(tq, tk, tv, p);
-    return cudaGetLastError();
+    return launch_variant<false>(a.in_bf16, tq, tk, tv, p, grid_for(a.B, a.H, a.max_seqlen, num_sms), smem, stream);
+}
+
+cudaError_t launch_fused(const FusedArgs &a, int num_sms, cudaStream_t stream)
+{
+    if (a.B == 0) {
+        if (a.cu_out != nullptr)
+            return cudaMemsetAsync(a.cu_out, 0, sizeof(int32_t), stream);
+        return cudaSuccess;
+    }
+    const int64_t rows = static_cast<int64_t>(a.B) * a.N;
+    alignas(64) CUtensorMap tq, tk, tv;
+    if (!make_gather_tmap(&tq, a.q, rows, a.H, a.in_bf16) || !make_gather_tmap(&tk, a.k, rows, a.H, a.in_bf16) ||
+        !make_gather_tmap(&tv, a.v, rows, a.H, a.in_bf16))
+        return cudaErrorInvalidValue;
+    Params p{};
+    p.mask = a.mask;
+    p.cu_out = a.cu_out;
+    p.out = a.y;
+    p.B = a.B;
+    p.H = a.H;
+    p.N = a.N;
+    p.capacity = rows;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.out_dt = a.out_dt;
+    p.err = a.err;
+    p.wait_ns = a.wait_ns;
+    const int smem = kSmemFixed + 2 * (a.B + 1) * 4;
+    return launch_variant<true>(a.in_bf16, tq, tk, tv, p, grid_for(a.B, a.H, a.N, num_sms), smem, stream);
 }
 
 }  // namespace rra

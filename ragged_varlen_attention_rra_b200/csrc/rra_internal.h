@@ -34,4 +34,22 @@ constexpr int kAttendMaxBatch = 8192;
 
 cudaError_t launch_attend(const AttendArgs &a, int num_sms, cudaStream_t stream);
 
+struct FusedArgs {
+    const uint8_t *mask;
+    const void *q, *k, *v;
+    void *y;
+    int32_t *cu_out;
+    int B, N, H;
+    float scale;
+    bool in_bf16;
+    int out_dt;
+    int32_t *err;
+    uint64_t wait_ns;
+};
+
+// Largest N the single-launch path accepts (its kept-row list lives in shared memory).
+constexpr int kFusedMaxN = 4096;
+
+cudaError_t launch_fused(const FusedArgs &a, int num_sms, cudaStream_t stream);
+
 }  // namespace rra

@@ -5,9 +5,9 @@ supplies device memory and the current stream.  If librra.so is missing or canno
 every function here raises -- there is no fallback.
 
 Names follow the C ABI: :func:`rra_pack`, :func:`rra_attend`, :func:`rra_unpack`,
-:func:`rra_get_device_error`, :func:`rra_status_string`, :func:`rra_attend_workspace_size`,
-:func:`rra_set_wait_timeout_ns`.  :func:`forward` chains the three calls (the whole
-pack-attend-unpack call of one pruning stage).
+:func:`rra_pack_attend_unpack`, :func:`rra_get_device_error`, :func:`rra_status_string`,
+:func:`rra_attend_workspace_size`, :func:`rra_set_wait_timeout_ns`.  :func:`forward` runs the
+whole pack-attend-unpack call of one pruning stage, as three calls or as the single launch.
 """
 from __future__ import annotations
 
@@ -51,6 +51,9 @@ def _declare(lib):
     lib.rra_unpack.argtypes = [vp, i32p, vp, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int,
                                c.c_int64, vp, i32p, vp]
     lib.rra_unpack.restype = c.c_int
+    lib.rra_pack_attend_unpack.argtypes = [vp, vp, vp, vp, vp, i32p, c.c_int, c.c_int, c.c_int, c.c_int,
+                                           c.c_float, c.c_int, c.c_int, i32p, vp]
+    lib.rra_pack_attend_unpack.restype = c.c_int
     lib.rra_get_device_error.argtypes = [i32p, vp, c.POINTER(c.c_int32)]
     lib.rra_get_device_error.restype = c.c_int
     lib.rra_status_string.argtypes = [c.c_int]
@@ -162,6 +165,19 @@ def rra_unpack(packed: torch.Tensor, cu_seqlens: torch.Tensor, mask: torch.Tenso
     _check(st, "rra_unpack")
 
 
+def rra_pack_attend_unpack(mask: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, y: torch.Tensor,
+                           cu_seqlens: Optional[torch.Tensor] = None, softmax_scale: float = 0.0,
+                           dev_error: Optional[torch.Tensor] = None, stream=None) -> None:
+    """The whole call in one launch: padded q/k/v [B, N, H, 64] + mask [B, N] -> padded y (pruned rows zero)."""
+    _require_cuda(mask, q, k, v, y, cu_seqlens, dev_error)
+    B, N = mask.shape
+    H, d = q.shape[2], q.shape[3]
+    st = lib().rra_pack_attend_unpack(_ptr(mask), _ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(cu_seqlens), B, N, H, d,
+                                      float(softmax_scale), _DT[q.dtype], _DT[y.dtype], _ptr(dev_error),
+                                      _stream(stream))
+    _check(st, "rra_pack_attend_unpack")
+
+
 # ------------------------------------------------------------------------------------ whole call
 
 class Buffers:
@@ -180,11 +196,16 @@ class Buffers:
 
 
 def forward(mask: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bufs: Buffers,
-            softmax_scale: float = 0.0, stream=None) -> torch.Tensor:
+            softmax_scale: float = 0.0, stream=None, fused: bool = False) -> torch.Tensor:
     """One pruning stage: pack the kept tokens of q/k/v, attend per image and head, unpack to padded.
 
-    All three calls are enqueued on `stream` without any host synchronisation; the padded
-    result is bufs.y (pruned rows zero)."""
+    Enqueued on `stream` without any host synchronisation; the padded result is bufs.y (pruned
+    rows zero).  fused=True runs the same call as the single launch rra_pack_attend_unpack
+    (bufs.cu is written, the packed buffers are not used)."""
+    if fused:
+        rra_pack_attend_unpack(mask, q, k, v, bufs.y, bufs.cu, softmax_scale=softmax_scale, dev_error=bufs.err,
+                               stream=stream)
+        return bufs.y
     rra_pack(mask, [q, k, v], bufs.packed, bufs.cu, dev_error=bufs.err, stream=stream)
     rra_attend(bufs.packed[0], bufs.packed[1], bufs.packed[2], bufs.o, bufs.cu, max_seqlen=mask.shape[1],
                softmax_scale=softmax_scale, dev_error=bufs.err, stream=stream)

@@ -29,7 +29,7 @@ def declared_functions():
 
 def test_header_declares_the_path():
     names = declared_functions()
-    for required in ("rra_pack", "rra_attend", "rra_unpack", "rra_attend_workspace_size",
+    for required in ("rra_pack", "rra_attend", "rra_unpack", "rra_pack_attend_unpack", "rra_attend_workspace_size",
                      "rra_get_device_error", "rra_status_string"):
         assert required in names
 
@@ -101,6 +101,16 @@ def test_unpack_validation(L):
     assert f(FAKE, FAKE, FAKE, 2, 8, 1, 64, 1, 2, 16, FAKE, None, None) == rra.RRA_ERR_INVALID_ARG  # fill_mode
     assert f(FAKE, FAKE, FAKE, 2, 8, 1, 64, 9, 0, 16, FAKE, None, None) == rra.RRA_ERR_UNSUPPORTED
     assert f(FAKE, FAKE, FAKE, 2, 8, 1, 64, 1, 0, 16, FAKE + 2, None, None) == rra.RRA_ERR_INVALID_ARG
+
+
+def test_fused_validation(L):
+    f = L.rra_pack_attend_unpack
+    assert f(None, FAKE, FAKE, FAKE, FAKE, None, 2, 8, 1, 64, 0.0, 1, 1, None, None) == rra.RRA_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE + 8, None, 2, 8, 1, 64, 0.0, 1, 1, None, None) == rra.RRA_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 8, 1, 32, 0.0, 1, 1, None, None) == rra.RRA_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 5000, 1, 64, 0.0, 1, 1, None, None) == rra.RRA_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 9000, 8, 1, 64, 0.0, 1, 1, None, None) == rra.RRA_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 8, 1, 64, 0.0, 2, 2, None, None) == rra.RRA_ERR_UNSUPPORTED
 
 
 def test_get_device_error_validation(L):
