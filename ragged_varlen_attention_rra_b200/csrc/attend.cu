@@ -77,8 +77,12 @@ constexpr uint32_t kOffV = kOffK + kKVStages * kTileBytes;
 constexpr uint32_t kOffOnes = kOffV + kKVStages * kTileBytes;   // [128 keys x 64] MN-major, column 0 = 1
 constexpr uint32_t kOffBar = kOffOnes + kTileBytes;
 constexpr uint32_t kOffRed = kOffBar + 512;             // [2 parities][2 halves][128] row max
-constexpr uint32_t kOffIdx = kOffRed + 2 * 2 * 128 * 4;  // fused: kept-row list of one image (int16)
-constexpr uint32_t kOffTile = kOffIdx + kFusedMaxN * 2;   // tile_pre[B+1], then cu[B+1]
+// fused: 4 slots, each the kept positions of one item's image (int16 [kFusedMaxN]) and its
+// kept-bit mask (uint32 [kFusedMaxN / 32])
+constexpr int kIdxSlots = 4;
+constexpr uint32_t kIdxSlotBytes = kFusedMaxN * 2 + kFusedMaxN / 8;
+constexpr uint32_t kOffIdx = kOffRed + 2 * 2 * 128 * 4;
+constexpr uint32_t kOffTile = kOffIdx + kIdxSlots * kIdxSlotBytes;  // tile_pre[B+1], then cu[B+1]
 constexpr int kSmemFixed = 1024 /*align slack*/ + kOffTile;
 
 struct Params {
@@ -101,6 +105,7 @@ struct Bars {
     uint64_t kv_full[kKVStages], kv_empty[kKVStages];
     uint64_t s_full[2], p_full[2], s_free[2];
     uint64_t o_full[2], o_free[2];
+    uint64_t idx_full[4], idx_free[4];  // fused: kept-row list slots, one per item in flight
     uint64_t drain;
     uint32_t tmem_slot;
     int abort;
@@ -298,7 +303,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *red = reinterpret_cast<float *>(base + kOffRed);            // row max exchange [2][2][128]
     int32_t *tile_pre = reinterpret_cast<int32_t *>(base + kOffTile);  // [B+1]
     int32_t *cu_s = tile_pre + (p.B + 1);                               // [B+1]
-    int16_t *idx = reinterpret_cast<int16_t *>(base + kOffIdx);         // fused: kept rows of one image
+    auto idx_list = [&](int slot) { return reinterpret_cast<int16_t *>(base + kOffIdx + slot * kIdxSlotBytes); };
+    auto idx_bits = [&](int slot) {
+        return reinterpret_cast<uint32_t *>(base + kOffIdx + slot * kIdxSlotBytes + kFusedMaxN * 2);
+    };
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -323,6 +331,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->s_free[s], 1);
             mbar_init(&bars->o_full[s], 1);
             mbar_init(&bars->o_free[s], kSoftmaxWarps);
+        }
+        for (int s = 0; s < kIdxSlots; ++s) {
+            mbar_init(&bars->idx_full[s], 1);
+            mbar_init(&bars->idx_free[s], kSoftmaxWarps);
         }
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
@@ -455,7 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // phase 0 counts as complete, so waiting on parity (phase ^ 1) passes at once for the
         // first fill of each slot, then tracks the consumer's releases.
         uint32_t q_phase = 0, kv_phase = 0;  // one bit per slot
-        int cur_b = -1;                      // fused: image whose kept-row list is in idx[]
+        int cur_b = -1, prev_slot = 0;       // fused: image of the previous item, and its list slot
+        uint32_t idx_phase = 0, n_items = 0;
         uint32_t q_issued = 0, kv_issued = 0;
         int qs = 0, ks = 0;
         bool ok = true;
@@ -463,31 +476,66 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Item it = decode_item(item, H, B, tile_pre, cu_s);
             const int nkc = (it.L + BN - 1) / BN;
             const int row_off = it.b * p.N;  // fused: first padded row of this image
+            const int islot = static_cast<int>(n_items & (kIdxSlots - 1));
             if constexpr (kFused) {
-                if (it.b != cur_b) {
-                    // kept positions of this image, in order (warp ballot scan of its mask row)
+                // list slot of this item: free once the epilogue of item n-4 has used it
+                ok = warp_wait(&bars->idx_free[islot], ((idx_phase >> islot) & 1u) ^ 1u, bars, p);
+                if (!ok)
+                    break;
+                idx_phase ^= 1u << islot;
+                int16_t *list = idx_list(islot);
+                uint32_t *bits = idx_bits(islot);
+                const int nwords = (p.N + 31) / 32;
+                if (it.b == cur_b) {
+                    // same image as the previous item: copy its list
+                    const int16_t *pl = idx_list(prev_slot);
+                    const uint32_t *pb = idx_bits(prev_slot);
+                    for (int i = lane; i < it.L; i += 32)
+                        list[i] = pl[i];
+                    for (int i = lane; i < nwords; i += 32)
+                        bits[i] = pb[i];
+                } else {
+                    // kept positions of this image in order: mask bytes fetched 8 words of 32 at
+                    // a time (independent loads), then one ballot per word
                     int running = 0;
-                    for (int c0 = 0; c0 < p.N; c0 += 32) {
-                        const int n = c0 + lane;
-                        const bool keep = n < p.N && p.mask[row_off + n] != 0;
-                        const unsigned bal = __ballot_sync(0xffffffffu, keep);
-                        if (keep)
-                            idx[running + __popc(bal & ((1u << lane) - 1u))] = static_cast<int16_t>(n);
-                        running += __popc(bal);
+                    for (int w0 = 0; w0 < nwords; w0 += 8) {
+                        bool keep[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int n = (w0 + u) * 32 + lane;
+                            keep[u] = n < p.N && p.mask[row_off + n] != 0;
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const unsigned bal = __ballot_sync(0xffffffffu, keep[u]);
+                            if (w0 + u < nwords) {
+                                if (keep[u])
+                                    list[running + __popc(bal & ((1u << lane) - 1u))] =
+                                        static_cast<int16_t>((w0 + u) * 32 + lane);
+                                if (lane == 0)
+                                    bits[w0 + u] = bal;
+                                running += __popc(bal);
+                            }
+                        }
                     }
-                    __syncwarp();
-                    cur_b = it.b;
                 }
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bars->idx_full[islot]);
+                cur_b = it.b;
+                prev_slot = islot;
                 if (it.qt == 0) {
                     // pruned rows of this (image, head) in the padded output become zero
                     const int out_vecs = (p.out_dt == RRA_F32 ? 4 * kD : 2 * kD) / 16;
-                    for (int n = lane; n < p.N; n += 32) {
-                        if (p.mask[row_off + n] != 0)
-                            continue;
-                        uint4 *y = reinterpret_cast<uint4 *>(p.out) +
-                                   (static_cast<int64_t>(row_off + n) * H + it.h) * out_vecs;
-                        for (int v2 = 0; v2 < out_vecs; ++v2)
-                            y[v2] = make_uint4(0, 0, 0, 0);
+                    for (int wd = 0; wd < nwords; ++wd) {
+                        const uint32_t pruned = ~bits[wd];
+                        const int n = wd * 32 + lane;
+                        if (n < p.N && ((pruned >> lane) & 1u)) {
+                            uint4 *y = reinterpret_cast<uint4 *>(p.out) +
+                                       (static_cast<int64_t>(row_off + n) * H + it.h) * out_vecs;
+                            for (int v2 = 0; v2 < out_vecs; ++v2)
+                                y[v2] = make_uint4(0, 0, 0, 0);
+                        }
                     }
                 }
             }
@@ -499,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive_expect_tx(&bars->q_full[qs], kTileBytes);
             __syncwarp();
             if constexpr (kFused) {
-                gather_tile(base + kOffQ + qs * kTileBytes, &tm_q, &bars->q_full[qs], idx, it.qt * BM,
+                gather_tile(base + kOffQ + qs * kTileBytes, &tm_q, &bars->q_full[qs], idx_list(islot), it.qt * BM,
                             min(BM, it.L - it.qt * BM), row_off, it.h * kD, lane);
             } else {
                 if (lane == 0)
@@ -518,10 +566,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if constexpr (kFused) {
                     const int cnt = min(BN, it.L - kc * BN);
-                    gather_tile(base + kOffK + ks * kTileBytes, &tm_k, &bars->kv_full[ks], idx, kc * BN, cnt, row_off,
-                                it.h * kD, lane);
-                    gather_tile(base + kOffV + ks * kTileBytes, &tm_v, &bars->kv_full[ks], idx, kc * BN, cnt, row_off,
-                                it.h * kD, lane);
+                    gather_tile(base + kOffK + ks * kTileBytes, &tm_k, &bars->kv_full[ks], idx_list(islot), kc * BN, cnt,
+                                row_off, it.h * kD, lane);
+                    gather_tile(base + kOffV + ks * kTileBytes, &tm_v, &bars->kv_full[ks], idx_list(islot), kc * BN, cnt,
+                                row_off, it.h * kD, lane);
                 } else {
                     if (lane == 0) {
                         tma_load_3d(base + kOffK + ks * kTileBytes, &tm_k, &bars->kv_full[ks], 0, it.h, it.seq0 + kc * BN);
@@ -532,6 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++kv_issued;
                 ks = (ks + 1 == kKVStages) ? 0 : ks + 1;
             }
+            ++n_items;
         }
         // drain: every issued fill has landed before the block may leave
         for (int s = 0; s < kQStages; ++s) {
@@ -683,11 +732,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // deferred epilogue of the previous item
         bool pending = false;
-        int pend_row0 = 0, pend_h = 0, pend_qrows = 0, pend_ob = 0, pend_b = 0, pend_q0 = 0;
+        int pend_row0 = 0, pend_h = 0, pend_qrows = 0, pend_ob = 0, pend_b = 0, pend_q0 = 0, pend_slot = 0;
+        uint32_t idxf_ph = 0;
         auto epilogue = [&]() -> bool {
             if (!warp_wait(&bars->o_full[pend_ob], (o_ph >> pend_ob) & 1u, bars, p))
                 return false;
             o_ph ^= 1u << pend_ob;
+            if constexpr (kFused) {
+                // the producer's list of this item (written long before; this orders the reads)
+                if (!warp_wait(&bars->idx_full[pend_slot], (idxf_ph >> pend_slot) & 1u, bars, p))
+                    return false;
+                idxf_ph ^= 1u << pend_slot;
+            }
             tc_fence_after();
             if (q4 * 32 < pend_qrows) {
                 uint32_t r[32], sum[1];
@@ -695,20 +751,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld1(lane_base + kColO0 + kOCols * pend_ob + 64, sum);
                 int64_t out_row = static_cast<int64_t>(pend_row0) + row;
                 if constexpr (kFused) {
-                    // padded position of kept token (q0 + row) of image b: warp select over its mask row
-                    const int target = pend_q0 + row;
-                    const int last = pend_q0 + q4 * 32 + 31;
-                    const uint8_t *mrow = p.mask + static_cast<int64_t>(pend_b) * p.N;
-                    int pos = 0, running = 0;
-                    for (int c0 = 0; c0 < p.N && running <= last; c0 += 32) {
-                        const bool keep = c0 + lane < p.N && mrow[c0 + lane] != 0;
-                        const unsigned bal = __ballot_sync(0xffffffffu, keep);
-                        const int cnt = __popc(bal);
-                        if (target >= running && target < running + cnt)
-                            pos = c0 + static_cast<int>(__fns(bal, 0, target - running + 1));
-                        running += cnt;
-                    }
-                    out_row = static_cast<int64_t>(pend_b) * p.N + pos;
+                    // padded position of kept token (q0 + row), from the item's list slot
+                    const int r = row < pend_qrows ? row : 0;
+                    out_row = static_cast<int64_t>(pend_b) * p.N + idx_list(pend_slot)[pend_q0 + r];
                 }
                 tmem_wait_ld();
                 const float inv = 1.f / __uint_as_float(sum[0]);
@@ -749,8 +794,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++n_epi;
             tc_fence_before();
             __syncwarp();
-            if (lane == 0)
+            if (lane == 0) {
                 mbar_arrive(&bars->o_free[pend_ob]);
+                if constexpr (kFused)
+                    mbar_arrive(&bars->idx_free[pend_slot]);
+            }
             pending = false;
             return true;
         };
@@ -848,6 +896,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             pend_row0 = it.seq0 + q0;
             pend_b = it.b;
             pend_q0 = q0;
+            pend_slot = n & (kIdxSlots - 1);
             pend_h = it.h;
             pend_qrows = qrows;
             pend_ob = ob;

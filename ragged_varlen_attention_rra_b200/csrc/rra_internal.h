@@ -48,7 +48,7 @@ struct FusedArgs {
 };
 
 // Largest N the single-launch path accepts (its kept-row list lives in shared memory).
-constexpr int kFusedMaxN = 4096;
+constexpr int kFusedMaxN = 2048;
 
 cudaError_t launch_fused(const FusedArgs &a, int num_sms, cudaStream_t stream);
 
