@@ -63,6 +63,21 @@ def dist_env():
     return ws, rank, local
 
 
+def reduce_max(x: float, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world_size: int, steps: int, tokens_per_call: int, max_total_ms: float) -> float:
+    """Whole-job tokens/s: every rank runs `steps` calls of `tokens_per_call` tokens (independent
+    replicas), and the job takes as long as its slowest rank."""
+    return world_size * steps * tokens_per_call / (max_total_ms * 1e-3)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -371,13 +386,9 @@ def main_gpu(args):
         raise RuntimeError(f"device error {rra.rra_status_string(err)} on the {other.path} path")
     same = all(torch.equal(a.view(torch.uint8), b.view(torch.uint8)) for a, b in zip(pipe.ys, other.ys))
 
-    total_ms = float(sum(step_ms))
-    if ws > 1:
-        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(float(sum(step_ms)), device="cuda")
     ms_per_step = total_ms / args.steps
-    value = ws * args.steps * T_call / (total_ms * 1e-3)
+    value = job_throughput(ws, args.steps, T_call, total_ms)
 
     # dispatch floor: host time to enqueue one graph replay, and one eager call through the API
     torch.cuda.synchronize()
@@ -469,14 +480,10 @@ def main_gpu(args):
                 e_end.record(stream)
             stream.synchronize()
             e2e_ms.append(e_start.elapsed_time(e_end))
-        tot = float(sum(e2e_ms))
-        if ws > 1:
-            t = torch.tensor([tot], device="cuda", dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            tot = float(t.item())
+        tot = reduce_max(float(sum(e2e_ms)), device="cuda")
         h2d = 3 * w.q.numel() * w.q.element_size() + sum(m.numel() for m in w.masks)
         d2h = sum(t.numel() * t.element_size() for t in host_out)
-        e2e = {"value": ws * args.steps * T_call / (tot * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+        e2e = {"value": job_throughput(ws, args.steps, T_call, tot), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": tot / args.steps,
                "api": f"rra.forward (eager, {args.path} path)"}
         if err == 0:
