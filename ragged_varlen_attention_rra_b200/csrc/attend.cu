@@ -13,12 +13,12 @@
 //     (fp32 [128 x 64]), so the tensor core computes S of the next step while the softmax
 //     warps work on the current one, and PV of one item runs under the next item's softmax;
 //   * warps specialise:
-//       warp 0      TMA producer: Q tiles (2-slot ring) and 128-key K/V chunks (3-slot ring)
-//                   of one head, fetched straight from the packed [T, H, 64] layout (3-D tensor
-//                   map, head = coordinate, 128-byte swizzle);
-//       warp 1      tensor-core issuer: S = Q K^T (smem x smem) and O += P V (P from TMEM as the
+//       warps 0..2  producer: Q tiles (2-slot ring) and 128-key K/V chunks (3-slot ring) of one
+//                   head; on the packed path warp 0 fetches them straight from the [T, H, 64]
+//                   layout with TMA (3-D tensor map, head = coordinate, 128-byte swizzle);
+//       warp 3      tensor-core issuer: S = Q K^T (smem x smem) and O += P V (P from TMEM as the
 //                   A operand), fp32 accumulation, completion signalled through mbarriers;
-//       warps 2..9  softmax: a pair of warps owns each quarter of the rows (TMEM lanes); within
+//       warps 4..11 softmax: a pair of warps owns each quarter of the rows (TMEM lanes); within
 //                   a step the two warps take alternate 32-key slices, keep them in registers
 //                   for both passes (row max, then exponentials), exchange the row max once,
 //                   write P back over their own S columns, and rescale their half of O in TMEM
@@ -38,10 +38,9 @@
 // The same kernel body, instantiated with kFused, runs the whole pack -> attend -> unpack call
 // in one launch (the pages' pipeline without its two copies through HBM): the block derives
 // the kept counts of every image from the keep mask itself, the producer gathers the kept rows
-// of the padded Q/K/V straight into the swizzled tiles with TMA tile::gather4 (four rows per
-// instruction, one instruction per lane of the producer warp), zero-fills the pruned rows of
-// the padded output for its (image, head), and the epilogue writes each output row back to
-// its padded position.
+// of the padded Q/K/V straight into the swizzled tiles with 16-byte cp.async (32 lanes, one
+// coalesced 128-byte row segment per 8 lanes), zero-fills the pruned rows of the padded output
+// for its (image, head), and the epilogue writes each output row back to its padded position.
 #include <cuda.h>
 
 #include <mutex>
@@ -56,7 +55,10 @@ namespace {
 constexpr int BM = 128;                 // query rows per tile (TMEM lanes)
 constexpr int BN = 128;                 // keys per step
 constexpr int kD = 64;                  // head dim
-constexpr int kThreads = 320;           // 10 warps: producer, MMA, 8 x softmax
+constexpr int kThreads = 384;           // 12 warps: 3 x producer, MMA, 8 x softmax
+constexpr int kProducerWarps = 3;       // fused path: all three copy; packed path: warp 0 issues TMA
+constexpr int kMmaWarp = 3;
+constexpr int kSoftmaxWarp0 = 4;
 constexpr int kSoftmaxWarps = 8;
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: S buffers at 0 and 128 (the P of each 32-key slice is written back over the
@@ -88,6 +90,7 @@ constexpr int kSmemFixed = 1024 /*align slack*/ + kOffTile;
 struct Params {
     const int32_t *cu;      // packed path: cu_seqlens in
     const uint8_t *mask;    // fused path: keep mask [B, N]
+    const uint8_t *src[3];  // fused path: padded Q, K, V [B*N, H, 64]
     int32_t *cu_out;        // fused path: cu_seqlens out (may be null)
     void *out;
     int B, H, N;
@@ -267,29 +270,25 @@ struct PvStep {
     bool wait_free;  // first PV of an item whose O buffer held an earlier item
 };
 
-// 2-D gather of four rows (row coordinates r0..r3) of 64 elements starting at column x.
-__device__ __forceinline__ void tma_gather4(void *smem_dst, const void *tmap, uint64_t *bar, int x, int r0, int r1,
-                                            int r2, int r3)
+// Fused path: producer warp w (of kProducerWarps) copies its share of one 128-row tile of one
+// head from the padded tensor into the 128-byte-swizzled layout with 16-byte cp.async: row r of
+// the tile is padded row row_off + list[base + r] (entries at or past `count` repeat the tile's
+// first row, whose result is masked later).  The 1024 chunks go in groups of 32 (one per lane,
+// 8 lanes per 128-byte row, so each row is one coalesced segment), group g to warp g % 3.
+// Completion arrives on `bar` once per producer lane.
+__device__ __forceinline__ void copy_tile_async(uint8_t *tile, const uint8_t *src, uint64_t *bar, const int16_t *list,
+                                                int base, int count, int row_off, int h, int H, int w, int lane)
 {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_addr(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_addr(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-        : "memory");
-}
-
-// Fused path: the producer lane gathers rows list[base + 4*lane .. +3] of one 128-row tile
-// (entries at or past `count` repeat the tile's first row, whose result is masked later).
-__device__ __forceinline__ void gather_tile(void *tile, const void *tmap, uint64_t *bar, const int16_t *list, int base,
-                                            int count, int row_off, int x, int lane)
-{
-    int r[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int i = 4 * lane + k;
-        r[k] = row_off + list[base + (i < count ? i : 0)];
+#pragma unroll 4
+    for (int grp = w; grp < 32; grp += kProducerWarps) {
+        const int i = lane + 32 * grp;
+        const int r = i >> 3, c = i & 7;
+        const int grow = row_off + list[base + (r < count ? r : 0)];
+        const uint8_t *gsrc = src + ((static_cast<int64_t>(grow) * H + h) * kD) * 2 + c * 16;
+        const uint32_t d = smem_addr(tile + r * 128 + ((c ^ (r & 7)) << 4));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
     }
-    tma_gather4(static_cast<uint8_t *>(tile) + 512 * lane, tmap, bar, x, r[0], r[1], r[2], r[3]);
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 template <bool kBF16, bool kFused>
@@ -314,15 +313,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int B = p.B, H = p.H;
 
     if (tid == 0) {
-        prefetch_tmap(&tm_q);
-        prefetch_tmap(&tm_k);
-        prefetch_tmap(&tm_v);
+        if constexpr (!kFused) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+        }
+        // full barriers: one TMA arrival with transaction bytes, or (fused) one cp.async
+        // arrival per producer lane
+        const uint32_t fills = kFused ? 32u * kProducerWarps : 1u;
         for (int s = 0; s < kQStages; ++s) {
-            mbar_init(&bars->q_full[s], 1);
+            mbar_init(&bars->q_full[s], fills);
             mbar_init(&bars->q_empty[s], 1);
         }
         for (int s = 0; s < kKVStages; ++s) {
-            mbar_init(&bars->kv_full[s], 1);
+            mbar_init(&bars->kv_full[s], kFused ? 2u * fills : fills);
             mbar_init(&bars->kv_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -461,14 +465,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = bars->tmem_slot;
     const int total_items = tile_pre[B] * H;
 
-    if (warp == 0) {
-        // ================================================================ TMA producer
+    if (warp < kProducerWarps && (kFused || warp == 0)) {
+        // ================================================================ producer
         // Empty-slot waits use the usual parity idiom: on a fresh barrier the phase "before"
         // phase 0 counts as complete, so waiting on parity (phase ^ 1) passes at once for the
         // first fill of each slot, then tracks the consumer's releases.
         uint32_t q_phase = 0, kv_phase = 0;  // one bit per slot
         int cur_b = -1, prev_slot = 0;       // fused: image of the previous item, and its list slot
-        uint32_t idx_phase = 0, n_items = 0;
+        uint32_t idx_phase = 0, idxf_phase = 0, n_items = 0;
         uint32_t q_issued = 0, kv_issued = 0;
         int qs = 0, ks = 0;
         bool ok = true;
@@ -478,15 +482,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int row_off = it.b * p.N;  // fused: first padded row of this image
             const int islot = static_cast<int>(n_items & (kIdxSlots - 1));
             if constexpr (kFused) {
-                // list slot of this item: free once the epilogue of item n-4 has used it
-                ok = warp_wait(&bars->idx_free[islot], ((idx_phase >> islot) & 1u) ^ 1u, bars, p);
-                if (!ok)
-                    break;
-                idx_phase ^= 1u << islot;
                 int16_t *list = idx_list(islot);
                 uint32_t *bits = idx_bits(islot);
                 const int nwords = (p.N + 31) / 32;
-                if (it.b == cur_b) {
+                // list slot of this item: free once the epilogue of item n-4 has used it; producer
+                // warp 0 fills it, the other producer warps wait until it is full (bounded waits
+                // only, so an aborting warp can never strand the others)
+                if (warp == 0) {
+                    ok = warp_wait(&bars->idx_free[islot], ((idx_phase >> islot) & 1u) ^ 1u, bars, p);
+                    if (!ok)
+                        break;
+                    idx_phase ^= 1u << islot;
+                }
+                if (warp != 0) {
+                    ok = warp_wait(&bars->idx_full[islot], (idxf_phase >> islot) & 1u, bars, p);
+                    if (!ok)
+                        break;
+                    idxf_phase ^= 1u << islot;
+                } else if (it.b == cur_b) {
                     // same image as the previous item: copy its list
                     const int16_t *pl = idx_list(prev_slot);
                     const uint32_t *pb = idx_bits(prev_slot);
@@ -520,14 +533,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 __syncwarp();
-                if (lane == 0)
+                if (warp == 0 && lane == 0)
                     mbar_arrive(&bars->idx_full[islot]);
                 cur_b = it.b;
                 prev_slot = islot;
                 if (it.qt == 0) {
                     // pruned rows of this (image, head) in the padded output become zero
                     const int out_vecs = (p.out_dt == RRA_F32 ? 4 * kD : 2 * kD) / 16;
-                    for (int wd = 0; wd < nwords; ++wd) {
+                    for (int wd = warp; wd < nwords; wd += kProducerWarps) {
                         const uint32_t pruned = ~bits[wd];
                         const int n = wd * 32 + lane;
                         if (n < p.N && ((pruned >> lane) & 1u)) {
@@ -543,15 +556,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok)
                 break;
             q_phase ^= 1u << qs;
-            if (lane == 0)
-                mbar_arrive_expect_tx(&bars->q_full[qs], kTileBytes);
-            __syncwarp();
             if constexpr (kFused) {
-                gather_tile(base + kOffQ + qs * kTileBytes, &tm_q, &bars->q_full[qs], idx_list(islot), it.qt * BM,
-                            min(BM, it.L - it.qt * BM), row_off, it.h * kD, lane);
+                copy_tile_async(base + kOffQ + qs * kTileBytes, p.src[0], &bars->q_full[qs], idx_list(islot),
+                                it.qt * BM, min(BM, it.L - it.qt * BM), row_off, it.h, H, warp, lane);
             } else {
-                if (lane == 0)
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&bars->q_full[qs], kTileBytes);
                     tma_load_3d(base + kOffQ + qs * kTileBytes, &tm_q, &bars->q_full[qs], 0, it.h, it.seq0 + it.qt * BM);
+                }
             }
             __syncwarp();
             ++q_issued;
@@ -561,16 +573,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok)
                     break;
                 kv_phase ^= 1u << ks;
-                if (lane == 0)
-                    mbar_arrive_expect_tx(&bars->kv_full[ks], 2 * kTileBytes);
-                __syncwarp();
                 if constexpr (kFused) {
                     const int cnt = min(BN, it.L - kc * BN);
-                    gather_tile(base + kOffK + ks * kTileBytes, &tm_k, &bars->kv_full[ks], idx_list(islot), kc * BN, cnt,
-                                row_off, it.h * kD, lane);
-                    gather_tile(base + kOffV + ks * kTileBytes, &tm_v, &bars->kv_full[ks], idx_list(islot), kc * BN, cnt,
-                                row_off, it.h * kD, lane);
+                    copy_tile_async(base + kOffK + ks * kTileBytes, p.src[1], &bars->kv_full[ks], idx_list(islot),
+                                    kc * BN, cnt, row_off, it.h, H, warp, lane);
+                    copy_tile_async(base + kOffV + ks * kTileBytes, p.src[2], &bars->kv_full[ks], idx_list(islot),
+                                    kc * BN, cnt, row_off, it.h, H, warp, lane);
                 } else {
+                    if (lane == 0)
+                        mbar_arrive_expect_tx(&bars->kv_full[ks], 2 * kTileBytes);
                     if (lane == 0) {
                         tma_load_3d(base + kOffK + ks * kTileBytes, &tm_k, &bars->kv_full[ks], 0, it.h, it.seq0 + kc * BN);
                         tma_load_3d(base + kOffV + ks * kTileBytes, &tm_v, &bars->kv_full[ks], 0, it.h, it.seq0 + kc * BN);
@@ -583,6 +594,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++n_items;
         }
         // drain: every issued fill has landed before the block may leave
+        if constexpr (kFused)
+            asm volatile("cp.async.wait_all;" ::: "memory");
         for (int s = 0; s < kQStages; ++s) {
             const uint32_t n = q_issued / kQStages + (static_cast<uint32_t>(s) < q_issued % kQStages ? 1u : 0u);
             if (n > 0)
@@ -593,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (n > 0)
                 mbar_wait_bounded(&bars->kv_full[s], (n - 1) & 1u, kDrainNs);
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ================================================================ tcgen05 issuer
         // Order: S(t) then PV(t-1), so the next step's QK^T runs while the softmax warps work.
         // phase parities, one bit per slot / buffer
@@ -687,6 +700,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (lane == 0) {
                     tc_fence_after();
+                    if constexpr (kFused)
+                        fence_proxy_async_smem();  // Q/K/V arrived through cp.async (generic proxy)
                     const uint64_t kd = slot_desc(kdesc0, ks);
                     const uint32_t idS = idesc_f16(BM, nk16, kBF16 ? 1u : 0u, 0u);
 #pragma unroll
@@ -719,10 +734,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait_bounded(&bars->drain, 0, kDrainNs);
         }
         __syncwarp();
-    } else {
+    } else if (warp >= kSoftmaxWarp0) {
         // ================================================================ softmax + epilogue
         const int q4 = warp & 3;                     // TMEM lane quarter of this warp
-        const int hf = (warp - 2) >> 2;              // which of the pair: slices hf, hf+2; O columns 32hf..
+        const int hf = (warp - kSoftmaxWarp0) >> 2;  // which of the pair: slices hf, hf+2; O columns 32hf..
         const int row = q4 * 32 + lane;              // row of S / O owned by this thread
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
         float *red_max = red;                        // [2][2][128]
@@ -1048,6 +1063,9 @@ cudaError_t launch_fused(const FusedArgs &a, int num_sms, cudaStream_t stream)
         !make_gather_tmap(&tv, a.v, rows, a.H, a.in_bf16))
         return cudaErrorInvalidValue;
     Params p{};
+    p.src[0] = static_cast<const uint8_t *>(a.q);
+    p.src[1] = static_cast<const uint8_t *>(a.k);
+    p.src[2] = static_cast<const uint8_t *>(a.v);
     p.mask = a.mask;
     p.cu_out = a.cu_out;
     p.out = a.y;
