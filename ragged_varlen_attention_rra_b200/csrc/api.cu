@@ -134,7 +134,7 @@ rra_status rra_pack_attend_unpack(const uint8_t *keep_mask, const void *q, const
         return RRA_ERR_INVALID_ARG;
     if (d != 64 || (in_dt != RRA_F16 && in_dt != RRA_BF16) || (out_dt != in_dt && out_dt != RRA_F32))
         return RRA_ERR_UNSUPPORTED;
-    if (B > rra::kAttendMaxBatch || N > rra::kFusedMaxN || H > 65535 || static_cast<int64_t>(B) * N > kMaxRows)
+    if (B > rra::kFusedMaxBatch || N > rra::kFusedMaxN || H > 65535 || static_cast<int64_t>(B) * N > kMaxRows)
         return RRA_ERR_UNSUPPORTED;
     if (!(softmax_scale == softmax_scale))
         return RRA_ERR_INVALID_ARG;

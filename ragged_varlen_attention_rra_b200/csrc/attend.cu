@@ -79,13 +79,23 @@ constexpr uint32_t kOffV = kOffK + kKVStages * kTileBytes;
 constexpr uint32_t kOffOnes = kOffV + kKVStages * kTileBytes;   // [128 keys x 64] MN-major, column 0 = 1
 constexpr uint32_t kOffBar = kOffOnes + kTileBytes;
 constexpr uint32_t kOffRed = kOffBar + 512;             // [2 parities][2 halves][128] row max
-// fused: 4 slots, each the kept positions of one item's image (int16 [kFusedMaxN]) and its
-// kept-bit mask (uint32 [kFusedMaxN / 32])
+// fused: 4 slots, each the kept positions of one item's image (int16 [kFusedMaxN]), the byte
+// offsets of those padded rows' first head (int32 [kFusedMaxN]) and the kept-bit mask
+// (uint32 [kFusedMaxN / 32])
 constexpr int kIdxSlots = 4;
-constexpr uint32_t kIdxSlotBytes = kFusedMaxN * 2 + kFusedMaxN / 8;
+constexpr uint32_t kIdxSlotBytes = kFusedMaxN * 2 + kFusedMaxN * 4 + kFusedMaxN / 8;
 constexpr uint32_t kOffIdx = kOffRed + 2 * 2 * 128 * 4;
-constexpr uint32_t kOffTile = kOffIdx + kIdxSlots * kIdxSlotBytes;  // tile_pre[B+1], then cu[B+1]
-constexpr int kSmemFixed = 1024 /*align slack*/ + kOffTile;
+// tile_pre[B+1], then cu[B+1]: after the list slots on the fused path, in their place otherwise
+template <bool kFused>
+constexpr uint32_t off_tile()
+{
+    return kFused ? kOffIdx + kIdxSlots * kIdxSlotBytes : kOffIdx;
+}
+template <bool kFused>
+constexpr int smem_bytes(int B)
+{
+    return 1024 /*align slack*/ + static_cast<int>(off_tile<kFused>()) + 2 * (B + 1) * 4;
+}
 
 struct Params {
     const int32_t *cu;      // packed path: cu_seqlens in
@@ -115,6 +125,8 @@ struct Bars {
     int warp_sums[2][kThreads / 32];
 };
 static_assert(sizeof(Bars) <= 512, "barrier block overflows its slot");
+static_assert(smem_bytes<false>(kAttendMaxBatch) <= 232448, "packed path exceeds shared memory");
+static_assert(smem_bytes<true>(kFusedMaxBatch) <= 232448, "single-launch path exceeds shared memory");
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 {
@@ -251,17 +263,24 @@ __device__ __forceinline__ void softmax_slice(uint32_t (&r)[32], int c, int nk, 
 
 __device__ __forceinline__ float slice_max(const uint32_t (&r)[32], int c, int nk, float mx)
 {
+    // pairwise tree (depth 5) rather than a 32-long dependent chain
+    float t[16];
     if (c + 32 <= nk) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-            mx = fmaxf(mx, __uint_as_float(r[j]));
+        for (int j = 0; j < 16; ++j)
+            t[j] = fmaxf(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
     } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-            if (c + j < nk)
-                mx = fmaxf(mx, __uint_as_float(r[j]));
+        for (int j = 0; j < 16; ++j)
+            t[j] = fmaxf(c + 2 * j < nk ? __uint_as_float(r[2 * j]) : -INFINITY,
+                         c + 2 * j + 1 < nk ? __uint_as_float(r[2 * j + 1]) : -INFINITY);
     }
-    return mx;
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+        for (int j = 0; j < w; ++j)
+            t[j] = fmaxf(t[j], t[j + w]);
+    return fmaxf(mx, t[0]);
 }
 
 // One PV step as the MMA warp sees it.
@@ -270,22 +289,34 @@ struct PvStep {
     bool wait_free;  // first PV of an item whose O buffer held an earlier item
 };
 
+// 2-D gather of four rows (row coordinates r0..r3) of 64 elements starting at column x.
+__device__ __forceinline__ void tma_gather4(void *smem_dst, const void *tmap, uint64_t *bar, int x, int r0, int r1,
+                                            int r2, int r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_addr(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_addr(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
+
 // Fused path: producer warp w (of kProducerWarps) copies its share of one 128-row tile of one
 // head from the padded tensor into the 128-byte-swizzled layout with 16-byte cp.async: row r of
 // the tile is padded row row_off + list[base + r] (entries at or past `count` repeat the tile's
 // first row, whose result is masked later).  The 1024 chunks go in groups of 32 (one per lane,
 // 8 lanes per 128-byte row, so each row is one coalesced segment), group g to warp g % 3.
 // Completion arrives on `bar` once per producer lane.
-__device__ __forceinline__ void copy_tile_async(uint8_t *tile, const uint8_t *src, uint64_t *bar, const int16_t *list,
-                                                int base, int count, int row_off, int h, int H, int w, int lane)
+__device__ __forceinline__ void copy_tile_async(uint8_t *tile, const uint8_t *src, uint64_t *bar, const int32_t *offs,
+                                                int base, int count, int w, int lane)
 {
+    // src already points at this head's 128 bytes of padded row 0; offs[] holds row offsets
+    const uint32_t tile_s = smem_addr(tile);
 #pragma unroll 4
     for (int grp = w; grp < 32; grp += kProducerWarps) {
         const int i = lane + 32 * grp;
         const int r = i >> 3, c = i & 7;
-        const int grow = row_off + list[base + (r < count ? r : 0)];
-        const uint8_t *gsrc = src + ((static_cast<int64_t>(grow) * H + h) * kD) * 2 + c * 16;
-        const uint32_t d = smem_addr(tile + r * 128 + ((c ^ (r & 7)) << 4));
+        const uint8_t *gsrc = src + offs[base + (r < count ? r : 0)] + c * 16;
+        const uint32_t d = tile_s + r * 128 + ((c ^ (r & 7)) << 4);
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
     }
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
@@ -300,11 +331,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars *bars = reinterpret_cast<Bars *>(base + kOffBar);
     float *red = reinterpret_cast<float *>(base + kOffRed);            // row max exchange [2][2][128]
-    int32_t *tile_pre = reinterpret_cast<int32_t *>(base + kOffTile);  // [B+1]
+    int32_t *tile_pre = reinterpret_cast<int32_t *>(base + off_tile<kFused>());  // [B+1]
     int32_t *cu_s = tile_pre + (p.B + 1);                               // [B+1]
     auto idx_list = [&](int slot) { return reinterpret_cast<int16_t *>(base + kOffIdx + slot * kIdxSlotBytes); };
+    auto idx_offs = [&](int slot) {
+        return reinterpret_cast<int32_t *>(base + kOffIdx + slot * kIdxSlotBytes + kFusedMaxN * 2);
+    };
     auto idx_bits = [&](int slot) {
-        return reinterpret_cast<uint32_t *>(base + kOffIdx + slot * kIdxSlotBytes + kFusedMaxN * 2);
+        return reinterpret_cast<uint32_t *>(base + kOffIdx + slot * kIdxSlotBytes + kFusedMaxN * 6);
     };
 
     const int tid = threadIdx.x;
@@ -313,8 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int B = p.B, H = p.H;
 
     if (tid == 0) {
+        prefetch_tmap(&tm_q);
         if constexpr (!kFused) {
-            prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
         }
@@ -322,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // arrival per producer lane
         const uint32_t fills = kFused ? 32u * kProducerWarps : 1u;
         for (int s = 0; s < kQStages; ++s) {
-            mbar_init(&bars->q_full[s], fills);
+            mbar_init(&bars->q_full[s], 1);  // Q always arrives by TMA (tile, or fused: gather4)
             mbar_init(&bars->q_empty[s], 1);
         }
         for (int s = 0; s < kKVStages; ++s) {
@@ -502,9 +536,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 } else if (it.b == cur_b) {
                     // same image as the previous item: copy its list
                     const int16_t *pl = idx_list(prev_slot);
+                    const int32_t *po = idx_offs(prev_slot);
                     const uint32_t *pb = idx_bits(prev_slot);
-                    for (int i = lane; i < it.L; i += 32)
+                    int32_t *offs = idx_offs(islot);
+                    for (int i = lane; i < it.L; i += 32) {
                         list[i] = pl[i];
+                        offs[i] = po[i];
+                    }
                     for (int i = lane; i < nwords; i += 32)
                         bits[i] = pb[i];
                 } else {
@@ -522,9 +560,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int u = 0; u < 8; ++u) {
                             const unsigned bal = __ballot_sync(0xffffffffu, keep[u]);
                             if (w0 + u < nwords) {
-                                if (keep[u])
-                                    list[running + __popc(bal & ((1u << lane) - 1u))] =
-                                        static_cast<int16_t>((w0 + u) * 32 + lane);
+                                if (keep[u]) {
+                                    const int slot_i = running + __popc(bal & ((1u << lane) - 1u));
+                                    const int n = (w0 + u) * 32 + lane;
+                                    list[slot_i] = static_cast<int16_t>(n);
+                                    idx_offs(islot)[slot_i] = (row_off + n) * H * kD * 2;
+                                }
                                 if (lane == 0)
                                     bits[w0 + u] = bal;
                                 running += __popc(bal);
@@ -557,8 +598,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             q_phase ^= 1u << qs;
             if constexpr (kFused) {
-                copy_tile_async(base + kOffQ + qs * kTileBytes, p.src[0], &bars->q_full[qs], idx_list(islot),
-                                it.qt * BM, min(BM, it.L - it.qt * BM), row_off, it.h, H, warp, lane);
+                // Q by the TMA engine (tile::gather4, four rows per lane of producer warp 0), in
+                // parallel with the K/V copies of the load/store path below
+                if (warp == 0) {
+                    if (lane == 0)
+                        mbar_arrive_expect_tx(&bars->q_full[qs], kTileBytes);
+                    __syncwarp();
+                    const int16_t *list = idx_list(islot);
+                    const int q0 = it.qt * BM, cnt = min(BM, it.L - q0);
+                    int r[4];
+#pragma unroll
+                    for (int k2 = 0; k2 < 4; ++k2) {
+                        const int i = 4 * lane + k2;
+                        r[k2] = row_off + list[q0 + (i < cnt ? i : 0)];
+                    }
+                    tma_gather4(base + kOffQ + qs * kTileBytes + 512 * lane, &tm_q, &bars->q_full[qs], it.h * kD, r[0],
+                                r[1], r[2], r[3]);
+                }
             } else {
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&bars->q_full[qs], kTileBytes);
@@ -575,10 +631,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 kv_phase ^= 1u << ks;
                 if constexpr (kFused) {
                     const int cnt = min(BN, it.L - kc * BN);
-                    copy_tile_async(base + kOffK + ks * kTileBytes, p.src[1], &bars->kv_full[ks], idx_list(islot),
-                                    kc * BN, cnt, row_off, it.h, H, warp, lane);
-                    copy_tile_async(base + kOffV + ks * kTileBytes, p.src[2], &bars->kv_full[ks], idx_list(islot),
-                                    kc * BN, cnt, row_off, it.h, H, warp, lane);
+                    copy_tile_async(base + kOffK + ks * kTileBytes, p.src[1] + it.h * kD * 2, &bars->kv_full[ks],
+                                    idx_offs(islot), kc * BN, cnt, warp, lane);
+                    copy_tile_async(base + kOffV + ks * kTileBytes, p.src[2] + it.h * kD * 2, &bars->kv_full[ks],
+                                    idx_offs(islot), kc * BN, cnt, warp, lane);
                 } else {
                     if (lane == 0)
                         mbar_arrive_expect_tx(&bars->kv_full[ks], 2 * kTileBytes);
@@ -1046,7 +1102,7 @@ cudaError_t launch_attend(const AttendArgs &a, int num_sms, cudaStream_t stream)
     p.out_dt = a.out_dt;
     p.err = a.err;
     p.wait_ns = a.wait_ns;
-    const int smem = kSmemFixed + 2 * (a.B + 1) * 4;
+    const int smem = smem_bytes<false>(a.B);
     return launch_variant<false>(a.in_bf16, tq, tk, tv, p, grid_for(a.B, a.H, a.max_seqlen, num_sms), smem, stream);
 }
 
@@ -1077,7 +1133,7 @@ cudaError_t launch_fused(const FusedArgs &a, int num_sms, cudaStream_t stream)
     p.out_dt = a.out_dt;
     p.err = a.err;
     p.wait_ns = a.wait_ns;
-    const int smem = kSmemFixed + 2 * (a.B + 1) * 4;
+    const int smem = smem_bytes<true>(a.B);
     return launch_variant<true>(a.in_bf16, tq, tk, tv, p, grid_for(a.B, a.H, a.N, num_sms), smem, stream);
 }
 

@@ -47,8 +47,10 @@ struct FusedArgs {
     uint64_t wait_ns;
 };
 
-// Largest N the single-launch path accepts (its kept-row list lives in shared memory).
-constexpr int kFusedMaxN = 2048;
+// Largest N and B the single-launch path accepts (its kept-row lists and per-image tables live
+// in shared memory next to the Q/K/V rings).
+constexpr int kFusedMaxN = 1024;
+constexpr int kFusedMaxBatch = 4096;
 
 cudaError_t launch_fused(const FusedArgs &a, int num_sms, cudaStream_t stream);
 

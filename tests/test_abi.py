@@ -108,8 +108,8 @@ def test_fused_validation(L):
     assert f(None, FAKE, FAKE, FAKE, FAKE, None, 2, 8, 1, 64, 0.0, 1, 1, None, None) == rra.RRA_ERR_INVALID_ARG
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE + 8, None, 2, 8, 1, 64, 0.0, 1, 1, None, None) == rra.RRA_ERR_INVALID_ARG
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 8, 1, 32, 0.0, 1, 1, None, None) == rra.RRA_ERR_UNSUPPORTED
-    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 2049, 1, 64, 0.0, 1, 1, None, None) == rra.RRA_ERR_UNSUPPORTED
-    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 9000, 8, 1, 64, 0.0, 1, 1, None, None) == rra.RRA_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 1025, 1, 64, 0.0, 1, 1, None, None) == rra.RRA_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 4097, 8, 1, 64, 0.0, 1, 1, None, None) == rra.RRA_ERR_UNSUPPORTED
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 8, 1, 64, 0.0, 2, 2, None, None) == rra.RRA_ERR_UNSUPPORTED
 
 
