@@ -9,21 +9,20 @@
 //   * one persistent block per SM walks a list of (image, 128-row q-tile, head) work items
 //     derived from cu_seqlens on the device, so the host never learns T; each item is taken
 //     in steps of 128 keys;
-//   * the block owns all 512 TMEM columns: two S buffers (fp32 [128 x 128]) and two O buffers
-//     (fp32 [128 x 64]), so the tensor core computes S of the next step while the softmax
-//     warps work on the current one, and PV of one item runs under the next item's softmax;
+//   * the block owns all 512 TMEM columns: an S buffer (fp32 [128 x 128]) and an O buffer
+//     (fp32 [128 x 80]) for each of two softmax groups that work on alternate items, so one
+//     group's QK^T and PV run on the tensor core while the other group's softmax runs;
 //   * warps specialise:
 //       warps 0..2  producer: Q tiles (2-slot ring) and 128-key K/V chunks (3-slot ring) of one
 //                   head; on the packed path warp 0 fetches them straight from the [T, H, 64]
 //                   layout with TMA (3-D tensor map, head = coordinate, 128-byte swizzle);
 //       warp 3      tensor-core issuer: S = Q K^T (smem x smem) and O += P V (P from TMEM as the
 //                   A operand), fp32 accumulation, completion signalled through mbarriers;
-//       warps 4..11 softmax: a pair of warps owns each quarter of the rows (TMEM lanes); within
-//                   a step the two warps take alternate 32-key slices, keep them in registers
-//                   for both passes (row max, then exponentials), exchange the row max once,
-//                   write P back over their own S columns, and rescale their half of O in TMEM
-//                   when a row's running max rises; an item's normalise-and-store epilogue runs
-//                   after the next item's softmax, when its last PV has long finished;
+//       warps 4..11 softmax: two groups of four warps take alternate items; in a group, thread
+//                   r owns row r of its S and O buffers (TMEM lane r), so the row max and row sum
+//                   need no exchange; it writes P back over its own S columns, rescales its row
+//                   of O in TMEM when the running max rises, and finally normalises and stores
+//                   the row -- while the other group's QK^T, softmax and PV run alongside;
 //   * for bf16 inputs P is split into a bf16 head and a bf16 remainder (two PV MMAs), which
 //     keeps P at ~16 significant bits; fp16 P (11 bits) is used as is;
 //   * the PV MMA runs with N = 80: the 64 columns of V plus a constant tile whose first column
@@ -59,7 +58,9 @@ constexpr int kThreads = 384;           // 12 warps: 3 x producer, MMA, 8 x soft
 constexpr int kProducerWarps = 3;       // fused path: all three copy; packed path: warp 0 issues TMA
 constexpr int kMmaWarp = 3;
 constexpr int kSoftmaxWarp0 = 4;
-constexpr int kSoftmaxWarps = 8;
+constexpr int kSoftmaxWarps = 8;        // two groups of four, one per TMEM lane quarter each
+constexpr int kGroupWarps = 4;
+static_assert(kSoftmaxWarp0 + kSoftmaxWarps == kThreads / 32 && kSoftmaxWarps == 2 * kGroupWarps, "warp roles");
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: S buffers at 0 and 128 (the P of each 32-key slice is written back over the
 // slice's own S columns: 16 columns of packed head values, then 16 of bf16 remainders), O
@@ -78,13 +79,12 @@ constexpr uint32_t kOffK = kOffQ + kQStages * kTileBytes;
 constexpr uint32_t kOffV = kOffK + kKVStages * kTileBytes;
 constexpr uint32_t kOffOnes = kOffV + kKVStages * kTileBytes;   // [128 keys x 64] MN-major, column 0 = 1
 constexpr uint32_t kOffBar = kOffOnes + kTileBytes;
-constexpr uint32_t kOffRed = kOffBar + 512;             // [2 parities][2 halves][128] row max
 // fused: 4 slots, each the kept positions of one item's image (int16 [kFusedMaxN]), the byte
 // offsets of those padded rows' first head (int32 [kFusedMaxN]) and the kept-bit mask
 // (uint32 [kFusedMaxN / 32])
 constexpr int kIdxSlots = 4;
 constexpr uint32_t kIdxSlotBytes = kFusedMaxN * 2 + kFusedMaxN * 4 + kFusedMaxN / 8;
-constexpr uint32_t kOffIdx = kOffRed + 2 * 2 * 128 * 4;
+constexpr uint32_t kOffIdx = kOffBar + 512;
 // tile_pre[B+1], then cu[B+1]: after the list slots on the fused path, in their place otherwise
 template <bool kFused>
 constexpr uint32_t off_tile()
@@ -220,12 +220,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-// Barrier between the two softmax warps that share a quarter of the rows (64 threads).
-__device__ __forceinline__ void pair_sync(int quarter)
-{
-    asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
-}
-
 // Exponentials of one 32-key slice of a row (keys c .. c+31, those >= nk masked to 0), written
 // back over the slice's own TMEM columns as the PV A operand: 16 columns of packed head values
 // (bf16 or fp16 pairs), then for bf16 16 columns of remainders.
@@ -283,6 +277,40 @@ __device__ __forceinline__ float slice_max(const uint32_t (&r)[32], int c, int n
     return fmaxf(mx, t[0]);
 }
 
+// Store 32 normalised output values (columns col0 .. col0+31 of one row) in the output type.
+__device__ __forceinline__ void store_row(const Params &p, int64_t off, const uint32_t (&r)[32], int col0, float inv)
+{
+    if (p.out_dt == RRA_F32) {
+        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off + col0);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            dst[j] = make_float4(__uint_as_float(r[4 * j]) * inv, __uint_as_float(r[4 * j + 1]) * inv,
+                                 __uint_as_float(r[4 * j + 2]) * inv, __uint_as_float(r[4 * j + 3]) * inv);
+    } else {
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + off + col0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                f[e] = __uint_as_float(r[8 * j + e]) * inv;
+            uint4 w;
+            if (p.out_dt == RRA_BF16) {
+                w.x = pack_bf16(f[0], f[1]);
+                w.y = pack_bf16(f[2], f[3]);
+                w.z = pack_bf16(f[4], f[5]);
+                w.w = pack_bf16(f[6], f[7]);
+            } else {
+                w.x = pack_f16(f[0], f[1]);
+                w.y = pack_f16(f[2], f[3]);
+                w.z = pack_f16(f[4], f[5]);
+                w.w = pack_f16(f[6], f[7]);
+            }
+            dst[j] = w;
+        }
+    }
+}
+
 // One PV step as the MMA warp sees it.
 struct PvStep {
     int sb, ks, ob, kc, nk16;
@@ -330,7 +358,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars *bars = reinterpret_cast<Bars *>(base + kOffBar);
-    float *red = reinterpret_cast<float *>(base + kOffRed);            // row max exchange [2][2][128]
     int32_t *tile_pre = reinterpret_cast<int32_t *>(base + off_tile<kFused>());  // [B+1]
     int32_t *cu_s = tile_pre + (p.B + 1);                               // [B+1]
     auto idx_list = [&](int slot) { return reinterpret_cast<int16_t *>(base + kOffIdx + slot * kIdxSlotBytes); };
@@ -365,14 +392,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->s_full[s], 1);
-            mbar_init(&bars->p_full[s], kSoftmaxWarps);  // one arrival per softmax warp
+            mbar_init(&bars->p_full[s], kGroupWarps);  // one arrival per warp of softmax group s
             mbar_init(&bars->s_free[s], 1);
             mbar_init(&bars->o_full[s], 1);
-            mbar_init(&bars->o_free[s], kSoftmaxWarps);
+            mbar_init(&bars->o_free[s], kGroupWarps);
         }
         for (int s = 0; s < kIdxSlots; ++s) {
             mbar_init(&bars->idx_full[s], 1);
-            mbar_init(&bars->idx_free[s], kSoftmaxWarps);
+            mbar_init(&bars->idx_free[s], kGroupWarps);
         }
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
@@ -664,16 +691,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kMmaWarp) {
         // ================================================================ tcgen05 issuer
-        // Order: S(t) then PV(t-1), so the next step's QK^T runs while the softmax warps work.
-        // phase parities, one bit per slot / buffer
-        uint32_t q_ph = 0, kv_ph = 0, p_ph = 0, sfree_ph = 0, ofree_ph = 0;
+        // Steps (item, 128-key chunk) come in production order; item n belongs to softmax group
+        // g = n & 1, which owns S buffer g and O buffer g.  For each step the issuer issues the
+        // group's own pending PV first when the step continues the same item (the S buffer is
+        // reused), then S of the step, then the other group's pending PV -- so one group's QK^T
+        // and PV run while the other group's softmax works.
+        uint32_t q_ph = 0, kv_ph = 0, p_ph = 0, sfree_ph = 0, ofree_ph = 0;  // one bit per slot / group
         const uint32_t idPV = idesc_f16(BM, kPvN, kBF16 ? 1u : 0u, 1u);
-        // shared-memory descriptors of every ring slot, built once; stepping K inside a 128-byte
-        // swizzled row adds 32 bytes (2 units) to the start address, stepping 16 key rows adds
-        // 2048 bytes (128 units).  V descriptors carry, as leading offset, the distance to the
-        // ones tile that supplies PV columns 64..79.
-        // The start-address field is linear in the slot index (a tile is 1024 units of 16 bytes);
-        // for V the leading offset to the ones tile shrinks by the same amount.
+        // shared-memory descriptors of the ring slots: stepping K inside a 128-byte swizzled row
+        // adds 32 bytes (2 units) to the start address, stepping 16 key rows adds 2048 bytes (128
+        // units), and a slot is 1024 units further.  V descriptors carry, as leading offset, the
+        // distance to the ones tile that supplies PV columns 64..79.
         const uint64_t qdesc0 = smem_desc_sw128(smem_addr(base + kOffQ), 16, 1024);
         const uint64_t kdesc0 = smem_desc_sw128(smem_addr(base + kOffK), 16, 1024);
         const uint64_t vdesc0 = smem_desc_sw128(smem_addr(base + kOffV), kOffOnes - kOffV, 1024);
@@ -681,27 +709,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto v_desc = [&](int slot) {
             return slot_desc(vdesc0, slot) - (static_cast<uint64_t>(slot) * (kTileBytes >> 4) << 16);
         };
-        int qs = 0, ks = 0;
-        int t = 0, n = 0;
-        bool have_prev = false;
-        PvStep prev{0, 0, 0, 0, 0, false};
+        int qs = 0, ks = 0, n = 0;
+        // per-group pending PV (registers: selected by value, never indexed)
+        PvStep pend0{0, 0, 0, 0, 0, false}, pend1{0, 0, 0, 0, 0, false};
+        uint32_t has_pend = 0, s_used = 0;  // one bit per group
         bool ok = true;
 
-        auto issue_pv = [&](const PvStep &u) -> bool {
-            if (!warp_wait(&bars->p_full[u.sb], (p_ph >> u.sb) & 1u, bars, p))
+        auto issue_pv = [&](int g) -> bool {
+            const PvStep u = g ? pend1 : pend0;
+            if (!warp_wait(&bars->p_full[g], (p_ph >> g) & 1u, bars, p))
                 return false;
-            p_ph ^= 1u << u.sb;
+            p_ph ^= 1u << g;
             if (u.wait_free) {
-                // first PV of an item: the O buffer's previous item must have been read out
-                if (!warp_wait(&bars->o_free[u.ob], (ofree_ph >> u.ob) & 1u, bars, p))
+                // first PV of an item: the group's previous item must have been read out
+                if (!warp_wait(&bars->o_free[g], (ofree_ph >> g) & 1u, bars, p))
                     return false;
-                ofree_ph ^= 1u << u.ob;
+                ofree_ph ^= 1u << g;
             }
             if (lane == 0) {
                 tc_fence_after();
                 const uint64_t vd = v_desc(u.ks);
-                const uint32_t dO = tmem + kColO0 + kOCols * u.ob;
-                const uint32_t aP = tmem + kColS0 + 128 * u.sb;
+                const uint32_t dO = tmem + kColO0 + kOCols * g;
+                const uint32_t aP = tmem + kColS0 + 128 * g;
                 const int nj = u.nk16 >> 4;
                 // keys 16j..16j+15 live in slice j/2: head part at column 32(j/2) + 8(j%2),
                 // remainder 16 columns further
@@ -715,17 +744,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (j < nj)
                             mma_ts(dO, aP + 32 * (j >> 1) + 8 * (j & 1) + 16, vd + 128 * j, idPV, 1u);
                 }
-                mma_commit(&bars->o_full[u.ob]);
-                mma_commit(&bars->s_free[u.sb]);
+                mma_commit(&bars->o_full[g]);
+                mma_commit(&bars->s_free[g]);
                 mma_commit(&bars->kv_empty[u.ks]);
             }
             __syncwarp();
+            has_pend &= ~(1u << g);
             return true;
         };
 
-        for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+        for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++n) {
             const Item it = decode_item(item, H, B, tile_pre, cu_s);
             const int nkc = (it.L + BN - 1) / BN;
+            const int g = n & 1;
             ok = warp_wait(&bars->q_full[qs], (q_ph >> qs) & 1u, bars, p);
             if (!ok)
                 break;
@@ -734,7 +765,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kc = 0; kc < nkc; ++kc) {
                 const int nk = min(BN, it.L - kc * BN);
                 const int nk16 = (nk + 15) & ~15;
-                const int sb = t & 1;
                 ok = warp_wait(&bars->kv_full[ks], (kv_ph >> ks) & 1u, bars, p);
                 if (!ok)
                     break;
@@ -747,43 +777,52 @@ __global__ void __launch_bounds__(kThreads, 1)
                     fence_proxy_async_smem();
                 }
                 __syncwarp();
-                // S buffer sb holds P of step t-2 until that PV completes
-                if (t >= 2) {
-                    ok = warp_wait(&bars->s_free[sb], (sfree_ph >> sb) & 1u, bars, p);
+                // the previous chunk of this item: its PV must be issued (and finish) before S
+                // overwrites the group's S buffer, which holds that chunk's P
+                if (has_pend & (1u << g)) {
+                    ok = issue_pv(g);
                     if (!ok)
                         break;
-                    sfree_ph ^= 1u << sb;
+                }
+                if (s_used & (1u << g)) {
+                    ok = warp_wait(&bars->s_free[g], (sfree_ph >> g) & 1u, bars, p);
+                    if (!ok)
+                        break;
+                    sfree_ph ^= 1u << g;
                 }
                 if (lane == 0) {
                     tc_fence_after();
                     if constexpr (kFused)
-                        fence_proxy_async_smem();  // Q/K/V arrived through cp.async (generic proxy)
+                        fence_proxy_async_smem();  // K/V arrived through cp.async (generic proxy)
                     const uint64_t kd = slot_desc(kdesc0, ks);
                     const uint32_t idS = idesc_f16(BM, nk16, kBF16 ? 1u : 0u, 0u);
 #pragma unroll
                     for (int kk = 0; kk < kD / 16; ++kk)
-                        mma_ss(tmem + kColS0 + 128 * sb, qd + 2 * kk, kd + 2 * kk, idS, kk > 0 ? 1u : 0u);
-                    mma_commit(&bars->s_full[sb]);
+                        mma_ss(tmem + kColS0 + 128 * g, qd + 2 * kk, kd + 2 * kk, idS, kk > 0 ? 1u : 0u);
+                    mma_commit(&bars->s_full[g]);
                     if (kc == nkc - 1)
                         mma_commit(&bars->q_empty[qs]);  // last read of this Q tile
                 }
                 __syncwarp();
-                if (have_prev) {
-                    ok = issue_pv(prev);
+                s_used |= 1u << g;
+                const PvStep step{g, ks, g, kc, nk16, kc == 0 && n >= 2};
+                if (g)
+                    pend1 = step;
+                else
+                    pend0 = step;
+                has_pend |= 1u << g;
+                if (has_pend & (1u << (g ^ 1))) {
+                    ok = issue_pv(g ^ 1);
                     if (!ok)
                         break;
                 }
-                // this step's PV: O buffer n&1, released by the epilogue of item n-2
-                prev = PvStep{sb, ks, n & 1, kc, nk16, kc == 0 && n >= 2};
-                have_prev = true;
-                ++t;
                 ks = (ks + 1 == kKVStages) ? 0 : ks + 1;
             }
-            ++n;
             qs = (qs + 1 == kQStages) ? 0 : qs + 1;
         }
-        if (ok && have_prev)
-            issue_pv(prev);
+        for (int g = 0; ok && g < 2; ++g)
+            if (has_pend & (1u << g))
+                ok = issue_pv(g);
         // drain: every MMA this thread issued has completed
         if (lane == 0) {
             mma_commit(&bars->drain);
@@ -792,189 +831,133 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp >= kSoftmaxWarp0) {
         // ================================================================ softmax + epilogue
+        // Group g (4 warps) takes items n = g, g+2, ...; thread r of the group owns row r of
+        // S buffer g and O buffer g (its TMEM lane), so row max and row sum need no exchange.
         const int q4 = warp & 3;                     // TMEM lane quarter of this warp
-        const int hf = (warp - kSoftmaxWarp0) >> 2;  // which of the pair: slices hf, hf+2; O columns 32hf..
+        const int g = (warp - kSoftmaxWarp0) >> 2;   // softmax group
         const int row = q4 * 32 + lane;              // row of S / O owned by this thread
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-        float *red_max = red;                        // [2][2][128]
-        uint32_t s_ph = 0, o_ph = 0;  // one bit per buffer
-        int t = 0, n = 0, n_epi = 0;
+        const uint32_t sbase = lane_base + kColS0 + 128 * g;
+        const uint32_t obase = lane_base + kColO0 + kOCols * g;
+        uint32_t s_ph = 0, o_ph = 0, idxf_ph = 0;
         bool ok = true;
-
-        // deferred epilogue of the previous item
-        bool pending = false;
-        int pend_row0 = 0, pend_h = 0, pend_qrows = 0, pend_ob = 0, pend_b = 0, pend_q0 = 0, pend_slot = 0;
-        uint32_t idxf_ph = 0;
-        auto epilogue = [&]() -> bool {
-            if (!warp_wait(&bars->o_full[pend_ob], (o_ph >> pend_ob) & 1u, bars, p))
-                return false;
-            o_ph ^= 1u << pend_ob;
-            if constexpr (kFused) {
-                // the producer's list of this item (written long before; this orders the reads)
-                if (!warp_wait(&bars->idx_full[pend_slot], (idxf_ph >> pend_slot) & 1u, bars, p))
-                    return false;
-                idxf_ph ^= 1u << pend_slot;
-            }
-            tc_fence_after();
-            if (q4 * 32 < pend_qrows) {
-                uint32_t r[32], sum[1];
-                tmem_ld32(lane_base + kColO0 + kOCols * pend_ob + 32 * hf, r);
-                tmem_ld1(lane_base + kColO0 + kOCols * pend_ob + 64, sum);
-                int64_t out_row = static_cast<int64_t>(pend_row0) + row;
-                if constexpr (kFused) {
-                    // padded position of kept token (q0 + row), from the item's list slot
-                    const int r = row < pend_qrows ? row : 0;
-                    out_row = static_cast<int64_t>(pend_b) * p.N + idx_list(pend_slot)[pend_q0 + r];
-                }
-                tmem_wait_ld();
-                const float inv = 1.f / __uint_as_float(sum[0]);
-                if (row < pend_qrows) {
-                    const int64_t off = (out_row * H + pend_h) * kD + 32 * hf;
-                    if (p.out_dt == RRA_F32) {
-                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            dst[j] = make_float4(__uint_as_float(r[4 * j]) * inv, __uint_as_float(r[4 * j + 1]) * inv,
-                                                 __uint_as_float(r[4 * j + 2]) * inv,
-                                                 __uint_as_float(r[4 * j + 3]) * inv);
-                    } else {
-                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + off);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            float f[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                f[e] = __uint_as_float(r[8 * j + e]) * inv;
-                            uint4 w;
-                            if (p.out_dt == RRA_BF16) {
-                                w.x = pack_bf16(f[0], f[1]);
-                                w.y = pack_bf16(f[2], f[3]);
-                                w.z = pack_bf16(f[4], f[5]);
-                                w.w = pack_bf16(f[6], f[7]);
-                            } else {
-                                w.x = pack_f16(f[0], f[1]);
-                                w.y = pack_f16(f[2], f[3]);
-                                w.z = pack_f16(f[4], f[5]);
-                                w.w = pack_f16(f[6], f[7]);
-                            }
-                            dst[j] = w;
-                        }
-                    }
-                }
-            }
-            ++n_epi;
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bars->o_free[pend_ob]);
-                if constexpr (kFused)
-                    mbar_arrive(&bars->idx_free[pend_slot]);
-            }
-            pending = false;
-            return true;
-        };
-
-        for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+        int n = 0;
+        for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++n) {
+            if ((n & 1) != g)
+                continue;
             const Item it = decode_item(item, H, B, tile_pre, cu_s);
             const int nkc = (it.L + BN - 1) / BN;
             const int q0 = it.qt * BM;
             const int qrows = min(BM, it.L - q0);
             const bool warp_active = q4 * 32 < qrows;
-            const int ob = n & 1;
             float m_run = -INFINITY;
             for (int kc = 0; kc < nkc; ++kc) {
                 const int nk = min(BN, it.L - kc * BN);
                 const int nk16 = (nk + 15) & ~15;
-                const int sb = t & 1;
-                const uint32_t sbase = lane_base + kColS0 + 128 * sb;
-                ok = warp_wait(&bars->s_full[sb], (s_ph >> sb) & 1u, bars, p);
+                ok = warp_wait(&bars->s_full[g], s_ph, bars, p);
                 if (!ok)
                     break;
-                s_ph ^= 1u << sb;
+                s_ph ^= 1u;
                 tc_fence_after();
-                const int c0 = 32 * hf, c1 = c0 + 64;
-                uint32_t r0[32], r1[32];
                 float m_new = m_run;
                 if (warp_active) {
-                    // both slices of this warp in registers for both passes
-                    if (c0 < nk16)
-                        tmem_ld32(sbase + c0, r0);
-                    if (c1 < nk16)
-                        tmem_ld32(sbase + c1, r1);
-                    tmem_wait_ld();
+                    // pass 1: row max, two 32-key slices per TMEM round trip
                     float mx = -INFINITY;
-                    if (c0 < nk16)
-                        mx = slice_max(r0, c0, nk, mx);
-                    if (c1 < nk16)
-                        mx = slice_max(r1, c1, nk, mx);
-                    float *rm = red_max + (t & 1) * 256;
-                    rm[hf * 128 + row] = mx;
-                    pair_sync(q4);
-                    m_new = fmaxf(m_run, fmaxf(rm[row], rm[128 + row]));
+                    for (int c = 0; c < nk16; c += 64) {
+                        uint32_t r0[32], r1[32];
+                        tmem_ld32(sbase + c, r0);
+                        if (c + 32 < nk16)
+                            tmem_ld32(sbase + c + 32, r1);
+                        tmem_wait_ld();
+                        mx = slice_max(r0, c, nk, mx);
+                        if (c + 32 < nk16)
+                            mx = slice_max(r1, c + 32, nk, mx);
+                    }
+                    m_new = fmaxf(m_run, mx);
                 }
-                // later steps of an item: the previous PV has landed in O; rescale rows whose max rose
+                // later chunks: the previous PV has landed in O; rescale rows whose max rose
                 if (kc > 0) {
-                    ok = warp_wait(&bars->o_full[ob], (o_ph >> ob) & 1u, bars, p);
+                    ok = warp_wait(&bars->o_full[g], o_ph, bars, p);
                     if (!ok)
                         break;
-                    o_ph ^= 1u << ob;
+                    o_ph ^= 1u;
                     tc_fence_after();
                     if (warp_active && __any_sync(0xffffffffu, m_new > m_run)) {
-                        // each warp of the pair rescales 32 output columns; the first also the sum
                         const float alpha = ex2_approx((m_run - m_new) * p.scale_log2);
-                        const uint32_t oaddr = lane_base + kColO0 + kOCols * ob + 32 * hf;
                         uint32_t r[32], rs[16];
-                        tmem_ld32(oaddr, r);
-                        if (hf == 0)
-                            tmem_ld16(lane_base + kColO0 + kOCols * ob + 64, rs);
+                        tmem_ld16(obase + 64, rs);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-                        tmem_st32(oaddr, r);
-                        if (hf == 0) {
+                        for (int j = 0; j < 16; ++j)
+                            rs[j] = __float_as_uint(__uint_as_float(rs[j]) * alpha);
+                        tmem_st16(obase + 64, rs);
 #pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                rs[j] = __float_as_uint(__uint_as_float(rs[j]) * alpha);
-                            tmem_st16(lane_base + kColO0 + kOCols * ob + 64, rs);
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            tmem_ld32(obase + 32 * h2, r);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
+                            tmem_st32(obase + 32 * h2, r);
                         }
                     }
                 }
                 if (warp_active) {
                     m_run = m_new;
                     const float neg_m = -m_new * p.scale_log2;
-                    if (c0 < nk16)
-                        softmax_slice<kBF16>(r0, c0, nk, p.scale_log2, neg_m, sbase + c0);
-                    if (c1 < nk16)
-                        softmax_slice<kBF16>(r1, c1, nk, p.scale_log2, neg_m, sbase + c1);
+                    // pass 2: P = exp2(scale*log2e*(s - m)) written back over each slice's S columns
+                    for (int c = 0; c < nk16; c += 32) {
+                        uint32_t r[32];
+                        tmem_ld32(sbase + c, r);
+                        tmem_wait_ld();
+                        softmax_slice<kBF16>(r, c, nk, p.scale_log2, neg_m, sbase + c);
+                    }
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
-                    mbar_arrive(&bars->p_full[sb]);
-                ++t;
+                    mbar_arrive(&bars->p_full[g]);
             }
             if (!ok)
                 break;
-            // the previous item's PV is long done: store it now, under this item's PV
-            if (pending) {
-                ok = epilogue();
+            // epilogue: the last PV has landed; normalise by the row sum (O column 64) and store
+            ok = warp_wait(&bars->o_full[g], o_ph, bars, p);
+            if (!ok)
+                break;
+            o_ph ^= 1u;
+            const int islot = n & (kIdxSlots - 1);
+            if constexpr (kFused) {
+                ok = warp_wait(&bars->idx_full[islot], (idxf_ph >> islot) & 1u, bars, p);
                 if (!ok)
                     break;
+                idxf_ph ^= 1u << islot;
             }
-            pending = true;
-            pend_row0 = it.seq0 + q0;
-            pend_b = it.b;
-            pend_q0 = q0;
-            pend_slot = n & (kIdxSlots - 1);
-            pend_h = it.h;
-            pend_qrows = qrows;
-            pend_ob = ob;
-            ++n;
+            tc_fence_after();
+            if (warp_active) {
+                uint32_t r0[32], r1[32], sum[1];
+                tmem_ld32(obase, r0);
+                tmem_ld32(obase + 32, r1);
+                tmem_ld1(obase + 64, sum);
+                int64_t out_row = static_cast<int64_t>(it.seq0) + q0 + row;
+                if constexpr (kFused)
+                    out_row = static_cast<int64_t>(it.b) * p.N + idx_list(islot)[q0 + (row < qrows ? row : 0)];
+                tmem_wait_ld();
+                if (row < qrows) {
+                    const float inv = 1.f / __uint_as_float(sum[0]);
+                    const int64_t off = (out_row * H + it.h) * kD;
+                    store_row(p, off, r0, 0, inv);
+                    store_row(p, off, r1, 32, inv);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars->o_free[g]);
+                if constexpr (kFused)
+                    mbar_arrive(&bars->idx_free[islot]);
+            }
         }
-        if (ok && pending)
-            epilogue();
     }
 
     tc_fence_before();
