@@ -252,7 +252,10 @@ def run_reference(args):
 # ------------------------------------------------------------------------------------ GPU arm
 
 class Pipeline:
-    """Device buffers + one CUDA graph of the whole call (all stages), with per-kernel events."""
+    """Device buffers + CUDA graphs of the whole call (all stages): `graph` holds the kernels
+    alone (the timed one: kernels that follow one another may overlap their start-up through
+    programmatic dependent launch), `graph_ev` the same kernels with an event between each pair
+    (for the per-kernel breakdown; the events serialise the kernels)."""
 
     def __init__(self, w, out_dtype, stream, path):
         self.w = w
@@ -264,6 +267,7 @@ class Pipeline:
         self.ys = [torch.empty(w.B, w.N, w.H, 64, dtype=self.bufs.y.dtype, device=dev) for _ in self.masks]
         self.stream = stream
         self.graph = None
+        self.graph_ev = None
         self.events = None
 
     @property
@@ -295,18 +299,19 @@ class Pipeline:
         with torch.cuda.stream(self.stream):
             self.enqueue()
         torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            self.enqueue()
+        self.graph = g
         n_ev = len(self.kernels) * len(self.masks) + 1
         events = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_ev)]
-        g = torch.cuda.CUDAGraph()
+        ge = torch.cuda.CUDAGraph()
         try:
-            with torch.cuda.graph(g, stream=self.stream):
+            with torch.cuda.graph(ge, stream=self.stream):
                 self.enqueue(events)
-            self.graph, self.events = g, events
-        except Exception:  # event-record nodes unavailable: graph without per-kernel events
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=self.stream):
-                self.enqueue()
-            self.graph, self.events = g, None
+            self.graph_ev, self.events = ge, events
+        except Exception:  # event-record nodes unavailable: no per-kernel breakdown
+            self.graph_ev, self.events = None, None
         torch.cuda.synchronize()
 
     def kernel_times(self):
@@ -322,8 +327,9 @@ class Pipeline:
 
 
 def time_path(pipe, flush, steps, warmup, stream):
-    """Warm-up, then `steps` timed replays, each after an untimed L2 flush; per-step ms and
-    per-kernel per-launch ms."""
+    """Warm-up, then `steps` timed replays of the kernels-only graph, each after an untimed L2
+    flush (per-step ms); then as many replays of the graph with per-kernel events, same protocol
+    (per-kernel per-launch ms)."""
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for i in range(warmup):
         with torch.cuda.stream(stream):
@@ -339,9 +345,13 @@ def time_path(pipe, flush, steps, warmup, stream):
             end.record(stream)
         stream.synchronize()
         step_ms.append(start.elapsed_time(end))
-        kt = pipe.kernel_times()
-        if kt:
-            for k, v in kt.items():
+    if pipe.graph_ev is not None:
+        for i in range(steps):
+            with torch.cuda.stream(stream):
+                flush.fill_((i + 11) & 0xFF)
+                pipe.graph_ev.replay()
+            stream.synchronize()
+            for k, v in pipe.kernel_times().items():
                 kern[k].extend(v)
     return step_ms, kern
 

@@ -153,7 +153,7 @@ rra_status rra_unpack(const void *packed, const int32_t *cu_seqlens, const uint8
  *   y           device [B, N, H, d] in out_dt (in_dt or RRA_F32): kept rows receive the attention
  *               output, pruned rows are set to zero bytes
  *   cu_seqlens  device int32 [B+1] written with the running kept counts, or NULL
- *   B, N, H, d  B <= 4096, N <= 1024
+ *   B, N, H, d  B <= 4096, N <= 1024, N*H*d*2 < 2^31
  *   softmax_scale <= 0 selects 1/sqrt(d)
  *   dev_error   device int32 or NULL (only RRA_ERR_TIMEOUT can be raised)
  */

@@ -136,6 +136,8 @@ rra_status rra_pack_attend_unpack(const uint8_t *keep_mask, const void *q, const
         return RRA_ERR_UNSUPPORTED;
     if (B > rra::kFusedMaxBatch || N > rra::kFusedMaxN || H > 65535 || static_cast<int64_t>(B) * N > kMaxRows)
         return RRA_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(N) * H * d * 2 > kMaxRows)  // byte offsets inside one image are 32-bit
+        return RRA_ERR_UNSUPPORTED;
     if (!(softmax_scale == softmax_scale))
         return RRA_ERR_INVALID_ARG;
     int sms = 0;

@@ -38,8 +38,8 @@
 // in one launch (the pages' pipeline without its two copies through HBM): the block derives
 // the kept counts of every image from the keep mask itself, the producer gathers the kept rows
 // of the padded Q/K/V straight into the swizzled tiles with 16-byte cp.async (32 lanes, one
-// coalesced 128-byte row segment per 8 lanes), zero-fills the pruned rows of the padded output
-// for its (image, head), and the epilogue writes each output row back to its padded position.
+// coalesced 128-byte row segment per 8 lanes), and the epilogue writes each output row back to
+// its padded position and zero-fills the pruned rows of its (image, head).
 #include <cuda.h>
 
 #include <mutex>
@@ -220,61 +220,72 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-// Exponentials of one 32-key slice of a row (keys c .. c+31, those >= nk masked to 0), written
-// back over the slice's own TMEM columns as the PV A operand: 16 columns of packed head values
-// (bf16 or fp16 pairs), then for bf16 16 columns of remainders.
+template <bool kBF16>
+__device__ __forceinline__ void pack_pair(uint32_t (&r)[32], int i, float p0, float p1)
+{
+    if constexpr (kBF16) {
+        const uint32_t a = __float_as_uint(p0), b = __float_as_uint(p1);
+        float l0, l1;
+        sub2(l0, l1, p0, p1, __uint_as_float(a & 0xFFFF0000u), __uint_as_float(b & 0xFFFF0000u));
+        r[2 * i] = __byte_perm(a, b, 0x7632);
+        r[2 * i + 1] = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
+    } else {
+        r[2 * i] = pack_f16(p0, p1);
+    }
+}
+
+// Exponentials of one 32-key slice of a row (keys c .. c+31, those >= nk masked to 0), packed
+// in place and written back over the slice's own TMEM columns as the PV A operand: 16 columns of
+// packed head values, then for bf16 16 columns of remainders.
+//   bf16: head = the top 16 bits of each fp32 value (truncation), remainder = the exact
+//         difference truncated the same way, so head + remainder carries p to a relative error
+//         below 2^-14 and the split costs integer byte permutes only (no conversions);
+//   fp16: p rounded to nearest fp16 (11 significant bits).
+// Packed pairs land in r[2i] (head) and r[2i+1] (remainder).
 template <bool kBF16>
 __device__ __forceinline__ void softmax_slice(uint32_t (&r)[32], int c, int nk, float scale_log2, float neg_m,
                                               uint32_t taddr)
 {
     if (c + 32 <= nk) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-            r[j] = __float_as_uint(ex2_approx(fmaf(__uint_as_float(r[j]), scale_log2, neg_m)));
+        for (int i = 0; i < 16; ++i) {
+            float x0, x1;
+            fma2_scalar(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scale_log2, neg_m);
+            pack_pair<kBF16>(r, i, ex2_approx(x0), ex2_approx(x1));
+        }
     } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-            r[j] = __float_as_uint((c + j < nk) ? ex2_approx(fmaf(__uint_as_float(r[j]), scale_log2, neg_m)) : 0.f);
-    }
-    uint32_t hi[16];
-#pragma unroll
-    for (int jj = 0; jj < 16; ++jj) {
-        hi[jj] = kBF16 ? pack_bf16(__uint_as_float(r[2 * jj]), __uint_as_float(r[2 * jj + 1]))
-                       : pack_f16(__uint_as_float(r[2 * jj]), __uint_as_float(r[2 * jj + 1]));
-    }
-    tmem_st16(taddr, hi);
-    if (kBF16) {
-        uint32_t lo[16];
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-            const float a = __uint_as_float(r[2 * jj]) - __uint_as_float(hi[jj] << 16);
-            const float b = __uint_as_float(r[2 * jj + 1]) - __uint_as_float(hi[jj] & 0xFFFF0000u);
-            lo[jj] = pack_bf16(a, b);
+        for (int i = 0; i < 16; ++i) {
+            float x0, x1;
+            fma2_scalar(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scale_log2, neg_m);
+            pack_pair<kBF16>(r, i, c + 2 * i < nk ? ex2_approx(x0) : 0.f, c + 2 * i + 1 < nk ? ex2_approx(x1) : 0.f);
         }
-        tmem_st16(taddr + 16, lo);
     }
+    tmem_st16_strided<0>(taddr, r);
+    if constexpr (kBF16)
+        tmem_st16_strided<1>(taddr + 16, r);
 }
 
 __device__ __forceinline__ float slice_max(const uint32_t (&r)[32], int c, int nk, float mx)
 {
-    // pairwise tree (depth 5) rather than a 32-long dependent chain
-    float t[16];
+    // two independent chains of three-input maxima
+    float t0 = mx, t1 = -INFINITY;
     if (c + 32 <= nk) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            t[j] = fmaxf(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+        for (int j = 0; j < 32; j += 4) {
+            t0 = fmax3(t0, __uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+            t1 = fmax3(t1, __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+        }
     } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            t[j] = fmaxf(c + 2 * j < nk ? __uint_as_float(r[2 * j]) : -INFINITY,
-                         c + 2 * j + 1 < nk ? __uint_as_float(r[2 * j + 1]) : -INFINITY);
+        for (int j = 0; j < 32; j += 4) {
+            t0 = fmax3(t0, c + j < nk ? __uint_as_float(r[j]) : -INFINITY,
+                       c + j + 1 < nk ? __uint_as_float(r[j + 1]) : -INFINITY);
+            t1 = fmax3(t1, c + j + 2 < nk ? __uint_as_float(r[j + 2]) : -INFINITY,
+                       c + j + 3 < nk ? __uint_as_float(r[j + 3]) : -INFINITY);
+        }
     }
-#pragma unroll
-    for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-        for (int j = 0; j < w; ++j)
-            t[j] = fmaxf(t[j], t[j + w]);
-    return fmaxf(mx, t[0]);
+    return fmaxf(t0, t1);
 }
 
 // Store 32 normalised output values (columns col0 .. col0+31 of one row) in the output type.
@@ -313,39 +324,32 @@ __device__ __forceinline__ void store_row(const Params &p, int64_t off, const ui
 
 // One PV step as the MMA warp sees it.
 struct PvStep {
-    int sb, ks, ob, kc, nk16;
+    int ks, kc, nk16;
     bool wait_free;  // first PV of an item whose O buffer held an earlier item
 };
 
-// 2-D gather of four rows (row coordinates r0..r3) of 64 elements starting at column x.
-__device__ __forceinline__ void tma_gather4(void *smem_dst, const void *tmap, uint64_t *bar, int x, int r0, int r1,
-                                            int r2, int r3)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_addr(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_addr(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-        : "memory");
-}
-
-// Fused path: producer warp w (of kProducerWarps) copies its share of one 128-row tile of one
-// head from the padded tensor into the 128-byte-swizzled layout with 16-byte cp.async: row r of
-// the tile is padded row row_off + list[base + r] (entries at or past `count` repeat the tile's
-// first row, whose result is masked later).  The 1024 chunks go in groups of 32 (one per lane,
-// 8 lanes per 128-byte row, so each row is one coalesced segment), group g to warp g % 3.
-// Completion arrives on `bar` once per producer lane.
+// Fused path: producer warp w (of kProducerWarps) copies its share of one tile of up to 128
+// kept rows of one head from the padded tensor into the 128-byte-swizzled layout with 16-byte
+// cp.async: row r of the tile is the image's kept row base + r.  The chunks go in groups of 32
+// (one per lane, 8 lanes per 128-byte row, so each row is one coalesced segment), group g to
+// warp g % 3.  Completion arrives on `bar` once per producer lane.
 __device__ __forceinline__ void copy_tile_async(uint8_t *tile, const uint8_t *src, uint64_t *bar, const int32_t *offs,
                                                 int base, int count, int w, int lane)
 {
-    // src already points at this head's 128 bytes of padded row 0; offs[] holds row offsets
+    // src points at this head's 128 bytes of the image's padded row 0; offs[] holds the byte
+    // offsets of the kept rows from there.  Rows at or past `count` are not copied: their S
+    // columns are masked, their V rows zeroed before use, or (Q) their output never stored.
     const uint32_t tile_s = smem_addr(tile);
+    const int groups = (count * 8 + 31) >> 5;
 #pragma unroll 4
-    for (int grp = w; grp < 32; grp += kProducerWarps) {
+    for (int grp = w; grp < groups; grp += kProducerWarps) {
         const int i = lane + 32 * grp;
         const int r = i >> 3, c = i & 7;
-        const uint8_t *gsrc = src + offs[base + (r < count ? r : 0)] + c * 16;
-        const uint32_t d = tile_s + r * 128 + ((c ^ (r & 7)) << 4);
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+        if (r < count) {
+            const uint8_t *gsrc = src + offs[base + r] + c * 16;
+            const uint32_t d = tile_s + r * 128 + ((c ^ (r & 7)) << 4);
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+        }
     }
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
@@ -372,10 +376,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int B = p.B, H = p.H;
+    pdl_trigger();
 
     if (tid == 0) {
-        prefetch_tmap(&tm_q);
         if constexpr (!kFused) {
+            prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
         }
@@ -383,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // arrival per producer lane
         const uint32_t fills = kFused ? 32u * kProducerWarps : 1u;
         for (int s = 0; s < kQStages; ++s) {
-            mbar_init(&bars->q_full[s], 1);  // Q always arrives by TMA (tile, or fused: gather4)
+            mbar_init(&bars->q_full[s], fills);
             mbar_init(&bars->q_empty[s], 1);
         }
         for (int s = 0; s < kKVStages; ++s) {
@@ -423,6 +428,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
     }
 
+    // everything above is private to the block; the inputs may come from the previous kernel
+    pdl_wait();
+
     // ---- work list: tile_pre[b] = number of 128-row query tiles of images < b; cu staged too.
     if constexpr (kFused) {
         // kept tokens per image, counted from 16-byte chunks of the flat mask into cu_s[b+1]
@@ -434,15 +442,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int off = static_cast<int>(addr & 15u);
         const uint4 *m16 = reinterpret_cast<const uint4 *>(addr - off);
         const int64_t nchunks = (off + total + 15) >> 4;
-        for (int64_t j = tid; j < nchunks; j += kThreads) {
-            const int64_t s0 = j * 16 - off;  // byte index of the chunk's first byte
-            uint32_t bits = kept_bits16_(__ldg(m16 + j)) & range16_(s0, 0, total);
-            while (bits != 0u) {
-                const int64_t first = s0 + (__ffs(bits) - 1);
-                const int b = static_cast<int>(first / p.N);
-                const uint32_t in_b = bits & range16_(s0, static_cast<int64_t>(b) * p.N, static_cast<int64_t>(b + 1) * p.N);
-                atomicAdd(&cu_s[b + 1], __popc(in_b));
-                bits &= ~in_b;
+        // every thread loads its chunks first (independent loads in flight together), then the
+        // counts are added per image with one shared atomic per (warp, image) -- lanes whose
+        // chunks hit the same image are grouped with a match and summed with a warp reduction
+        constexpr int kU = 4;
+        // (the loop bound is warp-uniform: every lane takes part in the warp collectives)
+        for (int64_t jw = static_cast<int64_t>(warp) * 32 * kU; jw < nchunks; jw += kThreads * kU) {
+            const int64_t j0 = jw + lane;
+            uint4 w[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int64_t j = j0 + u * 32;
+                w[u] = j < nchunks ? __ldg(m16 + j) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int64_t s0 = (j0 + u * 32) * 16 - off;  // byte index of the chunk's first byte
+                uint32_t bits = kept_bits16_(w[u]) & range16_(s0, 0, total);
+                while (__any_sync(0xffffffffu, bits != 0u)) {
+                    int b = -1, cnt = 0;
+                    if (bits != 0u) {
+                        // total <= 2^31 - 1, so the byte index fits a 32-bit division
+                        const uint32_t first = static_cast<uint32_t>(s0 + (__ffs(bits) - 1));
+                        b = static_cast<int>(first / static_cast<uint32_t>(p.N));
+                        const uint32_t in_b =
+                            bits & range16_(s0, static_cast<int64_t>(b) * p.N, static_cast<int64_t>(b + 1) * p.N);
+                        cnt = __popc(in_b);
+                        bits &= ~in_b;
+                    }
+                    const unsigned same = __match_any_sync(0xffffffffu, b);
+                    const int sum = __reduce_add_sync(same, cnt);
+                    if (b >= 0 && lane == __ffs(same) - 1)
+                        atomicAdd(&cu_s[b + 1], sum);
+                }
             }
         }
         __syncthreads();
@@ -525,6 +557,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bars->tmem_slot;
     const int total_items = tile_pre[B] * H;
+    // work items of this block, dealt round-robin: a block's items come from unrelated images,
+    // which evens out the per-block cost
+    const int item_first = static_cast<int>(blockIdx.x);
+    const int item_end = total_items;
+    const int item_step = static_cast<int>(gridDim.x);
 
     if (warp < kProducerWarps && (kFused || warp == 0)) {
         // ================================================================ producer
@@ -537,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t q_issued = 0, kv_issued = 0;
         int qs = 0, ks = 0;
         bool ok = true;
-        for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+        for (int item = item_first; ok && item < item_end; item += item_step) {
             const Item it = decode_item(item, H, B, tile_pre, cu_s);
             const int nkc = (it.L + BN - 1) / BN;
             const int row_off = it.b * p.N;  // fused: first padded row of this image
@@ -591,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     const int slot_i = running + __popc(bal & ((1u << lane) - 1u));
                                     const int n = (w0 + u) * 32 + lane;
                                     list[slot_i] = static_cast<int16_t>(n);
-                                    idx_offs(islot)[slot_i] = (row_off + n) * H * kD * 2;
+                                    idx_offs(islot)[slot_i] = n * H * kD * 2;  // < 2^31 (checked on the host)
                                 }
                                 if (lane == 0)
                                     bits[w0 + u] = bal;
@@ -605,43 +642,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive(&bars->idx_full[islot]);
                 cur_b = it.b;
                 prev_slot = islot;
-                if (it.qt == 0) {
-                    // pruned rows of this (image, head) in the padded output become zero
-                    const int out_vecs = (p.out_dt == RRA_F32 ? 4 * kD : 2 * kD) / 16;
-                    for (int wd = warp; wd < nwords; wd += kProducerWarps) {
-                        const uint32_t pruned = ~bits[wd];
-                        const int n = wd * 32 + lane;
-                        if (n < p.N && ((pruned >> lane) & 1u)) {
-                            uint4 *y = reinterpret_cast<uint4 *>(p.out) +
-                                       (static_cast<int64_t>(row_off + n) * H + it.h) * out_vecs;
-                            for (int v2 = 0; v2 < out_vecs; ++v2)
-                                y[v2] = make_uint4(0, 0, 0, 0);
-                        }
-                    }
-                }
             }
             ok = warp_wait(&bars->q_empty[qs], ((q_phase >> qs) & 1u) ^ 1u, bars, p);
             if (!ok)
                 break;
             q_phase ^= 1u << qs;
+            // fused: this head's 128 bytes of the image's padded row 0 in Q, K, V
+            const int64_t head0 = (static_cast<int64_t>(row_off) * H + it.h) * kD * 2;
             if constexpr (kFused) {
-                // Q by the TMA engine (tile::gather4, four rows per lane of producer warp 0), in
-                // parallel with the K/V copies of the load/store path below
-                if (warp == 0) {
-                    if (lane == 0)
-                        mbar_arrive_expect_tx(&bars->q_full[qs], kTileBytes);
-                    __syncwarp();
-                    const int16_t *list = idx_list(islot);
-                    const int q0 = it.qt * BM, cnt = min(BM, it.L - q0);
-                    int r[4];
-#pragma unroll
-                    for (int k2 = 0; k2 < 4; ++k2) {
-                        const int i = 4 * lane + k2;
-                        r[k2] = row_off + list[q0 + (i < cnt ? i : 0)];
-                    }
-                    tma_gather4(base + kOffQ + qs * kTileBytes + 512 * lane, &tm_q, &bars->q_full[qs], it.h * kD, r[0],
-                                r[1], r[2], r[3]);
-                }
+                const int q0 = it.qt * BM;
+                copy_tile_async(base + kOffQ + qs * kTileBytes, p.src[0] + head0, &bars->q_full[qs], idx_offs(islot), q0,
+                                min(BM, it.L - q0), warp, lane);
             } else {
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&bars->q_full[qs], kTileBytes);
@@ -658,9 +669,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 kv_phase ^= 1u << ks;
                 if constexpr (kFused) {
                     const int cnt = min(BN, it.L - kc * BN);
-                    copy_tile_async(base + kOffK + ks * kTileBytes, p.src[1] + it.h * kD * 2, &bars->kv_full[ks],
+                    copy_tile_async(base + kOffK + ks * kTileBytes, p.src[1] + head0, &bars->kv_full[ks],
                                     idx_offs(islot), kc * BN, cnt, warp, lane);
-                    copy_tile_async(base + kOffV + ks * kTileBytes, p.src[2] + it.h * kD * 2, &bars->kv_full[ks],
+                    copy_tile_async(base + kOffV + ks * kTileBytes, p.src[2] + head0, &bars->kv_full[ks],
                                     idx_offs(islot), kc * BN, cnt, warp, lane);
                 } else {
                     if (lane == 0)
@@ -691,11 +702,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kMmaWarp) {
         // ================================================================ tcgen05 issuer
-        // Steps (item, 128-key chunk) come in production order; item n belongs to softmax group
-        // g = n & 1, which owns S buffer g and O buffer g.  For each step the issuer issues the
-        // group's own pending PV first when the step continues the same item (the S buffer is
-        // reused), then S of the step, then the other group's pending PV -- so one group's QK^T
-        // and PV run while the other group's softmax works.
+        // An event loop over two kinds of work: S = Q K^T of the next step (item, 128-key chunk)
+        // in production order, and O += P V of a step whose P its softmax group has written.
+        // Item n belongs to softmax group g = n & 1 (S buffer g, O buffer g).  Whatever is ready
+        // is issued, waiting PVs first, so a PV never queues behind the next step's loads and an
+        // S never queues behind the other group's softmax.  Readiness is polled with
+        // non-blocking barrier tests; the loop gives up (RRA_ERR_TIMEOUT) when nothing has
+        // become ready for the wait limit.
         uint32_t q_ph = 0, kv_ph = 0, p_ph = 0, sfree_ph = 0, ofree_ph = 0;  // one bit per slot / group
         const uint32_t idPV = idesc_f16(BM, kPvN, kBF16 ? 1u : 0u, 1u);
         // shared-memory descriptors of the ring slots: stepping K inside a 128-byte swizzled row
@@ -709,120 +722,158 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto v_desc = [&](int slot) {
             return slot_desc(vdesc0, slot) - (static_cast<uint64_t>(slot) * (kTileBytes >> 4) << 16);
         };
-        int qs = 0, ks = 0, n = 0;
+        auto ready = [&](uint64_t *bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_test_wait(bar, parity));
+        };
+        // the next S step
+        int item = item_first, n = 0, kc = 0, qs = 0, ks = 0, nkc = 0;
+        bool q_landed = false;
+        int it_L = item < item_end ? decode_item(item, H, B, tile_pre, cu_s).L : 0;
+        nkc = (it_L + BN - 1) / BN;
         // per-group pending PV (registers: selected by value, never indexed)
-        PvStep pend0{0, 0, 0, 0, 0, false}, pend1{0, 0, 0, 0, 0, false};
-        uint32_t has_pend = 0, s_used = 0;  // one bit per group
+        PvStep pend0{0, 0, 0, false}, pend1{0, 0, 0, false};
+        uint32_t has_pend = 0;  // group g has an S whose PV is not issued yet
+        uint32_t s_busy = 0;    // group g's S buffer waits for its last PV to complete
         bool ok = true;
-
-        auto issue_pv = [&](int g) -> bool {
-            const PvStep u = g ? pend1 : pend0;
-            if (!warp_wait(&bars->p_full[g], (p_ph >> g) & 1u, bars, p))
-                return false;
-            p_ph ^= 1u << g;
-            if (u.wait_free) {
-                // first PV of an item: the group's previous item must have been read out
-                if (!warp_wait(&bars->o_free[g], (ofree_ph >> g) & 1u, bars, p))
-                    return false;
-                ofree_ph ^= 1u << g;
-            }
-            if (lane == 0) {
-                tc_fence_after();
-                const uint64_t vd = v_desc(u.ks);
-                const uint32_t dO = tmem + kColO0 + kOCols * g;
-                const uint32_t aP = tmem + kColS0 + 128 * g;
-                const int nj = u.nk16 >> 4;
-                // keys 16j..16j+15 live in slice j/2: head part at column 32(j/2) + 8(j%2),
-                // remainder 16 columns further
+        uint64_t idle_since = 0;
+        while (true) {
+            const bool more_s = item < item_end;
+            if (!more_s && has_pend == 0)
+                break;
+            bool progressed = false;
+            // ---- PVs whose P is in TMEM: one burst per chunk (each burst of tensor-core
+            // instructions pays a start-up cost of a few hundred cycles)
 #pragma unroll
-                for (int j = 0; j < BN / 16; ++j)
-                    if (j < nj)
-                        mma_ts(dO, aP + 32 * (j >> 1) + 8 * (j & 1), vd + 128 * j, idPV, (u.kc > 0 || j > 0) ? 1u : 0u);
-                if (kBF16) {
+            for (int g = 0; g < 2; ++g) {
+                if (!((has_pend >> g) & 1u))
+                    continue;
+                const PvStep u = g ? pend1 : pend0;
+                if (!ready(&bars->p_full[g], (p_ph >> g) & 1u))
+                    continue;
+                // first PV of an item: the group's previous item must have been read out
+                if (u.wait_free && !ready(&bars->o_free[g], (ofree_ph >> g) & 1u))
+                    continue;
+                p_ph ^= 1u << g;
+                if (u.wait_free)
+                    ofree_ph ^= 1u << g;
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint64_t vd = v_desc(u.ks);
+                    const uint32_t dO = tmem + kColO0 + kOCols * g;
+                    const uint32_t aP = tmem + kColS0 + 128 * g;
+                    const int nj = u.nk16 >> 4;
+                    // keys 16j..16j+15 live in slice j/2: head part at column 32(j/2) + 8(j%2),
+                    // remainder 16 columns further
 #pragma unroll
                     for (int j = 0; j < BN / 16; ++j)
                         if (j < nj)
-                            mma_ts(dO, aP + 32 * (j >> 1) + 8 * (j & 1) + 16, vd + 128 * j, idPV, 1u);
-                }
-                mma_commit(&bars->o_full[g]);
-                mma_commit(&bars->s_free[g]);
-                mma_commit(&bars->kv_empty[u.ks]);
-            }
-            __syncwarp();
-            has_pend &= ~(1u << g);
-            return true;
-        };
-
-        for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++n) {
-            const Item it = decode_item(item, H, B, tile_pre, cu_s);
-            const int nkc = (it.L + BN - 1) / BN;
-            const int g = n & 1;
-            ok = warp_wait(&bars->q_full[qs], (q_ph >> qs) & 1u, bars, p);
-            if (!ok)
-                break;
-            q_ph ^= 1u << qs;
-            const uint64_t qd = slot_desc(qdesc0, qs);
-            for (int kc = 0; kc < nkc; ++kc) {
-                const int nk = min(BN, it.L - kc * BN);
-                const int nk16 = (nk + 15) & ~15;
-                ok = warp_wait(&bars->kv_full[ks], (kv_ph >> ks) & 1u, bars, p);
-                if (!ok)
-                    break;
-                kv_ph ^= 1u << ks;
-                uint8_t *sV = base + kOffV + ks * kTileBytes;
-                // zero V rows [nk, nk16): they enter the PV MMA with probability 0
-                if (nk < nk16) {
-                    for (int i = lane; i < (nk16 - nk) * 8; i += 32)
-                        *reinterpret_cast<uint4 *>(sV + (nk + (i >> 3)) * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
-                    fence_proxy_async_smem();
-                }
-                __syncwarp();
-                // the previous chunk of this item: its PV must be issued (and finish) before S
-                // overwrites the group's S buffer, which holds that chunk's P
-                if (has_pend & (1u << g)) {
-                    ok = issue_pv(g);
-                    if (!ok)
-                        break;
-                }
-                if (s_used & (1u << g)) {
-                    ok = warp_wait(&bars->s_free[g], (sfree_ph >> g) & 1u, bars, p);
-                    if (!ok)
-                        break;
-                    sfree_ph ^= 1u << g;
-                }
-                if (lane == 0) {
-                    tc_fence_after();
-                    if constexpr (kFused)
-                        fence_proxy_async_smem();  // K/V arrived through cp.async (generic proxy)
-                    const uint64_t kd = slot_desc(kdesc0, ks);
-                    const uint32_t idS = idesc_f16(BM, nk16, kBF16 ? 1u : 0u, 0u);
+                            mma_ts(dO, aP + 32 * (j >> 1) + 8 * (j & 1), vd + 128 * j, idPV,
+                                   (u.kc > 0 || j > 0) ? 1u : 0u);
+                    if (kBF16) {
 #pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk)
-                        mma_ss(tmem + kColS0 + 128 * g, qd + 2 * kk, kd + 2 * kk, idS, kk > 0 ? 1u : 0u);
-                    mma_commit(&bars->s_full[g]);
-                    if (kc == nkc - 1)
-                        mma_commit(&bars->q_empty[qs]);  // last read of this Q tile
+                        for (int j = 0; j < BN / 16; ++j)
+                            if (j < nj)
+                                mma_ts(dO, aP + 32 * (j >> 1) + 8 * (j & 1) + 16, vd + 128 * j, idPV, 1u);
+                    }
+                    mma_commit(&bars->o_full[g]);
+                    mma_commit(&bars->s_free[g]);
+                    mma_commit(&bars->kv_empty[u.ks]);
                 }
                 __syncwarp();
-                s_used |= 1u << g;
-                const PvStep step{g, ks, g, kc, nk16, kc == 0 && n >= 2};
-                if (g)
-                    pend1 = step;
-                else
-                    pend0 = step;
-                has_pend |= 1u << g;
-                if (has_pend & (1u << (g ^ 1))) {
-                    ok = issue_pv(g ^ 1);
-                    if (!ok)
-                        break;
-                }
-                ks = (ks + 1 == kKVStages) ? 0 : ks + 1;
+                has_pend &= ~(1u << g);
+                progressed = true;
             }
-            qs = (qs + 1 == kQStages) ? 0 : qs + 1;
+            // ---- the next S
+            if (more_s) {
+                const int g = n & 1;
+                bool go = !((has_pend >> g) & 1u);  // the S buffer still holds P that no PV has read
+                if (go && ((s_busy >> g) & 1u)) {
+                    go = ready(&bars->s_free[g], (sfree_ph >> g) & 1u);
+                    if (go) {
+                        sfree_ph ^= 1u << g;
+                        s_busy &= ~(1u << g);
+                    }
+                }
+                if (go && !q_landed) {
+                    go = ready(&bars->q_full[qs], (q_ph >> qs) & 1u);
+                    if (go) {
+                        q_ph ^= 1u << qs;
+                        q_landed = true;
+                    }
+                }
+                if (go)
+                    go = ready(&bars->kv_full[ks], (kv_ph >> ks) & 1u);
+                if (go) {
+                    kv_ph ^= 1u << ks;
+                    const int nk = min(BN, it_L - kc * BN);
+                    const int nk16 = (nk + 15) & ~15;
+                    uint8_t *sV = base + kOffV + ks * kTileBytes;
+                    // zero V rows [nk, nk16): they enter the PV MMA with probability 0
+                    if (nk < nk16) {
+                        for (int i = lane; i < (nk16 - nk) * 8; i += 32)
+                            *reinterpret_cast<uint4 *>(sV + (nk + (i >> 3)) * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+                        fence_proxy_async_smem();
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        tc_fence_after();
+                        if constexpr (kFused)
+                            fence_proxy_async_smem();  // K/V arrived through cp.async (generic proxy)
+                        const uint64_t qd = slot_desc(qdesc0, qs);
+                        const uint64_t kd = slot_desc(kdesc0, ks);
+                        const uint32_t idS = idesc_f16(BM, nk16, kBF16 ? 1u : 0u, 0u);
+#pragma unroll
+                        for (int kk = 0; kk < kD / 16; ++kk)
+                            mma_ss(tmem + kColS0 + 128 * g, qd + 2 * kk, kd + 2 * kk, idS, kk > 0 ? 1u : 0u);
+                        mma_commit(&bars->s_full[g]);
+                        if (kc == nkc - 1)
+                            mma_commit(&bars->q_empty[qs]);  // last read of this Q tile
+                    }
+                    __syncwarp();
+                    s_busy |= 1u << g;
+                    const PvStep step{ks, kc, nk16, kc == 0 && n >= 2};
+                    if (g)
+                        pend1 = step;
+                    else
+                        pend0 = step;
+                    has_pend |= 1u << g;
+                    ks = (ks + 1 == kKVStages) ? 0 : ks + 1;
+                    if (++kc == nkc) {
+                        kc = 0;
+                        qs = (qs + 1 == kQStages) ? 0 : qs + 1;
+                        q_landed = false;
+                        item += item_step;
+                        ++n;
+                        if (item < item_end) {
+                            it_L = decode_item(item, H, B, tile_pre, cu_s).L;
+                            nkc = (it_L + BN - 1) / BN;
+                        }
+                    }
+                    progressed = true;
+                }
+            }
+            if (progressed) {
+                idle_since = 0;
+                continue;
+            }
+            if (*reinterpret_cast<volatile int *>(&bars->abort)) {
+                ok = false;
+                break;
+            }
+            __nanosleep(64);  // leave issue slots to the softmax warps sharing this scheduler
+            const uint64_t now = global_timer_ns();
+            if (idle_since == 0) {
+                idle_since = now;
+            } else if (now - idle_since >= p.wait_ns) {
+                if (lane == 0) {
+                    *reinterpret_cast<volatile int *>(&bars->abort) = 1;
+                    raise_error(p.err, RRA_ERR_TIMEOUT);
+                }
+                ok = false;
+                break;
+            }
         }
-        for (int g = 0; ok && g < 2; ++g)
-            if (has_pend & (1u << g))
-                ok = issue_pv(g);
+        (void)ok;
         // drain: every MMA this thread issued has completed
         if (lane == 0) {
             mma_commit(&bars->drain);
@@ -842,7 +893,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t s_ph = 0, o_ph = 0, idxf_ph = 0;
         bool ok = true;
         int n = 0;
-        for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x, ++n) {
+        for (int item = item_first; ok && item < item_end; item += item_step, ++n) {
             if ((n & 1) != g)
                 continue;
             const Item it = decode_item(item, H, B, tile_pre, cu_s);
@@ -859,23 +910,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 s_ph ^= 1u;
                 tc_fence_after();
+                // pass 1, row max: two 32-key slices per TMEM round trip (a rolled loop: every
+                // slice runs the same code, which keeps the kernel's instruction footprint small)
                 float m_new = m_run;
                 if (warp_active) {
-                    // pass 1: row max, two 32-key slices per TMEM round trip
                     float mx = -INFINITY;
-                    for (int c = 0; c < nk16; c += 64) {
-                        uint32_t r0[32], r1[32];
-                        tmem_ld32(sbase + c, r0);
-                        if (c + 32 < nk16)
-                            tmem_ld32(sbase + c + 32, r1);
-                        tmem_wait_ld();
-                        mx = slice_max(r0, c, nk, mx);
-                        if (c + 32 < nk16)
-                            mx = slice_max(r1, c + 32, nk, mx);
+#pragma unroll 1
+                    for (int c = 0; c < nk; c += 64) {
+                        uint32_t ra[32], rb[32];
+                        tmem_ld32(sbase + c, ra);
+                        tmem_ld32(sbase + c + 32, rb);  // columns past the chunk are ignored below
+                        tmem_wait_ld_dep(ra);
+                        tmem_wait_ld_dep(rb);
+                        mx = slice_max(ra, c, nk, mx);
+                        if (c + 32 < nk)
+                            mx = slice_max(rb, c + 32, nk, mx);
                     }
                     m_new = fmaxf(m_run, mx);
                 }
                 // later chunks: the previous PV has landed in O; rescale rows whose max rose
+                // (before any P of this chunk is handed over, so no PV of it can start earlier)
                 if (kc > 0) {
                     ok = warp_wait(&bars->o_full[g], o_ph, bars, p);
                     if (!ok)
@@ -884,33 +938,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     if (warp_active && __any_sync(0xffffffffu, m_new > m_run)) {
                         const float alpha = ex2_approx((m_run - m_new) * p.scale_log2);
-                        uint32_t r[32], rs[16];
-                        tmem_ld16(obase + 64, rs);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            rs[j] = __float_as_uint(__uint_as_float(rs[j]) * alpha);
-                        tmem_st16(obase + 64, rs);
-#pragma unroll
-                        for (int h2 = 0; h2 < 2; ++h2) {
-                            tmem_ld32(obase + 32 * h2, r);
+#pragma unroll 1
+                        for (uint32_t c = 0; c < kPvN; c += 16) {
+                            uint32_t o[16];
+                            tmem_ld16(obase + c, o);
                             tmem_wait_ld();
 #pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-                            tmem_st32(obase + 32 * h2, r);
+                            for (int j = 0; j < 16; ++j)
+                                o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                            tmem_st16(obase + c, o);
                         }
                     }
                 }
+                m_run = m_new;
+                const float neg_m = -m_new * p.scale_log2;
+                // pass 2: P = exp2(scale*log2e*(s - m)), one 32-key slice per round trip
                 if (warp_active) {
-                    m_run = m_new;
-                    const float neg_m = -m_new * p.scale_log2;
-                    // pass 2: P = exp2(scale*log2e*(s - m)) written back over each slice's S columns
+#pragma unroll 1
                     for (int c = 0; c < nk16; c += 32) {
-                        uint32_t r[32];
-                        tmem_ld32(sbase + c, r);
-                        tmem_wait_ld();
-                        softmax_slice<kBF16>(r, c, nk, p.scale_log2, neg_m, sbase + c);
+                        uint32_t ra[32];
+                        tmem_ld32(sbase + c, ra);
+                        tmem_wait_ld_dep(ra);
+                        softmax_slice<kBF16>(ra, c, nk, p.scale_log2, neg_m, sbase + c);
                     }
                 }
                 tmem_wait_st();
@@ -939,11 +988,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(obase, r0);
                 tmem_ld32(obase + 32, r1);
                 tmem_ld1(obase + 64, sum);
-                int64_t out_row = static_cast<int64_t>(it.seq0) + q0 + row;
-                if constexpr (kFused)
-                    out_row = static_cast<int64_t>(it.b) * p.N + idx_list(islot)[q0 + (row < qrows ? row : 0)];
                 tmem_wait_ld();
                 if (row < qrows) {
+                    int64_t out_row = static_cast<int64_t>(it.seq0) + q0 + row;
+                    if constexpr (kFused)
+                        out_row = static_cast<int64_t>(it.b) * p.N + idx_list(islot)[q0 + row];
                     const float inv = 1.f / __uint_as_float(sum[0]);
                     const int64_t off = (out_row * H + it.h) * kD;
                     store_row(p, off, r0, 0, inv);
@@ -952,9 +1001,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
+            if (lane == 0)
                 mbar_arrive(&bars->o_free[g]);
-                if constexpr (kFused)
+            if constexpr (kFused) {
+                if (it.qt == 0) {
+                    // pruned rows of this (image, head) in the padded output become zero: 16-byte
+                    // stores, consecutive threads along a row
+                    const uint32_t *bits = idx_bits(islot);
+                    const int lg = p.out_dt == RRA_F32 ? 4 : 3;  // log2 of 16-byte vectors per head row
+                    const int nvec = p.N << lg;
+                    for (int i = q4 * 32 + lane; i < nvec; i += kGroupWarps * 32) {
+                        const int tok = i >> lg;
+                        if (!((bits[tok >> 5] >> (tok & 31)) & 1u))
+                            reinterpret_cast<uint4 *>(p.out)[(((static_cast<int64_t>(it.b) * p.N + tok) * H + it.h) << lg) +
+                                                             (i & ((1 << lg) - 1))] = make_uint4(0, 0, 0, 0);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0)
                     mbar_arrive(&bars->idx_free[islot]);
             }
         }
@@ -1006,24 +1070,6 @@ bool make_tmap(CUtensorMap *map, const void *ptr, int64_t capacity, int H, bool 
     return r == CUDA_SUCCESS;
 }
 
-// Padded [rows, H*64] 16-bit tensor seen as 2-D (element, token row) for tile::gather4: the box
-// is one row high and 64 elements (one head) wide.
-bool make_gather_tmap(CUtensorMap *map, const void *ptr, int64_t rows, int H, bool bf16)
-{
-    EncodeTiledFn enc = get_encode_fn();
-    if (enc == nullptr)
-        return false;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H) * kD, static_cast<cuuint64_t>(rows)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * kD * 2};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kD), 1u};
-    const cuuint32_t estr[2] = {1u, 1u};
-    const CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                           const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 template <bool kBF16, bool kFused>
 cudaError_t set_smem_attr(int bytes)
 {
@@ -1049,11 +1095,9 @@ cudaError_t launch_variant(bool bf16, const CUtensorMap &tq, const CUtensorMap &
     cudaError_t e = bf16 ? set_smem_attr<true, kFused>(smem) : set_smem_attr<false, kFused>(smem);
     if (e != cudaSuccess)
         return e;
-    if (bf16)
-        attend_kernel<true, kFused><<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(tq, tk, tv, p);
-    else
-        attend_kernel<false, kFused><<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(tq, tk, tv, p);
-    return cudaGetLastError();
+    const dim3 g(static_cast<unsigned>(grid)), blk(kThreads);
+    return bf16 ? launch_pdl(attend_kernel<true, kFused>, g, blk, smem, stream, tq, tk, tv, p)
+                : launch_pdl(attend_kernel<false, kFused>, g, blk, smem, stream, tq, tk, tv, p);
 }
 
 int64_t grid_for(int B, int H, int max_seqlen, int num_sms)
@@ -1097,10 +1141,7 @@ cudaError_t launch_fused(const FusedArgs &a, int num_sms, cudaStream_t stream)
         return cudaSuccess;
     }
     const int64_t rows = static_cast<int64_t>(a.B) * a.N;
-    alignas(64) CUtensorMap tq, tk, tv;
-    if (!make_gather_tmap(&tq, a.q, rows, a.H, a.in_bf16) || !make_gather_tmap(&tk, a.k, rows, a.H, a.in_bf16) ||
-        !make_gather_tmap(&tv, a.v, rows, a.H, a.in_bf16))
-        return cudaErrorInvalidValue;
+    alignas(64) CUtensorMap unused{};  // the single-launch path copies with cp.async, not TMA
     Params p{};
     p.src[0] = static_cast<const uint8_t *>(a.q);
     p.src[1] = static_cast<const uint8_t *>(a.k);
@@ -1117,7 +1158,7 @@ cudaError_t launch_fused(const FusedArgs &a, int num_sms, cudaStream_t stream)
     p.err = a.err;
     p.wait_ns = a.wait_ns;
     const int smem = smem_bytes<true>(a.B);
-    return launch_variant<true>(a.in_bf16, tq, tk, tv, p, grid_for(a.B, a.H, a.N, num_sms), smem, stream);
+    return launch_variant<true>(a.in_bf16, unused, unused, unused, p, grid_for(a.B, a.H, a.N, num_sms), smem, stream);
 }
 
 }  // namespace rra

@@ -145,12 +145,14 @@ __global__ void __launch_bounds__(kThreads) pack_kernel(const uint8_t *__restric
     __shared__ int16_t slot_of[kThreads];
     __shared__ int16_t n_of_slot[kThreads];
 
+    pdl_trigger();
     const int b = blockIdx.y;
     const int n0 = blockIdx.x * rows_per_split;
     if (n0 >= N)
         return;
     const int n1 = min(N, n0 + rows_per_split);
     const int64_t img0 = static_cast<int64_t>(b) * N;
+    pdl_wait();  // the mask and the padded tensors may come from the previous kernel
 
     // Phase 1: image start, rank of row n0 inside the image, image length -- one pass.
     const Counts c = count_ranges(mask, img0, img0 + n0, img0 + N);
@@ -208,12 +210,14 @@ __global__ void __launch_bounds__(kThreads) unpack_kernel(const uint8_t *__restr
     __shared__ int16_t slot_of[kThreads];
     __shared__ int16_t n_of_slot[kThreads];
 
+    pdl_trigger();
     const int b = blockIdx.y;
     const int n0 = blockIdx.x * rows_per_split;
     if (n0 >= N)
         return;
     const int n1 = min(N, n0 + rows_per_split);
     const int64_t img0 = static_cast<int64_t>(b) * N;
+    pdl_wait();  // cu_seqlens and the packed rows come from the previous kernels
     const int64_t start = cu[b];
     const int64_t end = cu[b + 1];
 
@@ -308,9 +312,8 @@ cudaError_t launch_pack(const uint8_t *mask, int B, int N, int64_t row_bytes, in
     const int V = static_cast<int>(row_bytes / 16);
     const dim3 grid(splits, B);
     return dispatch_vpl(V, [&](auto vpl) {
-        pack_kernel<decltype(vpl)::value><<<grid, kThreads, 0, stream>>>(mask, N, rows, V, n_tensors, s, d,
-                                                                         capacity, cu, err);
-        return cudaGetLastError();
+        return launch_pdl(pack_kernel<decltype(vpl)::value>, grid, dim3(kThreads), 0, stream, mask, N, rows, V,
+                          n_tensors, s, d, capacity, cu, err);
     });
 }
 
@@ -325,10 +328,9 @@ cudaError_t launch_unpack(const void *packed, const int32_t *cu, const uint8_t *
     const int V = static_cast<int>(row_bytes / 16);
     const dim3 grid(splits, B);
     return dispatch_vpl(V, [&](auto vpl) {
-        unpack_kernel<decltype(vpl)::value><<<grid, kThreads, 0, stream>>>(
-            static_cast<const uint8_t *>(packed), cu, mask, N, rows, V, fill_mode, capacity,
-            static_cast<uint8_t *>(dst), err);
-        return cudaGetLastError();
+        return launch_pdl(unpack_kernel<decltype(vpl)::value>, grid, dim3(kThreads), 0, stream,
+                          static_cast<const uint8_t *>(packed), cu, mask, N, rows, V, fill_mode, capacity,
+                          static_cast<uint8_t *>(dst), err);
     });
 }
 

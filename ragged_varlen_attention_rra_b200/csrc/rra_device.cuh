@@ -20,6 +20,14 @@ __device__ __forceinline__ void raise_error(int32_t *err, int code)
         atomicCAS(reinterpret_cast<int *>(err), 0, code);
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization may
+// start while the previous kernel in the stream is still running; pdl_wait() blocks until that
+// kernel has completed and its memory writes are visible (it returns at once when there is no
+// such dependency), and pdl_trigger() lets the next kernel in the stream start its own
+// preamble early.  Neither changes what a kernel computes.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t global_timer_ns()
 {
     uint64_t t;
@@ -207,6 +215,35 @@ __device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t (&r)[1])
 }
 
 // Each thread of the warp writes 16 consecutive 32-bit columns of its own TMEM lane.
+// Wait for this thread's outstanding tcgen05.ld and make the 32 registers of r depend on the
+// wait, so no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32])
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
+// Store 16 columns taken from every other register of r (start 0: r[0], r[2], ..., r[30];
+// start 1: r[1], r[3], ..., r[31]).
+template <int kStart>
+__device__ __forceinline__ void tmem_st16_strided(uint32_t taddr, const uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[kStart]), "r"(r[kStart + 2]), "r"(r[kStart + 4]), "r"(r[kStart + 6]), "r"(r[kStart + 8]),
+        "r"(r[kStart + 10]), "r"(r[kStart + 12]), "r"(r[kStart + 14]), "r"(r[kStart + 16]), "r"(r[kStart + 18]),
+        "r"(r[kStart + 20]), "r"(r[kStart + 22]), "r"(r[kStart + 24]), "r"(r[kStart + 26]), "r"(r[kStart + 28]),
+        "r"(r[kStart + 30])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
 {
     asm volatile(
@@ -273,6 +310,32 @@ __device__ __forceinline__ float ex2_approx(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// (y0, y1) = (x0, x1) * s + c, one paired fp32 instruction.
+__device__ __forceinline__ void fma2_scalar(float &y0, float &y1, float x0, float x1, float s, float c)
+{
+    asm("{\n\t.reg .b64 x, s2, c2, d;\n\tmov.b64 x, {%2, %3};\n\tmov.b64 s2, {%4, %4};\n\t"
+        "mov.b64 c2, {%5, %5};\n\tfma.rn.f32x2 d, x, s2, c2;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(y0), "=f"(y1)
+        : "f"(x0), "f"(x1), "f"(s), "f"(c));
+}
+
+// (y0, y1) = (a0, a1) - (b0, b1), one paired fp32 instruction.
+__device__ __forceinline__ void sub2(float &y0, float &y1, float a0, float a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(y0), "=f"(y1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
 // Number of nonzero bytes in a 32-bit word: bit 7 of each byte is set iff the byte is nonzero.

@@ -111,6 +111,7 @@ def test_fused_validation(L):
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 1025, 1, 64, 0.0, 1, 1, None, None) == rra.RRA_ERR_UNSUPPORTED
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 4097, 8, 1, 64, 0.0, 1, 1, None, None) == rra.RRA_ERR_UNSUPPORTED
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 8, 1, 64, 0.0, 2, 2, None, None) == rra.RRA_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 1024, 16384, 64, 0.0, 1, 1, None, None) == rra.RRA_ERR_UNSUPPORTED
 
 
 def test_get_device_error_validation(L):
