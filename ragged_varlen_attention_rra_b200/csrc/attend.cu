@@ -13,11 +13,13 @@
 //     (fp32 [128 x 80]) for each of two softmax groups that work on alternate items, so one
 //     group's QK^T and PV run on the tensor core while the other group's softmax runs;
 //   * warps specialise:
-//       warps 0..2  producer: Q tiles (2-slot ring) and 128-key K/V chunks (3-slot ring) of one
+//       warps 0..1  producer: Q tiles (2-slot ring) and 128-key K/V chunks (3-slot ring) of one
 //                   head; on the packed path warp 0 fetches them straight from the [T, H, 64]
 //                   layout with TMA (3-D tensor map, head = coordinate, 128-byte swizzle);
-//       warp 3      tensor-core issuer: S = Q K^T (smem x smem) and O += P V (P from TMEM as the
-//                   A operand), fp32 accumulation, completion signalled through mbarriers;
+//       warps 2..3  tensor-core issuers, one per softmax group: S = Q K^T (smem x smem) and
+//                   O += P V (P from TMEM as the A operand), fp32 accumulation, completion
+//                   signalled through mbarriers -- two issuing threads keep the tensor core busy
+//                   with both groups' short instruction bursts at once;
 //       warps 4..11 softmax: two groups of four warps take alternate items; in a group, thread
 //                   r owns row r of its S and O buffers (TMEM lane r), so the row max and row sum
 //                   need no exchange; it writes P back over its own S columns, rescales its row
@@ -54,9 +56,9 @@ namespace {
 constexpr int BM = 128;                 // query rows per tile (TMEM lanes)
 constexpr int BN = 128;                 // keys per step
 constexpr int kD = 64;                  // head dim
-constexpr int kThreads = 384;           // 12 warps: 3 x producer, MMA, 8 x softmax
-constexpr int kProducerWarps = 3;       // fused path: all three copy; packed path: warp 0 issues TMA
-constexpr int kMmaWarp = 3;
+constexpr int kThreads = 384;           // 12 warps: 2 x producer, 2 x MMA issuer, 8 x softmax
+constexpr int kProducerWarps = 2;       // fused path: both copy; packed path: warp 0 issues TMA
+constexpr int kMmaWarp0 = 2;            // warp 2 issues group 1's tensor-core work, warp 3 group 0's
 constexpr int kSoftmaxWarp0 = 4;
 constexpr int kSoftmaxWarps = 8;        // two groups of four, one per TMEM lane quarter each
 constexpr int kGroupWarps = 4;
@@ -84,7 +86,10 @@ constexpr uint32_t kOffBar = kOffOnes + kTileBytes;
 // (uint32 [kFusedMaxN / 32])
 constexpr int kIdxSlots = 4;
 constexpr uint32_t kIdxSlotBytes = kFusedMaxN * 2 + kFusedMaxN * 4 + kFusedMaxN / 8;
-constexpr uint32_t kOffIdx = kOffBar + 512;
+// the block's first work items, decoded once in the prologue (Item: 5 ints each)
+constexpr int kItemTable = 64;
+constexpr uint32_t kOffItems = kOffBar + 512;
+constexpr uint32_t kOffIdx = kOffItems + kItemTable * 20;
 // tile_pre[B+1], then cu[B+1]: after the list slots on the fused path, in their place otherwise
 template <bool kFused>
 constexpr uint32_t off_tile()
@@ -119,7 +124,7 @@ struct Bars {
     uint64_t s_full[2], p_full[2], s_free[2];
     uint64_t o_full[2], o_free[2];
     uint64_t idx_full[4], idx_free[4];  // fused: kept-row list slots, one per item in flight
-    uint64_t drain;
+    uint64_t drain[2];
     uint32_t tmem_slot;
     int abort;
     int warp_sums[2][kThreads / 32];
@@ -166,6 +171,7 @@ __device__ __forceinline__ uint32_t range16_(int64_t s, int64_t lo, int64_t hi)
 struct Item {
     int b, h, qt, seq0, L;
 };
+static_assert(sizeof(Item) == 20, "item table entry size");
 
 __device__ __forceinline__ Item decode_item(int item, int H, int B, const int32_t *tile_pre, const int32_t *cu)
 {
@@ -189,10 +195,8 @@ __device__ __forceinline__ Item decode_item(int item, int H, int B, const int32_
 
 // Bounded wait used by every role: returns false when the block is aborting or the wait ran
 // out (which itself raises the abort flag and the timeout error).
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Bars *bars, const Params &p)
+__device__ __noinline__ bool wait_or_abort_slow(uint64_t *bar, uint32_t parity, Bars *bars, const Params &p)
 {
-    if (mbar_test_wait(bar, parity))
-        return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
         if (*reinterpret_cast<volatile int *>(&bars->abort))
@@ -205,6 +209,11 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Ba
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Bars *bars, const Params &p)
+{
+    return mbar_test_wait(bar, parity) || wait_or_abort_slow(bar, parity, bars, p);
 }
 
 // Warp-uniform version: every lane waits, and the warp proceeds only if all lanes saw the
@@ -322,12 +331,6 @@ __device__ __forceinline__ void store_row(const Params &p, int64_t off, const ui
     }
 }
 
-// One PV step as the MMA warp sees it.
-struct PvStep {
-    int ks, kc, nk16;
-    bool wait_free;  // first PV of an item whose O buffer held an earlier item
-};
-
 // Fused path: producer warp w (of kProducerWarps) copies its share of one tile of up to 128
 // kept rows of one head from the padded tensor into the 128-byte-swizzled layout with 16-byte
 // cp.async: row r of the tile is the image's kept row base + r.  The chunks go in groups of 32
@@ -406,7 +409,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->idx_full[s], 1);
             mbar_init(&bars->idx_free[s], kGroupWarps);
         }
-        mbar_init(&bars->drain, 1);
+        mbar_init(&bars->drain[0], 1);
+        mbar_init(&bars->drain[1], 1);
         bars->abort = 0;
         fence_mbarrier_init();
     }
@@ -434,47 +438,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- work list: tile_pre[b] = number of 128-row query tiles of images < b; cu staged too.
     if constexpr (kFused) {
         // kept tokens per image, counted from 16-byte chunks of the flat mask into cu_s[b+1]
-        for (int b = tid; b <= B; b += kThreads)
-            cu_s[b] = 0;
-        __syncthreads();
-        const int64_t total = static_cast<int64_t>(B) * p.N;
         const uintptr_t addr = reinterpret_cast<uintptr_t>(p.mask);
         const int off = static_cast<int>(addr & 15u);
         const uint4 *m16 = reinterpret_cast<const uint4 *>(addr - off);
-        const int64_t nchunks = (off + total + 15) >> 4;
-        // every thread loads its chunks first (independent loads in flight together), then the
-        // counts are added per image with one shared atomic per (warp, image) -- lanes whose
-        // chunks hit the same image are grouped with a match and summed with a warp reduction
-        constexpr int kU = 4;
-        // (the loop bound is warp-uniform: every lane takes part in the warp collectives)
-        for (int64_t jw = static_cast<int64_t>(warp) * 32 * kU; jw < nchunks; jw += kThreads * kU) {
-            const int64_t j0 = jw + lane;
-            uint4 w[kU];
+        // a warp per image, six images per warp at a time: lane l loads 16-byte chunks l,
+        // l + 32, ... of each image's byte range (coalesced), all loads of a round issued before
+        // any is used; the counts are summed with one warp reduction per image
+        constexpr int kImg = 6;
+        for (int bw = warp * kImg; bw < B; bw += (kThreads / 32) * kImg) {
+            int64_t lo[kImg], c0[kImg], c1[kImg];
+            int cnt[kImg];
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int64_t j = j0 + u * 32;
-                w[u] = j < nchunks ? __ldg(m16 + j) : make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < kImg; ++i) {
+                const int b = min(bw + i, B - 1);
+                lo[i] = static_cast<int64_t>(b) * p.N;
+                c0[i] = (off + lo[i]) >> 4;
+                c1[i] = (off + lo[i] + p.N + 15) >> 4;
+                cnt[i] = 0;
+            }
+            for (int k = 0; k * 32 < p.N / 16 + 2; ++k) {
+                uint4 w[kImg];
+#pragma unroll
+                for (int i = 0; i < kImg; ++i) {
+                    const int64_t j = c0[i] + lane + 32 * k;
+                    w[i] = j < c1[i] ? __ldg(m16 + j) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int i = 0; i < kImg; ++i)
+                    cnt[i] += __popc(kept_bits16_(w[i]) &
+                                     range16_((c0[i] + lane + 32 * k) * 16 - off, lo[i], lo[i] + p.N));
             }
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int64_t s0 = (j0 + u * 32) * 16 - off;  // byte index of the chunk's first byte
-                uint32_t bits = kept_bits16_(w[u]) & range16_(s0, 0, total);
-                while (__any_sync(0xffffffffu, bits != 0u)) {
-                    int b = -1, cnt = 0;
-                    if (bits != 0u) {
-                        // total <= 2^31 - 1, so the byte index fits a 32-bit division
-                        const uint32_t first = static_cast<uint32_t>(s0 + (__ffs(bits) - 1));
-                        b = static_cast<int>(first / static_cast<uint32_t>(p.N));
-                        const uint32_t in_b =
-                            bits & range16_(s0, static_cast<int64_t>(b) * p.N, static_cast<int64_t>(b + 1) * p.N);
-                        cnt = __popc(in_b);
-                        bits &= ~in_b;
-                    }
-                    const unsigned same = __match_any_sync(0xffffffffu, b);
-                    const int sum = __reduce_add_sync(same, cnt);
-                    if (b >= 0 && lane == __ffs(same) - 1)
-                        atomicAdd(&cu_s[b + 1], sum);
-                }
+            for (int i = 0; i < kImg; ++i) {
+                const int sum = __reduce_add_sync(0xffffffffu, cnt[i]);
+                if (lane == 0 && bw + i < B)
+                    cu_s[bw + i + 1] = sum;
             }
         }
         __syncthreads();
@@ -552,6 +550,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
+    // decode the block's first items once: every role walks the same list
+    Item *items = reinterpret_cast<Item *>(base + kOffItems);
+    {
+        const int total = tile_pre[B] * H;
+        for (int k = tid; k < kItemTable; k += kThreads) {
+            const int item = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
+            if (item < total)
+                items[k] = decode_item(item, H, B, tile_pre, cu_s);
+        }
+    }
+    auto item_at = [&](int k, int item) {
+        return k < kItemTable ? items[k] : decode_item(item, H, B, tile_pre, cu_s);
+    };
+
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -575,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int qs = 0, ks = 0;
         bool ok = true;
         for (int item = item_first; ok && item < item_end; item += item_step) {
-            const Item it = decode_item(item, H, B, tile_pre, cu_s);
+            const Item it = item_at(static_cast<int>(n_items), item);
             const int nkc = (it.L + BN - 1) / BN;
             const int row_off = it.b * p.N;  // fused: first padded row of this image
             const int islot = static_cast<int>(n_items & (kIdxSlots - 1));
@@ -700,16 +712,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (n > 0)
                 mbar_wait_bounded(&bars->kv_full[s], (n - 1) & 1u, kDrainNs);
         }
-    } else if (warp == kMmaWarp) {
-        // ================================================================ tcgen05 issuer
-        // An event loop over two kinds of work: S = Q K^T of the next step (item, 128-key chunk)
-        // in production order, and O += P V of a step whose P its softmax group has written.
-        // Item n belongs to softmax group g = n & 1 (S buffer g, O buffer g).  Whatever is ready
-        // is issued, waiting PVs first, so a PV never queues behind the next step's loads and an
-        // S never queues behind the other group's softmax.  Readiness is polled with
-        // non-blocking barrier tests; the loop gives up (RRA_ERR_TIMEOUT) when nothing has
-        // become ready for the wait limit.
-        uint32_t q_ph = 0, kv_ph = 0, p_ph = 0, sfree_ph = 0, ofree_ph = 0;  // one bit per slot / group
+    } else if (warp == kMmaWarp0 || warp == kMmaWarp0 + 1) {
+        // ================================================================ tcgen05 issuers
+        // One issuing thread per softmax group (warp 3: group 0, warp 2: group 1), so the two
+        // groups' tensor-core work is issued concurrently.  Group g owns the items n = g, g+2, ...
+        // of the block, S buffer g and O buffer g; for each 128-key chunk of its items its issuer
+        // runs S = Q K^T, waits for the softmax to write P over S, then O += P V.  The Q/K/V rings
+        // are filled in item order for both groups, so each issuer walks every item and, for the
+        // other group's, only advances its ring positions and phase bits.
+        const int g = kMmaWarp0 + 1 - warp;
+        uint32_t q_ph = 0, kv_ph = 0, p_ph = 0, sfree_ph = 0, ofree_ph = 0;
         const uint32_t idPV = idesc_f16(BM, kPvN, kBF16 ? 1u : 0u, 1u);
         // shared-memory descriptors of the ring slots: stepping K inside a 128-byte swizzled row
         // adds 32 bytes (2 units) to the start address, stepping 16 key rows adds 2048 bytes (128
@@ -719,165 +731,106 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t kdesc0 = smem_desc_sw128(smem_addr(base + kOffK), 16, 1024);
         const uint64_t vdesc0 = smem_desc_sw128(smem_addr(base + kOffV), kOffOnes - kOffV, 1024);
         auto slot_desc = [](uint64_t d0, int slot) { return d0 + static_cast<uint64_t>(slot) * (kTileBytes >> 4); };
-        auto v_desc = [&](int slot) {
-            return slot_desc(vdesc0, slot) - (static_cast<uint64_t>(slot) * (kTileBytes >> 4) << 16);
-        };
-        auto ready = [&](uint64_t *bar, uint32_t parity) {
-            return __all_sync(0xffffffffu, mbar_test_wait(bar, parity));
-        };
-        // the next S step
-        int item = item_first, n = 0, kc = 0, qs = 0, ks = 0, nkc = 0;
-        bool q_landed = false;
-        int it_L = item < item_end ? decode_item(item, H, B, tile_pre, cu_s).L : 0;
-        nkc = (it_L + BN - 1) / BN;
-        // per-group pending PV (registers: selected by value, never indexed)
-        PvStep pend0{0, 0, 0, false}, pend1{0, 0, 0, false};
-        uint32_t has_pend = 0;  // group g has an S whose PV is not issued yet
-        uint32_t s_busy = 0;    // group g's S buffer waits for its last PV to complete
-        bool ok = true;
-        uint64_t idle_since = 0;
-        while (true) {
-            const bool more_s = item < item_end;
-            if (!more_s && has_pend == 0)
+        const uint32_t dS = tmem + kColS0 + 128 * g;
+        const uint32_t dO = tmem + kColO0 + kOCols * g;
+        int qs = 0, ks = 0, n = 0;
+        bool s_busy = false, ok = true;
+        for (int item = item_first; ok && item < item_end; item += item_step, ++n) {
+            const int nkc = (item_at(n, item).L + BN - 1) / BN;
+            if ((n & 1) != g) {
+                // the other group's item: its fills pass through the same ring slots
+                q_ph ^= 1u << qs;
+                qs = (qs + 1 == kQStages) ? 0 : qs + 1;
+                for (int kc = 0; kc < nkc; ++kc) {
+                    kv_ph ^= 1u << ks;
+                    ks = (ks + 1 == kKVStages) ? 0 : ks + 1;
+                }
+                continue;
+            }
+            const int L = item_at(n, item).L;
+            ok = warp_wait(&bars->q_full[qs], (q_ph >> qs) & 1u, bars, p);
+            if (!ok)
                 break;
-            bool progressed = false;
-            // ---- PVs whose P is in TMEM: one burst per chunk (each burst of tensor-core
-            // instructions pays a start-up cost of a few hundred cycles)
-#pragma unroll
-            for (int g = 0; g < 2; ++g) {
-                if (!((has_pend >> g) & 1u))
-                    continue;
-                const PvStep u = g ? pend1 : pend0;
-                if (!ready(&bars->p_full[g], (p_ph >> g) & 1u))
-                    continue;
-                // first PV of an item: the group's previous item must have been read out
-                if (u.wait_free && !ready(&bars->o_free[g], (ofree_ph >> g) & 1u))
-                    continue;
-                p_ph ^= 1u << g;
-                if (u.wait_free)
-                    ofree_ph ^= 1u << g;
+            q_ph ^= 1u << qs;
+            for (int kc = 0; kc < nkc; ++kc) {
+                const int nk = min(BN, L - kc * BN);
+                const int nk16 = (nk + 15) & ~15;
+                ok = warp_wait(&bars->kv_full[ks], (kv_ph >> ks) & 1u, bars, p);
+                if (!ok)
+                    break;
+                kv_ph ^= 1u << ks;
+                uint8_t *sV = base + kOffV + ks * kTileBytes;
+                // zero V rows [nk, nk16): they enter the PV MMA with probability 0
+                if (nk < nk16) {
+                    for (int i = lane; i < (nk16 - nk) * 8; i += 32)
+                        *reinterpret_cast<uint4 *>(sV + (nk + (i >> 3)) * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
+                    fence_proxy_async_smem();
+                }
+                __syncwarp();
+                // the S buffer holds the previous chunk's P until that chunk's PV has completed
+                if (s_busy) {
+                    ok = warp_wait(&bars->s_free[g], sfree_ph, bars, p);
+                    if (!ok)
+                        break;
+                    sfree_ph ^= 1u;
+                }
                 if (lane == 0) {
                     tc_fence_after();
-                    const uint64_t vd = v_desc(u.ks);
-                    const uint32_t dO = tmem + kColO0 + kOCols * g;
-                    const uint32_t aP = tmem + kColS0 + 128 * g;
-                    const int nj = u.nk16 >> 4;
+                    if constexpr (kFused)
+                        fence_proxy_async_smem();  // Q/K/V arrived through cp.async (generic proxy)
+                    const uint64_t qd = slot_desc(qdesc0, qs);
+                    const uint64_t kd = slot_desc(kdesc0, ks);
+                    const uint32_t idS = idesc_f16(BM, nk16, kBF16 ? 1u : 0u, 0u);
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk)
+                        mma_ss(dS, qd + 2 * kk, kd + 2 * kk, idS, kk > 0 ? 1u : 0u);
+                    mma_commit(&bars->s_full[g]);
+                    if (kc == nkc - 1)
+                        mma_commit(&bars->q_empty[qs]);  // last read of this Q tile
+                }
+                __syncwarp();
+                // P of this chunk in TMEM; before the first PV of an item, the group's previous
+                // item must have been read out of O
+                ok = warp_wait(&bars->p_full[g], p_ph, bars, p);
+                if (!ok)
+                    break;
+                p_ph ^= 1u;
+                if (kc == 0 && n >= 2) {
+                    ok = warp_wait(&bars->o_free[g], ofree_ph, bars, p);
+                    if (!ok)
+                        break;
+                    ofree_ph ^= 1u;
+                }
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint64_t vd = slot_desc(vdesc0, ks) - (static_cast<uint64_t>(ks) * (kTileBytes >> 4) << 16);
+                    const int nj = nk16 >> 4;
                     // keys 16j..16j+15 live in slice j/2: head part at column 32(j/2) + 8(j%2),
-                    // remainder 16 columns further
+                    // remainder (bf16) 16 columns further
 #pragma unroll
                     for (int j = 0; j < BN / 16; ++j)
                         if (j < nj)
-                            mma_ts(dO, aP + 32 * (j >> 1) + 8 * (j & 1), vd + 128 * j, idPV,
-                                   (u.kc > 0 || j > 0) ? 1u : 0u);
+                            mma_ts(dO, dS + 32 * (j >> 1) + 8 * (j & 1), vd + 128 * j, idPV, (kc > 0 || j > 0) ? 1u : 0u);
                     if (kBF16) {
 #pragma unroll
                         for (int j = 0; j < BN / 16; ++j)
                             if (j < nj)
-                                mma_ts(dO, aP + 32 * (j >> 1) + 8 * (j & 1) + 16, vd + 128 * j, idPV, 1u);
+                                mma_ts(dO, dS + 32 * (j >> 1) + 8 * (j & 1) + 16, vd + 128 * j, idPV, 1u);
                     }
                     mma_commit(&bars->o_full[g]);
                     mma_commit(&bars->s_free[g]);
-                    mma_commit(&bars->kv_empty[u.ks]);
+                    mma_commit(&bars->kv_empty[ks]);
                 }
                 __syncwarp();
-                has_pend &= ~(1u << g);
-                progressed = true;
+                s_busy = true;
+                ks = (ks + 1 == kKVStages) ? 0 : ks + 1;
             }
-            // ---- the next S
-            if (more_s) {
-                const int g = n & 1;
-                bool go = !((has_pend >> g) & 1u);  // the S buffer still holds P that no PV has read
-                if (go && ((s_busy >> g) & 1u)) {
-                    go = ready(&bars->s_free[g], (sfree_ph >> g) & 1u);
-                    if (go) {
-                        sfree_ph ^= 1u << g;
-                        s_busy &= ~(1u << g);
-                    }
-                }
-                if (go && !q_landed) {
-                    go = ready(&bars->q_full[qs], (q_ph >> qs) & 1u);
-                    if (go) {
-                        q_ph ^= 1u << qs;
-                        q_landed = true;
-                    }
-                }
-                if (go)
-                    go = ready(&bars->kv_full[ks], (kv_ph >> ks) & 1u);
-                if (go) {
-                    kv_ph ^= 1u << ks;
-                    const int nk = min(BN, it_L - kc * BN);
-                    const int nk16 = (nk + 15) & ~15;
-                    uint8_t *sV = base + kOffV + ks * kTileBytes;
-                    // zero V rows [nk, nk16): they enter the PV MMA with probability 0
-                    if (nk < nk16) {
-                        for (int i = lane; i < (nk16 - nk) * 8; i += 32)
-                            *reinterpret_cast<uint4 *>(sV + (nk + (i >> 3)) * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
-                        fence_proxy_async_smem();
-                    }
-                    __syncwarp();
-                    if (lane == 0) {
-                        tc_fence_after();
-                        if constexpr (kFused)
-                            fence_proxy_async_smem();  // K/V arrived through cp.async (generic proxy)
-                        const uint64_t qd = slot_desc(qdesc0, qs);
-                        const uint64_t kd = slot_desc(kdesc0, ks);
-                        const uint32_t idS = idesc_f16(BM, nk16, kBF16 ? 1u : 0u, 0u);
-#pragma unroll
-                        for (int kk = 0; kk < kD / 16; ++kk)
-                            mma_ss(tmem + kColS0 + 128 * g, qd + 2 * kk, kd + 2 * kk, idS, kk > 0 ? 1u : 0u);
-                        mma_commit(&bars->s_full[g]);
-                        if (kc == nkc - 1)
-                            mma_commit(&bars->q_empty[qs]);  // last read of this Q tile
-                    }
-                    __syncwarp();
-                    s_busy |= 1u << g;
-                    const PvStep step{ks, kc, nk16, kc == 0 && n >= 2};
-                    if (g)
-                        pend1 = step;
-                    else
-                        pend0 = step;
-                    has_pend |= 1u << g;
-                    ks = (ks + 1 == kKVStages) ? 0 : ks + 1;
-                    if (++kc == nkc) {
-                        kc = 0;
-                        qs = (qs + 1 == kQStages) ? 0 : qs + 1;
-                        q_landed = false;
-                        item += item_step;
-                        ++n;
-                        if (item < item_end) {
-                            it_L = decode_item(item, H, B, tile_pre, cu_s).L;
-                            nkc = (it_L + BN - 1) / BN;
-                        }
-                    }
-                    progressed = true;
-                }
-            }
-            if (progressed) {
-                idle_since = 0;
-                continue;
-            }
-            if (*reinterpret_cast<volatile int *>(&bars->abort)) {
-                ok = false;
-                break;
-            }
-            __nanosleep(64);  // leave issue slots to the softmax warps sharing this scheduler
-            const uint64_t now = global_timer_ns();
-            if (idle_since == 0) {
-                idle_since = now;
-            } else if (now - idle_since >= p.wait_ns) {
-                if (lane == 0) {
-                    *reinterpret_cast<volatile int *>(&bars->abort) = 1;
-                    raise_error(p.err, RRA_ERR_TIMEOUT);
-                }
-                ok = false;
-                break;
-            }
+            qs = (qs + 1 == kQStages) ? 0 : qs + 1;
         }
-        (void)ok;
         // drain: every MMA this thread issued has completed
         if (lane == 0) {
-            mma_commit(&bars->drain);
-            mbar_wait_bounded(&bars->drain, 0, kDrainNs);
+            mma_commit(&bars->drain[g]);
+            mbar_wait_bounded(&bars->drain[g], 0, kDrainNs);
         }
         __syncwarp();
     } else if (warp >= kSoftmaxWarp0) {
@@ -896,7 +849,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int item = item_first; ok && item < item_end; item += item_step, ++n) {
             if ((n & 1) != g)
                 continue;
-            const Item it = decode_item(item, H, B, tile_pre, cu_s);
+            const Item it = item_at(n, item);
             const int nkc = (it.L + BN - 1) / BN;
             const int q0 = it.qt * BM;
             const int qrows = min(BM, it.L - q0);
@@ -984,19 +937,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             if (warp_active) {
-                uint32_t r0[32], r1[32], sum[1];
-                tmem_ld32(obase, r0);
-                tmem_ld32(obase + 32, r1);
+                uint32_t sum[1];
                 tmem_ld1(obase + 64, sum);
                 tmem_wait_ld();
-                if (row < qrows) {
-                    int64_t out_row = static_cast<int64_t>(it.seq0) + q0 + row;
-                    if constexpr (kFused)
-                        out_row = static_cast<int64_t>(it.b) * p.N + idx_list(islot)[q0 + row];
-                    const float inv = 1.f / __uint_as_float(sum[0]);
-                    const int64_t off = (out_row * H + it.h) * kD;
-                    store_row(p, off, r0, 0, inv);
-                    store_row(p, off, r1, 32, inv);
+                const float inv = 1.f / __uint_as_float(sum[0]);
+                int64_t out_row = static_cast<int64_t>(it.seq0) + q0 + row;
+                if constexpr (kFused)
+                    out_row = static_cast<int64_t>(it.b) * p.N + idx_list(islot)[q0 + (row < qrows ? row : 0)];
+                const int64_t off = (out_row * H + it.h) * kD;
+#pragma unroll 1
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t r[32];
+                    tmem_ld32(obase + 32 * h2, r);
+                    tmem_wait_ld_dep(r);
+                    if (row < qrows)
+                        store_row(p, off, r, 32 * h2, inv);
                 }
             }
             tc_fence_before();

@@ -22,11 +22,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-#ifdef RRA_AB_NO_PDL
-    cfg.numAttrs = 0;
-#else
     cfg.numAttrs = 1;
-#endif
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
