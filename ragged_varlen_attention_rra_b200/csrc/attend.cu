@@ -56,13 +56,19 @@ namespace {
 constexpr int BM = 128;                 // query rows per tile (TMEM lanes)
 constexpr int BN = 128;                 // keys per step
 constexpr int kD = 64;                  // head dim
-constexpr int kThreads = 384;           // 12 warps: 2 x producer, 2 x MMA issuer, 8 x softmax
-constexpr int kProducerWarps = 2;       // fused path: both copy; packed path: warp 0 issues TMA
+constexpr int kThreads = 416;           // 13 warps: 2 x copier, 2 x MMA issuer, 8 x softmax, list builder
+// producer warps: warp 0 fills the Q/K/V rings (TMA on the packed path; on the single-launch path
+// warps 0 and 1 share the cp.async gathers), warp 12 (single-launch path) builds the kept-row
+// lists ahead of them
+constexpr int kCopyWarps = 2;
+constexpr int kListWarp = 12;
 constexpr int kMmaWarp0 = 2;            // warp 2 issues group 1's tensor-core work, warp 3 group 0's
 constexpr int kSoftmaxWarp0 = 4;
 constexpr int kSoftmaxWarps = 8;        // two groups of four, one per TMEM lane quarter each
 constexpr int kGroupWarps = 4;
-static_assert(kSoftmaxWarp0 + kSoftmaxWarps == kThreads / 32 && kSoftmaxWarps == 2 * kGroupWarps, "warp roles");
+static_assert(kSoftmaxWarp0 + kSoftmaxWarps == kListWarp && kListWarp + 1 == kThreads / 32 &&
+                  kSoftmaxWarps == 2 * kGroupWarps,
+              "warp roles");
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: S buffers at 0 and 128 (the P of each 32-key slice is written back over the
 // slice's own S columns: 16 columns of packed head values, then 16 of bf16 remainders), O
@@ -120,7 +126,11 @@ constexpr uint64_t kDrainNs = 2000000000ull;
 
 struct Bars {
     uint64_t q_full[kQStages], q_empty[kQStages];
-    uint64_t kv_full[kKVStages], kv_empty[kKVStages];
+    // kv_full[slot][g]: the fill of a K/V slot for an item of softmax group g.  A slot carries
+    // both groups' chunks, but each group's issuer waits only on its own barrier, whose phases
+    // then advance one fill at a time from its point of view (a parity wait never sees a phase
+    // two ahead or two behind).
+    uint64_t kv_full[kKVStages][2], kv_empty[kKVStages];
     uint64_t s_full[2], p_full[2], s_free[2];
     uint64_t o_full[2], o_free[2];
     uint64_t idx_full[4], idx_free[4];  // fused: kept-row list slots, one per item in flight
@@ -331,11 +341,11 @@ __device__ __forceinline__ void store_row(const Params &p, int64_t off, const ui
     }
 }
 
-// Fused path: producer warp w (of kProducerWarps) copies its share of one tile of up to 128
-// kept rows of one head from the padded tensor into the 128-byte-swizzled layout with 16-byte
-// cp.async: row r of the tile is the image's kept row base + r.  The chunks go in groups of 32
-// (one per lane, 8 lanes per 128-byte row, so each row is one coalesced segment), group g to
-// warp g % 3.  Completion arrives on `bar` once per producer lane.
+// Fused path: copier warp w (of kCopyWarps) copies its share of one tile of up to 128 kept rows
+// of one head from the padded tensor into the 128-byte-swizzled layout with 16-byte cp.async:
+// row r of the tile is the image's kept row base + r.  The chunks go in groups of 32 (one per
+// lane, 8 lanes per 128-byte row, so each row is one coalesced segment), group g to warp g % 2.
+// Completion arrives on `bar` once per copier lane.
 __device__ __forceinline__ void copy_tile_async(uint8_t *tile, const uint8_t *src, uint64_t *bar, const int32_t *offs,
                                                 int base, int count, int w, int lane)
 {
@@ -345,7 +355,7 @@ __device__ __forceinline__ void copy_tile_async(uint8_t *tile, const uint8_t *sr
     const uint32_t tile_s = smem_addr(tile);
     const int groups = (count * 8 + 31) >> 5;
 #pragma unroll 4
-    for (int grp = w; grp < groups; grp += kProducerWarps) {
+    for (int grp = w; grp < groups; grp += kCopyWarps) {
         const int i = lane + 32 * grp;
         const int r = i >> 3, c = i & 7;
         if (r < count) {
@@ -389,13 +399,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // full barriers: one TMA arrival with transaction bytes, or (fused) one cp.async
         // arrival per producer lane
-        const uint32_t fills = kFused ? 32u * kProducerWarps : 1u;
+        const uint32_t fills = kFused ? 32u * kCopyWarps : 1u;
         for (int s = 0; s < kQStages; ++s) {
             mbar_init(&bars->q_full[s], fills);
             mbar_init(&bars->q_empty[s], 1);
         }
         for (int s = 0; s < kKVStages; ++s) {
-            mbar_init(&bars->kv_full[s], kFused ? 2u * fills : fills);
+            mbar_init(&bars->kv_full[s][0], kFused ? 2u * fills : fills);
+            mbar_init(&bars->kv_full[s][1], kFused ? 2u * fills : fills);
             mbar_init(&bars->kv_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -575,15 +586,80 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int item_end = total_items;
     const int item_step = static_cast<int>(gridDim.x);
 
-    if (warp < kProducerWarps && (kFused || warp == 0)) {
+    if (kFused && warp == kListWarp) {
+        // ================================================================ kept-row lists
+        // Item n's list goes to slot n % 4, free once the epilogue of item n-4 has used it (the
+        // copier is done with a list before that epilogue can run); this warp runs up to four
+        // items ahead of the copier.
+        uint32_t idx_phase = 0;
+        int cur_b = -1, prev_slot = 0, n = 0;
+        bool ok = true;
+        for (int item = item_first; ok && item < item_end; item += item_step, ++n) {
+            const Item it = item_at(n, item);
+            const int row_off = it.b * p.N;
+            const int islot = n & (kIdxSlots - 1);
+            int16_t *list = idx_list(islot);
+            uint32_t *bits = idx_bits(islot);
+            int32_t *offs = idx_offs(islot);
+            const int nwords = (p.N + 31) / 32;
+            ok = warp_wait(&bars->idx_free[islot], ((idx_phase >> islot) & 1u) ^ 1u, bars, p);
+            if (!ok)
+                break;
+            idx_phase ^= 1u << islot;
+            if (it.b == cur_b) {
+                // same image as the previous item: copy its list
+                const int16_t *pl = idx_list(prev_slot);
+                const int32_t *po = idx_offs(prev_slot);
+                const uint32_t *pb = idx_bits(prev_slot);
+                for (int i = lane; i < it.L; i += 32) {
+                    list[i] = pl[i];
+                    offs[i] = po[i];
+                }
+                for (int i = lane; i < nwords; i += 32)
+                    bits[i] = pb[i];
+            } else {
+                // kept positions of this image in order: mask bytes fetched 8 words of 32 at a
+                // time (independent loads), then one ballot per word
+                int running = 0;
+                for (int w0 = 0; w0 < nwords; w0 += 8) {
+                    bool keep[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int tok = (w0 + u) * 32 + lane;
+                        keep[u] = tok < p.N && p.mask[row_off + tok] != 0;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const unsigned bal = __ballot_sync(0xffffffffu, keep[u]);
+                        if (w0 + u < nwords) {
+                            if (keep[u]) {
+                                const int slot_i = running + __popc(bal & ((1u << lane) - 1u));
+                                const int tok = (w0 + u) * 32 + lane;
+                                list[slot_i] = static_cast<int16_t>(tok);
+                                offs[slot_i] = tok * H * kD * 2;  // < 2^31 (checked on the host)
+                            }
+                            if (lane == 0)
+                                bits[w0 + u] = bal;
+                            running += __popc(bal);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&bars->idx_full[islot]);
+            cur_b = it.b;
+            prev_slot = islot;
+        }
+    } else if (warp < (kFused ? kCopyWarps : 1)) {
         // ================================================================ producer
         // Empty-slot waits use the usual parity idiom: on a fresh barrier the phase "before"
         // phase 0 counts as complete, so waiting on parity (phase ^ 1) passes at once for the
         // first fill of each slot, then tracks the consumer's releases.
         uint32_t q_phase = 0, kv_phase = 0;  // one bit per slot
-        int cur_b = -1, prev_slot = 0;       // fused: image of the previous item, and its list slot
-        uint32_t idx_phase = 0, idxf_phase = 0, n_items = 0;
-        uint32_t q_issued = 0, kv_issued = 0;
+        uint32_t idxf_phase = 0, n_items = 0;
+        uint32_t q_issued = 0;
+        uint32_t kv_par = 0, kv_any = 0;  // per kv_full barrier (bit 2*slot+group): fill-count parity, any fill
         int qs = 0, ks = 0;
         bool ok = true;
         for (int item = item_first; ok && item < item_end; item += item_step) {
@@ -592,68 +668,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int row_off = it.b * p.N;  // fused: first padded row of this image
             const int islot = static_cast<int>(n_items & (kIdxSlots - 1));
             if constexpr (kFused) {
-                int16_t *list = idx_list(islot);
-                uint32_t *bits = idx_bits(islot);
-                const int nwords = (p.N + 31) / 32;
-                // list slot of this item: free once the epilogue of item n-4 has used it; producer
-                // warp 0 fills it, the other producer warps wait until it is full (bounded waits
-                // only, so an aborting warp can never strand the others)
-                if (warp == 0) {
-                    ok = warp_wait(&bars->idx_free[islot], ((idx_phase >> islot) & 1u) ^ 1u, bars, p);
-                    if (!ok)
-                        break;
-                    idx_phase ^= 1u << islot;
-                }
-                if (warp != 0) {
-                    ok = warp_wait(&bars->idx_full[islot], (idxf_phase >> islot) & 1u, bars, p);
-                    if (!ok)
-                        break;
-                    idxf_phase ^= 1u << islot;
-                } else if (it.b == cur_b) {
-                    // same image as the previous item: copy its list
-                    const int16_t *pl = idx_list(prev_slot);
-                    const int32_t *po = idx_offs(prev_slot);
-                    const uint32_t *pb = idx_bits(prev_slot);
-                    int32_t *offs = idx_offs(islot);
-                    for (int i = lane; i < it.L; i += 32) {
-                        list[i] = pl[i];
-                        offs[i] = po[i];
-                    }
-                    for (int i = lane; i < nwords; i += 32)
-                        bits[i] = pb[i];
-                } else {
-                    // kept positions of this image in order: mask bytes fetched 8 words of 32 at
-                    // a time (independent loads), then one ballot per word
-                    int running = 0;
-                    for (int w0 = 0; w0 < nwords; w0 += 8) {
-                        bool keep[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int n = (w0 + u) * 32 + lane;
-                            keep[u] = n < p.N && p.mask[row_off + n] != 0;
-                        }
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const unsigned bal = __ballot_sync(0xffffffffu, keep[u]);
-                            if (w0 + u < nwords) {
-                                if (keep[u]) {
-                                    const int slot_i = running + __popc(bal & ((1u << lane) - 1u));
-                                    const int n = (w0 + u) * 32 + lane;
-                                    list[slot_i] = static_cast<int16_t>(n);
-                                    idx_offs(islot)[slot_i] = n * H * kD * 2;  // < 2^31 (checked on the host)
-                                }
-                                if (lane == 0)
-                                    bits[w0 + u] = bal;
-                                running += __popc(bal);
-                            }
-                        }
-                    }
-                }
-                __syncwarp();
-                if (warp == 0 && lane == 0)
-                    mbar_arrive(&bars->idx_full[islot]);
-                cur_b = it.b;
-                prev_slot = islot;
+                // the kept-row list of this item (built by the list warp)
+                ok = warp_wait(&bars->idx_full[islot], (idxf_phase >> islot) & 1u, bars, p);
+                if (!ok)
+                    break;
+                idxf_phase ^= 1u << islot;
             }
             ok = warp_wait(&bars->q_empty[qs], ((q_phase >> qs) & 1u) ^ 1u, bars, p);
             if (!ok)
@@ -679,22 +698,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok)
                     break;
                 kv_phase ^= 1u << ks;
+                uint64_t *full = &bars->kv_full[ks][n_items & 1u];  // the owning group's barrier
                 if constexpr (kFused) {
                     const int cnt = min(BN, it.L - kc * BN);
-                    copy_tile_async(base + kOffK + ks * kTileBytes, p.src[1] + head0, &bars->kv_full[ks],
-                                    idx_offs(islot), kc * BN, cnt, warp, lane);
-                    copy_tile_async(base + kOffV + ks * kTileBytes, p.src[2] + head0, &bars->kv_full[ks],
-                                    idx_offs(islot), kc * BN, cnt, warp, lane);
+                    copy_tile_async(base + kOffK + ks * kTileBytes, p.src[1] + head0, full, idx_offs(islot), kc * BN,
+                                    cnt, warp, lane);
+                    copy_tile_async(base + kOffV + ks * kTileBytes, p.src[2] + head0, full, idx_offs(islot), kc * BN,
+                                    cnt, warp, lane);
                 } else {
-                    if (lane == 0)
-                        mbar_arrive_expect_tx(&bars->kv_full[ks], 2 * kTileBytes);
                     if (lane == 0) {
-                        tma_load_3d(base + kOffK + ks * kTileBytes, &tm_k, &bars->kv_full[ks], 0, it.h, it.seq0 + kc * BN);
-                        tma_load_3d(base + kOffV + ks * kTileBytes, &tm_v, &bars->kv_full[ks], 0, it.h, it.seq0 + kc * BN);
+                        mbar_arrive_expect_tx(full, 2 * kTileBytes);
+                        tma_load_3d(base + kOffK + ks * kTileBytes, &tm_k, full, 0, it.h, it.seq0 + kc * BN);
+                        tma_load_3d(base + kOffV + ks * kTileBytes, &tm_v, full, 0, it.h, it.seq0 + kc * BN);
                     }
                 }
                 __syncwarp();
-                ++kv_issued;
+                {
+                    const uint32_t bit = 1u << (2 * ks + (n_items & 1u));  // barrier kv_full[ks][group]
+                    kv_par ^= bit;
+                    kv_any |= bit;
+                }
                 ks = (ks + 1 == kKVStages) ? 0 : ks + 1;
             }
             ++n_items;
@@ -707,11 +730,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (n > 0)
                 mbar_wait_bounded(&bars->q_full[s], (n - 1) & 1u, kDrainNs);
         }
-        for (int s = 0; s < kKVStages; ++s) {
-            const uint32_t n = kv_issued / kKVStages + (static_cast<uint32_t>(s) < kv_issued % kKVStages ? 1u : 0u);
-            if (n > 0)
-                mbar_wait_bounded(&bars->kv_full[s], (n - 1) & 1u, kDrainNs);
-        }
+        for (int s = 0; s < kKVStages; ++s)
+            for (int gg = 0; gg < 2; ++gg) {
+                const uint32_t bit = 1u << (2 * s + gg);
+                if (kv_any & bit)  // the last fill has parity (count - 1) & 1
+                    mbar_wait_bounded(&bars->kv_full[s][gg], (kv_par & bit) ? 0u : 1u, kDrainNs);
+            }
     } else if (warp == kMmaWarp0 || warp == kMmaWarp0 + 1) {
         // ================================================================ tcgen05 issuers
         // One issuing thread per softmax group (warp 3: group 0, warp 2: group 1), so the two
@@ -738,13 +762,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int item = item_first; ok && item < item_end; item += item_step, ++n) {
             const int nkc = (item_at(n, item).L + BN - 1) / BN;
             if ((n & 1) != g) {
-                // the other group's item: its fills pass through the same ring slots
+                // the other group's item: its Q slot is never ours (item n uses slot n % 2), and
+                // its K/V chunks pass through the same slots but signal the other group's
+                // barriers -- only the ring positions advance
                 q_ph ^= 1u << qs;
                 qs = (qs + 1 == kQStages) ? 0 : qs + 1;
-                for (int kc = 0; kc < nkc; ++kc) {
-                    kv_ph ^= 1u << ks;
-                    ks = (ks + 1 == kKVStages) ? 0 : ks + 1;
-                }
+                ks = (ks + nkc) % kKVStages;
                 continue;
             }
             const int L = item_at(n, item).L;
@@ -755,7 +778,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kc = 0; kc < nkc; ++kc) {
                 const int nk = min(BN, L - kc * BN);
                 const int nk16 = (nk + 15) & ~15;
-                ok = warp_wait(&bars->kv_full[ks], (kv_ph >> ks) & 1u, bars, p);
+                ok = warp_wait(&bars->kv_full[ks][g], (kv_ph >> ks) & 1u, bars, p);
                 if (!ok)
                     break;
                 kv_ph ^= 1u << ks;
@@ -833,7 +856,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait_bounded(&bars->drain[g], 0, kDrainNs);
         }
         __syncwarp();
-    } else if (warp >= kSoftmaxWarp0) {
+    } else if (warp >= kSoftmaxWarp0 && warp < kSoftmaxWarp0 + kSoftmaxWarps) {
         // ================================================================ softmax + epilogue
         // Group g (4 warps) takes items n = g, g+2, ...; thread r of the group owns row r of
         // S buffer g and O buffer g (its TMEM lane), so row max and row sum need no exchange.
