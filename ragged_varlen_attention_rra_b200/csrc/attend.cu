@@ -15,7 +15,8 @@
 //   * warps specialise:
 //       warps 0..1  producer: Q tiles (2-slot ring) and 128-key K/V chunks (3-slot ring) of one
 //                   head; on the packed path warp 0 fetches them straight from the [T, H, 64]
-//                   layout with TMA (3-D tensor map, head = coordinate, 128-byte swizzle);
+//                   layout with TMA (3-D tensor map, head = coordinate, 128-byte swizzle), on
+//                   the single-launch path warps 0 and 1 gather them with cp.async;
 //       warps 2..3  tensor-core issuers, one per softmax group: S = Q K^T (smem x smem) and
 //                   O += P V (P from TMEM as the A operand), fp32 accumulation, completion
 //                   signalled through mbarriers -- two issuing threads keep the tensor core busy
@@ -25,6 +26,7 @@
 //                   need no exchange; it writes P back over its own S columns, rescales its row
 //                   of O in TMEM when the running max rises, and finally normalises and stores
 //                   the row -- while the other group's QK^T, softmax and PV run alongside;
+//       warp 12     (single-launch path) builds each item's kept-row list ahead of the gathers;
 //   * for bf16 inputs P is split into a bf16 head and a bf16 remainder (two PV MMAs), which
 //     keeps P at ~16 significant bits; fp16 P (11 bits) is used as is;
 //   * the PV MMA runs with N = 80: the 64 columns of V plus a constant tile whose first column
