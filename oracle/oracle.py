@@ -62,6 +62,9 @@ def _declare(lib):
     lib.rra_oracle_unpack.argtypes = [vp, i32p, u8p, ctypes.c_int, ctypes.c_int, ctypes.c_int64,
                                       ctypes.c_int, ctypes.c_int64, vp]
     lib.rra_oracle_unpack.restype = ctypes.c_int
+    lib.rra_oracle_l2_mask.argtypes = [vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, i32p,
+                                       ctypes.c_double, u8p, u8p]
+    lib.rra_oracle_l2_mask.restype = ctypes.c_int
     return lib
 
 
@@ -206,4 +209,24 @@ def unpack(packed, cu, mask, fill_mode: int = 0, dst=None, capacity: int | None 
     if capacity is None:
         capacity = p.shape[0]
     lib.rra_oracle_unpack(_ptr(p), _i32p(cua), _ptr(m), B, N, row_bytes, int(fill_mode), int(capacity), _ptr(out))
+    return out
+
+
+def l2_mask(x, k_keep=None, threshold_sq: float = 0.0, prev=None, dtype: str | None = None, lib=None) -> np.ndarray:
+    """Threshold-l2 selection: embeddings x [B, N, C] (16-bit or float) -> keep mask uint8 [B, N].
+
+    With k_keep ([B] ints) each image keeps CLS and its k_b highest-norm candidates (lower
+    index first among ties); otherwise CLS and every candidate whose squared norm reaches
+    threshold_sq.  Candidates are tokens n >= 1 kept in `prev` (all of them without it)."""
+    lib = lib or load()
+    xa = _np(x)
+    code = _dtype_code(x, dtype)
+    B, N, C = xa.shape
+    out = np.zeros((B, N), dtype=np.uint8)
+    kk = None if k_keep is None else np.ascontiguousarray(np.asarray(k_keep, dtype=np.int32))
+    pv = None if prev is None else np.ascontiguousarray(_np(prev).astype(np.uint8))
+    rc = lib.rra_oracle_l2_mask(_ptr(xa), code, B, N, C, None if kk is None else _i32p(kk), float(threshold_sq),
+                                None if pv is None else _ptr(pv), _ptr(out))
+    if rc != 0:
+        raise ValueError("rra_oracle_l2_mask: bad arguments")
     return out

@@ -234,3 +234,75 @@ int rra_oracle_unpack(const uint8_t *packed, const int32_t *cu, const uint8_t *m
     }
     return 0;
 }
+
+/*
+ * Threshold-l2 token selection, the step in front of the pipeline (aissential.tech summary,
+ * Summary: the DeiT models are pruned with Threshold-l2, EViT and other methods -- the pages
+ * name the method and nothing more).  Readings, each also listed in the design notes:
+ *   - a token's score is the l2 norm of its embedding row x[b, n, 0..C-1]; the squared norm,
+ *     which orders tokens the same way, is what is compared;
+ *   - the squared norm is accumulated as acc = fma(x_c, x_c, acc) for c = 0, 1, ..., C-1 in
+ *     IEEE double from the exactly widened 16-bit inputs, so it is one reproducible number;
+ *     a NaN score ranks below every other score;
+ *   - the CLS token (n = 0) is always kept;
+ *   - the candidates are the tokens n >= 1 kept by the previous stage (`prev`, or every token
+ *     n >= 1 when there is none), which makes multi-stage masks nested (EViT-like schedules);
+ *   - with `k_keep`, image b keeps its k_b best candidates: highest score first, the lower
+ *     index first among equal scores (k_b clamped to [0, #candidates]); without it, every
+ *     candidate whose squared norm is >= threshold_sq.
+ * Returns 0, or -1 on a bad argument.
+ */
+static double l2_sq(const void *x, int dtype, int64_t row, int C)
+{
+    double acc = 0.0;
+    for (int c = 0; c < C; ++c) {
+        double v = load_elem(x, dtype, row * C + c);
+        acc = fma(v, v, acc);
+    }
+    return acc;
+}
+
+int rra_oracle_l2_mask(const void *x, int dtype, int B, int N, int C, const int32_t *k_keep, double threshold_sq,
+                       const uint8_t *prev, uint8_t *mask)
+{
+    if (B < 0 || N < 1 || C < 1)
+        return -1;
+    double *score = (double *)malloc(sizeof(double) * (size_t)N);
+    char *cand = (char *)malloc((size_t)N);
+    if (score == NULL || cand == NULL) {
+        free(score);
+        free(cand);
+        return -1;
+    }
+    for (int b = 0; b < B; ++b) {
+        int ncand = 0;
+        for (int n = 0; n < N; ++n) {
+            double s = l2_sq(x, dtype, (int64_t)b * N + n, C);
+            score[n] = isnan(s) ? -INFINITY : s;
+            cand[n] = (char)(n >= 1 && (prev == NULL || prev[(int64_t)b * N + n] != 0));
+            ncand += cand[n];
+            mask[(int64_t)b * N + n] = 0;
+        }
+        mask[(int64_t)b * N] = 1;
+        if (k_keep != NULL) {
+            int k = k_keep[b] < 0 ? 0 : (k_keep[b] > ncand ? ncand : k_keep[b]);
+            /* pick the best remaining candidate k times; a strict '>' over ascending n keeps
+             * the lowest index among equal scores */
+            for (int t = 0; t < k; ++t) {
+                int best = -1;
+                for (int n = 1; n < N; ++n)
+                    if (cand[n] && (best < 0 || score[n] > score[best]))
+                        best = n;
+                mask[(int64_t)b * N + best] = 1;
+                cand[best] = 0;
+            }
+        } else {
+            for (int n = 1; n < N; ++n)
+                if (cand[n] && score[n] >= threshold_sq)
+                    mask[(int64_t)b * N + n] = 1;
+        }
+    }
+    free(score);
+    free(cand);
+    return 0;
+}

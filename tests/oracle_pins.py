@@ -349,6 +349,71 @@ def pin_unpack_ranks_and_fill(lib):
                 assert np.all(y[b, n].view(np.uint32) == 0)
 
 
+# ------------------------------------------------------------------------------------ token selection
+
+def _int_bf16(rng, shape, lo=-6, hi=7):
+    """Small integers stored as bf16: every square and every sum of squares is exact, so ties are
+    real ties and the accumulation order cannot change a score."""
+    return torch.from_numpy(rng.integers(lo, hi, size=shape).astype(np.float32)).to(torch.bfloat16)
+
+
+def _scores(x):
+    return x.float().double().pow(2).sum(-1).numpy()  # exact for small-integer inputs
+
+
+def pin_l2_mask_topk_matches_sorted(lib):
+    """Top-k Threshold-l2 selection: CLS plus the k_b candidates of highest squared norm, the lower
+    index first among equal norms; candidates restricted by the previous stage's mask."""
+    rng = np.random.default_rng(41)
+    B, N, C = 6, 37, 8
+    x = _int_bf16(rng, (B, N, C), -3, 4)  # few distinct norms: many exact ties
+    prev = _rand_mask(rng, B, N, 0.7)
+    prev[1, 0] = 0  # CLS is kept even when the previous stage dropped it
+    k = rng.integers(0, 30, size=B).astype(np.int32)
+    sc = _scores(x)
+    for use_prev in (False, True):
+        got = O.l2_mask(x, k_keep=k, prev=prev if use_prev else None, lib=lib)
+        for b in range(B):
+            cand = [n for n in range(1, N) if (not use_prev or prev[b, n])]
+            order = sorted(cand, key=lambda n: (-sc[b, n], n))
+            want = np.zeros(N, np.uint8)
+            want[0] = 1
+            want[order[:max(0, min(int(k[b]), len(cand)))]] = 1
+            assert np.array_equal(got[b], want), (use_prev, b)
+
+
+def pin_l2_mask_threshold_and_extremes(lib):
+    """Threshold mode keeps exactly the candidates with squared norm >= threshold (equality kept);
+    k = 0 keeps only CLS, k >= #candidates keeps every candidate."""
+    rng = np.random.default_rng(42)
+    B, N, C = 3, 21, 4
+    x = _int_bf16(rng, (B, N, C))
+    sc = _scores(x)
+    thr = float(np.median(sc[:, 1:]))  # an attained value: the >= boundary is exercised
+    got = O.l2_mask(x, threshold_sq=thr, lib=lib)
+    want = (sc >= thr).astype(np.uint8)
+    want[:, 0] = 1
+    assert np.array_equal(got, want)
+    assert np.array_equal(O.l2_mask(x, threshold_sq=0.0, lib=lib), np.ones((B, N), np.uint8))
+    only_cls = np.zeros((B, N), np.uint8)
+    only_cls[:, 0] = 1
+    assert np.array_equal(O.l2_mask(x, threshold_sq=math.inf, lib=lib), only_cls)
+    assert np.array_equal(O.l2_mask(x, k_keep=np.zeros(B, np.int32), lib=lib), only_cls)
+    assert np.array_equal(O.l2_mask(x, k_keep=np.full(B, 10 * N, np.int32), lib=lib), np.ones((B, N), np.uint8))
+
+
+def pin_l2_mask_norm_not_l1(lib):
+    """The score is the l2 norm: (3, 0, 0, 0) (|.|_2 = 3, |.|_1 = 3) must beat (1, 1, 1, 1) and
+    (2, 2, 0, 0) (|.|_2 = 2, 2.83; |.|_1 = 4); a NaN row ranks last and never passes a threshold."""
+    x = torch.tensor([[[0, 0, 0, 0], [1, 1, 1, 1], [2, 2, 0, 0], [3, 0, 0, 0], [float("nan"), 0, 0, 0]]],
+                     dtype=torch.float32).to(torch.bfloat16)
+    assert np.array_equal(O.l2_mask(x, k_keep=[1], lib=lib)[0], [1, 0, 0, 1, 0])
+    assert np.array_equal(O.l2_mask(x, k_keep=[2], lib=lib)[0], [1, 0, 1, 1, 0])
+    assert np.array_equal(O.l2_mask(x, k_keep=[4], lib=lib)[0], [1, 1, 1, 1, 1])
+    assert np.array_equal(O.l2_mask(x, threshold_sq=4.0, lib=lib)[0], [1, 1, 1, 1, 0])
+    assert np.array_equal(O.l2_mask(x, threshold_sq=8.5, lib=lib)[0], [1, 0, 0, 1, 0])
+
+
 ALL_PINS = [
     pin_cu_seqlens_matches_cumsum,
     pin_rank_matches_nonzero,
@@ -365,4 +430,7 @@ ALL_PINS = [
     pin_attend_golden_hand_cases,
     pin_widening_exact,
     pin_unpack_ranks_and_fill,
+    pin_l2_mask_topk_matches_sorted,
+    pin_l2_mask_threshold_and_extremes,
+    pin_l2_mask_norm_not_l1,
 ]

@@ -39,6 +39,14 @@ MUTANTS = {
     "f16_bias": ("v = ldexp((double)(1024 + m), e - 25);", "v = ldexp((double)(1024 + m), e - 24);"),
     "f16_subnormal": ("v = ldexp((double)m, -24);", "v = ldexp((double)m, -25);"),
     "bf16_truncated": ("uint32_t u = ((uint32_t)b) << 16;", "uint32_t u = ((uint32_t)(b & 0xFFF0)) << 16;"),
+    "l2_tie_takes_higher_index": ("if (cand[n] && (best < 0 || score[n] > score[best]))",
+                                  "if (cand[n] && (best < 0 || score[n] >= score[best]))"),
+    "l2_cls_not_forced": ("        mask[(int64_t)b * N] = 1;\n        if (k_keep != NULL) {",
+                          "        if (k_keep != NULL) {"),
+    "l2_ignores_previous_stage": ("cand[n] = (char)(n >= 1 && (prev == NULL || prev[(int64_t)b * N + n] != 0));",
+                                  "cand[n] = (char)(n >= 1);"),
+    "l2_threshold_strict": ("if (cand[n] && score[n] >= threshold_sq)", "if (cand[n] && score[n] > threshold_sq)"),
+    "l2_is_l1": ("acc = fma(v, v, acc);", "acc += fabs(v);"),
     "mask_byte_is_bool": ("if (mask[(int64_t)b * N + n] != 0)\n                run += 1;",
                           "if (mask[(int64_t)b * N + n] == 1)\n                run += 1;"),
 }
