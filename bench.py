@@ -356,6 +356,32 @@ def time_path(pipe, flush, steps, warmup, stream):
     return step_ms, kern
 
 
+def time_mask_producer(w, flush, stream, steps, warmup, hbm_peak):
+    """The token-selection step in front of the path (rra_l2_mask, top-k mode) on embeddings of
+    the workload's width (C = 64 H, DeiT's embedding size) and keep counts from the configs'
+    recipe: per-launch device time (L2 flushed before each launch), algorithmic bytes, GB/s."""
+    C = 64 * w.H
+    x = workloads.embeddings(w.B, w.N, C, "bf16", seed=w.seed).cuda()
+    k = torch.from_numpy(workloads.keep_counts(w.B, w.N, seed=w.seed)).cuda()
+    mask = torch.empty(w.B, w.N, dtype=torch.uint8, device="cuda")
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = []
+    for i in range(warmup + steps):
+        with torch.cuda.stream(stream):
+            flush.fill_((i + 3) & 0xFF)
+            start.record(stream)
+            rra.rra_l2_mask(x, mask, k_keep=k, stream=stream)
+            end.record(stream)
+        stream.synchronize()
+        if i >= warmup:
+            ms.append(start.elapsed_time(end))
+    us = 1e3 * statistics.mean(ms)
+    nbytes = w.B * w.N * C * 2 + w.B * w.N + 4 * w.B
+    gbs = nbytes / (us * 1e3)
+    return {"call": "rra_l2_mask (top-k)", "B": w.B, "N": w.N, "C": C, "us_per_launch": us,
+            "alg_bytes_per_launch": nbytes, "gbs": gbs, "frac_of_hbm": gbs / hbm_peak}
+
+
 def main_gpu(args):
     ws, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -501,6 +527,8 @@ def main_gpu(args):
             if err2 != 0:
                 raise RuntimeError(f"device error {rra.rra_status_string(err2)} in the e2e region")
 
+    mask_producer = None if args.profile else time_mask_producer(w, flush, stream, args.steps, args.warmup, hbm_peak)
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and not args.profile:
         cpu = cpu_baseline(w, args.cpu_seconds)
@@ -524,6 +552,7 @@ def main_gpu(args):
                            "tokens_per_s": T_call / (1e-3 * statistics.mean(o_step_ms)), "kernels": other_kernels,
                            "identical_output": bool(same)},
             "attention_tflops": attn_tflops,
+            "mask_producer": mask_producer,
             "roofline": roofline,
             "e2e": e2e,
             "cpu_baseline": cpu,

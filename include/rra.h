@@ -162,6 +162,32 @@ rra_status rra_pack_attend_unpack(const uint8_t *keep_mask, const void *q, const
                                   rra_dtype in_dt, rra_dtype out_dt, int32_t *dev_error, rra_stream_t stream);
 
 /*
+ * rra_l2_mask -- Threshold-l2 token selection, the step in front of the pipeline (aissential.tech
+ * summary, Summary: the DeiT models are pruned with Threshold-l2, EViT and other methods; the
+ * pages name the method only).  For every image b:
+ *   score(n)   = squared l2 norm of x[b, n, :], accumulated in double as acc = fma(x_c, x_c, acc)
+ *                for c = 0 .. C-1 from the exactly widened 16-bit inputs; a NaN score ranks
+ *                below every other;
+ *   candidates = tokens n >= 1 with prev_mask[b, n] != 0 (every n >= 1 when prev_mask is NULL),
+ *                which makes the masks of successive stages nested (EViT-like schedules);
+ *   keep_mask[b, 0] = 1 (the CLS token is always kept);
+ *   with k_keep:  keep_mask[b, n] = 1 for the k_keep[b] best candidates -- higher score first,
+ *                 lower n first among equal scores, k clamped to [0, number of candidates];
+ *   without:      keep_mask[b, n] = 1 for the candidates with score >= threshold_sq;
+ *   every other keep_mask[b, n] = 0.
+ *
+ *   x             device [B, N, C] in dt (RRA_F16 or RRA_BF16), 16-byte aligned, C a multiple of 8
+ *   k_keep        device int32 [B], or NULL for threshold mode
+ *   threshold_sq  threshold on the squared norm (threshold mode only)
+ *   prev_mask     device uint8 [B, N] or NULL; may be the same buffer as keep_mask
+ *   keep_mask     device uint8 [B, N], written
+ *   B <= 65535, 1 <= N <= 4096
+ */
+rra_status rra_l2_mask(const void *x, int B, int N, int C, rra_dtype dt, const int32_t *k_keep,
+                       double threshold_sq, const uint8_t *prev_mask, uint8_t *keep_mask,
+                       rra_stream_t stream);
+
+/*
  * rra_get_device_error -- copy the device error word to *host_out.  This SYNCHRONISES `stream`
  * (it is the only call that does) and so must not be used inside stream capture.
  */

@@ -162,6 +162,24 @@ rra_status rra_pack_attend_unpack(const uint8_t *keep_mask, const void *q, const
     return e == cudaSuccess ? RRA_OK : RRA_ERR_CUDA;
 }
 
+rra_status rra_l2_mask(const void *x, int B, int N, int C, rra_dtype dt, const int32_t *k_keep, double threshold_sq,
+                       const uint8_t *prev_mask, uint8_t *keep_mask, rra_stream_t stream)
+{
+    if (x == nullptr || keep_mask == nullptr)
+        return RRA_ERR_INVALID_ARG;
+    if (B < 0 || N < 1 || C < 1 || !aligned16(x))
+        return RRA_ERR_INVALID_ARG;
+    if ((dt != RRA_F16 && dt != RRA_BF16) || C % 8 != 0)
+        return RRA_ERR_UNSUPPORTED;
+    if (B > 65535 || N > rra::kMaskMaxN || static_cast<int64_t>(B) * N * C > (int64_t{1} << 40))
+        return RRA_ERR_UNSUPPORTED;
+    if (k_keep == nullptr && threshold_sq != threshold_sq)
+        return RRA_ERR_INVALID_ARG;
+    const cudaError_t e = rra::launch_l2_mask(x, B, N, C, dt == RRA_BF16, k_keep, threshold_sq, prev_mask, keep_mask,
+                                              reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RRA_OK : RRA_ERR_CUDA;
+}
+
 size_t rra_attend_workspace_size(int B, int H, int max_seqlen)
 {
     (void)B;

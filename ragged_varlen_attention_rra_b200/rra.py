@@ -5,9 +5,10 @@ supplies device memory and the current stream.  If librra.so is missing or canno
 every function here raises -- there is no fallback.
 
 Names follow the C ABI: :func:`rra_pack`, :func:`rra_attend`, :func:`rra_unpack`,
-:func:`rra_pack_attend_unpack`, :func:`rra_get_device_error`, :func:`rra_status_string`,
-:func:`rra_attend_workspace_size`, :func:`rra_set_wait_timeout_ns`.  :func:`forward` runs the
-whole pack-attend-unpack call of one pruning stage, as three calls or as the single launch.
+:func:`rra_pack_attend_unpack`, :func:`rra_l2_mask`, :func:`rra_get_device_error`,
+:func:`rra_status_string`, :func:`rra_attend_workspace_size`, :func:`rra_set_wait_timeout_ns`.
+:func:`forward` runs the whole pack-attend-unpack call of one pruning stage, as three calls or
+as the single launch.
 """
 from __future__ import annotations
 
@@ -54,6 +55,8 @@ def _declare(lib):
     lib.rra_pack_attend_unpack.argtypes = [vp, vp, vp, vp, vp, i32p, c.c_int, c.c_int, c.c_int, c.c_int,
                                            c.c_float, c.c_int, c.c_int, i32p, vp]
     lib.rra_pack_attend_unpack.restype = c.c_int
+    lib.rra_l2_mask.argtypes = [vp, c.c_int, c.c_int, c.c_int, c.c_int, i32p, c.c_double, vp, vp, vp]
+    lib.rra_l2_mask.restype = c.c_int
     lib.rra_get_device_error.argtypes = [i32p, vp, c.POINTER(c.c_int32)]
     lib.rra_get_device_error.restype = c.c_int
     lib.rra_status_string.argtypes = [c.c_int]
@@ -176,6 +179,19 @@ def rra_pack_attend_unpack(mask: torch.Tensor, q: torch.Tensor, k: torch.Tensor,
                                       float(softmax_scale), _DT[q.dtype], _DT[y.dtype], _ptr(dev_error),
                                       _stream(stream))
     _check(st, "rra_pack_attend_unpack")
+
+
+def rra_l2_mask(x: torch.Tensor, keep_mask: torch.Tensor, k_keep: Optional[torch.Tensor] = None,
+                threshold_sq: float = 0.0, prev_mask: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Threshold-l2 selection: embeddings x [B, N, C] (fp16/bf16) -> keep_mask uint8 [B, N] (CLS kept).
+
+    With k_keep (int32 [B]) image b keeps its k_b highest-norm candidates; otherwise every
+    candidate whose squared norm reaches threshold_sq.  Candidates: n >= 1 kept in prev_mask."""
+    _require_cuda(x, keep_mask, k_keep, prev_mask)
+    B, N, C = x.shape
+    st = lib().rra_l2_mask(_ptr(x), B, N, C, _DT[x.dtype], _ptr(k_keep), float(threshold_sq), _ptr(prev_mask),
+                           _ptr(keep_mask), _stream(stream))
+    _check(st, "rra_l2_mask")
 
 
 # ------------------------------------------------------------------------------------ whole call

@@ -197,6 +197,29 @@ def config5_staged(B: int, seed: int = 0, ratio: float = 0.7, stages: int = 3) -
                ratio=ratio, batch=B, stages=stages)
 
 
+def embeddings(B: int, N: int, C: int = 384, dtype: str = "bf16", seed: int = 0, kind: str = "normal") -> torch.Tensor:
+    """Token embeddings [B, N, C] for the token-selection step (DeiT-S width 384 by default).
+
+    kind "normal": N(0, 1) rounded to the 16-bit type; kind "ties": small integers in [-3, 3]
+    (many tokens share a norm); kind "nan": normal with the embedding of a few tokens set to NaN."""
+    rng = np.random.default_rng(np.random.SeedSequence([int(seed), 77, int(B), int(N), int(C)]))
+    if kind == "ties":
+        x = rng.integers(-3, 4, size=(B, N, C)).astype(np.float32)
+    else:
+        x = rng.standard_normal((B, N, C), dtype=np.float32)
+        if kind == "nan":
+            bad = rng.integers(1, N, size=(B, 3))
+            for b in range(B):
+                x[b, bad[b], 0] = np.nan
+    return torch.from_numpy(x).to(_TORCH_DTYPES[dtype]).contiguous()
+
+
+def keep_counts(B: int, N: int, lo: float = 0.3, hi: float = 0.7, seed: int = 0) -> np.ndarray:
+    """Patches kept per image at ratios r_b ~ U[lo, hi] (the configs' recipe), int32 [B]."""
+    rng = np.random.default_rng(np.random.SeedSequence([int(seed), 78, int(B), int(N)]))
+    return np.array([keep_count(r, N - 1) for r in rng.uniform(lo, hi, size=B)], dtype=np.int32)
+
+
 def from_lengths(lengths: Sequence[int], N: int, H: int, dtype: str = "bf16", seed: int = 0,
                  std: float = 1.0, contiguous_prefix: bool = False) -> Workload:
     """Edge-case workload with given per-image kept lengths (0 <= L_b <= N)."""

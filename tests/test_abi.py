@@ -114,6 +114,20 @@ def test_fused_validation(L):
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 1024, 16384, 64, 0.0, 1, 1, None, None) == rra.RRA_ERR_UNSUPPORTED
 
 
+def test_l2_mask_validation(L):
+    f = L.rra_l2_mask
+    assert f(None, 2, 8, 16, 1, None, 1.0, None, FAKE, None) == rra.RRA_ERR_INVALID_ARG
+    assert f(FAKE, 2, 8, 16, 1, None, 1.0, None, None, None) == rra.RRA_ERR_INVALID_ARG
+    assert f(FAKE + 8, 2, 8, 16, 1, None, 1.0, None, FAKE, None) == rra.RRA_ERR_INVALID_ARG  # misaligned
+    assert f(FAKE, -1, 8, 16, 1, None, 1.0, None, FAKE, None) == rra.RRA_ERR_INVALID_ARG
+    assert f(FAKE, 2, 0, 16, 1, None, 1.0, None, FAKE, None) == rra.RRA_ERR_INVALID_ARG
+    assert f(FAKE, 2, 8, 12, 1, None, 1.0, None, FAKE, None) == rra.RRA_ERR_UNSUPPORTED  # C not a multiple of 8
+    assert f(FAKE, 2, 8, 16, 2, None, 1.0, None, FAKE, None) == rra.RRA_ERR_UNSUPPORTED  # fp32 embeddings
+    assert f(FAKE, 2, 4097, 16, 1, None, 1.0, None, FAKE, None) == rra.RRA_ERR_UNSUPPORTED
+    assert f(FAKE, 2, 8, 16, 1, None, float("nan"), None, FAKE, None) == rra.RRA_ERR_INVALID_ARG
+    assert f(FAKE, 0, 8, 16, 1, None, 1.0, None, FAKE, None) == rra.RRA_OK  # nothing to do, no launch
+
+
 def test_get_device_error_validation(L):
     out = ctypes.c_int32(0)
     assert L.rra_get_device_error(None, None, ctypes.byref(out)) == rra.RRA_ERR_INVALID_ARG

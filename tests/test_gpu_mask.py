@@ -1,0 +1,86 @@
+"""Threshold-l2 token selection on the GPU (rra_l2_mask) against the float64 oracle: the masks
+must be identical, bit for bit, on the same seeded embeddings -- top-k and threshold modes,
+nested stages, exact ties, NaN tokens, fp16 and bf16, and the configs' sizes."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from ragged_varlen_attention_rra_b200 import rra
+from ragged_varlen_attention_rra_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_mask(x, k=None, thr=0.0, prev=None, inplace=False):
+    B, N, _ = x.shape
+    xd = x.cuda()
+    kd = None if k is None else torch.as_tensor(k, dtype=torch.int32).cuda()
+    pd = None if prev is None else torch.as_tensor(prev, dtype=torch.uint8).cuda().contiguous()
+    out = pd if inplace else torch.full((B, N), 7, dtype=torch.uint8, device="cuda")  # garbage to overwrite
+    rra.rra_l2_mask(xd, out, k_keep=kd, threshold_sq=thr, prev_mask=pd)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("kind", ["normal", "ties", "nan"])
+def test_topk_matches_oracle(dtype, kind):
+    B, N, C = 64, 197, 384
+    x = W.embeddings(B, N, C, dtype, seed=3, kind=kind)
+    k = W.keep_counts(B, N, seed=3)
+    want = O.l2_mask(x, k_keep=k)
+    got = gpu_mask(x, k)
+    assert np.array_equal(got, want)
+    assert np.array_equal(got.sum(1), 1 + np.minimum(k, N - 1))  # CLS + k_b
+
+
+@pytest.mark.parametrize("kind", ["normal", "ties", "nan"])
+def test_threshold_matches_oracle(kind):
+    B, N, C = 16, 197, 384
+    x = W.embeddings(B, N, C, "bf16", seed=5, kind=kind)
+    for thr in (0.0, 350.0, 384.0, 420.0, float("inf")):
+        assert np.array_equal(gpu_mask(x, thr=thr), O.l2_mask(x, threshold_sq=thr)), thr
+
+
+def test_nested_stages_match_oracle():
+    """EViT-like schedule: three stages each keeping 0.7 of the previous survivors, chained on the
+    device through prev_mask (the last stage in place)."""
+    B, N, C = 64, 197, 384
+    x = W.embeddings(B, N, C, "bf16", seed=9)
+    prev_gpu = prev_cpu = None
+    kk = N - 1
+    for stage in range(3):
+        kk = W.keep_count(0.7, kk)
+        k = np.full(B, kk, np.int32)
+        want = O.l2_mask(x, k_keep=k, prev=prev_cpu)
+        got = gpu_mask(x, k, prev=prev_gpu, inplace=stage == 2)
+        assert np.array_equal(got, want), stage
+        if prev_cpu is not None:
+            assert np.all(want <= prev_cpu | (np.arange(N) == 0))  # nested
+        prev_gpu = prev_cpu = want
+
+
+@pytest.mark.parametrize("B,N,C", [(1, 1, 8), (3, 2, 8), (64, 577, 768), (512, 197, 384), (4, 4096, 64)])
+def test_sizes_match_oracle(B, N, C):
+    x = W.embeddings(B, N, C, "bf16", seed=B + N, kind="ties" if N % 2 else "normal")
+    k = np.random.default_rng(N).integers(-2, N + 2, size=B).astype(np.int32)  # incl. k < 0 and k > N-1
+    assert np.array_equal(gpu_mask(x, k), O.l2_mask(x, k_keep=k))
+
+
+def test_mask_feeds_the_pipeline():
+    """The device-made mask drives the single-launch call exactly as the same mask from the host."""
+    B, N, H = 8, 197, 6
+    x = W.embeddings(B, N, 384, "bf16", seed=11)
+    k = W.keep_counts(B, N, seed=11)
+    w = W.from_lengths([1] * B, N, H, seed=11)  # only its Q/K/V are used
+    q, kk, v = w.q.cuda(), w.k.cuda(), w.v.cuda()
+    dmask = torch.empty(B, N, dtype=torch.uint8, device="cuda")
+    rra.rra_l2_mask(x.cuda(), dmask, k_keep=torch.as_tensor(k).cuda())
+    hmask = torch.from_numpy(O.l2_mask(x, k_keep=k)).cuda()
+    y1 = torch.empty(B, N, H, 64, dtype=q.dtype, device="cuda")
+    y2 = torch.empty_like(y1)
+    rra.rra_pack_attend_unpack(dmask, q, kk, v, y1)
+    rra.rra_pack_attend_unpack(hmask, q, kk, v, y2)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))

@@ -74,3 +74,15 @@ def test_config5_staged_nested():
 def test_from_lengths():
     w = W.from_lengths([0, 1, 17, 197], 197, 2)
     assert list(w.lengths[0]) == [0, 1, 17, 197]
+
+
+def test_embeddings_and_keep_counts_are_seeded():
+    a = W.embeddings(3, 17, 16, "bf16", seed=4)
+    b = W.embeddings(3, 17, 16, "bf16", seed=4)
+    assert a.shape == (3, 17, 16) and a.dtype == torch.bfloat16 and torch.equal(a, b)
+    t = W.embeddings(2, 9, 8, "f16", seed=1, kind="ties")
+    assert t.dtype == torch.float16 and torch.all(t == t.round()) and t.abs().max() <= 3
+    n = W.embeddings(2, 9, 8, "bf16", seed=1, kind="nan")
+    assert torch.isnan(n.float()).any() and not torch.isnan(n[:, 0].float()).any()
+    k = W.keep_counts(64, 197, seed=2)
+    assert k.dtype == np.int32 and k.min() >= W.keep_count(0.3, 196) and k.max() <= W.keep_count(0.7, 196)
