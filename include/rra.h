@@ -165,9 +165,10 @@ rra_status rra_pack_attend_unpack(const uint8_t *keep_mask, const void *q, const
  * rra_l2_mask -- Threshold-l2 token selection, the step in front of the pipeline (aissential.tech
  * summary, Summary: the DeiT models are pruned with Threshold-l2, EViT and other methods; the
  * pages name the method only).  For every image b:
- *   score(n)   = squared l2 norm of x[b, n, :], accumulated in double as acc = fma(x_c, x_c, acc)
- *                for c = 0 .. C-1 from the exactly widened 16-bit inputs; a NaN score ranks
- *                below every other;
+ *   score(n)   = squared l2 norm of x[b, n, :], accumulated in single precision as
+ *                acc = fmaf(x_c, x_c, acc) for c = 0 .. C-1 (in that order) from the exactly
+ *                widened 16-bit inputs; a NaN score ranks below every other; the threshold is
+ *                compared with the score widened to double;
  *   candidates = tokens n >= 1 with prev_mask[b, n] != 0 (every n >= 1 when prev_mask is NULL),
  *                which makes the masks of successive stages nested (EViT-like schedules);
  *   keep_mask[b, 0] = 1 (the CLS token is always kept);

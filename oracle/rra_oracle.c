@@ -241,9 +241,11 @@ int rra_oracle_unpack(const uint8_t *packed, const int32_t *cu, const uint8_t *m
  * name the method and nothing more).  Readings, each also listed in the design notes:
  *   - a token's score is the l2 norm of its embedding row x[b, n, 0..C-1]; the squared norm,
  *     which orders tokens the same way, is what is compared;
- *   - the squared norm is accumulated as acc = fma(x_c, x_c, acc) for c = 0, 1, ..., C-1 in
- *     IEEE double from the exactly widened 16-bit inputs, so it is one reproducible number;
- *     a NaN score ranks below every other score;
+ *   - the squared norm is accumulated in IEEE single precision -- the precision the selection
+ *     kernel decides in -- as acc = fmaf(x_c, x_c, acc) for c = 0, 1, ..., C-1 from the exactly
+ *     widened 16-bit inputs, so it is one reproducible number (each square is exact in single
+ *     precision; the running sum rounds the same way on both sides); a NaN score ranks below
+ *     every other score;
  *   - the CLS token (n = 0) is always kept;
  *   - the candidates are the tokens n >= 1 kept by the previous stage (`prev`, or every token
  *     n >= 1 when there is none), which makes multi-stage masks nested (EViT-like schedules);
@@ -254,12 +256,12 @@ int rra_oracle_unpack(const uint8_t *packed, const int32_t *cu, const uint8_t *m
  */
 static double l2_sq(const void *x, int dtype, int64_t row, int C)
 {
-    double acc = 0.0;
+    float acc = 0.0f;
     for (int c = 0; c < C; ++c) {
-        double v = load_elem(x, dtype, row * C + c);
-        acc = fma(v, v, acc);
+        float v = (float)load_elem(x, dtype, row * C + c); /* exact: a 16-bit value */
+        acc = fmaf(v, v, acc);
     }
-    return acc;
+    return (double)acc;
 }
 
 int rra_oracle_l2_mask(const void *x, int dtype, int B, int N, int C, const int32_t *k_keep, double threshold_sq,

@@ -46,7 +46,7 @@ MUTANTS = {
     "l2_ignores_previous_stage": ("cand[n] = (char)(n >= 1 && (prev == NULL || prev[(int64_t)b * N + n] != 0));",
                                   "cand[n] = (char)(n >= 1);"),
     "l2_threshold_strict": ("if (cand[n] && score[n] >= threshold_sq)", "if (cand[n] && score[n] > threshold_sq)"),
-    "l2_is_l1": ("acc = fma(v, v, acc);", "acc += fabs(v);"),
+    "l2_is_l1": ("acc = fmaf(v, v, acc);", "acc += fabsf(v);"),
     "mask_byte_is_bool": ("if (mask[(int64_t)b * N + n] != 0)\n                run += 1;",
                           "if (mask[(int64_t)b * N + n] == 1)\n                run += 1;"),
 }
