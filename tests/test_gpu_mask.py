@@ -84,3 +84,50 @@ def test_mask_feeds_the_pipeline():
     rra.rra_pack_attend_unpack(hmask, q, kk, v, y2)
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+def test_three_stage_schedule_in_one_graph():
+    """EViT-like schedule entirely on the device inside one CUDA graph: for each of three stages,
+    select (nested in the previous stage's mask) then run the single-launch call; replayed with
+    new embeddings in the same buffers, every stage's mask and output match the host path."""
+    B, N, H = 16, 197, 6
+    w = W.from_lengths([1] * B, N, H, seed=21)
+    q, kk, v = w.q.cuda(), w.k.cuda(), w.v.cuda()
+    ks = []
+    kprev = N - 1
+    for _ in range(3):
+        kprev = W.keep_count(0.7, kprev)
+        ks.append(torch.full((B,), kprev, dtype=torch.int32, device="cuda"))
+    x = torch.empty(B, N, 384, dtype=torch.bfloat16, device="cuda")
+    masks = [torch.empty(B, N, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    ys = [torch.empty(B, N, H, 64, dtype=q.dtype, device="cuda") for _ in range(3)]
+    s = torch.cuda.Stream()
+
+    def enqueue():
+        for i in range(3):
+            rra.rra_l2_mask(x, masks[i], k_keep=ks[i], prev_mask=masks[i - 1] if i else None, stream=s)
+            rra.rra_pack_attend_unpack(masks[i], q, kk, v, ys[i], stream=s)
+
+    x.copy_(W.embeddings(B, N, 384, "bf16", seed=1).cuda())
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        enqueue()  # eager once (sets function attributes outside capture)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        enqueue()
+    for seed in (2, 3):
+        xe = W.embeddings(B, N, 384, "bf16", seed=seed)
+        x.copy_(xe.cuda())
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        prev = None
+        for i in range(3):
+            want = O.l2_mask(xe, k_keep=ks[i].cpu().numpy(), prev=prev)
+            assert np.array_equal(masks[i].cpu().numpy(), want), (seed, i)
+            y_ref = torch.empty_like(ys[i])
+            rra.rra_pack_attend_unpack(torch.from_numpy(want).cuda(), q, kk, v, y_ref)
+            torch.cuda.synchronize()
+            assert torch.equal(ys[i].view(torch.int16), y_ref.view(torch.int16)), (seed, i)
+            prev = want
