@@ -142,3 +142,13 @@ def test_missing_library_fails_loudly(tmp_path):
             "sys.exit(1)\n") % (str(tmp_path / "nope.so"), ROOT)
     p = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True)
     assert p.returncode == 0 and "RAISED" in p.stdout, p.stdout + p.stderr
+
+
+def test_binding_matches_header_arity(L):
+    """Every declared call is bound in Python with as many arguments as the header declares."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    for name, params in re.findall(r"\b(rra_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", text):
+        params = params.strip()
+        arity = 0 if params in ("", "void") else params.count(",") + 1
+        fn = getattr(L, name)
+        assert fn.argtypes is not None and len(fn.argtypes) == arity, (name, arity, fn.argtypes)
