@@ -13,7 +13,7 @@
  * The pages give no formula beyond "attention", so the oracle is the plain definition of
  * softmax(Q K^T * scale) V restricted to the kept tokens of one image and one head.
  *
- * Readings where the pages are silent (each also listed in the design notes):
+ * Readings where the pages are silent:
  *   - keep mask: one byte per (image, token); nonzero = keep;
  *   - kept tokens keep their original order (stable ascending index), images in batch order;
  *   - cu_seqlens[0] = 0, cu_seqlens[b+1] = cu_seqlens[b] + L_b (varlen descriptor);
@@ -238,7 +238,7 @@ int rra_oracle_unpack(const uint8_t *packed, const int32_t *cu, const uint8_t *m
 /*
  * Threshold-l2 token selection, the step in front of the pipeline (aissential.tech summary,
  * Summary: the DeiT models are pruned with Threshold-l2, EViT and other methods -- the pages
- * name the method and nothing more).  Readings, each also listed in the design notes:
+ * name the method and nothing more).  Readings taken where they are silent:
  *   - a token's score is the l2 norm of its embedding row x[b, n, 0..C-1]; the squared norm,
  *     which orders tokens the same way, is what is compared;
  *   - the squared norm is accumulated in IEEE single precision -- the precision the selection

@@ -8,8 +8,9 @@ exactly as the kernel does, and a wait passes when the barrier's phase parity di
 Besides that, the model tracks which phase each wait is *meant* to see, and fails when a wait
 passes before that phase completed, or when a schedule can make no progress.
 
-The roles' orders of waits and arrivals restate the kernel's: see the synchronisation table of
-the attention kernel's design (per-group K/V full barriers, Q slot n % 2, list slot n % 4, ...).
+The roles' orders of waits and arrivals restate the kernel's (csrc/attend.cu): item n belongs to
+softmax group n % 2 and uses Q slot n % 2 and kept-row list slot n % 4; K/V chunks go round a
+3-slot ring in production order, with one "full" barrier per slot and group.
 """
 import random
 
