@@ -152,3 +152,42 @@ def test_binding_matches_header_arity(L):
         arity = 0 if params in ("", "void") else params.count(",") + 1
         fn = getattr(L, name)
         assert fn.argtypes is not None and len(fn.argtypes) == arity, (name, arity, fn.argtypes)
+
+
+try:
+    from hypothesis import given, settings, strategies as st
+
+    bad_field = st.sampled_from(["B", "H", "d", "cap", "ms", "align", "idt", "odt", "scale", "null"])
+
+    @settings(max_examples=200, deadline=None)
+    @given(bad=bad_field, B=st.integers(0, 8192), H=st.integers(1, 64), ms=st.integers(0, 4096),
+           cap=st.integers(1, 1 << 20), odt_same=st.booleans(), idt=st.sampled_from([0, 1]))
+    def test_attend_rejects_any_invalid_field_before_launch(L, bad, B, H, ms, cap, odt_same, idt):
+        """Whatever else the arguments are, one invalid field makes rra_attend return an error code
+        without touching a device (these calls never reach a launch, on any machine)."""
+        args = dict(q=FAKE, o=FAKE, cu=FAKE, B=B, H=H, d=64, ms=ms, cap=cap, scale=0.0, idt=idt,
+                    odt=idt if odt_same else 2)
+        if bad == "B":
+            args["B"] = -1 - B
+        elif bad == "H":
+            args["H"] = -H
+        elif bad == "d":
+            args["d"] = 64 + H
+        elif bad == "cap":
+            args["cap"] = -cap
+        elif bad == "ms":
+            args["ms"] = -1 - ms
+        elif bad == "align":
+            args["q"] = FAKE + 2 * (1 + H % 7)
+        elif bad == "idt":
+            args["idt"] = 2 + H % 3
+        elif bad == "odt":
+            args["odt"] = 1 - idt  # the other 16-bit type
+        elif bad == "scale":
+            args["scale"] = float("nan")
+        else:
+            args["cu"] = None
+        st_code = _attend(L, **args)
+        assert st_code in (rra.RRA_ERR_INVALID_ARG, rra.RRA_ERR_UNSUPPORTED), (bad, args, st_code)
+except ImportError:  # pragma: no cover
+    pass
