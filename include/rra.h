@@ -34,6 +34,11 @@
  *     `dev_error` may be NULL, in which case those errors are not reported -- the kernels
  *     still never read or write outside the buffers described here.
  *   - Device pointers must be 16-byte aligned (the kernels move 16-byte vectors).
+ *   - No output may overlap an input of the same call, nor another output: blocks read the
+ *     inputs of an image while other blocks write the outputs of that image, so an in-place
+ *     call would race.  Every call compares the byte ranges its sizes describe and returns
+ *     RRA_ERR_INVALID_ARG, before any launch, when two of them intersect.  The one exception
+ *     is rra_l2_mask, whose keep_mask may be exactly the same buffer as prev_mask.
  */
 #ifndef RRA_H
 #define RRA_H

@@ -46,6 +46,15 @@ inline int elem_size(rra_dtype dt)
 
 constexpr int64_t kMaxRows = 0x7fffffffLL;
 
+// True when the byte ranges [a, a+na) and [b, b+nb) do not intersect (empty ranges never do).
+inline bool disjoint(const void *a, uint64_t na, const void *b, uint64_t nb)
+{
+    if (a == nullptr || b == nullptr || na == 0 || nb == 0)
+        return true;
+    const uint64_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 + na <= b0 || b0 + nb <= a0;
+}
+
 }  // namespace
 
 extern "C" {
@@ -70,6 +79,21 @@ rra_status rra_pack(const uint8_t *keep_mask, int B, int N, int H, int d, rra_dt
         if (src[i] == nullptr || dst[i] == nullptr)
             return RRA_ERR_INVALID_ARG;
         if (!aligned16(src[i]) || !aligned16(dst[i]))
+            return RRA_ERR_INVALID_ARG;
+    }
+    {
+        // outputs (packed rows, cu_seqlens) must not overlap the inputs (mask, padded rows) or each other
+        const uint64_t mask_b = static_cast<uint64_t>(B) * N, cu_b = 4ull * (B + 1);
+        const uint64_t src_b = mask_b * row_bytes, dst_b = static_cast<uint64_t>(capacity) * row_bytes;
+        for (int i = 0; i < n_tensors; ++i) {
+            if (!disjoint(dst[i], dst_b, keep_mask, mask_b) || !disjoint(dst[i], dst_b, cu_seqlens, cu_b) ||
+                !disjoint(cu_seqlens, cu_b, src[i], src_b))
+                return RRA_ERR_INVALID_ARG;
+            for (int j = 0; j < n_tensors; ++j)
+                if (!disjoint(dst[i], dst_b, src[j], src_b) || (j != i && !disjoint(dst[i], dst_b, dst[j], dst_b)))
+                    return RRA_ERR_INVALID_ARG;
+        }
+        if (!disjoint(cu_seqlens, cu_b, keep_mask, mask_b))
             return RRA_ERR_INVALID_ARG;
     }
     int sms = 0;
@@ -100,6 +124,13 @@ rra_status rra_attend(const void *q, const void *k, const void *v, void *o, cons
         return RRA_ERR_INVALID_ARG;
     if (!(softmax_scale == softmax_scale))
         return RRA_ERR_INVALID_ARG;
+    {
+        const uint64_t rows = static_cast<uint64_t>(capacity) * H * d;
+        const uint64_t in_b = rows * 2, out_b = rows * (out_dt == RRA_F32 ? 4 : 2), cu_b = 4ull * (B + 1);
+        if (!disjoint(o, out_b, q, in_b) || !disjoint(o, out_b, k, in_b) || !disjoint(o, out_b, v, in_b) ||
+            !disjoint(o, out_b, cu_seqlens, cu_b))
+            return RRA_ERR_INVALID_ARG;
+    }
     int sms = 0;
     if (num_sms_of_current_device(&sms) != 0)
         return RRA_ERR_CUDA;
@@ -140,6 +171,17 @@ rra_status rra_pack_attend_unpack(const uint8_t *keep_mask, const void *q, const
         return RRA_ERR_UNSUPPORTED;
     if (!(softmax_scale == softmax_scale))
         return RRA_ERR_INVALID_ARG;
+    {
+        const uint64_t mask_b = static_cast<uint64_t>(B) * N, elems = mask_b * H * d, cu_b = 4ull * (B + 1);
+        const uint64_t in_b = elems * 2, out_b = elems * (out_dt == RRA_F32 ? 4 : 2);
+        const void *ins[4] = {q, k, v, keep_mask};
+        const uint64_t in_sz[4] = {in_b, in_b, in_b, mask_b};
+        for (int i = 0; i < 4; ++i)
+            if (!disjoint(y, out_b, ins[i], in_sz[i]) || !disjoint(cu_seqlens, cu_b, ins[i], in_sz[i]))
+                return RRA_ERR_INVALID_ARG;
+        if (!disjoint(y, out_b, cu_seqlens, cu_b))
+            return RRA_ERR_INVALID_ARG;
+    }
     int sms = 0;
     if (num_sms_of_current_device(&sms) != 0)
         return RRA_ERR_CUDA;
@@ -175,6 +217,12 @@ rra_status rra_l2_mask(const void *x, int B, int N, int C, rra_dtype dt, const i
         return RRA_ERR_UNSUPPORTED;
     if (k_keep == nullptr && threshold_sq != threshold_sq)
         return RRA_ERR_INVALID_ARG;
+    {
+        const uint64_t mask_b = static_cast<uint64_t>(B) * N;
+        if (!disjoint(keep_mask, mask_b, x, mask_b * C * 2) || !disjoint(keep_mask, mask_b, k_keep, 4ull * B) ||
+            (prev_mask != keep_mask && !disjoint(keep_mask, mask_b, prev_mask, mask_b)))
+            return RRA_ERR_INVALID_ARG;
+    }
     const cudaError_t e = rra::launch_l2_mask(x, B, N, C, dt == RRA_BF16, k_keep, threshold_sq, prev_mask, keep_mask,
                                               reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? RRA_OK : RRA_ERR_CUDA;
@@ -206,6 +254,13 @@ rra_status rra_unpack(const void *packed, const int32_t *cu_seqlens, const uint8
         return RRA_ERR_UNSUPPORTED;
     if (B > 65535 || static_cast<int64_t>(B) * N > kMaxRows || capacity > kMaxRows)
         return RRA_ERR_UNSUPPORTED;
+    {
+        const uint64_t mask_b = static_cast<uint64_t>(B) * N;
+        const uint64_t dst_b = mask_b * row_bytes;
+        if (!disjoint(dst, dst_b, packed, static_cast<uint64_t>(capacity) * row_bytes) ||
+            !disjoint(dst, dst_b, cu_seqlens, 4ull * (B + 1)) || !disjoint(dst, dst_b, keep_mask, mask_b))
+            return RRA_ERR_INVALID_ARG;
+    }
     int sms = 0;
     if (num_sms_of_current_device(&sms) != 0)
         return RRA_ERR_CUDA;

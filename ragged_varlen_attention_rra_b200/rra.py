@@ -105,6 +105,46 @@ def _require_cuda(*ts):
             raise ValueError("rra calls take contiguous CUDA tensors")
 
 
+def _expect(cond: bool, msg: str):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _is_mask(t: torch.Tensor) -> bool:
+    return t.dtype in (torch.uint8, torch.bool)
+
+
+def _span(t: torch.Tensor):
+    a = t.data_ptr()
+    return a, a + t.numel() * t.element_size()
+
+
+def _disjoint(outs, ins, what: str):
+    """Each output's bytes must not overlap any input's: the kernels read inputs of an image while
+    other blocks write outputs of the same image, so an in-place call would race."""
+    for o in outs:
+        if o is None or o.numel() == 0:
+            continue
+        o0, o1 = _span(o)
+        for i in ins:
+            if i is None or i.numel() == 0:
+                continue
+            i0, i1 = _span(i)
+            _expect(o1 <= i0 or i1 <= o0, f"{what}: an output overlaps an input")
+
+
+def _check_cu(cu: Optional[torch.Tensor], B: int, what: str):
+    if cu is None:
+        return
+    _expect(cu.dtype == torch.int32 and cu.dim() == 1 and cu.numel() >= B + 1,
+            f"{what}: cu_seqlens must be int32 [B+1] (B = {B}), got {cu.dtype} {tuple(cu.shape)}")
+
+
+def _check_err(err: Optional[torch.Tensor], what: str):
+    if err is not None:
+        _expect(err.dtype == torch.int32 and err.numel() >= 1, f"{what}: dev_error must be an int32 word")
+
+
 # ------------------------------------------------------------------------------------ calls
 
 def rra_status_string(status: int) -> str:
@@ -130,22 +170,49 @@ def rra_pack(mask: torch.Tensor, srcs: Sequence[torch.Tensor], dsts: Sequence[to
              cu_seqlens: torch.Tensor, capacity: Optional[int] = None,
              dev_error: Optional[torch.Tensor] = None, stream=None) -> None:
     """Keep mask [B, N] + padded srcs [B, N, H, d] -> packed dsts [capacity, H, d] and cu_seqlens [B+1]."""
-    _require_cuda(mask, cu_seqlens, dev_error, *srcs, *dsts)
+    what = "rra_pack"
+    _expect(1 <= len(srcs) <= 3 and len(srcs) == len(dsts), f"{what}: 1..3 sources and as many destinations")
+    _expect(_is_mask(mask) and mask.dim() == 2, f"{what}: mask must be uint8/bool [B, N]")
     B, N = mask.shape
-    H, d = srcs[0].shape[2], srcs[0].shape[3]
-    cap = dsts[0].shape[0] if capacity is None else capacity
+    s0 = srcs[0]
+    _expect(s0.dim() == 4 and tuple(s0.shape[:2]) == (B, N) and s0.dtype in _DT,
+            f"{what}: sources must be [B, N, H, d] = [{B}, {N}, H, d] fp16/bf16/fp32")
+    H, d = s0.shape[2], s0.shape[3]
+    for t in srcs:
+        _expect(t.shape == s0.shape and t.dtype == s0.dtype, f"{what}: sources differ in shape or dtype")
+    for t in dsts:
+        _expect(t.dim() == 3 and tuple(t.shape[1:]) == (H, d) and t.dtype == s0.dtype,
+                f"{what}: destinations must be [capacity, {H}, {d}] of the sources' dtype")
+    rows = min(t.shape[0] for t in dsts)
+    cap = rows if capacity is None else int(capacity)
+    _expect(1 <= cap <= rows, f"{what}: capacity {cap} outside [1, {rows}] (rows of the destinations)")
+    _check_cu(cu_seqlens, B, what)
+    _check_err(dev_error, what)
+    _disjoint([*dsts, cu_seqlens], [mask, *srcs], what)
+    _disjoint(list(dsts), [cu_seqlens], what)
+    _require_cuda(mask, cu_seqlens, dev_error, *srcs, *dsts)
     n = len(srcs)
-    src_arr = (ctypes.c_void_p * n)(*[s.data_ptr() for s in srcs])
+    src_arr = (ctypes.c_void_p * n)(*[t.data_ptr() for t in srcs])
     dst_arr = (ctypes.c_void_p * n)(*[t.data_ptr() for t in dsts])
-    st = lib().rra_pack(_ptr(mask), B, N, H, d, _DT[srcs[0].dtype], n, src_arr, dst_arr, cap,
+    st = lib().rra_pack(_ptr(mask), B, N, H, d, _DT[s0.dtype], n, src_arr, dst_arr, cap,
                         _ptr(cu_seqlens), _ptr(dev_error), _stream(stream))
-    _check(st, "rra_pack")
+    _check(st, what)
 
 
 def rra_attend(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, cu_seqlens: torch.Tensor,
                max_seqlen: int, softmax_scale: float = 0.0, dev_error: Optional[torch.Tensor] = None,
                workspace: Optional[torch.Tensor] = None, stream=None) -> None:
     """Packed q/k/v [capacity, H, 64] + cu_seqlens [B+1] -> packed o (o's dtype selects the output type)."""
+    what = "rra_attend"
+    _expect(q.dim() == 3 and q.dtype in (torch.float16, torch.bfloat16), f"{what}: q must be fp16/bf16 [capacity, H, d]")
+    for t in (k, v):
+        _expect(t.shape == q.shape and t.dtype == q.dtype, f"{what}: k and v must match q's shape and dtype")
+    _expect(o.shape == q.shape and o.dtype in (q.dtype, torch.float32),
+            f"{what}: o must be {tuple(q.shape)} in q's dtype or fp32")
+    _expect(cu_seqlens.dtype == torch.int32 and cu_seqlens.dim() == 1 and cu_seqlens.numel() >= 1,
+            f"{what}: cu_seqlens must be int32 [B+1]")
+    _check_err(dev_error, what)
+    _disjoint([o], [q, k, v, cu_seqlens, workspace], what)
     _require_cuda(q, k, v, o, cu_seqlens, dev_error, workspace)
     B = cu_seqlens.shape[0] - 1
     cap, H, d = q.shape
@@ -153,32 +220,54 @@ def rra_attend(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tenso
     st = lib().rra_attend(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cu_seqlens), B, H, d, int(max_seqlen), cap,
                           float(softmax_scale), _DT[q.dtype], _DT[o.dtype], _ptr(workspace), ws_bytes,
                           _ptr(dev_error), _stream(stream))
-    _check(st, "rra_attend")
+    _check(st, what)
 
 
 def rra_unpack(packed: torch.Tensor, cu_seqlens: torch.Tensor, mask: torch.Tensor, dst: torch.Tensor,
                fill_mode: int = 0, capacity: Optional[int] = None, dev_error: Optional[torch.Tensor] = None,
                stream=None) -> None:
     """Packed [capacity, H, d] -> padded dst [B, N, H, d]; pruned rows zero (fill_mode 0) or untouched (1)."""
-    _require_cuda(packed, cu_seqlens, mask, dst, dev_error)
+    what = "rra_unpack"
+    _expect(packed.dim() == 3 and packed.dtype in _DT, f"{what}: packed must be [capacity, H, d]")
+    _expect(_is_mask(mask) and mask.dim() == 2, f"{what}: mask must be uint8/bool [B, N]")
     B, N = mask.shape
-    cap, H, d = packed.shape if capacity is None else (capacity,) + tuple(packed.shape[1:])
+    cap = packed.shape[0] if capacity is None else int(capacity)
+    _expect(1 <= cap <= packed.shape[0], f"{what}: capacity {cap} outside [1, {packed.shape[0]}] (rows of packed)")
+    H, d = packed.shape[1], packed.shape[2]
+    _expect(tuple(dst.shape) == (B, N, H, d) and dst.dtype == packed.dtype,
+            f"{what}: dst must be [{B}, {N}, {H}, {d}] in packed's dtype")
+    _check_cu(cu_seqlens, B, what)
+    _check_err(dev_error, what)
+    _disjoint([dst], [packed, cu_seqlens, mask], what)
+    _require_cuda(packed, cu_seqlens, mask, dst, dev_error)
     st = lib().rra_unpack(_ptr(packed), _ptr(cu_seqlens), _ptr(mask), B, N, H, d, _DT[packed.dtype],
                           int(fill_mode), cap, _ptr(dst), _ptr(dev_error), _stream(stream))
-    _check(st, "rra_unpack")
+    _check(st, what)
 
 
 def rra_pack_attend_unpack(mask: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, y: torch.Tensor,
                            cu_seqlens: Optional[torch.Tensor] = None, softmax_scale: float = 0.0,
                            dev_error: Optional[torch.Tensor] = None, stream=None) -> None:
     """The whole call in one launch: padded q/k/v [B, N, H, 64] + mask [B, N] -> padded y (pruned rows zero)."""
-    _require_cuda(mask, q, k, v, y, cu_seqlens, dev_error)
+    what = "rra_pack_attend_unpack"
+    _expect(_is_mask(mask) and mask.dim() == 2, f"{what}: mask must be uint8/bool [B, N]")
     B, N = mask.shape
+    _expect(q.dim() == 4 and tuple(q.shape[:2]) == (B, N) and q.dtype in (torch.float16, torch.bfloat16),
+            f"{what}: q must be fp16/bf16 [{B}, {N}, H, d]")
+    for t in (k, v):
+        _expect(t.shape == q.shape and t.dtype == q.dtype, f"{what}: k and v must match q's shape and dtype")
+    _expect(y.shape == q.shape and y.dtype in (q.dtype, torch.float32),
+            f"{what}: y must be {tuple(q.shape)} in q's dtype or fp32")
+    _check_cu(cu_seqlens, B, what)
+    _check_err(dev_error, what)
+    _disjoint([y, cu_seqlens], [mask, q, k, v], what)
+    _disjoint([y], [cu_seqlens], what)
+    _require_cuda(mask, q, k, v, y, cu_seqlens, dev_error)
     H, d = q.shape[2], q.shape[3]
     st = lib().rra_pack_attend_unpack(_ptr(mask), _ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(cu_seqlens), B, N, H, d,
                                       float(softmax_scale), _DT[q.dtype], _DT[y.dtype], _ptr(dev_error),
                                       _stream(stream))
-    _check(st, "rra_pack_attend_unpack")
+    _check(st, what)
 
 
 def rra_l2_mask(x: torch.Tensor, keep_mask: torch.Tensor, k_keep: Optional[torch.Tensor] = None,
@@ -186,12 +275,24 @@ def rra_l2_mask(x: torch.Tensor, keep_mask: torch.Tensor, k_keep: Optional[torch
     """Threshold-l2 selection: embeddings x [B, N, C] (fp16/bf16) -> keep_mask uint8 [B, N] (CLS kept).
 
     With k_keep (int32 [B]) image b keeps its k_b highest-norm candidates; otherwise every
-    candidate whose squared norm reaches threshold_sq.  Candidates: n >= 1 kept in prev_mask."""
-    _require_cuda(x, keep_mask, k_keep, prev_mask)
+    candidate whose squared norm reaches threshold_sq.  Candidates: n >= 1 kept in prev_mask
+    (which may be keep_mask itself)."""
+    what = "rra_l2_mask"
+    _expect(x.dim() == 3 and x.dtype in (torch.float16, torch.bfloat16), f"{what}: x must be fp16/bf16 [B, N, C]")
     B, N, C = x.shape
+    _expect(keep_mask.dtype == torch.uint8 and tuple(keep_mask.shape) == (B, N),
+            f"{what}: keep_mask must be uint8 [{B}, {N}]")
+    if k_keep is not None:
+        _expect(k_keep.dtype == torch.int32 and k_keep.numel() >= B, f"{what}: k_keep must be int32 [{B}]")
+    if prev_mask is not None:
+        _expect(_is_mask(prev_mask) and tuple(prev_mask.shape) == (B, N), f"{what}: prev_mask must be uint8 [{B}, {N}]")
+    _disjoint([keep_mask], [x, k_keep], what)
+    if prev_mask is not None and prev_mask.data_ptr() != keep_mask.data_ptr():
+        _disjoint([keep_mask], [prev_mask], what)
+    _require_cuda(x, keep_mask, k_keep, prev_mask)
     st = lib().rra_l2_mask(_ptr(x), B, N, C, _DT[x.dtype], _ptr(k_keep), float(threshold_sq), _ptr(prev_mask),
                            _ptr(keep_mask), _stream(stream))
-    _check(st, "rra_l2_mask")
+    _check(st, what)
 
 
 # ------------------------------------------------------------------------------------ whole call
@@ -218,6 +319,10 @@ def forward(mask: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tenso
     Enqueued on `stream` without any host synchronisation; the padded result is bufs.y (pruned
     rows zero).  fused=True runs the same call as the single launch rra_pack_attend_unpack
     (bufs.cu is written, the packed buffers are not used)."""
+    _expect(tuple(mask.shape) == (bufs.B, bufs.N), f"forward: mask {tuple(mask.shape)} != buffers' [{bufs.B}, {bufs.N}]")
+    for t in (q, k, v):
+        _expect(tuple(t.shape) == (bufs.B, bufs.N, bufs.H, 64) and t.dtype == bufs.packed[0].dtype,
+                f"forward: q/k/v must be [{bufs.B}, {bufs.N}, {bufs.H}, 64] {bufs.packed[0].dtype}")
     if fused:
         rra_pack_attend_unpack(mask, q, k, v, bufs.y, bufs.cu, softmax_scale=softmax_scale, dev_error=bufs.err,
                                stream=stream)

@@ -191,3 +191,94 @@ try:
         assert st_code in (rra.RRA_ERR_INVALID_ARG, rra.RRA_ERR_UNSUPPORTED), (bad, args, st_code)
 except ImportError:  # pragma: no cover
     pass
+
+
+def test_overlapping_output_is_rejected_before_launch(L):
+    """An output whose bytes intersect an input's is refused with RRA_ERR_INVALID_ARG before any
+    CUDA call (every other argument here is valid, so only the overlap check can answer)."""
+    # rra_attend, o == q
+    assert _attend(L, q=FAKE, o=FAKE) == rra.RRA_ERR_INVALID_ARG
+    # o starts inside q (capacity 16 rows x 128 bytes of bf16 = 2048 bytes)
+    assert _attend(L, q=FAKE, o=FAKE + 1024) == rra.RRA_ERR_INVALID_ARG
+    # single launch: y overlaps v, or cu_seqlens overlaps q
+    f = L.rra_pack_attend_unpack
+    assert f(FAKE, 0x100000, 0x200000, 0x300000, 0x300000, None, 2, 8, 1, 64, 0.0, 1, 1, None, None) == \
+        rra.RRA_ERR_INVALID_ARG
+    assert f(FAKE, 0x100000, 0x200000, 0x300000, 0x400000, 0x100010, 2, 8, 1, 64, 0.0, 1, 1, None, None) == \
+        rra.RRA_ERR_INVALID_ARG
+    # unpack: dst overlaps the mask
+    assert L.rra_unpack(0x100000, 0x200000, 0x300000, 2, 8, 1, 64, 1, 0, 16, 0x300000, None, None) == \
+        rra.RRA_ERR_INVALID_ARG
+    # pack: a destination overlaps a source
+    assert _pack(L, srcp=0x100000, dstp=0x100000, cu=0x900000) == rra.RRA_ERR_INVALID_ARG
+    # l2 mask: keep_mask overlaps the embeddings; keep_mask partially overlapping prev_mask
+    g = L.rra_l2_mask
+    assert g(0x100000, 2, 8, 16, 1, None, 1.0, None, 0x100000, None) == rra.RRA_ERR_INVALID_ARG
+    assert g(0x100000, 2, 8, 16, 1, None, 1.0, 0x200008, 0x200000, None) == rra.RRA_ERR_INVALID_ARG
+
+
+class _T:
+    """CPU tensors with the shapes of a call: the binding's shape and dtype checks run before its
+    device check, so every mismatch below is reported without a GPU."""
+
+    def __init__(self, B=2, N=8, H=2, dt=None):
+        import torch
+        dt = dt or torch.bfloat16
+        self.torch = torch
+        self.mask = torch.ones(B, N, dtype=torch.uint8)
+        self.q, self.k, self.v = (torch.zeros(B, N, H, 64, dtype=dt) for _ in range(3))
+        self.y = torch.zeros(B, N, H, 64, dtype=dt)
+        self.cu = torch.zeros(B + 1, dtype=torch.int32)
+        self.packed = [torch.zeros(B * N, H, 64, dtype=dt) for _ in range(3)]
+        self.o = torch.zeros(B * N, H, 64, dtype=dt)
+
+
+def _raises(fn, match):
+    with pytest.raises(ValueError, match=match):
+        fn()
+
+
+def test_binding_checks_shapes_and_dtypes():
+    t = _T()
+    torch = t.torch
+    # a well-formed call on CPU tensors reaches the device check
+    _raises(lambda: rra.rra_pack_attend_unpack(t.mask, t.q, t.k, t.v, t.y, t.cu), "CUDA")
+    _raises(lambda: rra.rra_attend(*t.packed, t.o, t.cu, max_seqlen=8), "CUDA")
+    # rra_attend: k/v/o shape or dtype different from q, cu_seqlens of the wrong type
+    _raises(lambda: rra.rra_attend(t.packed[0], t.packed[1][:5], t.packed[2], t.o, t.cu, 8), "k and v")
+    _raises(lambda: rra.rra_attend(t.packed[0], t.packed[1].half(), t.packed[2], t.o, t.cu, 8), "k and v")
+    _raises(lambda: rra.rra_attend(*t.packed, t.o[:, :1], t.cu, 8), "o must be")
+    _raises(lambda: rra.rra_attend(*t.packed, t.o.half(), t.cu, 8), "o must be")
+    _raises(lambda: rra.rra_attend(*t.packed, t.o, t.cu.long(), 8), "cu_seqlens")
+    _raises(lambda: rra.rra_attend(t.packed[0], t.packed[1], t.packed[2], t.packed[0], t.cu, 8), "overlaps")
+    # rra_unpack: capacity beyond packed rows, dst shape or dtype, mask dtype, short cu_seqlens
+    _raises(lambda: rra.rra_unpack(t.o, t.cu, t.mask, t.y, capacity=t.o.shape[0] + 1), "capacity")
+    _raises(lambda: rra.rra_unpack(t.o, t.cu, t.mask, t.y[:1]), "dst must be")
+    _raises(lambda: rra.rra_unpack(t.o, t.cu, t.mask, t.y.float()), "dst must be")
+    _raises(lambda: rra.rra_unpack(t.o, t.cu, t.mask.int(), t.y), "mask")
+    _raises(lambda: rra.rra_unpack(t.o, t.cu[:2], t.mask, t.y), "cu_seqlens")
+    # rra_pack: destination row size, destination dtype, capacity, source shapes
+    _raises(lambda: rra.rra_pack(t.mask, [t.q], [t.o[:, :1]], t.cu), "destinations")
+    _raises(lambda: rra.rra_pack(t.mask, [t.q], [t.o.half()], t.cu), "destinations")
+    _raises(lambda: rra.rra_pack(t.mask, [t.q], [t.o], t.cu, capacity=t.o.shape[0] + 1), "capacity")
+    _raises(lambda: rra.rra_pack(t.mask, [t.q, t.k[:1]], t.packed[:2], t.cu), "sources")
+    _raises(lambda: rra.rra_pack(t.mask[:1], [t.q], [t.o], t.cu), "sources")
+    _raises(lambda: rra.rra_pack(t.mask, [t.q], [t.o, t.o], t.cu), "destinations")
+    # single launch: y shape/dtype, k/v dtype, mask vs q, cu_seqlens length
+    _raises(lambda: rra.rra_pack_attend_unpack(t.mask, t.q, t.k, t.v, t.y[:1]), "y must be")
+    _raises(lambda: rra.rra_pack_attend_unpack(t.mask, t.q, t.k, t.v, t.y.half()), "y must be")
+    _raises(lambda: rra.rra_pack_attend_unpack(t.mask, t.q, t.k.half(), t.v, t.y), "k and v")
+    _raises(lambda: rra.rra_pack_attend_unpack(t.mask[:, :4], t.q, t.k, t.v, t.y), "q must be")
+    _raises(lambda: rra.rra_pack_attend_unpack(t.mask, t.q, t.k, t.v, t.y, t.cu[:1]), "cu_seqlens")
+    _raises(lambda: rra.rra_pack_attend_unpack(t.mask, t.q, t.k, t.v, t.q), "overlaps")
+    # rra_l2_mask: mask shape, k_keep dtype, prev_mask shape
+    x = torch.zeros(2, 8, 16, dtype=torch.bfloat16)
+    _raises(lambda: rra.rra_l2_mask(x, torch.zeros(2, 7, dtype=torch.uint8)), "keep_mask")
+    _raises(lambda: rra.rra_l2_mask(x, t.mask, k_keep=torch.zeros(2, dtype=torch.int64)), "k_keep")
+    _raises(lambda: rra.rra_l2_mask(x, t.mask, prev_mask=t.mask[:1]), "prev_mask")
+    _raises(lambda: rra.rra_l2_mask(x, t.mask, prev_mask=t.mask), "CUDA")  # in place is allowed
+    # forward: mask or q/k/v that do not match the buffers
+    bufs = type("Bufs", (), {"B": 2, "N": 8, "H": 2, "packed": t.packed, "y": t.y, "cu": t.cu, "err": None,
+                             "o": t.o})()
+    _raises(lambda: rra.forward(t.mask[:1], t.q, t.k, t.v, bufs), "mask")
+    _raises(lambda: rra.forward(t.mask, t.q[:, :, :1], t.k, t.v, bufs), "q/k/v")
