@@ -1,10 +1,12 @@
 #!/usr/bin/env python
 """Benchmark of the pack -> attend -> unpack call on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c5:1.0:512] [--impl ours|reference]
 
 One step = one whole pack -> attend -> unpack call for every pruning stage of the workload,
-replayed from a CUDA graph over inputs resident in HBM.  The call runs either as the single
+replayed from a CUDA graph over inputs resident in HBM.  The default workload is the largest
+single-GPU configuration: DeiT-B head shape (H=12, d=64, N=197), keep ratio 1.0, B=512 images
+(100,864 tokens per call).  The call runs either as the single
 launch rra_pack_attend_unpack (--path fused, the default: identical bytes out) or as the three
 launches rra_pack, rra_attend, rra_unpack (--path three); the other path is timed afterwards
 and reported beside it.  L2 is flushed (a 256 MiB write, untimed) before every timed step, and
@@ -13,15 +15,19 @@ inside the graph give the per-kernel times.
 
 Prints ONE JSON line on rank 0: packed tokens/s (whole job), us per call, the roofline of the
 dominant kernel, end-to-end throughput through the public API with pinned host buffers,
-the float64 CPU oracle on a bounded sample, clocks sampled during the timed region, and how
-many of this library's kernels ran in the timed region.
+the float64 CPU oracle on a bounded sample (one core and all of the host's cores), clocks
+sampled during the timed region, how many of this library's kernels ran in the timed region,
+and (N = 1, unless --no-sweep) a `sweep` over every configured cell: config 5's keep ratio x
+batch grid and three-stage rows, configs 1-4 -- per cell the graph-replayed us per call with L2
+cold and warm, eager us per call, packed tokens/s, attention TFLOP/s, the kernel's fraction of
+the HBM roofline, and the same for the three-call path.
 
 With torchrun (N > 1) every rank runs an independent replica of the workload on its own GPU
 (images are independent, so the path shards with no exchange): weak scaling, timings reduced
 as the max over ranks.
 
---impl reference times the float64 CPU oracle itself (rank 0 only) on the same workload,
-metric and unit, one bounded sample of images per step.
+--impl reference times the float64 CPU oracle itself (rank 0 only, all host cores, one thread
+per image) on the same workload, metric and unit, one bounded sample of images per step.
 """
 from __future__ import annotations
 
@@ -105,9 +111,8 @@ def ncu_traffic(kernel, workload):
     return e.get("dram_bytes_per_launch")
 
 
-def algorithmic_bytes(w, lengths, row_bytes, out_row_bytes):
+def algorithmic_bytes(B, N, lengths, row_bytes, out_row_bytes):
     """Per-stage algorithmic HBM bytes of each kernel (the minimal reads + writes)."""
-    B, N = w.B, w.N
     T = int(lengths.sum())
     return {
         "pack": B * N + 2 * 3 * T * row_bytes + 4 * (B + 1),
@@ -119,16 +124,16 @@ def algorithmic_bytes(w, lengths, row_bytes, out_row_bytes):
 
 
 class ClockSampler:
-    """SM clock and clock-event (throttle) reasons sampled through NVML every ~2 ms by a
+    """SM clock and clock-event (throttle) reasons sampled through NVML every ~0.5 ms by a
     background thread while the timed region runs (nvidia-smi's 200 ms loop is too coarse
-    for a timed region of tens of milliseconds)."""
+    for a timed region of milliseconds)."""
 
     REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
                "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
                "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
                "sw_power_cap": "nvmlClocksEventReasonSwPowerCap"}
 
-    def __init__(self, torch_index, period_s=0.002):
+    def __init__(self, torch_index, period_s=0.0005):
         self.torch_index = torch_index
         self.period = period_s
         self.samples = []
@@ -179,40 +184,63 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------------ CPU oracle
 
-def oracle_call(w, stage_masks, images):
-    """One oracle pack-attend-unpack over the given images of every stage; returns tokens done."""
-    sys.path.insert(0, ROOT)
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def oracle_call(q, k, v, H, dtype, stage_masks, images):
+    """One oracle pack-attend-unpack over the given images of every stage; returns tokens done.
+    The oracle's C calls release the GIL, so threads running this on disjoint images run on
+    separate cores."""
     from oracle import oracle as O
     sel = torch.as_tensor(images, dtype=torch.long)
-    q, k, v = w.q[sel], w.k[sel], w.v[sel]
+    qs, ks, vs = q[sel], k[sel], v[sel]
     tokens = 0
     for m in stage_masks:
         ms = m[sel]
-        qp, cu = O.pack(ms, q)
-        kp, _ = O.pack(ms, k)
-        vp, _ = O.pack(ms, v)
-        o = O.attend(qp, kp, vp, cu, w.H, 64, dtype=w.dtype)
+        qp, cu = O.pack(ms, qs)
+        kp, _ = O.pack(ms, ks)
+        vp, _ = O.pack(ms, vs)
+        o = O.attend(qp, kp, vp, cu, H, 64, dtype=dtype)
         O.unpack(o, cu, ms)
         tokens += int(cu[-1])
     return tokens
 
 
+def oracle_images(w, images, threads):
+    """The oracle over `images` (every stage), one image per task on `threads` threads; tokens."""
+    if threads <= 1:
+        return sum(oracle_call(w.q, w.k, w.v, w.H, w.dtype, w.masks, [i]) for i in images)
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        return sum(ex.map(lambda i: oracle_call(w.q, w.k, w.v, w.H, w.dtype, w.masks, [i]), images))
+
+
 def cpu_baseline(w, budget_s=10.0):
-    """The oracle, as it stands, on whole calls of the workload until about `budget_s` of CPU time."""
+    """The oracle, as it stands, on a bounded sample of the workload's images: first on one core
+    for about budget_s / 3, then on all host cores (one thread per image) for about the rest."""
     from oracle import oracle as O
     O.load()
-    imgs = list(range(w.B))
-    t0 = time.perf_counter()
-    tokens, calls = 0, 0
-    while True:
-        tokens += oracle_call(w, w.masks, imgs)
-        calls += 1
-        if time.perf_counter() - t0 >= budget_s:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": tokens / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{calls} whole call(s) of {w.name} (all {w.B} images, {len(w.masks)} stage(s)), "
-                      f"single-threaded float64 C, {dt:.1f} s"}
+    cores = host_cores()
+    out = {}
+    for leg, threads, budget in (("single", 1, budget_s / 3), ("multi", cores, 2 * budget_s / 3)):
+        t0 = time.perf_counter()
+        tokens, done = 0, 0
+        while time.perf_counter() - t0 < budget and done < 4 * w.B:
+            batch = [(done + j) % w.B for j in range(threads)]
+            tokens += oracle_images(w, batch, threads)
+            done += len(batch)
+        dt = time.perf_counter() - t0
+        out[leg] = {"value": tokens / dt, "images": done, "seconds": dt, "threads": threads}
+    m = out["multi"]
+    return {"value": m["value"], "unit": UNIT, "cores": m["threads"], "kind": "oracle",
+            "sample": f"{m['images']} image(s) of {w.name} (every stage) on {m['threads']} threads, one image "
+                      f"per thread, float64 C, {m['seconds']:.1f} s; host has {cores} usable cores",
+            "single_core": {"value": out["single"]["value"], "unit": UNIT, "cores": 1,
+                            "sample": f"{out['single']['images']} image(s), {out['single']['seconds']:.1f} s"}}
 
 
 def run_reference(args):
@@ -222,27 +250,29 @@ def run_reference(args):
     w = workloads.by_name(args.workload)
     from oracle import oracle as O
     O.load()
-    per_step = max(1, min(w.B, args.ref_images))
-    order = list(range(w.B))
+    cores = host_cores()
+    per_step = max(1, min(w.B, args.ref_images if args.ref_images > 0 else cores))
     step_tokens, step_times = [], []
     for i in range(args.warmup + args.steps):
-        imgs = [order[(i * per_step + j) % w.B] for j in range(per_step)]
+        imgs = [(i * per_step + j) % w.B for j in range(per_step)]
         t0 = time.perf_counter()
-        tok = oracle_call(w, w.masks, imgs)
+        tok = oracle_images(w, imgs, min(cores, per_step))
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             step_tokens.append(tok)
             step_times.append(dt)
     total_t = sum(step_times)
     value = sum(step_tokens) / total_t
+    threads = min(cores, per_step)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d": 64, "stages": len(w.masks),
                    "seed": w.seed, "recipe": w.recipe, "l2": "n/a (CPU)"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"{per_step} image(s) of {w.name} per step, every stage, single-threaded"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{per_step} image(s) of {w.name} per step, every stage, {threads} threads "
+                                   f"(one image each); host has {cores} usable cores"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -252,19 +282,21 @@ def run_reference(args):
 # ------------------------------------------------------------------------------------ GPU arm
 
 class Pipeline:
-    """Device buffers + CUDA graphs of the whole call (all stages): `graph` holds the kernels
-    alone (the timed one: kernels that follow one another may overlap their start-up through
-    programmatic dependent launch), `graph_ev` the same kernels with an event between each pair
-    (for the per-kernel breakdown; the events serialise the kernels)."""
+    """Device buffers + CUDA graphs of the whole call (all stages) on device-resident inputs:
+    `graph` holds the kernels alone (the timed one: kernels that follow one another may overlap
+    their start-up through programmatic dependent launch), `graph_ev` the same kernels with an
+    event between each pair (for the per-kernel breakdown; the events serialise the kernels)."""
 
-    def __init__(self, w, out_dtype, stream, path):
-        self.w = w
+    def __init__(self, q, k, v, masks, out_dtype, stream, path):
         self.path = path
-        dev = "cuda"
-        self.masks = [m.to(dev) for m in w.masks]
-        self.q, self.k, self.v = (t.to(dev) for t in (w.q, w.k, w.v))
-        self.bufs = rra.Buffers(w.B, w.N, w.H, w.q.dtype, out_dtype=out_dtype)
-        self.ys = [torch.empty(w.B, w.N, w.H, 64, dtype=self.bufs.y.dtype, device=dev) for _ in self.masks]
+        self.q, self.k, self.v = q, k, v
+        self.masks = masks
+        self.B, self.N, self.H = q.shape[0], q.shape[1], q.shape[2]
+        self.bufs = rra.Buffers(self.B, self.N, self.H, q.dtype, out_dtype=out_dtype)
+        if path == "fused":  # the single launch uses no packed buffers
+            self.bufs.packed = [t[:1] for t in self.bufs.packed]
+            self.bufs.o = self.bufs.o[:1]
+        self.ys = [torch.empty(self.B, self.N, self.H, 64, dtype=self.bufs.y.dtype, device="cuda") for _ in masks]
         self.stream = stream
         self.graph = None
         self.graph_ev = None
@@ -287,7 +319,7 @@ class Pipeline:
             rra.rra_pack(m, [self.q, self.k, self.v], b.packed, b.cu, dev_error=b.err, stream=s)
             if events:
                 events[nk * i + 1].record(s)
-            rra.rra_attend(b.packed[0], b.packed[1], b.packed[2], b.o, b.cu, max_seqlen=self.w.N,
+            rra.rra_attend(b.packed[0], b.packed[1], b.packed[2], b.o, b.cu, max_seqlen=self.N,
                            dev_error=b.err, stream=s)
             if events:
                 events[nk * i + 2].record(s)
@@ -356,14 +388,14 @@ def time_path(pipe, flush, steps, warmup, stream):
     return step_ms, kern
 
 
-def time_mask_producer(w, flush, stream, steps, warmup, hbm_peak):
+def time_mask_producer(B, N, H, seed, flush, stream, steps, warmup, hbm_peak):
     """The token-selection step in front of the path (rra_l2_mask, top-k mode) on embeddings of
     the workload's width (C = 64 H, DeiT's embedding size) and keep counts from the configs'
     recipe: per-launch device time (L2 flushed before each launch), algorithmic bytes, GB/s."""
-    C = 64 * w.H
-    x = workloads.embeddings(w.B, w.N, C, "bf16", seed=w.seed).cuda()
-    k = torch.from_numpy(workloads.keep_counts(w.B, w.N, seed=w.seed)).cuda()
-    mask = torch.empty(w.B, w.N, dtype=torch.uint8, device="cuda")
+    C = 64 * H
+    x = workloads.embeddings(B, N, C, "bf16", seed=seed).cuda()
+    k = torch.from_numpy(workloads.keep_counts(B, N, seed=seed)).cuda()
+    mask = torch.empty(B, N, dtype=torch.uint8, device="cuda")
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ms = []
     for i in range(warmup + steps):
@@ -376,10 +408,147 @@ def time_mask_producer(w, flush, stream, steps, warmup, hbm_peak):
         if i >= warmup:
             ms.append(start.elapsed_time(end))
     us = 1e3 * statistics.mean(ms)
-    nbytes = w.B * w.N * C * 2 + w.B * w.N + 4 * w.B
+    nbytes = B * N * C * 2 + B * N + 4 * B
     gbs = nbytes / (us * 1e3)
-    return {"call": "rra_l2_mask (top-k)", "B": w.B, "N": w.N, "C": C, "us_per_launch": us,
+    return {"call": "rra_l2_mask (top-k)", "B": B, "N": N, "C": C, "us_per_launch": us,
             "alg_bytes_per_launch": nbytes, "gbs": gbs, "frac_of_hbm": gbs / hbm_peak}
+
+
+def kernel_table(kms, alg, stages, hbm_peak):
+    table = {}
+    for k, v in kms.items():
+        if not v:
+            return None
+        per_launch_us = 1e3 * statistics.mean(v)
+        per_launch_bytes = alg[k] / stages
+        gbs = per_launch_bytes / (per_launch_us * 1e3)
+        table[k] = {"us_per_launch": per_launch_us, "gbs": gbs, "alg_bytes_per_launch": per_launch_bytes,
+                    "frac_of_hbm": gbs / hbm_peak}
+    return table
+
+
+def attention_flops(lengths):
+    return sum(4 * 64 * int(H_) * int((l.astype(np.int64) ** 2).sum()) for H_, l in lengths)
+
+
+def empty_graph_floor(stream, reps=200):
+    """Device time per replay of a graph holding one trivial kernel (a 4-byte fill): the floor
+    that graph launch and kernel start-up put under any call."""
+    x = torch.zeros(1, dtype=torch.int32, device="cuda")
+    with torch.cuda.stream(stream):
+        x.fill_(1)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        x.fill_(2)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(10):
+            g.replay()
+        start.record(stream)
+        for _ in range(reps):
+            g.replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / reps * 1e3
+
+
+def run_sweep(names, flush, stream, hbm_peak, cold_reps=10, warm_reps=100, eager_reps=30):
+    """Every named cell on inputs drawn on the device (values of the largest batch of each shape,
+    sliced for the smaller ones; masks from the cell's recipe).  Per cell: the single launch's
+    graph replay us per call with L2 flushed before each replay (cold) and back to back (warm),
+    eager us per call through the API, tokens/s, attention TFLOP/s, its HBM roofline fraction
+    from in-graph events, and the three-call path's cold us per call with its output checked
+    byte for byte against the single launch's."""
+    shapes = {}
+    for n in names:
+        B, N, H, dt, std = workloads.shape_of(n)
+        key = (N, H, dt, std)
+        shapes[key] = max(shapes.get(key, 0), B)
+    order = sorted(names, key=lambda n: workloads.shape_of(n)[1:])
+    cells, cur_key, vals = {}, None, None
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for name in order:
+        B, N, H, dt, std = workloads.shape_of(name)
+        key = (N, H, dt, std)
+        if key != cur_key:
+            vals = None
+            torch.cuda.empty_cache()
+            vals = workloads.device_values(shapes[key], N, H, dt, seed=0, std=std)
+            cur_key = key
+        q, k, v = (t[:B] for t in vals)
+        masks_np = workloads.sweep_masks(name)
+        masks = [torch.from_numpy(np.ascontiguousarray(m)).cuda() for m in masks_np]
+        lengths = [m.astype(bool).sum(axis=1) for m in masks_np]
+        T_call = int(sum(int(l.sum()) for l in lengths))
+        row_bytes = H * 64 * 2
+        entry = {"B": B, "N": N, "H": H, "stages": len(masks), "tokens_per_call": T_call}
+        res = {}
+        for path in ("fused", "three"):
+            pipe = Pipeline(q, k, v, masks, None, stream, path)
+            pipe.capture()
+            cold = []
+            for i in range(cold_reps + 2):
+                with torch.cuda.stream(stream):
+                    flush.fill_(i & 0xFF)
+                    start.record(stream)
+                    pipe.graph.replay()
+                    end.record(stream)
+                stream.synchronize()
+                if i >= 2:
+                    cold.append(start.elapsed_time(end))
+            kern = {kk: [] for kk in pipe.kernels}
+            for i in range(cold_reps):
+                with torch.cuda.stream(stream):
+                    flush.fill_((i + 5) & 0xFF)
+                    pipe.graph_ev.replay()
+                stream.synchronize()
+                for kk, vv in pipe.kernel_times().items():
+                    kern[kk].extend(vv)
+            res[path] = (pipe, 1e3 * statistics.mean(cold), kern)
+            if path == "fused":
+                with torch.cuda.stream(stream):
+                    start.record(stream)
+                    for _ in range(warm_reps):
+                        pipe.graph.replay()
+                    end.record(stream)
+                torch.cuda.synchronize()
+                entry["us_warm"] = start.elapsed_time(end) / warm_reps * 1e3
+                with torch.cuda.stream(stream):
+                    pipe.enqueue()
+                    start.record(stream)
+                    for _ in range(eager_reps):
+                        pipe.enqueue()
+                    end.record(stream)
+                torch.cuda.synchronize()
+                entry["us_eager"] = start.elapsed_time(end) / eager_reps * 1e3
+        fused_pipe, us_cold, kern = res["fused"]
+        three_pipe, us_cold3, kern3 = res["three"]
+        for pipe in (fused_pipe, three_pipe):
+            err = rra.rra_get_device_error(pipe.bufs.err, stream)
+            if err != 0:
+                raise RuntimeError(f"device error {rra.rra_status_string(err)} in sweep cell {name}")
+        alg = {}
+        for l in lengths:
+            for kk, bb in algorithmic_bytes(B, N, l, row_bytes, row_bytes).items():
+                alg[kk] = alg.get(kk, 0) + bb
+        kt = kernel_table(kern, alg, len(masks), hbm_peak)
+        kt3 = kernel_table(kern3, alg, len(masks), hbm_peak)
+        flops = attention_flops([(H, l) for l in lengths])
+        k_us = kt["pack_attend_unpack"]["us_per_launch"] * len(masks)
+        entry.update({
+            "us_cold": us_cold, "tokens_per_s": T_call / (us_cold * 1e-6),
+            "kernel_us": kt["pack_attend_unpack"]["us_per_launch"],
+            "frac_of_hbm": kt["pack_attend_unpack"]["frac_of_hbm"],
+            "attention_tflops": flops / (k_us * 1e-6) / 1e12,
+            "three_calls": {"us_cold": us_cold3, "kernels_us": {kk: vv["us_per_launch"] for kk, vv in kt3.items()},
+                            "frac_of_hbm": {kk: vv["frac_of_hbm"] for kk, vv in kt3.items()},
+                            "identical_output": all(torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+                                                    for a, b in zip(fused_pipe.ys, three_pipe.ys))},
+        })
+        cells[name] = entry
+        del res, fused_pipe, three_pipe
+    return {n: cells[n] for n in names}
 
 
 def main_gpu(args):
@@ -392,15 +561,15 @@ def main_gpu(args):
     w = workloads.by_name(args.workload)
     stream = torch.cuda.Stream()
     out_dtype = torch.float32 if args.out == "f32" else None
-    pipe = Pipeline(w, out_dtype, stream, args.path)
+    dq, dk, dv = (t.cuda() for t in (w.q, w.k, w.v))
+    dmasks = [m.cuda() for m in w.masks]
+    pipe = Pipeline(dq, dk, dv, dmasks, out_dtype, stream, args.path)
     pipe.capture()
-    other = Pipeline(w, out_dtype, stream, "three" if args.path == "fused" else "fused")
-    other.capture()
     stages = len(w.masks)
     lengths = w.lengths
     T_call = int(sum(int(l.sum()) for l in lengths))
     row_bytes = w.H * 64 * w.q.element_size()
-    out_row_bytes = w.H * 64 * pipe.bufs.o.element_size()
+    out_row_bytes = w.H * 64 * pipe.bufs.y.element_size()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
     if ws > 1:
@@ -415,16 +584,18 @@ def main_gpu(args):
     err = rra.rra_get_device_error(pipe.bufs.err, stream)
     if err != 0:
         raise RuntimeError(f"device error {rra.rra_status_string(err)} in the timed region")
+    total_ms = reduce_max(float(sum(step_ms)), device="cuda")
+    ms_per_step = total_ms / args.steps
+    value = job_throughput(ws, args.steps, T_call, total_ms)
+
     # the other path, same workload, same protocol (reported beside the headline)
+    other = Pipeline(dq, dk, dv, dmasks, out_dtype, stream, "three" if args.path == "fused" else "fused")
+    other.capture()
     o_step_ms, o_kern_ms = time_path(other, flush, args.steps, args.warmup, stream)
     err = rra.rra_get_device_error(other.bufs.err, stream)
     if err != 0:
         raise RuntimeError(f"device error {rra.rra_status_string(err)} on the {other.path} path")
     same = all(torch.equal(a.view(torch.uint8), b.view(torch.uint8)) for a, b in zip(pipe.ys, other.ys))
-
-    total_ms = reduce_max(float(sum(step_ms)), device="cuda")
-    ms_per_step = total_ms / args.steps
-    value = job_throughput(ws, args.steps, T_call, total_ms)
 
     # dispatch floor: host time to enqueue one graph replay, and one eager call through the API
     torch.cuda.synchronize()
@@ -456,30 +627,19 @@ def main_gpu(args):
     hbm_peak, peak_kind = peaks()
     alg = {}
     for l in lengths:
-        for k, b in algorithmic_bytes(w, l, row_bytes, out_row_bytes).items():
+        for k, b in algorithmic_bytes(w.B, w.N, l, row_bytes, out_row_bytes).items():
             alg[k] = alg.get(k, 0) + b
-
-    def kernel_table(kms):
-        table = {}
-        for k, v in kms.items():
-            if not v:
-                return None
-            per_launch_us = 1e3 * statistics.mean(v)
-            per_launch_bytes = alg[k] / stages
-            gbs = per_launch_bytes / (per_launch_us * 1e3)
-            table[k] = {"us_per_launch": per_launch_us, "gbs": gbs, "alg_bytes_per_launch": per_launch_bytes,
-                        "frac_of_hbm": gbs / hbm_peak}
-        return table
-
-    per_kernel = kernel_table(kern_ms)
-    other_kernels = kernel_table(o_kern_ms)
+    per_kernel = kernel_table(kern_ms, alg, stages, hbm_peak)
+    other_kernels = kernel_table(o_kern_ms, alg, stages, hbm_peak)
     roofline = None
     if per_kernel:
         dom = max(per_kernel, key=lambda k: per_kernel[k]["us_per_launch"])
         ach = per_kernel[dom]["gbs"]
         roofline = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": ach / hbm_peak, "peak_source": peak_kind, "traffic": ncu_traffic(dom, w.name)}
-    flops = sum(4 * 64 * w.H * int((l.astype(np.int64) ** 2).sum()) for l in lengths)
+                    "frac": ach / hbm_peak, "peak_source": peak_kind, "traffic": ncu_traffic(dom, w.name),
+                    "alg_bytes_per_launch": per_kernel[dom]["alg_bytes_per_launch"],
+                    "us_per_launch": per_kernel[dom]["us_per_launch"]}
+    flops = attention_flops([(w.H, l) for l in lengths])
     attn_key = "pack_attend_unpack" if args.path == "fused" else "attend"
     attn_tflops = (flops / (per_kernel[attn_key]["us_per_launch"] * stages * 1e-6) / 1e12) if per_kernel else None
 
@@ -489,19 +649,19 @@ def main_gpu(args):
         host_in = [t.pin_memory() for t in (w.q, w.k, w.v)]
         host_masks = [m.pin_memory() for m in w.masks]
         host_out = [torch.empty(pipe.ys[0].shape, dtype=pipe.ys[0].dtype).pin_memory() for _ in w.masks]
-        dq, dk, dv = (torch.empty(w.q.shape, dtype=w.q.dtype, device="cuda") for _ in range(3))
-        dmasks = [torch.empty(m.shape, dtype=m.dtype, device="cuda") for m in w.masks]
+        eq, ek, ev = (torch.empty(w.q.shape, dtype=w.q.dtype, device="cuda") for _ in range(3))
+        emasks = [torch.empty(m.shape, dtype=m.dtype, device="cuda") for m in w.masks]
         bufs = rra.Buffers(w.B, w.N, w.H, w.q.dtype, out_dtype=out_dtype)
         e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
         def e2e_step():
             with torch.cuda.stream(stream):
-                for d, h in zip((dq, dk, dv), host_in):
+                for d, h in zip((eq, ek, ev), host_in):
                     d.copy_(h, non_blocking=True)
-                for d, h in zip(dmasks, host_masks):
+                for d, h in zip(emasks, host_masks):
                     d.copy_(h, non_blocking=True)
-                for i, m in enumerate(dmasks):
-                    y = rra.forward(m, dq, dk, dv, bufs, stream=stream, fused=args.path == "fused")
+                for i, m in enumerate(emasks):
+                    y = rra.forward(m, eq, ek, ev, bufs, stream=stream, fused=args.path == "fused")
                     host_out[i].copy_(y, non_blocking=True)
         for _ in range(max(3, args.warmup)):
             e2e_step()
@@ -522,12 +682,26 @@ def main_gpu(args):
         e2e = {"value": job_throughput(ws, args.steps, T_call, tot), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": tot / args.steps,
                "api": f"rra.forward (eager, {args.path} path)"}
-        if err == 0:
-            err2 = rra.rra_get_device_error(bufs.err, stream)
-            if err2 != 0:
-                raise RuntimeError(f"device error {rra.rra_status_string(err2)} in the e2e region")
+        err2 = rra.rra_get_device_error(bufs.err, stream)
+        if err2 != 0:
+            raise RuntimeError(f"device error {rra.rra_status_string(err2)} in the e2e region")
+        del bufs, eq, ek, ev
 
-    mask_producer = None if args.profile else time_mask_producer(w, flush, stream, args.steps, args.warmup, hbm_peak)
+    mask_producer = None if args.profile else time_mask_producer(w.B, w.N, w.H, w.seed, flush, stream, args.steps,
+                                                                 args.warmup, hbm_peak)
+    del pipe.graph_ev, other.graph_ev
+
+    sweep = None
+    if ws == 1 and not args.no_sweep and not args.profile:
+        del other
+        torch.cuda.empty_cache()
+        with ClockSampler(dev_index, period_s=0.005) as sclk:
+            floor = empty_graph_floor(stream)
+            cells = run_sweep(workloads.sweep_names() if args.sweep == "all" else args.sweep.split(","), flush,
+                              stream, hbm_peak)
+        sweep = {"inputs": "Q/K/V drawn on the device (seeded, N(0, std^2) as each config), masks from each "
+                           "config's recipe; L2 flushed (256 MiB write) before every cold replay",
+                 "empty_graph_floor_us": floor, "clocks": sclk.summary(), "cells": cells}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and not args.profile:
@@ -541,14 +715,15 @@ def main_gpu(args):
             "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d": 64, "stages": stages,
                        "tokens_per_call": T_call, "seed": w.seed, "recipe": w.recipe, "path": args.path,
-                       "out_dtype": str(pipe.bufs.o.dtype).replace("torch.", ""),
-                       "l2": "flushed before every timed step (256 MiB write, untimed)",
+                       "out_dtype": str(pipe.bufs.y.dtype).replace("torch.", ""),
+                       "l2": "flushed before every timed step (256 MiB write, untimed); inputs also exceed L2",
                        "parallelism": f"replicas x{ws}"},
             "us_per_call": ms_per_step * 1e3,
             "us_per_call_warm_back_to_back": warm_us,
-            "host_dispatch_us": {"graph_replay": host_graph_us, "eager_three_calls": host_eager_us},
+            "host_dispatch_us": {"graph_replay": host_graph_us, "eager_call": host_eager_us},
             "kernels": per_kernel,
-            "other_path": {"path": other.path, "us_per_call": 1e3 * statistics.mean(o_step_ms),
+            "other_path": {"path": "three" if args.path == "fused" else "fused",
+                           "us_per_call": 1e3 * statistics.mean(o_step_ms),
                            "tokens_per_s": T_call / (1e-3 * statistics.mean(o_step_ms)), "kernels": other_kernels,
                            "identical_output": bool(same)},
             "attention_tflops": attn_tflops,
@@ -558,9 +733,10 @@ def main_gpu(args):
             "cpu_baseline": cpu,
             "clocks": clk.summary(),
             "gpu_launches": args.steps * len(pipe.kernels) * stages,
+            "sweep": sweep,
         }
         print(json.dumps(line), flush=True)
-    del pipe, other
+    del pipe
     if ws > 1:
         torch.distributed.destroy_process_group()
     return 0
@@ -572,16 +748,19 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="c2", help="c1 | c2 | c3:B | c4 | c5:r:B | c5s:B")
+    ap.add_argument("--workload", default="c5:1.0:512", help="c1 | c2 | c3:B | c4 | c5:r:B | c5s:B")
     ap.add_argument("--out", choices=["native", "f32"], default="native")
     ap.add_argument("--path", choices=["fused", "three"], default="fused",
                     help="single launch (default) or the three calls pack, attend, unpack")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--sweep", default="all", help="'all' or a comma-separated list of workload names")
     ap.add_argument("--profile", action="store_true",
-                    help="timed steps only (no dispatch loops, e2e or CPU leg): the command ncu captures")
+                    help="timed steps only (no dispatch loops, e2e, sweep or CPU leg): the command ncu captures")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--ref-images", type=int, default=16, help="images per step of the reference arm")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-images", type=int, default=0,
+                    help="images per step of the reference arm (default: one per host core)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     if args.impl == "reference":

@@ -257,3 +257,94 @@ def by_name(name: str, seed: int = 0) -> Workload:
     if parts[0] == "c5s":
         return config5_staged(int(parts[1]), seed)
     raise ValueError(f"unknown workload {name!r}")
+
+
+# ------------------------------------------------------------------------------------ sweep inputs
+
+def device_values(B: int, N: int, H: int, dtype: str = "bf16", seed: int = 0, std: float = 1.0,
+                  device="cuda") -> List[torch.Tensor]:
+    """Padded Q, K, V [B, N, H, 64] drawn directly on the device (torch's seeded generator there),
+    for timing-only sweeps whose cells are never compared with the oracle: N(0, std^2) rounded to
+    the 16-bit type, the same distribution as the named configs' host draws."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(np.random.SeedSequence([int(seed), 55, int(B), int(N), int(H)]).generate_state(1)[0]))
+    out = []
+    for _ in range(3):
+        x = torch.randn(B, N, H, D_HEAD, generator=g, device=device, dtype=torch.float32)
+        if std != 1.0:
+            x.mul_(std)
+        out.append(x.to(_TORCH_DTYPES[dtype]).contiguous())
+    return out
+
+
+def sweep_masks(name: str, seed: int = 0) -> List[np.ndarray]:
+    """Keep masks of a named workload (same recipes and seeds as ``by_name``) without drawing its
+    Q/K/V: for c1/c3/c5 cells the lengths and kept positions come from a mask-only stream, so they
+    follow the config's recipe but are not the same draws as the full workload's."""
+    parts = name.split(":")
+    kind = parts[0]
+    if kind == "c1":
+        B, N = 4, 197
+        rng = np.random.default_rng(np.random.SeedSequence([seed, 1, B, 0, 1, 66]))
+        lengths = rng.integers(20, N + 1, size=B)
+        return [np.stack([_random_subset_row(rng, int(L), N) for L in lengths])]
+    if kind == "c2":
+        return [m.numpy() for m in config2(seed).masks]
+    if kind == "c3":
+        B, N = int(parts[1]), 197
+        rng = np.random.default_rng(np.random.SeedSequence([seed, 3, B, 0, 1, 66]))
+        lengths = 40 + rng.integers(-4, 5, size=B)
+        return [np.stack([_random_subset_row(rng, int(L), N) for L in lengths])]
+    if kind == "c4":
+        B, N = 64, 577
+        rng = np.random.default_rng(np.random.SeedSequence([seed, 4, B, 0, 1, 66]))
+        score = np.concatenate([np.zeros((B, 1)), rng.uniform(0.0, 1.0, size=(B, N - 1))], axis=1)
+        ratios = rng.uniform(0.3, 0.7, size=B)
+        return [np.stack([_topk_mask_row(score[b], keep_count(ratios[b], N - 1), N) for b in range(B)])]
+    if kind == "c5":
+        r, B, N = float(parts[1]), int(parts[2]), 197
+        rng = np.random.default_rng(np.random.SeedSequence([seed, 5, B, int(round(1000 * r)), 1, 66]))
+        score = np.concatenate([np.zeros((B, 1)), rng.uniform(0.0, 1.0, size=(B, N - 1))], axis=1)
+        k = keep_count(r, N - 1)
+        return [np.stack([_topk_mask_row(score[b], k, N) for b in range(B)])]
+    if kind == "c5s":
+        B, N, ratio = int(parts[1]), 197, 0.7
+        rng = np.random.default_rng(np.random.SeedSequence([seed, 5, B, 700, 3, 66]))
+        masks, prev, k = [], np.ones((B, N), dtype=np.uint8), N - 1
+        for _ in range(3):
+            k = keep_count(ratio, k)
+            score = np.concatenate([np.zeros((B, 1)), rng.uniform(0.0, 1.0, size=(B, N - 1))], axis=1)
+            cur = np.stack([_topk_mask_row(score[b], k, N, candidates=np.nonzero(prev[b, 1:])[0] + 1)
+                            for b in range(B)])
+            masks.append(cur)
+            prev = cur
+        return masks
+    raise ValueError(f"unknown workload {name!r}")
+
+
+def shape_of(name: str):
+    """(B, N, H, dtype, std) of a named workload."""
+    parts = name.split(":")
+    kind = parts[0]
+    if kind == "c1":
+        return 4, 197, 3, "f16", 1.0
+    if kind == "c2":
+        return 64, 197, 6, "bf16", 1.0
+    if kind == "c3":
+        return int(parts[1]), 197, 12, "bf16", 1.0
+    if kind == "c4":
+        return 64, 577, 12, "bf16", 0.5
+    if kind == "c5":
+        return int(parts[2]), 197, 12, "bf16", 1.0
+    if kind == "c5s":
+        return int(parts[1]), 197, 12, "bf16", 1.0
+    raise ValueError(f"unknown workload {name!r}")
+
+
+def sweep_names() -> List[str]:
+    """Every cell the configs name: config 5's keep-ratio x batch grid and its three-stage row per
+    batch, config 1, config 2, config 3's batch sweep and config 4."""
+    names = [f"c5:{r}:{B}" for r in (1.0, 0.7, 0.5, 0.3, 0.2, 0.1) for B in (1, 4, 16, 64, 256, 512)]
+    names += [f"c5s:{B}" for B in (1, 4, 16, 64, 256, 512)]
+    names += ["c1", "c2"] + [f"c3:{B}" for B in (1, 2, 4, 64, 256)] + ["c4"]
+    return names
