@@ -13,4 +13,6 @@ from .oracle import (  # noqa: F401
     attend_rows,
     unpack,
     library_path,
+    l2_mask,
+    l2_score,
 )

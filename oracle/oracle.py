@@ -65,6 +65,11 @@ def _declare(lib):
     lib.rra_oracle_l2_mask.argtypes = [vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, i32p,
                                        ctypes.c_double, u8p, u8p]
     lib.rra_oracle_l2_mask.restype = ctypes.c_int
+    lib.rra_oracle_l2_score.argtypes = [vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                                        ctypes.POINTER(ctypes.c_uint32)]
+    lib.rra_oracle_l2_score.restype = ctypes.c_int
+    lib.rra_oracle_l2_score_words.argtypes = []
+    lib.rra_oracle_l2_score_words.restype = ctypes.c_int
     return lib
 
 
@@ -229,4 +234,36 @@ def l2_mask(x, k_keep=None, threshold_sq: float = 0.0, prev=None, dtype: str | N
                                 None if pv is None else _ptr(pv), _ptr(out))
     if rc != 0:
         raise ValueError("rra_oracle_l2_mask: bad arguments")
+    return out
+
+
+SCORE_NAN, SCORE_FINITE, SCORE_INF = 0, 1, 2
+SCORE_EMIN = -298  # weight of the last bit of the oracle's fixed-point squared norm
+
+
+def l2_score(x, dtype: str | None = None, lib=None):
+    """Exact squared l2 norm of every row of x [..., C] as computed by the oracle: a list of
+    (class, value) with class SCORE_NAN / SCORE_FINITE / SCORE_INF and, for a finite score, the
+    exact value as a fractions.Fraction (None otherwise)."""
+    from fractions import Fraction
+    lib = lib or load()
+    xa = _np(x)
+    code = _dtype_code(x, dtype)
+    C = xa.shape[-1]
+    rows = int(np.prod(xa.shape[:-1], dtype=np.int64))
+    xa = np.ascontiguousarray(xa.reshape(rows, C))
+    nw = lib.rra_oracle_l2_score_words()
+    words = (ctypes.c_uint32 * nw)()
+    out = []
+    for r in range(rows):
+        cls = lib.rra_oracle_l2_score(_ptr(xa), code, r, C, words)
+        if cls < 0:
+            raise ValueError("rra_oracle_l2_score: unsupported dtype")
+        if cls == SCORE_FINITE:
+            v = 0
+            for i in reversed(range(nw)):
+                v = (v << 32) | int(words[i])
+            out.append((cls, Fraction(v, 1 << -SCORE_EMIN)))
+        else:
+            out.append((cls, None))
     return out

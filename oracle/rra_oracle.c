@@ -241,46 +241,174 @@ int rra_oracle_unpack(const uint8_t *packed, const int32_t *cu, const uint8_t *m
  * name the method and nothing more).  Readings taken where they are silent:
  *   - a token's score is the l2 norm of its embedding row x[b, n, 0..C-1]; the squared norm,
  *     which orders tokens the same way, is what is compared;
- *   - the squared norm is accumulated in IEEE single precision -- the precision the selection
- *     kernel decides in -- as acc = fmaf(x_c, x_c, acc) for c = 0, 1, ..., C-1 from the exactly
- *     widened 16-bit inputs, so it is one reproducible number (each square is exact in single
- *     precision; the running sum rounds the same way on both sides); a NaN score ranks below
- *     every other score;
+ *   - the squared norm is the EXACT sum of the squares, with no rounding anywhere: every
+ *     16-bit (or single-precision) input is an odd integer M times a power of two 2^e, its
+ *     square M^2 * 2^(2e) is added into a fixed-point integer whose last bit is 2^-298 (the
+ *     square of the smallest single-precision subnormal), so the comparison between two
+ *     tokens is the comparison between the two exact rational numbers, whatever the order of
+ *     the terms; a score with a NaN term is NaN and ranks below every other score, one with an
+ *     infinite term (and no NaN) is +infinity;
  *   - the CLS token (n = 0) is always kept;
  *   - the candidates are the tokens n >= 1 kept by the previous stage (`prev`, or every token
  *     n >= 1 when there is none), which makes multi-stage masks nested (EViT-like schedules);
  *   - with `k_keep`, image b keeps its k_b best candidates: highest score first, the lower
  *     index first among equal scores (k_b clamped to [0, #candidates]); without it, every
- *     candidate whose squared norm is >= threshold_sq.
- * Returns 0, or -1 on a bad argument.
+ *     candidate whose squared norm is >= threshold_sq (compared exactly; a NaN score never
+ *     passes).
  */
-static double l2_sq(const void *x, int dtype, int64_t row, int C)
+enum { SCORE_NAN = 0, SCORE_FINITE = 1, SCORE_INF = 2 };
+#define SCORE_WORDS 20    /* 640 bits: squares of single-precision values stay below 2^256,
+                             i.e. bit 554 above 2^-298, plus 31 bits of carries for C < 2^31 */
+#define SCORE_EMIN (-298) /* weight of bit 0 */
+
+typedef struct {
+    int cls;                      /* SCORE_NAN, SCORE_FINITE or SCORE_INF */
+    uint32_t w[SCORE_WORDS];      /* finite value = sum_i w[i] 2^(32 i) * 2^SCORE_EMIN */
+} Score;
+
+static void score_zero(Score *s)
 {
-    float acc = 0.0f;
-    for (int c = 0; c < C; ++c) {
-        float v = (float)load_elem(x, dtype, row * C + c); /* exact: a 16-bit value */
-        acc = fmaf(v, v, acc);
-    }
-    return (double)acc;
+    s->cls = SCORE_FINITE;
+    memset(s->w, 0, sizeof s->w);
 }
+
+/* Add the integer m * 2^shift (m < 2^48, shift >= 0) into the fixed-point words.  Returns 0 when
+ * the sum does not fit in SCORE_WORDS words. */
+static int words_add(uint32_t *w, uint64_t m, int shift)
+{
+    /* m * 2^(shift % 32) < 2^80: three 32-bit words, starting at word shift / 32 */
+    const int i0 = shift / 32, r = shift % 32;
+    uint32_t part[3];
+    part[0] = (uint32_t)(m << r);
+    part[1] = (uint32_t)(r ? (m >> (32 - r)) : (m >> 32));
+    part[2] = (uint32_t)(r ? (m >> (64 - r)) : 0);
+    uint64_t carry = 0;
+    int j = i0;
+    for (; j < SCORE_WORDS; ++j) {
+        const uint64_t add = (j - i0 < 3 ? (uint64_t)part[j - i0] : 0) + carry;
+        if (j - i0 >= 3 && add == 0)
+            return 1;
+        const uint64_t t = (uint64_t)w[j] + add;
+        w[j] = (uint32_t)t;
+        carry = t >> 32;
+    }
+    if (carry != 0)
+        return 0;
+    for (; j < i0 + 3; ++j)
+        if (part[j - i0] != 0)
+            return 0;
+    return 1;
+}
+
+/* s += x^2 exactly.  x is a value of one of the input types (at most 24 significant bits and a
+ * binary exponent of at least -149), widened exactly to double. */
+static void score_add_square(Score *s, double x)
+{
+    if (isnan(x)) {
+        s->cls = SCORE_NAN;
+        return;
+    }
+    if (isinf(x)) {
+        if (s->cls != SCORE_NAN)
+            s->cls = SCORE_INF;
+        return;
+    }
+    if (x == 0.0)
+        return;
+    int k;
+    double f = frexp(fabs(x), &k);       /* |x| = f * 2^k, 0.5 <= f < 1 */
+    uint64_t m = (uint64_t)ldexp(f, 53); /* exact: f has at most 53 significant bits */
+    int e = k - 53;
+    while ((m & 1u) == 0) {              /* |x| = m * 2^e with m odd */
+        m >>= 1;
+        e += 1;
+    }
+    /* m < 2^24, so m^2 < 2^48; x^2 = m^2 * 2^(2e) and 2e >= SCORE_EMIN for the input types */
+    words_add(s->w, m * m, 2 * e - SCORE_EMIN);
+}
+
+/* -1, 0, +1 as a < b, a == b, a > b, with NaN below every number. */
+static int score_cmp(const Score *a, const Score *b)
+{
+    if (a->cls != b->cls)
+        return a->cls < b->cls ? -1 : 1;
+    if (a->cls != SCORE_FINITE)
+        return 0;
+    for (int i = SCORE_WORDS - 1; i >= 0; --i)
+        if (a->w[i] != b->w[i])
+            return a->w[i] < b->w[i] ? -1 : 1;
+    return 0;
+}
+
+/* The smallest score value >= t, for comparing a score with a threshold t (not NaN):
+ * score >= t  <=>  score >= score_ceil(t).  A t beyond every finite score maps to +infinity. */
+static void score_ceil(Score *s, double t)
+{
+    score_zero(s);
+    if (t <= 0.0)
+        return;
+    if (isinf(t)) {
+        s->cls = SCORE_INF;
+        return;
+    }
+    int k;
+    double f = frexp(t, &k);
+    uint64_t m = (uint64_t)ldexp(f, 53);
+    int e = k - 53; /* t = m * 2^e */
+    int shift = e - SCORE_EMIN;
+    if (shift < 0) {
+        /* t / 2^SCORE_EMIN = m / 2^-shift: round up to the next integer */
+        uint64_t q = (-shift >= 64) ? 0 : (m >> -shift);
+        int exact = (-shift < 64) && ((q << -shift) == m);
+        m = q + (exact ? 0 : 1);
+        shift = 0;
+    }
+    if (shift + 64 > SCORE_WORDS * 32 || !words_add(s->w, m >> 16, shift + 16) || !words_add(s->w, m & 0xFFFF, shift))
+        s->cls = SCORE_INF; /* beyond every finite score */
+}
+
+static void l2_score(const void *x, int dtype, int64_t row, int C, Score *s)
+{
+    score_zero(s);
+    for (int c = 0; c < C; ++c)
+        score_add_square(s, load_elem(x, dtype, row * C + c));
+}
+
+/* The exact squared norm of row `row` of x [., C]: returns its class (0 NaN, 1 finite,
+ * 2 +infinity) and, for a finite one, writes the SCORE_WORDS 32-bit words of the integer
+ * value / 2^-298 (least significant first) to `words`. */
+int rra_oracle_l2_score(const void *x, int dtype, int64_t row, int C, uint32_t *words)
+{
+    if (dtype != ORACLE_F16 && dtype != ORACLE_BF16 && dtype != ORACLE_F32)
+        return -1;
+    Score s;
+    l2_score(x, dtype, row, C, &s);
+    memcpy(words, s.w, sizeof s.w);
+    return s.cls;
+}
+
+int rra_oracle_l2_score_words(void) { return SCORE_WORDS; }
 
 int rra_oracle_l2_mask(const void *x, int dtype, int B, int N, int C, const int32_t *k_keep, double threshold_sq,
                        const uint8_t *prev, uint8_t *mask)
 {
-    if (B < 0 || N < 1 || C < 1)
+    if (B < 0 || N < 1 || C < 1 || isnan(threshold_sq))
         return -1;
-    double *score = (double *)malloc(sizeof(double) * (size_t)N);
+    if (dtype != ORACLE_F16 && dtype != ORACLE_BF16 && dtype != ORACLE_F32)
+        return -1;
+    Score *score = (Score *)malloc(sizeof(Score) * (size_t)N);
     char *cand = (char *)malloc((size_t)N);
     if (score == NULL || cand == NULL) {
         free(score);
         free(cand);
         return -1;
     }
+    Score thr;
+    score_ceil(&thr, threshold_sq);
     for (int b = 0; b < B; ++b) {
         int ncand = 0;
         for (int n = 0; n < N; ++n) {
-            double s = l2_sq(x, dtype, (int64_t)b * N + n, C);
-            score[n] = isnan(s) ? -INFINITY : s;
+            l2_score(x, dtype, (int64_t)b * N + n, C, &score[n]);
             cand[n] = (char)(n >= 1 && (prev == NULL || prev[(int64_t)b * N + n] != 0));
             ncand += cand[n];
             mask[(int64_t)b * N + n] = 0;
@@ -293,14 +421,14 @@ int rra_oracle_l2_mask(const void *x, int dtype, int B, int N, int C, const int3
             for (int t = 0; t < k; ++t) {
                 int best = -1;
                 for (int n = 1; n < N; ++n)
-                    if (cand[n] && (best < 0 || score[n] > score[best]))
+                    if (cand[n] && (best < 0 || score_cmp(&score[n], &score[best]) > 0))
                         best = n;
                 mask[(int64_t)b * N + best] = 1;
                 cand[best] = 0;
             }
         } else {
             for (int n = 1; n < N; ++n)
-                if (cand[n] && score[n] >= threshold_sq)
+                if (cand[n] && score[n].cls != SCORE_NAN && score_cmp(&score[n], &thr) >= 0)
                     mask[(int64_t)b * N + n] = 1;
         }
     }

@@ -414,6 +414,68 @@ def pin_l2_mask_norm_not_l1(lib):
     assert np.array_equal(O.l2_mask(x, threshold_sq=8.5, lib=lib)[0], [1, 0, 0, 1, 0])
 
 
+def _exact_sq(row):
+    """(class, Fraction) of the exact squared norm of a list of Python floats (each the exact
+    value of a 16-bit or single-precision input)."""
+    from fractions import Fraction
+    if any(math.isnan(v) for v in row):
+        return (O.SCORE_NAN, None)
+    if any(math.isinf(v) for v in row):
+        return (O.SCORE_INF, None)
+    return (O.SCORE_FINITE, sum((Fraction(v) ** 2 for v in row), Fraction(0)))
+
+
+def pin_l2_score_is_exact_sum(lib):
+    """The oracle's squared norm is the exact rational sum of the squares (fractions.Fraction):
+    on N(0,1) rows of C = 384 and 768 in bf16 and fp16 (where a single-precision chain already
+    rounds), on rows mixing magnitudes from 2^-60 to 2^60 (where a double-precision chain rounds
+    too, in an order-dependent way), on subnormal and zero entries, and with inf / NaN entries."""
+    rng = np.random.default_rng(43)
+    cases = []
+    for dt in (torch.bfloat16, torch.float16):
+        for C in (384, 768):
+            cases.append(torch.from_numpy(rng.standard_normal((4, C), dtype=np.float32)).to(dt))
+    wide = (rng.standard_normal((6, 64)) * np.exp2(rng.integers(-60, 61, size=(6, 64)))).astype(np.float32)
+    cases.append(torch.from_numpy(wide).to(torch.bfloat16))
+    cases.append(torch.from_numpy(wide))  # single precision input
+    cases.append(torch.tensor([[2.0 ** -133, -(2.0 ** -126), 1.0, 3.0, 0.0, -0.0, 2.0 ** 100, 2.0 ** -100]],
+                              dtype=torch.float32).to(torch.bfloat16))
+    cases.append(torch.tensor([[2.0 ** -24, 2.0 ** -14, 0.5, 65504.0, 0.0, -3.0, 1.0 / 3.0, 1e-5]],
+                              dtype=torch.float32).to(torch.float16))
+    cases.append(torch.tensor([[1.0, float("inf"), 2.0], [float("nan"), float("inf"), 1.0], [3.0, 4.0, 0.0]],
+                              dtype=torch.float32).to(torch.bfloat16))
+    for x in cases:
+        got = O.l2_score(x, lib=lib)
+        for r, row in enumerate(x.reshape(-1, x.shape[-1]).tolist()):
+            assert got[r] == _exact_sq(row), (x.dtype, r)
+
+
+def pin_l2_mask_exact_where_rounding_ties(lib):
+    """Selection follows the exact sums where a rounded accumulation, in either order, sees a
+    tie: token 1 is exactly 1; tokens 2 and 3 are 1 + 100 * 2^-60 (the tiny terms after the 1,
+    or before it); token 4 is 1 + 99 * 2^-60; token 5 is 1 + 5 * 2^-54.  In double precision
+    every one of them sums to 1.  Exactly, 5 > 2 = 3 > 4 > 1; token 6 (= 1 + 2^-52) beats them
+    all, and of the others only 5 reaches the threshold 1 + 2^-52 that 6 attains."""
+    C = 128
+    t = 2.0 ** -30
+    rows = [[0.0] * C, [1.0] + [0.0] * (C - 1), [1.0] + [t] * 100 + [0.0] * 27, [t] * 100 + [1.0] + [0.0] * 27,
+            [1.0] + [t] * 99 + [0.0] * 28, [1.0] + [2.0 ** -27] * 5 + [0.0] * 122,
+            [1.0, 2.0 ** -26] + [0.0] * 126]
+    x = torch.tensor([rows], dtype=torch.float32).to(torch.bfloat16)
+    assert x.float().tolist() == [rows]  # every entry is a bf16 value
+    want = {1: [5], 2: [5, 2], 3: [5, 2, 3], 4: [5, 2, 3, 4], 5: [5, 2, 3, 4, 1]}
+    for k, keep in want.items():
+        # token 6 competes too: 1 + 2^-52 > 1 + 5 * 2^-54 (token 5), so it is always first
+        got = O.l2_mask(x, k_keep=[k + 1], lib=lib)[0]
+        exp = np.zeros(7, np.uint8)
+        exp[[0, 6] + keep[:k]] = 1
+        assert np.array_equal(got, exp), (k, got)
+    got = O.l2_mask(x, threshold_sq=1.0 + 2.0 ** -52, lib=lib)[0]
+    assert np.array_equal(got, [1, 0, 0, 0, 0, 1, 1]), got
+    got = O.l2_mask(x, threshold_sq=1.0, lib=lib)[0]
+    assert np.array_equal(got, [1, 1, 1, 1, 1, 1, 1]), got
+
+
 ALL_PINS = [
     pin_cu_seqlens_matches_cumsum,
     pin_rank_matches_nonzero,
@@ -433,4 +495,6 @@ ALL_PINS = [
     pin_l2_mask_topk_matches_sorted,
     pin_l2_mask_threshold_and_extremes,
     pin_l2_mask_norm_not_l1,
+    pin_l2_score_is_exact_sum,
+    pin_l2_mask_exact_where_rounding_ties,
 ]

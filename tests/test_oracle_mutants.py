@@ -14,6 +14,10 @@ from oracle import oracle as O
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "rra_oracle.c")
 
+L2_LOOP = """    score_zero(s);
+    for (int c = 0; c < C; ++c)
+        score_add_square(s, load_elem(x, dtype, row * C + c));"""
+
 MUTANTS = {
     "drop_scale": ("s[j] = acc * scale;", "s[j] = acc;"),
     "max_sign": ("s[j] = exp(s[j] - m);", "s[j] = exp(m - s[j]);"),
@@ -39,14 +43,25 @@ MUTANTS = {
     "f16_bias": ("v = ldexp((double)(1024 + m), e - 25);", "v = ldexp((double)(1024 + m), e - 24);"),
     "f16_subnormal": ("v = ldexp((double)m, -24);", "v = ldexp((double)m, -25);"),
     "bf16_truncated": ("uint32_t u = ((uint32_t)b) << 16;", "uint32_t u = ((uint32_t)(b & 0xFFF0)) << 16;"),
-    "l2_tie_takes_higher_index": ("if (cand[n] && (best < 0 || score[n] > score[best]))",
-                                  "if (cand[n] && (best < 0 || score[n] >= score[best]))"),
+    "l2_tie_takes_higher_index": ("if (cand[n] && (best < 0 || score_cmp(&score[n], &score[best]) > 0))",
+                                  "if (cand[n] && (best < 0 || score_cmp(&score[n], &score[best]) >= 0))"),
     "l2_cls_not_forced": ("        mask[(int64_t)b * N] = 1;\n        if (k_keep != NULL) {",
                           "        if (k_keep != NULL) {"),
     "l2_ignores_previous_stage": ("cand[n] = (char)(n >= 1 && (prev == NULL || prev[(int64_t)b * N + n] != 0));",
                                   "cand[n] = (char)(n >= 1);"),
-    "l2_threshold_strict": ("if (cand[n] && score[n] >= threshold_sq)", "if (cand[n] && score[n] > threshold_sq)"),
-    "l2_is_l1": ("acc = fmaf(v, v, acc);", "acc += fabsf(v);"),
+    "l2_threshold_strict": ("score_cmp(&score[n], &thr) >= 0)", "score_cmp(&score[n], &thr) > 0)"),
+    "l2_is_l1": ("words_add(s->w, m * m, 2 * e - SCORE_EMIN);", "words_add(s->w, m, e - SCORE_EMIN);"),
+    # the exact score replaced by rounded accumulations: single precision in index order,
+    # double precision in index order, double precision in reverse order
+    "l2_fp32_chain": (L2_LOOP, "    float f = 0.0f;\n    for (int c = 0; c < C; ++c) { float v = (float)load_elem(x, dtype, row * C + c); "
+                      "f = fmaf(v, v, f); }\n    if (isnan(f)) { score_zero(s); s->cls = SCORE_NAN; } else score_ceil(s, f);"),
+    "l2_fp64_chain": (L2_LOOP, "    double f = 0.0;\n    for (int c = 0; c < C; ++c) { double v = load_elem(x, dtype, row * C + c); "
+                      "f = fma(v, v, f); }\n    if (isnan(f)) { score_zero(s); s->cls = SCORE_NAN; } else score_ceil(s, f);"),
+    "l2_fp64_reversed": (L2_LOOP, "    double f = 0.0;\n    for (int c = C - 1; c >= 0; --c) { double v = load_elem(x, dtype, row * C + c); "
+                         "f = fma(v, v, f); }\n    if (isnan(f)) { score_zero(s); s->cls = SCORE_NAN; } else score_ceil(s, f);"),
+    "l2_carry_dropped": ("        carry = t >> 32;", "        carry = 0;"),
+    "l2_square_bit_off_by_one": ("words_add(s->w, m * m, 2 * e - SCORE_EMIN);", "words_add(s->w, m * m, 2 * e - SCORE_EMIN + 1);"),
+    "l2_inf_not_above_finite": ("        if (s->cls != SCORE_NAN)\n            s->cls = SCORE_INF;", "        ;"),
     "mask_byte_is_bool": ("if (mask[(int64_t)b * N + n] != 0)\n                run += 1;",
                           "if (mask[(int64_t)b * N + n] == 1)\n                run += 1;"),
 }
