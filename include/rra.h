@@ -170,16 +170,21 @@ rra_status rra_pack_attend_unpack(const uint8_t *keep_mask, const void *q, const
  * rra_l2_mask -- Threshold-l2 token selection, the step in front of the pipeline (aissential.tech
  * summary, Summary: the DeiT models are pruned with Threshold-l2, EViT and other methods; the
  * pages name the method only).  For every image b:
- *   score(n)   = squared l2 norm of x[b, n, :], accumulated in single precision as
- *                acc = fmaf(x_c, x_c, acc) for c = 0 .. C-1 (in that order) from the exactly
- *                widened 16-bit inputs; a NaN score ranks below every other; the threshold is
- *                compared with the score widened to double;
+ *   score(n)   = squared l2 norm of x[b, n, :], the exact sum of the squares of the (exactly
+ *                widened) 16-bit inputs: each square is exact in double precision and the sum is
+ *                carried in double-double arithmetic, normalised to (RN(S), S - RN(S)), which is a
+ *                function of the exact sum S alone -- so the order of the additions cannot matter,
+ *                and the selection is the exact one whenever a token's squares lie within 2^96 of
+ *                one another (otherwise only tokens whose exact scores agree to about 2^-96
+ *                relative can be ordered differently); a score with a NaN term ranks below every
+ *                other, one with an infinite term (and no NaN) above every finite one;
  *   candidates = tokens n >= 1 with prev_mask[b, n] != 0 (every n >= 1 when prev_mask is NULL),
  *                which makes the masks of successive stages nested (EViT-like schedules);
  *   keep_mask[b, 0] = 1 (the CLS token is always kept);
  *   with k_keep:  keep_mask[b, n] = 1 for the k_keep[b] best candidates -- higher score first,
  *                 lower n first among equal scores, k clamped to [0, number of candidates];
- *   without:      keep_mask[b, n] = 1 for the candidates with score >= threshold_sq;
+ *   without:      keep_mask[b, n] = 1 for the candidates with score >= threshold_sq, compared
+ *                 exactly (a NaN score never passes);
  *   every other keep_mask[b, n] = 0.
  *
  *   x             device [B, N, C] in dt (RRA_F16 or RRA_BF16), 16-byte aligned, C a multiple of 8

@@ -223,8 +223,13 @@ rra_status rra_l2_mask(const void *x, int B, int N, int C, rra_dtype dt, const i
             (prev_mask != keep_mask && !disjoint(keep_mask, mask_b, prev_mask, mask_b)))
             return RRA_ERR_INVALID_ARG;
     }
+    if (B == 0)
+        return RRA_OK;
+    int sms = 0;
+    if (num_sms_of_current_device(&sms) != 0)
+        return RRA_ERR_CUDA;
     const cudaError_t e = rra::launch_l2_mask(x, B, N, C, dt == RRA_BF16, k_keep, threshold_sq, prev_mask, keep_mask,
-                                              reinterpret_cast<cudaStream_t>(stream));
+                                              sms, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? RRA_OK : RRA_ERR_CUDA;
 }
 

@@ -2,19 +2,29 @@
 // pipeline ("Dispatch-Aware Ragged Attention for Pruned Vision Transformers", aissential.tech
 // summary, Summary: the DeiT models are pruned with Threshold-l2, EViT and other methods).
 //
-// One block per image.  The image's embeddings pass through shared memory in column chunks
-// (16-byte cp.async, coalesced along each token's row, double-buffered), and each thread extends
-// the squared-norm chain of its tokens chunk by chunk: acc = fmaf(x_c, x_c, acc) in single
-// precision over c = 0..C-1 in index order (16-bit inputs widen exactly and their squares are
-// exact, so the score is one reproducible number).  The scores go to shared memory as
-// order-preserving integer keys (0 = not a candidate, 1 = NaN, otherwise the bits of the
-// non-negative float plus 2).  A candidate's rank
-// is the number of candidates that beat it (higher key, or equal key and lower index); it is
-// kept when that rank is below k_b.  Ranking by counting costs N^2 comparisons per image -- 39 K
-// at N = 197, 1 M at N = 1024, spread over 256 threads -- and needs no sort.
+// Each image is scored by a thread-block cluster of up to eight CTAs, so every SM takes part even
+// at small batches (one CTA per image once the batch alone fills the GPU): CTA r of the cluster
+// owns a contiguous slice of the image's tokens, and a warp computes the squared norms of four
+// tokens at a time from coalesced 16-byte loads of their embedding rows.  The squared norm is first accumulated in plain double, one fused multiply-add per input
+// (each square of a 16-bit input is exact in double: at most 22 significant bits); that sum is
+// provably exact, in any order, when every square is a multiple of 2^q and the total stays below
+// 2^(q+52), which a token checks from the smallest exponent among its inputs -- true for almost
+// every token of realistic embeddings.  A token that fails the check (a tiny, subnormal, infinite
+// or NaN input) is recomputed in double-double arithmetic: each addition an error-free two-sum
+// whose rounding error is carried in a second double, the warp's partials combined the same way,
+// the pair normalised to (hi, lo) = (RN(S), S - RN(S)).  Either way the result is a function of
+// the exact sum S alone, so the selection does not depend on the order of the additions and
+// equals the exact selection whenever every token's squares lie within 2^96 of one another (any
+// realistic embedding; beyond that, only tokens whose exact scores agree to ~2^-96 relative could
+// be ordered differently).  A token's (hi, lo) becomes a 128-bit key whose unsigned order is the
+// score order (0 = not a candidate, then NaN, then the finite scores, then +infinity); each CTA
+// writes its keys into the shared memory of every CTA of the cluster (distributed shared memory),
+// one cluster barrier publishes them, and each CTA then ranks its own tokens: a candidate's rank
+// is the number of candidates that beat it (a higher key, or an equal key and a lower index), and
+// it is kept when that rank is below k_b -- N comparisons per token, spread over a warp, no sort.
 #include <cuda_fp16.h>
 
-#include <atomic>
+#include <mutex>
 
 #include "rra_device.cuh"
 #include "rra_internal.h"
@@ -24,171 +34,356 @@ namespace rra {
 namespace {
 
 constexpr int kMaskThreads = 256;
+constexpr int kMaskWarps = kMaskThreads / 32;
+constexpr int kMaxCluster = 8;  // portable cluster size
+constexpr int kChunksPerPass = 2;  // 16-byte loads in flight per lane and token
+constexpr int kTokPerWarp = 4;     // tokens a warp scores at once
+
+// Two copies of the value 1.0 in the 16-bit type.
+template <bool kBF16>
+struct One2 {
+    static constexpr uint32_t value = kBF16 ? 0x3F803F80u : 0x3C003C00u;
+};
+
+struct Key {
+    unsigned long long hi, lo;
+};
 
 template <bool kBF16>
-__device__ __forceinline__ float widen(uint32_t bits16)
+__device__ __forceinline__ double widen(uint32_t bits16)
 {
     if constexpr (kBF16)
-        return __uint_as_float(bits16 << 16);
+        return static_cast<double>(__uint_as_float(bits16 << 16));
     else
-        return __half2float(__ushort_as_half(static_cast<unsigned short>(bits16)));
+        return static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(bits16))));
 }
 
-// Shared memory: the keys [N] (8 bytes each), then two staging buffers of N token rows, each row
-// `w` embedding columns (w * 2 bytes), padded by 16 bytes when w >= 16 so that the 16-byte reads
-// of consecutive tokens fall in different banks.
-constexpr int kMaxTokPerThread = kMaskMaxN / kMaskThreads;
+// s + e == a + b exactly (Knuth's two-sum; explicit round-to-nearest operations, no contraction).
+__device__ __forceinline__ void two_sum(double a, double b, double &s, double &e)
+{
+    s = __dadd_rn(a, b);
+    const double bb = __dsub_rn(s, a);
+    e = __dadd_rn(__dsub_rn(a, __dsub_rn(s, bb)), __dsub_rn(b, bb));
+}
 
-__host__ __device__ constexpr int staging_stride(int w) { return w * 2 + (w >= 16 ? 16 : 0); }
+// (hi, lo) += (h2, l2)
+__device__ __forceinline__ void dd_add(double &hi, double &lo, double h2, double l2)
+{
+    double s, e;
+    two_sum(hi, h2, s, e);
+    hi = s;
+    lo = __dadd_rn(lo, __dadd_rn(e, l2));
+}
+
+// Unsigned 64-bit image of a double whose order is the numeric order (for the low part, which
+// may be negative).
+__device__ __forceinline__ unsigned long long ordered_bits(double d)
+{
+    const unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(d));
+    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+__device__ __forceinline__ bool key_greater(const Key &a, const Key &b)
+{
+    return a.hi > b.hi || (a.hi == b.hi && a.lo > b.lo);
+}
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_size()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+// Store a key into the shared memory of CTA `rank` of this cluster, at the address that `local`
+// has in this CTA.
+__device__ __forceinline__ void st_cluster_key(const Key *local, uint32_t rank, const Key &k)
+{
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+    asm volatile("st.shared::cluster.v2.u64 [%0], {%1, %2};" ::"r"(remote), "l"(k.hi), "l"(k.lo) : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// The two 16-bit values of w widened exactly to fp32 (low half first).
+template <bool kBF16>
+__device__ __forceinline__ float2 widen2(uint32_t w)
+{
+    if constexpr (kBF16)
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    else
+        return __half22float2(*reinterpret_cast<const __half2 *>(&w));
+}
+
+// True when the plain double accumulation of the squares was exact, so `acc` is the exact sum.
+// tmin2 / tmax2 hold, per 16-bit half, the minimum / maximum magnitude bits (sign cleared) seen.
+// Required: no zero input (a zero goes to the slow path, which is exact for it too), no
+// infinite or NaN input, and for bf16 every |x| in [2^-63, 2^64), so that each square x * x is
+// exact in fp32 (at most 16 significant bits, exponent in range; fp16 squares always are); and
+// every square is a multiple of 2^q (q = twice the last-bit exponent of the smallest-exponent
+// input) while the sum stays below 2^(q+52) -- then every partial sum, in any order, is an
+// integer multiple of 2^q below 2^(q+53), representable exactly, so no addition rounded (the
+// factor-2 margin covers the rounding of `acc` itself when the condition fails).
+template <bool kBF16>
+__device__ __forceinline__ bool fast_sum_exact(double acc, uint32_t tmin2, uint32_t tmax2)
+{
+    const uint32_t tmin = min(tmin2 & 0xFFFFu, tmin2 >> 16), tmax = max(tmax2 & 0xFFFFu, tmax2 >> 16);
+    int emin;
+    if constexpr (kBF16) {
+        if (tmin < (64u << 7) || tmax >= (191u << 7))
+            return false;
+        emin = static_cast<int>(tmin >> 7) - 127 - 7;  // last-bit exponent of the smallest input
+    } else {
+        if (tmin == 0u || tmax >= 0x7C00u)
+            return false;
+        emin = max(static_cast<int>(tmin >> 10), 1) - 15 - 10;
+    }
+    return acc < __hiloint2double((2 * emin + 52 + 1023) << 20, 0);  // 2^(q+52), a normal double here
+}
+
+// Key of a token that the fast path cannot settle: the squared norm in double-double arithmetic
+// (exact squares, error-free two-sum), normalised to (RN(S), S - RN(S)), with NaN / infinite
+// classes.  The whole warp calls it (warp-uniform condition); lane 0's result is used.
+template <bool kBF16>
+__device__ __noinline__ Key slow_key(const uint16_t *xrow, int nchunks, int lane)
+{
+    const uint4 *row = reinterpret_cast<const uint4 *>(xrow);
+    double hi = 0.0, lo = 0.0;
+    bool nan = false, inf = false;
+    for (int j = lane; j < nchunks; j += 32) {
+        const uint4 v = __ldg(row + j);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const double d = widen<kBF16>((i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu));
+            nan |= isnan(d);
+            inf |= isinf(d);
+            double s, e;
+            two_sum(hi, __dmul_rn(d, d), s, e);  // the square is exact in double
+            hi = s;
+            lo = __dadd_rn(lo, e);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const double h2 = __shfl_xor_sync(0xffffffffu, hi, off);
+        const double l2 = __shfl_xor_sync(0xffffffffu, lo, off);
+        dd_add(hi, lo, h2, l2);
+    }
+    nan = __any_sync(0xffffffffu, nan);
+    inf = __any_sync(0xffffffffu, inf);
+    if (nan)
+        return {1ull, 0ull};
+    if (inf)
+        return {0x7FF0000000000000ull + 2ull, ordered_bits(0.0)};
+    const double h = __dadd_rn(hi, lo);  // (h, l) = (RN(S), S - RN(S)): canonical
+    double l = __dsub_rn(lo, __dsub_rn(h, hi));
+    if (l == 0.0)
+        l = 0.0;  // one zero
+    return {static_cast<unsigned long long>(__double_as_longlong(h)) + 2ull, ordered_bits(l)};
+}
 
 template <bool kBF16>
-__global__ void __launch_bounds__(kMaskThreads) l2_mask_kernel(const uint16_t *__restrict__ x, int N, int C, int w,
+__global__ void __launch_bounds__(kMaskThreads) l2_mask_kernel(const uint16_t *__restrict__ x, int N, int C,
                                                                 const int32_t *__restrict__ k_keep, double thr_sq,
                                                                 const uint8_t *prev, uint8_t *mask)
 {
     extern __shared__ __align__(16) uint8_t sm[];
-    unsigned long long *key = reinterpret_cast<unsigned long long *>(sm);
-    const int stride = staging_stride(w);
-    uint8_t *buf0 = sm + ((static_cast<size_t>(N) * 8 + 15) & ~static_cast<size_t>(15));
-    uint8_t *buf1 = buf0 + static_cast<size_t>(N) * stride;
+    Key *keys = reinterpret_cast<Key *>(sm);  // [N]: the keys of every token of the image
+    const uint32_t cs = cluster_size();
+    const uint32_t rank = cluster_rank();
+    const int b = static_cast<int>(blockIdx.x / cs);
+    const int per_cta = (N + static_cast<int>(cs) - 1) / static_cast<int>(cs);
+    const int n0 = static_cast<int>(rank) * per_cta;
+    const int n1 = min(N, n0 + per_cta);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row0 = static_cast<int64_t>(b) * N;
+    const int nchunks = C / 8;
     pdl_trigger();
     pdl_wait();  // the embeddings and the previous stage's mask may come from the previous kernel
-    const int b = blockIdx.x;
-    const int64_t row0 = static_cast<int64_t>(b) * N;
-    const int tid = threadIdx.x;
 
-    // the image's embedding columns [c0, c0 + wj) into a staging buffer, 16 bytes per cp.async
-    auto stage = [&](int c0, uint8_t *dst) {
-        const int wj = min(w, C - c0);
-        const int parts = wj / 8;
-        const uint32_t d0 = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
-        for (int i = tid; i < N * parts; i += kMaskThreads) {
-            const int n = i / parts, q = i - n * parts;
-            const uint16_t *src = x + (row0 + n) * C + c0 + q * 8;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d0 + n * stride + q * 16), "l"(src)
-                         : "memory");
+    // ---- scores of this CTA's tokens: a warp takes kTokPerWarp tokens at a time (n, n + 8, ...,
+    // all their loads of a pass in flight together), then writes their keys to every CTA of the
+    // cluster
+    for (int nb = n0 + warp; nb < n1; nb += kTokPerWarp * kMaskWarps) {
+        double acc[kTokPerWarp];
+        uint32_t tmin[kTokPerWarp], tmax[kTokPerWarp];  // 16x2 magnitude bounds
+#pragma unroll
+        for (int t = 0; t < kTokPerWarp; ++t) {
+            acc[t] = 0.0;
+            tmin[t] = 0xFFFFFFFFu;
+            tmax[t] = 0u;
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-
-    // squared norms: each thread continues the fma chain of its tokens chunk by chunk, columns in
-    // index order, so the result is the one sequential accumulation the definition names
-    float acc[kMaxTokPerThread];
+        for (int j0 = 0; j0 < nchunks; j0 += 32 * kChunksPerPass) {
+            uint4 v[kTokPerWarp][kChunksPerPass];
 #pragma unroll
-    for (int t = 0; t < kMaxTokPerThread; ++t)
-        acc[t] = 0.0f;
-    const int nchunks = (C + w - 1) / w;
-    stage(0, buf0);
-    for (int j = 0; j < nchunks; ++j) {
-        if (j + 1 < nchunks)
-            stage((j + 1) * w, (j & 1) ? buf0 : buf1);
-        else
-            asm volatile("cp.async.commit_group;" ::: "memory");  // keep the group count uniform
-        asm volatile("cp.async.wait_group 1;" ::: "memory");      // this thread's copies of chunk j
-        __syncthreads();                                          // everyone's copies of chunk j
-        const uint8_t *cur = (j & 1) ? buf1 : buf0;
-        const int wj = min(w, C - j * w);
+            for (int t = 0; t < kTokPerWarp; ++t) {
+                const int n = nb + t * kMaskWarps;
+                const uint4 *row = reinterpret_cast<const uint4 *>(x + (row0 + n) * C);
 #pragma unroll
-        for (int t = 0; t < kMaxTokPerThread; ++t) {
-            const int n = tid + t * kMaskThreads;
-            if (n < N) {
-                const uint4 *row = reinterpret_cast<const uint4 *>(cur + n * stride);
-                float a = acc[t];
-                for (int q = 0; q < wj / 8; ++q) {
-                    const uint4 v4 = row[q];
-                    const uint32_t v[4] = {v4.x, v4.y, v4.z, v4.w};
+                for (int u = 0; u < kChunksPerPass; ++u) {
+                    const int j = j0 + lane + 32 * u;
+                    // padding lanes read the value 1.0 (in range, not zero): no effect on the bounds
+                    v[t][u] = (n < n1 && j < nchunks) ? __ldg(row + j) : make_uint4(One2<kBF16>::value, One2<kBF16>::value, One2<kBF16>::value, One2<kBF16>::value);
+                }
+            }
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float lo = widen<kBF16>(v[i] & 0xFFFFu), hi = widen<kBF16>(v[i] >> 16);
-                        a = __fmaf_rn(lo, lo, a);  // element 2i, then 2i + 1: index order
-                        a = __fmaf_rn(hi, hi, a);
+            for (int t = 0; t < kTokPerWarp; ++t) {
+#pragma unroll
+                for (int u = 0; u < kChunksPerPass; ++u) {
+                    const int j = j0 + lane + 32 * u;
+                    const uint32_t w[4] = {v[t][u].x, v[t][u].y, v[t][u].z, v[t][u].w};
+                    const uint32_t m0 = w[0] & 0x7FFF7FFFu, m1 = w[1] & 0x7FFF7FFFu, m2 = w[2] & 0x7FFF7FFFu,
+                                   m3 = w[3] & 0x7FFF7FFFu;
+                    tmin[t] = __vimin3_u16x2(tmin[t], __vimin3_u16x2(m0, m1, m2), m3);
+                    tmax[t] = __vimax3_u16x2(tmax[t], __vimax3_u16x2(m0, m1, m2), m3);
+                    if (j < nchunks) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float2 f = widen2<kBF16>(w[i]);
+                            // exact fp32 squares (checked by fast_sum_exact), exact widening, one
+                            // rounded-to-nearest double addition each
+                            acc[t] = __dadd_rn(acc[t], static_cast<double>(__fmul_rn(f.x, f.x)));
+                            acc[t] = __dadd_rn(acc[t], static_cast<double>(__fmul_rn(f.y, f.y)));
+                        }
                     }
                 }
-                acc[t] = a;
             }
         }
-        __syncthreads();  // the buffer is refilled two chunks later
-    }
 #pragma unroll
-    for (int t = 0; t < kMaxTokPerThread; ++t) {
-        const int n = tid + t * kMaskThreads;
-        if (n < N) {
-            const bool cand = n >= 1 && (prev == nullptr || prev[row0 + n] != 0);
-            const float a = acc[t];
-            key[n] = !cand ? 0ull : (a != a ? 1ull : static_cast<unsigned long long>(__float_as_uint(a)) + 2ull);
+        for (int t = 0; t < kTokPerWarp; ++t) {
+            const int n = nb + t * kMaskWarps;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                acc[t] = __dadd_rn(acc[t], __shfl_xor_sync(0xffffffffu, acc[t], off));
+                { const uint32_t o = __shfl_xor_sync(0xffffffffu, tmin[t], off); tmin[t] = __vimin3_u16x2(tmin[t], o, o); }
+                { const uint32_t o = __shfl_xor_sync(0xffffffffu, tmax[t], off); tmax[t] = __vimax3_u16x2(tmax[t], o, o); }
+            }
+            Key k;
+            if (!fast_sum_exact<kBF16>(acc[t], tmin[t], tmax[t]) && n < n1)
+                k = slow_key<kBF16>(x + (row0 + n) * C, nchunks, lane);  // warp-uniform, rare
+            else
+                k = {static_cast<unsigned long long>(__double_as_longlong(acc[t])) + 2ull, ordered_bits(0.0)};
+            if (lane == 0 && n < n1) {
+                const bool cand = n >= 1 && (prev == nullptr || prev[row0 + n] != 0);
+                if (!cand)
+                    k = {0ull, 0ull};
+                for (uint32_t r = 0; r < cs; ++r)
+                    st_cluster_key(keys + n, r, k);
+            }
         }
     }
-    __syncthreads();
+    cluster_sync_all();  // every key of the image is now in this CTA's shared memory
+
+    // ---- selection of this CTA's tokens
     const int kb = k_keep != nullptr ? k_keep[b] : 0;
-    for (int n = tid; n < N; n += kMaskThreads) {
-        const unsigned long long kn = key[n];
+    for (int n = n0 + warp; n < n1; n += kMaskWarps) {
+        const Key kn = keys[n];
         uint8_t keep;
         if (n == 0) {
             keep = 1;  // CLS
-        } else if (kn == 0) {
+        } else if (kn.hi == 0) {
             keep = 0;  // not a candidate
         } else if (k_keep != nullptr) {
+            // non-candidates have key 0 and never beat a candidate
             int r = 0;
-            for (int m = 1; m < N && r < kb; ++m) {
-                const unsigned long long km = key[m];
-                r += (km > kn || (km == kn && m < n)) ? 1 : 0;
+            for (int m = 1 + lane; m < N; m += 32) {
+                const Key km = keys[m];
+                r += (key_greater(km, kn) || (km.hi == kn.hi && km.lo == kn.lo && m < n)) ? 1 : 0;
             }
+            r = __reduce_add_sync(0xffffffffu, r);
             keep = r < kb ? 1 : 0;
+        } else if (kn.hi == 1) {
+            keep = 0;  // NaN never reaches a threshold
         } else {
-            keep = (kn != 1 && static_cast<double>(__uint_as_float(static_cast<uint32_t>(kn - 2))) >= thr_sq) ? 1 : 0;
+            // exact S >= t:  RN(S) > t, or RN(S) == t and S - RN(S) >= 0
+            const double h = __longlong_as_double(static_cast<long long>(kn.hi - 2ull));
+            keep = (h > thr_sq || (h == thr_sq && kn.lo >= 0x8000000000000000ull)) ? 1 : 0;
         }
-        mask[row0 + n] = keep;
+        if (lane == 0)
+            mask[row0 + n] = keep;
     }
 }
 
-// Staging width: the widest of 64, 32, 16 columns whose two buffers fit in 128 KB, else 8 (two
-// unpadded 16-byte rows per token: 128 KB at the largest N).
-int staging_width(int N)
+// CTAs per image: enough for about two CTAs per SM over the batch (one CTA per image once the
+// batch alone fills the GPU, where clusters would only limit how many CTAs can be resident), at
+// least 16 tokens per CTA, at most the portable cluster size; a power of two.
+int cluster_for(int B, int N, int num_sms)
 {
-    for (int w = 64; w > 8; w /= 2)
-        if (2 * static_cast<int64_t>(N) * staging_stride(w) <= 128 * 1024)
-            return w;
-    return 8;
+    int cs = 1;
+    while (cs < kMaxCluster && static_cast<int64_t>(B) * cs < 2 * num_sms && N >= 32 * cs)
+        cs *= 2;
+    return cs;
 }
-
-size_t mask_smem_bytes(int N, int w)
-{
-    return ((static_cast<size_t>(N) * 8 + 15) & ~static_cast<size_t>(15)) +
-           2 * static_cast<size_t>(N) * static_cast<size_t>(staging_stride(w));
-}
-static_assert(((kMaskMaxN * 8 + 15) & ~15) + 2 * kMaskMaxN * staging_stride(8) <= 227 * 1024,
-              "staging buffers exceed shared memory at the largest N");
 
 template <bool kBF16>
-cudaError_t set_mask_smem(size_t bytes)
+cudaError_t set_mask_smem(int bytes)
 {
-    static std::atomic<size_t> done{0};
-    if (done.load(std::memory_order_relaxed) >= bytes)
+    static std::mutex mu;
+    static int done_bytes[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 64 && done_bytes[dev] >= bytes)
         return cudaSuccess;
-    const cudaError_t e =
-        cudaFuncSetAttribute(l2_mask_kernel<kBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
-    if (e == cudaSuccess)
-        done.store(bytes, std::memory_order_relaxed);
+    e = cudaFuncSetAttribute(l2_mask_kernel<kBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && dev < 64)
+        done_bytes[dev] = bytes;
     return e;
+}
+
+template <bool kBF16>
+cudaError_t launch_mask_variant(const uint16_t *x, int B, int N, int C, const int32_t *k_keep, double thr_sq,
+                                const uint8_t *prev, uint8_t *mask, int num_sms, cudaStream_t stream)
+{
+    const int cs = cluster_for(B, N, num_sms);
+    const int smem = N * static_cast<int>(sizeof(Key));
+    cudaError_t e = set_mask_smem<kBF16>(smem);
+    if (e != cudaSuccess)
+        return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(B) * cs);
+    cfg.blockDim = dim3(kMaskThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cs);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, l2_mask_kernel<kBF16>, x, N, C, k_keep, thr_sq, prev, mask);
 }
 
 }  // namespace
 
+static_assert(kMaskMaxN * sizeof(Key) <= 227 * 1024, "keys exceed shared memory at the largest N");
+
 cudaError_t launch_l2_mask(const void *x, int B, int N, int C, bool bf16, const int32_t *k_keep, double thr_sq,
-                           const uint8_t *prev, uint8_t *mask, cudaStream_t stream)
+                           const uint8_t *prev, uint8_t *mask, int num_sms, cudaStream_t stream)
 {
     if (B == 0)
         return cudaSuccess;
-    const int w = staging_width(N);
-    const size_t smem = mask_smem_bytes(N, w);
-    const cudaError_t e = bf16 ? set_mask_smem<true>(smem) : set_mask_smem<false>(smem);
-    if (e != cudaSuccess)
-        return e;
     const auto *xs = static_cast<const uint16_t *>(x);
-    return bf16 ? launch_pdl(l2_mask_kernel<true>, dim3(B), dim3(kMaskThreads), smem, stream, xs, N, C, w, k_keep,
-                             thr_sq, prev, mask)
-                : launch_pdl(l2_mask_kernel<false>, dim3(B), dim3(kMaskThreads), smem, stream, xs, N, C, w, k_keep,
-                             thr_sq, prev, mask);
+    return bf16 ? launch_mask_variant<true>(xs, B, N, C, k_keep, thr_sq, prev, mask, num_sms, stream)
+                : launch_mask_variant<false>(xs, B, N, C, k_keep, thr_sq, prev, mask, num_sms, stream);
 }
 
 }  // namespace rra

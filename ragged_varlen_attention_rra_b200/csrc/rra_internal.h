@@ -74,10 +74,10 @@ constexpr int kFusedMaxBatch = 4096;
 
 cudaError_t launch_fused(const FusedArgs &a, int num_sms, cudaStream_t stream);
 
-// Largest N rra_l2_mask accepts (one 8-byte key per token in shared memory).
+// Largest N rra_l2_mask accepts (one 16-byte key per token in shared memory).
 constexpr int kMaskMaxN = 4096;
 
 cudaError_t launch_l2_mask(const void *x, int B, int N, int C, bool bf16, const int32_t *k_keep, double thr_sq,
-                           const uint8_t *prev, uint8_t *mask, cudaStream_t stream);
+                           const uint8_t *prev, uint8_t *mask, int num_sms, cudaStream_t stream);
 
 }  // namespace rra
