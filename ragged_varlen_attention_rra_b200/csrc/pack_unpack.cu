@@ -7,7 +7,9 @@
 // (grid = splits x images) and derives everything it needs from the keep mask in one pass:
 //   * pack: the packed start of its image (nonzero mask bytes of images < b), the rank of its
 //     first row inside the image, and the image length, counted together from 16-byte mask
-//     chunks and reduced once -- so no second launch and no inter-block wait is needed;
+//     chunks and reduced once -- so no second launch and no inter-block wait is needed; this
+//     reads B^2 N / 2 mask bytes over the grid, so from 1025 images on a one-block launch writes
+//     cu_seqlens first and the gather blocks read their image's start from it;
 //   * both: the slot of every kept row of its range (warp ballots + one block prefix).
 // Rows then move as 16-byte vectors, one warp per row, every load of a row (all tensors) in
 // flight before its stores.
@@ -136,7 +138,60 @@ __device__ __forceinline__ BlockScan block_scan(Counts c, const uint8_t *row, in
     return r;
 }
 
-template <int VPL>
+// cu_seqlens of the whole batch from one block of 1024 threads: thread t counts image base + t
+// from 16-byte mask chunks, then one block scan per 1024 images.  rra_pack launches it first
+// for large batches, so that its gather blocks read their image's start from cu_seqlens instead of
+// counting the mask bytes of every earlier image (B^2 N / 2 bytes in all).
+constexpr int kScanThreads = 1024;
+constexpr int kPackScanMinBatch = 1025;  // batches from this size on take the two-launch form
+
+__global__ void __launch_bounds__(kScanThreads) cu_kernel(const uint8_t *__restrict__ mask, int B, int N,
+                                                          int64_t capacity, int32_t *__restrict__ cu, int32_t *err)
+{
+    __shared__ int warp_tot[kScanThreads / 32];
+    pdl_trigger();
+    pdl_wait();  // the mask may come from the previous kernel
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uintptr_t addr = reinterpret_cast<uintptr_t>(mask);
+    const int off = static_cast<int>(addr & 15u);
+    const uint4 *base = reinterpret_cast<const uint4 *>(addr - off);
+    int64_t carry = 0;
+    for (int b0 = 0; b0 < B; b0 += kScanThreads) {
+        const int b = b0 + static_cast<int>(threadIdx.x);
+        int cnt = 0;
+        if (b < B) {
+            const int64_t lo = static_cast<int64_t>(b) * N, hi = lo + N;
+            for (int64_t j = (off + lo) >> 4; j < (off + hi + 15) >> 4; ++j)
+                cnt += __popc(kept_bits16(__ldg(base + j)) & range_bits16(j * 16 - off, lo, hi));
+        }
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o)
+                incl += t;
+        }
+        if (lane == 31)
+            warp_tot[warp] = incl;
+        __syncthreads();
+        int before = 0, total = 0;
+        for (int w = 0; w < kScanThreads / 32; ++w) {
+            before += (w < warp) ? warp_tot[w] : 0;
+            total += warp_tot[w];
+        }
+        if (b < B)
+            cu[b + 1] = static_cast<int32_t>(carry + before + incl);
+        carry += total;
+        __syncthreads();  // warp_tot is rewritten by the next round
+    }
+    if (threadIdx.x == 0) {
+        cu[0] = 0;
+        if (carry > capacity)
+            raise_error(err, RRA_ERR_CAPACITY);
+    }
+}
+
+template <int VPL, bool kFromCu>
 __global__ void __launch_bounds__(kThreads) pack_kernel(const uint8_t *__restrict__ mask, int N, int rows_per_split,
                                                         int V, int n_tensors, SrcPtrs src, DstPtrs dst,
                                                         int64_t capacity, int32_t *__restrict__ cu, int32_t *err)
@@ -154,11 +209,12 @@ __global__ void __launch_bounds__(kThreads) pack_kernel(const uint8_t *__restric
     const int64_t img0 = static_cast<int64_t>(b) * N;
     pdl_wait();  // the mask and the padded tensors may come from the previous kernel
 
-    // Phase 1: image start, rank of row n0 inside the image, image length -- one pass.
-    const Counts c = count_ranges(mask, img0, img0 + n0, img0 + N);
+    // Phase 1: image start, rank of row n0 inside the image, image length -- one pass (the image
+    // start read from cu_seqlens instead when the previous launch has written it).
+    const Counts c = kFromCu ? count_ranges(mask + img0, 0, n0, N) : count_ranges(mask, img0, img0 + n0, img0 + N);
     const BlockScan s = block_scan(c, mask + img0, n0, n1, slot_of, n_of_slot, part);
-    const int64_t image_start = s.before;
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
+    const int64_t image_start = kFromCu ? static_cast<int64_t>(cu[b]) : static_cast<int64_t>(s.before);
+    if (!kFromCu && blockIdx.x == 0 && threadIdx.x == 0) {
         if (b == 0)
             cu[0] = 0;
         cu[b + 1] = static_cast<int32_t>(image_start + s.total);
@@ -311,8 +367,17 @@ cudaError_t launch_pack(const uint8_t *mask, int B, int N, int64_t row_bytes, in
     const int rows = (N + splits - 1) / splits;
     const int V = static_cast<int>(row_bytes / 16);
     const dim3 grid(splits, B);
+    if (B >= kPackScanMinBatch) {
+        const cudaError_t e = launch_pdl(cu_kernel, dim3(1), dim3(kScanThreads), 0, stream, mask, B, N, capacity, cu, err);
+        if (e != cudaSuccess)
+            return e;
+        return dispatch_vpl(V, [&](auto vpl) {
+            return launch_pdl(pack_kernel<decltype(vpl)::value, true>, grid, dim3(kThreads), 0, stream, mask, N, rows,
+                              V, n_tensors, s, d, capacity, cu, err);
+        });
+    }
     return dispatch_vpl(V, [&](auto vpl) {
-        return launch_pdl(pack_kernel<decltype(vpl)::value>, grid, dim3(kThreads), 0, stream, mask, N, rows, V,
+        return launch_pdl(pack_kernel<decltype(vpl)::value, false>, grid, dim3(kThreads), 0, stream, mask, N, rows, V,
                           n_tensors, s, d, capacity, cu, err);
     });
 }
