@@ -6,32 +6,37 @@
 //     o_i = sum_j softmax_j(scale * q_i . k_j) v_j,   j over all L_b kept tokens of image b.
 //
 // How (B200-specific design, not the pages' Triton kernel):
-//   * one persistent block per SM walks a list of (image, 128-row q-tile, head) work items
-//     derived from cu_seqlens on the device, so the host never learns T; each item is taken
-//     in steps of 128 keys;
-//   * the block owns all 512 TMEM columns: an S buffer (fp32 [128 x 128]) and an O buffer
-//     (fp32 [128 x 80]) for each of two softmax groups that work on alternate items, so one
-//     group's QK^T and PV run on the tensor core while the other group's softmax runs;
+//   * one persistent block per SM walks a list of work items derived from cu_seqlens on the
+//     device, so the host never learns T: (image, 128-row q-tile, head) when some image keeps
+//     more than 64 tokens; otherwise (tile of 128 consecutive rows of the packed token space,
+//     head), each tile holding the rows of several images, every query row attending only to its
+//     own image's keys (a per-row key range, i.e. a block-diagonal mask); keys come in steps of
+//     128;
+//   * the block owns all 512 TMEM columns, 256 for each of two softmax groups that work on
+//     alternate items: S (fp32 [128 x 128]), P (16-bit [128 x 128]) and O (fp32 [128 x 64]).  P
+//     apart from S lets the next chunk's S = Q K^T run while this chunk's O += P V does, and one
+//     group's tensor-core work runs while the other group's softmax does;
 //   * warps specialise:
-//       warps 0..1  producer: Q tiles (2-slot ring) and 128-key K/V chunks (3-slot ring) of one
+//       warps 0..1  producer: Q tiles (2-slot ring) and 128-key K/V chunks (4-slot ring) of one
 //                   head; on the packed path warp 0 fetches them straight from the [T, H, 64]
 //                   layout with TMA (3-D tensor map, head = coordinate, 128-byte swizzle), on
 //                   the single-launch path warps 0 and 1 gather them with cp.async;
 //       warps 2..3  tensor-core issuers, one per softmax group: S = Q K^T (smem x smem) and
 //                   O += P V (P from TMEM as the A operand), fp32 accumulation, completion
-//                   signalled through mbarriers -- two issuing threads keep the tensor core busy
-//                   with both groups' short instruction bursts at once;
+//                   signalled through mbarriers; between bursts each prepares its group's next
+//                   V tile (zero tail; for bf16 inputs an in-place conversion to fp16);
 //       warps 4..11 softmax: two groups of four warps take alternate items; in a group, thread
-//                   r owns row r of its S and O buffers (TMEM lane r), so the row max and row sum
-//                   need no exchange; it writes P back over its own S columns, rescales its row
-//                   of O in TMEM when the running max rises, and finally normalises and stores
-//                   the row -- while the other group's QK^T, softmax and PV run alongside;
+//                   r owns row r of its S, P and O (TMEM lane r), so the row max and row sum
+//                   need no exchange (the row sum is kept in a register); it rescales its row of O
+//                   in TMEM when the running max rises, and finally normalises and stores the row;
 //       warp 12     (single-launch path) builds each item's kept-row list ahead of the gathers;
-//   * for bf16 inputs P is split into a bf16 head and a bf16 remainder (two PV MMAs), which
-//     keeps P at ~16 significant bits; fp16 P (11 bits) is used as is;
-//   * the PV MMA runs with N = 80: the 64 columns of V plus a constant tile whose first column
-//     is all ones, so column 64 of O accumulates the row sum of exactly the P that was used --
-//     the softmax warps never add up P themselves;
+//       warps 13-14 prepare each V tile as soon as it lands (alternate fills);
+//       warp 15     (single-launch path) zero-fills the block's share of pruned padded rows while
+//                   the rest of the block computes;
+//   * P is rounded to fp16 (11 significant bits) and meets an fp16 V: for bf16 inputs every V
+//     tile is converted in shared memory, exactly for |v| in [2^-14, 65504] and with an
+//     absolute error below 2^-25 under it; a tile holding a finite |v| >= 65536 keeps bf16 and
+//     meets a bf16 P;
 //   * key rows past the sequence end get probability 0 and the matching V rows are zeroed in
 //     shared memory, so whatever bytes lie there (the next image, or uninitialised capacity
 //     rows) never reach the output;
@@ -43,7 +48,7 @@
 // the kept counts of every image from the keep mask itself, the producer gathers the kept rows
 // of the padded Q/K/V straight into the swizzled tiles with 16-byte cp.async (32 lanes, one
 // coalesced 128-byte row segment per 8 lanes), and the epilogue writes each output row back to
-// its padded position and zero-fills the pruned rows of its (image, head).
+// its padded position.
 #include <cuda.h>
 
 #include <mutex>
@@ -58,46 +63,52 @@ namespace {
 constexpr int BM = 128;                 // query rows per tile (TMEM lanes)
 constexpr int BN = 128;                 // keys per step
 constexpr int kD = 64;                  // head dim
-constexpr int kThreads = 416;           // 13 warps: 2 x copier, 2 x MMA issuer, 8 x softmax, list builder
+constexpr int kThreads = 512;           // 16 warps: 2 x copier, 2 x MMA issuer, 8 x softmax, list, 2 x V, zero-fill
 // producer warps: warp 0 fills the Q/K/V rings (TMA on the packed path; on the single-launch path
 // warps 0 and 1 share the cp.async gathers), warp 12 (single-launch path) builds the kept-row
-// lists ahead of them
+// lists ahead of them, warps 13 and 14 prepare the V tiles for their PVs as soon as they land
+// (alternate fills), warp 15 (single-launch path) zero-fills the block's share of pruned rows
 constexpr int kCopyWarps = 2;
 constexpr int kListWarp = 12;
+constexpr int kVWarp0 = 13;
+constexpr int kVWarps = 2;
+constexpr int kZeroWarp = 15;
 constexpr int kMmaWarp0 = 2;            // warp 2 issues group 1's tensor-core work, warp 3 group 0's
 constexpr int kSoftmaxWarp0 = 4;
 constexpr int kSoftmaxWarps = 8;        // two groups of four, one per TMEM lane quarter each
 constexpr int kGroupWarps = 4;
-static_assert(kSoftmaxWarp0 + kSoftmaxWarps == kListWarp && kListWarp + 1 == kThreads / 32 &&
-                  kSoftmaxWarps == 2 * kGroupWarps,
+static_assert(kSoftmaxWarp0 + kSoftmaxWarps == kListWarp && kListWarp + 1 == kVWarp0 && kVWarp0 + kVWarps == kZeroWarp &&
+                  kZeroWarp + 1 == kThreads / 32 && kSoftmaxWarps == 2 * kGroupWarps,
               "warp roles");
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns: S buffers at 0 and 128 (the P of each 32-key slice is written back over the
-// slice's own S columns: 16 columns of packed head values, then 16 of bf16 remainders), O
-// buffers of 80 columns (64 outputs, the row sum, 15 zeros) at 256 and 352.
-constexpr uint32_t kColS0 = 0;
-constexpr uint32_t kColO0 = 256;
-constexpr uint32_t kOCols = 96;         // stride between the two O buffers
-constexpr uint32_t kPvN = 80;
+// TMEM columns: 256 per softmax group g, at 256 g: S (fp32 [128 x 128]) in columns 0..127, P
+// (16-bit [128 x 128], two keys per column) in 128..191, O (fp32 [128 x 64]) in 192..255.  With P
+// apart from S, the next chunk's S = Q K^T can be computed while this chunk's O += P V runs.
+constexpr uint32_t kGroupCols = 256;
+constexpr uint32_t kColS = 0;
+constexpr uint32_t kColP = 128;
+constexpr uint32_t kColO = 192;
 constexpr uint32_t kTileBytes = 128 * 128;
 constexpr int kQStages = 2;
-constexpr int kKVStages = 3;
+constexpr int kKVStages = 4;
 
 // shared-memory map (offsets from a 1024-byte aligned base)
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kQStages * kTileBytes;
 constexpr uint32_t kOffV = kOffK + kKVStages * kTileBytes;
-constexpr uint32_t kOffOnes = kOffV + kKVStages * kTileBytes;   // [128 keys x 64] MN-major, column 0 = 1
-constexpr uint32_t kOffBar = kOffOnes + kTileBytes;
-// fused: 4 slots, each the kept positions of one item's image (int16 [kFusedMaxN]), the byte
-// offsets of those padded rows' first head (int32 [kFusedMaxN]) and the kept-bit mask
-// (uint32 [kFusedMaxN / 32])
+constexpr uint32_t kOffBar = kOffV + kKVStages * kTileBytes;
+// fused: 4 slots, each the padded row index (b * N + n, int32) of every key row of one item, in
+// packed order
 constexpr int kIdxSlots = 4;
-constexpr uint32_t kIdxSlotBytes = kFusedMaxN * 2 + kFusedMaxN * 4 + kFusedMaxN / 8;
-// the block's first work items, decoded once in the prologue (Item: 5 ints each)
-constexpr int kItemTable = 64;
-constexpr uint32_t kOffItems = kOffBar + 512;
-constexpr uint32_t kOffIdx = kOffItems + kItemTable * 20;
+constexpr uint32_t kIdxSlotBytes = kFusedMaxN * 4;
+// short-sequence tiling: used when no image has more than kShortMax kept tokens; a tile's keys
+// then span at most 128 + 2 * (kShortMax - 1) <= 2 * BN rows
+constexpr int kShortMax = 64;
+// the block's first work items, decoded once in the prologue (Item: 6 ints each)
+constexpr int kItemTable = 56;
+constexpr uint32_t kBarBytes = 640;
+constexpr uint32_t kOffItems = kOffBar + kBarBytes;
+constexpr uint32_t kOffIdx = kOffItems + kItemTable * 24;
 // tile_pre[B+1], then cu[B+1]: after the list slots on the fused path, in their place otherwise
 template <bool kFused>
 constexpr uint32_t off_tile()
@@ -113,7 +124,7 @@ constexpr int smem_bytes(int B)
 struct Params {
     const int32_t *cu;      // packed path: cu_seqlens in
     const uint8_t *mask;    // fused path: keep mask [B, N]
-    const uint8_t *src[3];  // fused path: padded Q, K, V [B*N, H, 64]
+    const uint8_t *src[3];  // fused path: padded Q, K, V [B*N, H, 64]; packed path: V [capacity, H, 64] in src[2]
     int32_t *cu_out;        // fused path: cu_seqlens out (may be null)
     void *out;
     int B, H, N;
@@ -133,15 +144,21 @@ struct Bars {
     // then advance one fill at a time from its point of view (a parity wait never sees a phase
     // two ahead or two behind).
     uint64_t kv_full[kKVStages][2], kv_empty[kKVStages];
-    uint64_t s_full[2], p_full[2], s_free[2];
-    uint64_t o_full[2], o_free[2];
+    // per softmax group: S of a chunk computed / its P written (and S read) / its PV completed /
+    // its V tile ready for the PV (zero tail, fp16 or bf16 as v_fmt of its slot says) / O read out
+    uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
+    // v_ready[slot][g]: the V warp has prepared the slot's V tile of a chunk of group g (one
+    // barrier per slot and group, like kv_full: the V warp may run a few chunks ahead of a group,
+    // but never more than one fill of the same slot)
+    uint64_t v_ready[kKVStages][2];
     uint64_t idx_full[4], idx_free[4];  // fused: kept-row list slots, one per item in flight
     uint64_t drain[2];
     uint32_t tmem_slot;
     int abort;
-    int warp_sums[2][kThreads / 32];
+    int v_fmt[kKVStages];  // per K/V slot: 0 = its V tile (and so the chunk's P) is fp16, 1 = bf16
+    int warp_sums[3][kThreads / 32];
 };
-static_assert(sizeof(Bars) <= 512, "barrier block overflows its slot");
+static_assert(sizeof(Bars) <= kBarBytes, "barrier block overflows its slot");
 static_assert(smem_bytes<false>(kAttendMaxBatch) <= 232448, "packed path exceeds shared memory");
 static_assert(smem_bytes<true>(kFusedMaxBatch) <= 232448, "single-launch path exceeds shared memory");
 
@@ -179,29 +196,62 @@ __device__ __forceinline__ uint32_t range16_(int64_t s, int64_t lo, int64_t hi)
     return h > l ? (((1u << h) - 1u) & ~((1u << l) - 1u)) : 0u;
 }
 
-// One decoded work item.
+// One decoded work item: the query rows [q0, q0 + nq) of the packed token space (one head), and
+// the key rows [k0, k0 + nk) they attend to -- every kept token of each image that owns one of the
+// query rows (images are contiguous in the packed space, so this is one range).  b0 is the image
+// of row q0.
+//   per-image tiling (some image longer than kShortMax): item = (image b, 128-row q-tile qt, h),
+//     q0 = cu[b] + 128 qt, k0 = cu[b], nk = L_b: one image per item;
+//   short-sequence tiling: item = (tile t of the packed space, h), q0 = 128 t: the tile's rows
+//     may belong to several images, each query row attending only to its own image's keys.
 struct Item {
-    int b, h, qt, seq0, L;
+    int b0, h, q0, nq, k0, nk;
 };
-static_assert(sizeof(Item) == 20, "item table entry size");
+static_assert(sizeof(Item) == 24, "item table entry size");
 
-__device__ __forceinline__ Item decode_item(int item, int H, int B, const int32_t *tile_pre, const int32_t *cu)
+// Largest b in [lo, hi) with cu[b] <= p (cu non-decreasing, cu[lo] <= p): the image owning packed
+// row p (an empty image shares its start with the next one, which is then the one returned).
+__device__ __forceinline__ int image_of_row(const int32_t *cu, int lo, int hi, int p)
 {
-    Item it;
-    const int g = item / H;
-    it.h = item - g * H;
-    int lo = 0, hi = B;  // tile_pre[lo] <= g < tile_pre[hi]
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (tile_pre[mid] <= g)
+        if (cu[mid] <= p)
             lo = mid;
         else
             hi = mid;
     }
-    it.b = lo;
-    it.qt = g - tile_pre[lo];
-    it.seq0 = cu[lo];
-    it.L = cu[lo + 1] - it.seq0;
+    return lo;
+}
+
+__device__ __forceinline__ Item decode_item(int item, int H, int B, bool short_tiles, int T, const int32_t *tile_pre,
+                                            const int32_t *cu)
+{
+    Item it;
+    const int g = item / H;
+    it.h = item - g * H;
+    if (short_tiles) {
+        it.q0 = g * BM;
+        it.nq = min(BM, T - it.q0);
+        it.b0 = image_of_row(cu, 0, B, it.q0);
+        const int b1 = image_of_row(cu, it.b0, B, it.q0 + it.nq - 1);
+        it.k0 = cu[it.b0];
+        it.nk = cu[b1 + 1] - it.k0;
+    } else {
+        int lo = 0, hi = B;  // tile_pre[lo] <= g < tile_pre[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (tile_pre[mid] <= g)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        const int qt = g - tile_pre[lo];
+        it.b0 = lo;
+        it.k0 = cu[lo];
+        it.nk = cu[lo + 1] - it.k0;
+        it.q0 = it.k0 + qt * BM;
+        it.nq = min(BM, it.nk - qt * BM);
+    }
     return it;
 }
 
@@ -241,57 +291,75 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-template <bool kBF16>
-__device__ __forceinline__ void pack_pair(uint32_t (&r)[32], int i, float p0, float p1)
+// Two fp32 probabilities packed as two 16-bit values (low half = the first), fp16 or bf16, round
+// to nearest.
+__device__ __forceinline__ uint32_t pack_p(float a, float b, bool f16)
 {
-    if constexpr (kBF16) {
-        const uint32_t a = __float_as_uint(p0), b = __float_as_uint(p1);
-        float l0, l1;
-        sub2(l0, l1, p0, p1, __uint_as_float(a & 0xFFFF0000u), __uint_as_float(b & 0xFFFF0000u));
-        r[2 * i] = __byte_perm(a, b, 0x7632);
-        r[2 * i + 1] = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
-    } else {
-        r[2 * i] = pack_f16(p0, p1);
-    }
+    return f16 ? pack_f16(a, b) : pack_bf16(a, b);
 }
 
-// Exponentials of one 32-key slice of a row (keys c .. c+31, those >= nk masked to 0), packed
-// in place and written back over the slice's own TMEM columns as the PV A operand: 16 columns of
-// packed head values, then for bf16 16 columns of remainders.
-//   bf16: head = the top 16 bits of each fp32 value (truncation), remainder = the exact
-//         difference truncated the same way, so head + remainder carries p to a relative error
-//         below 2^-14 and the split costs integer byte permutes only (no conversions);
-//   fp16: p rounded to nearest fp16 (11 significant bits).
-// Packed pairs land in r[2i] (head) and r[2i+1] (remainder).
-template <bool kBF16>
-__device__ __forceinline__ void softmax_slice(uint32_t (&r)[32], int c, int nk, float scale_log2, float neg_m,
-                                              uint32_t taddr)
+// Exponentials of one 32-key slice of a row (keys c .. c+31; keys not set in `keys` masked to 0),
+// packed as 16 columns of 16-bit pairs and written to the row's P columns at `taddr`; returns the
+// slice's sum of the fp32 values.  `full` (warp-uniform) says every lane's keys cover the slice.
+__device__ __forceinline__ float softmax_slice(const uint32_t (&r)[32], uint32_t keys, bool full, bool f16,
+                                               float scale_log2, float neg_m, uint32_t taddr)
 {
-    if (c + 32 <= nk) {
+    uint32_t pk[16];
+    float s0 = 0.f, s1 = 0.f;
+    if (full) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             float x0, x1;
             fma2_scalar(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scale_log2, neg_m);
-            pack_pair<kBF16>(r, i, ex2_approx(x0), ex2_approx(x1));
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            s0 += p0;
+            s1 += p1;
+            pk[i] = pack_p(p0, p1, f16);
         }
     } else {
+        // masked keys enter the exponential as -inf (2^-inf = +0): a select per element, never a
+        // branch, so lanes with different key ranges do not diverge (and garbage S is dropped)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             float x0, x1;
             fma2_scalar(x0, x1, __uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]), scale_log2, neg_m);
-            pack_pair<kBF16>(r, i, c + 2 * i < nk ? ex2_approx(x0) : 0.f, c + 2 * i + 1 < nk ? ex2_approx(x1) : 0.f);
+            x0 = ((keys >> (2 * i)) & 1u) ? x0 : -INFINITY;
+            x1 = ((keys >> (2 * i + 1)) & 1u) ? x1 : -INFINITY;
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            s0 += p0;
+            s1 += p1;
+            pk[i] = pack_p(p0, p1, f16);
         }
     }
-    tmem_st16_strided<0>(taddr, r);
-    if constexpr (kBF16)
-        tmem_st16_strided<1>(taddr + 16, r);
+    tmem_st16(taddr, pk);
+    return s0 + s1;
 }
 
-__device__ __forceinline__ float slice_max(const uint32_t (&r)[32], int c, int nk, float mx)
+// P = 0 for a whole 32-key slice (no key of the slice belongs to any row of the warp).
+__device__ __forceinline__ void zero_p16(uint32_t taddr)
+{
+    uint32_t z[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        z[i] = 0u;
+    tmem_st16(taddr, z);
+}
+
+// Bit k set: key c + k of the slice lies in the row's range [lo, hi).
+__device__ __forceinline__ uint32_t key_bits(int c, int lo, int hi)
+{
+    const int a = max(lo - c, 0), b = min(hi - c, 32);
+    if (b <= a)
+        return 0u;
+    return (b == 32 ? 0xffffffffu : ((1u << b) - 1u)) & ~((1u << a) - 1u);
+}
+
+// Running max over the keys c .. c+31 of a row that are set in `keys`.
+__device__ __forceinline__ float slice_max(const uint32_t (&r)[32], uint32_t keys, bool full, float mx)
 {
     // two independent chains of three-input maxima
     float t0 = mx, t1 = -INFINITY;
-    if (c + 32 <= nk) {
+    if (full) {
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
             t0 = fmax3(t0, __uint_as_float(r[j]), __uint_as_float(r[j + 1]));
@@ -300,10 +368,10 @@ __device__ __forceinline__ float slice_max(const uint32_t (&r)[32], int c, int n
     } else {
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
-            t0 = fmax3(t0, c + j < nk ? __uint_as_float(r[j]) : -INFINITY,
-                       c + j + 1 < nk ? __uint_as_float(r[j + 1]) : -INFINITY);
-            t1 = fmax3(t1, c + j + 2 < nk ? __uint_as_float(r[j + 2]) : -INFINITY,
-                       c + j + 3 < nk ? __uint_as_float(r[j + 3]) : -INFINITY);
+            t0 = fmax3(t0, ((keys >> j) & 1u) ? __uint_as_float(r[j]) : -INFINITY,
+                       ((keys >> (j + 1)) & 1u) ? __uint_as_float(r[j + 1]) : -INFINITY);
+            t1 = fmax3(t1, ((keys >> (j + 2)) & 1u) ? __uint_as_float(r[j + 2]) : -INFINITY,
+                       ((keys >> (j + 3)) & 1u) ? __uint_as_float(r[j + 3]) : -INFINITY);
         }
     }
     return fmaxf(t0, t1);
@@ -343,17 +411,79 @@ __device__ __forceinline__ void store_row(const Params &p, int64_t off, const ui
     }
 }
 
+// Two bf16 values -> two fp16 values, round to nearest (exact for |v| in [2^-14, 65504]; smaller
+// magnitudes round to fp16's subnormal grid, an absolute error below 2^-25).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w)
+{
+    const __half2 h = __floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// A K/V slot's V tile before its PV, by one whole warp: rows [nk, nk16) are zeroed (they meet
+// P = 0 and must not hold NaN), and bf16 values are converted in place to fp16, so that P can be
+// rounded to fp16 (11 significant bits) rather than bf16 (8).  A value outside fp16's range (a
+// finite |v| >= 65536, or an infinity) becomes an fp16 infinity; if any does, the tile is put back
+// to its original bf16 bytes from global memory (row r of the tile is row rows[base + r], or
+// row0 + r when rows is null, of the tensor at vsrc) and stays bf16, and so does the P that meets
+// it.  Rows are 128 contiguous bytes in the swizzled layout, so rows [0, nk) are the first
+// 128 nk bytes.  Returns true when the tile (and the chunk's P) is fp16.
+template <bool kBF16>
+__device__ __noinline__ bool prepare_v(uint8_t *sV, int nk, int lane, const uint8_t *vsrc, int64_t row_bytes,
+                                       const int32_t *rows, int base, int64_t row0)
+{
+    const int nk16 = (nk + 15) & ~15;
+    for (int i = lane; i < (nk16 - nk) * 8; i += 32)
+        *reinterpret_cast<uint4 *>(sV + nk * 128 + i * 16) = make_uint4(0, 0, 0, 0);
+    bool fp16 = true;
+    if constexpr (kBF16) {
+        uint4 *v = reinterpret_cast<uint4 *>(sV);
+        const int n16 = nk * 8;  // 16-byte chunks of rows [0, nk)
+        uint32_t infs = 0;
+        for (int i0 = lane; i0 < n16; i0 += 128) {
+            uint4 w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                w[u] = i0 + 32 * u < n16 ? v[i0 + 32 * u] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                uint4 h;
+                h.x = bf16x2_to_f16x2(w[u].x);
+                h.y = bf16x2_to_f16x2(w[u].y);
+                h.z = bf16x2_to_f16x2(w[u].z);
+                h.w = bf16x2_to_f16x2(w[u].w);
+                infs |= __vcmpeq2(h.x & 0x7FFF7FFFu, 0x7C007C00u) | __vcmpeq2(h.y & 0x7FFF7FFFu, 0x7C007C00u) |
+                        __vcmpeq2(h.z & 0x7FFF7FFFu, 0x7C007C00u) | __vcmpeq2(h.w & 0x7FFF7FFFu, 0x7C007C00u);
+                if (i0 + 32 * u < n16)
+                    v[i0 + 32 * u] = h;
+            }
+        }
+        if (__any_sync(0xffffffffu, infs != 0u)) {
+            // rare: an infinity or a value beyond fp16's range -- the original bf16 tile again
+            __syncwarp();
+            for (int i = lane; i < n16; i += 32) {
+                const int r = i >> 3, c = i & 7;
+                const int64_t grow = rows != nullptr ? static_cast<int64_t>(rows[base + r]) : row0 + r;
+                v[r * 8 + (c ^ (r & 7))] = __ldg(reinterpret_cast<const uint4 *>(vsrc + grow * row_bytes) + c);
+            }
+            fp16 = false;
+        }
+    }
+    fence_proxy_async_smem();  // generic-proxy writes, read next by the tensor core
+    __syncwarp();
+    return fp16;
+}
+
 // Fused path: copier warp w (of kCopyWarps) copies its share of one tile of up to 128 kept rows
 // of one head from the padded tensor into the 128-byte-swizzled layout with 16-byte cp.async:
-// row r of the tile is the image's kept row base + r.  The chunks go in groups of 32 (one per
-// lane, 8 lanes per 128-byte row, so each row is one coalesced segment), group g to warp g % 2.
+// row r of the tile is padded row rows[base + r].  The chunks go in groups of 32 (one per lane,
+// 8 lanes per 128-byte row, so each row is one coalesced segment), group g to warp g % kCopyWarps.
 // Completion arrives on `bar` once per copier lane.
-__device__ __forceinline__ void copy_tile_async(uint8_t *tile, const uint8_t *src, uint64_t *bar, const int32_t *offs,
-                                                int base, int count, int w, int lane)
+__device__ __forceinline__ void copy_tile_async(uint8_t *tile, const uint8_t *src, int64_t row_bytes, uint64_t *bar,
+                                                const int32_t *rows, int base, int count, int w, int lane)
 {
-    // src points at this head's 128 bytes of the image's padded row 0; offs[] holds the byte
-    // offsets of the kept rows from there.  Rows at or past `count` are not copied: their S
-    // columns are masked, their V rows zeroed before use, or (Q) their output never stored.
+    // src points at this head's 128 bytes of padded row 0.  Rows at or past `count` are not
+    // copied: their S columns are masked, their V rows zeroed before use, or (Q) their output
+    // never stored.
     const uint32_t tile_s = smem_addr(tile);
     const int groups = (count * 8 + 31) >> 5;
 #pragma unroll 4
@@ -361,12 +491,33 @@ __device__ __forceinline__ void copy_tile_async(uint8_t *tile, const uint8_t *sr
         const int i = lane + 32 * grp;
         const int r = i >> 3, c = i & 7;
         if (r < count) {
-            const uint8_t *gsrc = src + offs[base + r] + c * 16;
+            const uint8_t *gsrc = src + static_cast<int64_t>(rows[base + r]) * row_bytes + c * 16;
             const uint32_t d = tile_s + r * 128 + ((c ^ (r & 7)) << 4);
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
         }
     }
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// Fused path: one tile of up to 128 kept rows of one head, as copy_tile_async does, but when the
+// rows are consecutive padded rows (every token of the range kept, e.g. an unpruned image) copier
+// lane 0 of warp 0 moves the whole 128-row box with one TMA load of the padded tensor instead
+// (rows past `count` land too and are masked like the gathered case's stale rows).  Either way each
+// copier lane arrives once on `bar`; the TMA bytes are added to the phase's transaction count.
+__device__ __forceinline__ void gather_tile(uint8_t *tile, const CUtensorMap *tm, int h, const uint8_t *src,
+                                            int64_t row_bytes, uint64_t *bar, const int32_t *rows, int base,
+                                            int count, int w, int lane)
+{
+    const int r0 = rows[base];
+    if (rows[base + count - 1] - r0 == count - 1) {  // the list is increasing: consecutive rows
+        if (w == 0 && lane == 0) {
+            mbar_expect_tx(bar, kTileBytes);
+            tma_load_3d(tile, tm, bar, 0, h, r0);
+        }
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+        return;
+    }
+    copy_tile_async(tile, src, row_bytes, bar, rows, base, count, w, lane);
 }
 
 template <bool kBF16, bool kFused>
@@ -379,13 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Bars *bars = reinterpret_cast<Bars *>(base + kOffBar);
     int32_t *tile_pre = reinterpret_cast<int32_t *>(base + off_tile<kFused>());  // [B+1]
     int32_t *cu_s = tile_pre + (p.B + 1);                               // [B+1]
-    auto idx_list = [&](int slot) { return reinterpret_cast<int16_t *>(base + kOffIdx + slot * kIdxSlotBytes); };
-    auto idx_offs = [&](int slot) {
-        return reinterpret_cast<int32_t *>(base + kOffIdx + slot * kIdxSlotBytes + kFusedMaxN * 2);
-    };
-    auto idx_bits = [&](int slot) {
-        return reinterpret_cast<uint32_t *>(base + kOffIdx + slot * kIdxSlotBytes + kFusedMaxN * 6);
-    };
+    auto idx_list = [&](int slot) { return reinterpret_cast<int32_t *>(base + kOffIdx + slot * kIdxSlotBytes); };
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -394,11 +539,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_trigger();
 
     if (tid == 0) {
-        if constexpr (!kFused) {
-            prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_v);
-        }
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
         // full barriers: one TMA arrival with transaction bytes, or (fused) one cp.async
         // arrival per producer lane
         const uint32_t fills = kFused ? 32u * kCopyWarps : 1u;
@@ -410,12 +553,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bars->kv_full[s][0], kFused ? 2u * fills : fills);
             mbar_init(&bars->kv_full[s][1], kFused ? 2u * fills : fills);
             mbar_init(&bars->kv_empty[s], 1);
+            mbar_init(&bars->v_ready[s][0], 1);
+            mbar_init(&bars->v_ready[s][1], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars->s_full[s], 1);
             mbar_init(&bars->p_full[s], kGroupWarps);  // one arrival per warp of softmax group s
-            mbar_init(&bars->s_free[s], 1);
-            mbar_init(&bars->o_full[s], 1);
+            mbar_init(&bars->pv_done[s], 1);
             mbar_init(&bars->o_free[s], kGroupWarps);
         }
         for (int s = 0; s < kIdxSlots; ++s) {
@@ -430,19 +574,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         tmem_alloc(&bars->tmem_slot, kTmemCols);
         tmem_relinquish();
-    }
-
-    // ---- constant ones tile: 128 key rows of 128 bytes in the 128-byte-swizzled layout, element 0
-    // of every row = 1.0 (the 16-byte chunk c of row r sits at chunk c ^ (r % 8))
-    {
-        uint8_t *ones = base + kOffOnes;
-        const uint32_t one = kBF16 ? 0x3F80u : 0x3C00u;
-        for (int i = tid; i < 128 * 8; i += kThreads) {
-            const int r = i >> 3, c = i & 7;
-            const uint4 v = make_uint4(c == (r & 7) ? one : 0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4 *>(ones + r * 128 + c * 16) = v;
-        }
-        fence_proxy_async_smem();
     }
 
     // everything above is private to the block; the inputs may come from the previous kernel
@@ -492,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (tid == 0)
         tile_pre[0] = 0;
-    int carry_t = 0, carry_l = 0;
+    int carry_t = 0, carry_l = 0, lmax = 0;  // lmax: longest sequence, or kShortMax + 1 if any image is malformed
     for (int c0 = 0; c0 < B; c0 += kThreads) {
         const int b = c0 + tid;
         int tiles = 0, len = 0;
@@ -500,6 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (kFused) {
                 len = cu_s[b + 1];
                 tiles = (len + BM - 1) / BM;
+                lmax = max(lmax, len);
             } else {
                 const int64_t s0 = p.cu[b], s1 = p.cu[b + 1];
                 cu_s[b] = static_cast<int32_t>(s0);
@@ -508,8 +640,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (s0 < 0 || s1 < s0 || s1 > p.capacity) {
                     if (blockIdx.x == 0)
                         raise_error(p.err, RRA_ERR_BAD_SEQLENS);
+                    lmax = kShortMax + 1;  // malformed: per-image tiles, which skip this image
                 } else {
                     tiles = static_cast<int>((s1 - s0 + BM - 1) / BM);
+                    // the packed space must start at row 0 for the short-sequence tiling
+                    lmax = max(lmax, (b == 0 && s0 != 0) ? kShortMax + 1 : static_cast<int>(s1 - s0));
                 }
             }
         }
@@ -523,9 +658,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l_incl += c;
             }
         }
+        const int wmax = __reduce_max_sync(0xffffffffu, lmax);
         if (lane == 31) {
             bars->warp_sums[0][warp] = it_incl;
             bars->warp_sums[1][warp] = l_incl;
+            bars->warp_sums[2][warp] = wmax;
         }
         __syncthreads();
         int before_t = carry_t, before_l = carry_l, chunk_t = 0, chunk_l = 0;
@@ -535,6 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             before_l += (w < warp) ? bars->warp_sums[1][w] : 0;
             chunk_t += bars->warp_sums[0][w];
             chunk_l += bars->warp_sums[1][w];
+            lmax = max(lmax, bars->warp_sums[2][w]);
         }
         if (b < B) {
             tile_pre[b + 1] = before_t + it_incl;
@@ -552,36 +690,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (blockIdx.x == 0 && p.cu_out != nullptr)
             for (int b = tid; b <= B; b += kThreads)
                 p.cu_out[b] = cu_s[b];
-        // images without kept tokens have no work item: their padded output rows are zeroed here
-        const int out_vecs = (p.out_dt == RRA_F32 ? 4 * kD : 2 * kD) / 16;  // 16-byte vectors per head row
-        for (int b = blockIdx.x; b < B; b += gridDim.x) {
-            if (cu_s[b + 1] != cu_s[b])
-                continue;
-            uint4 *y = reinterpret_cast<uint4 *>(p.out) + static_cast<int64_t>(b) * p.N * H * out_vecs;
-            for (int64_t i = tid; i < static_cast<int64_t>(p.N) * H * out_vecs; i += kThreads)
-                y[i] = make_uint4(0, 0, 0, 0);
-        }
     }
+
+    // tiling: when no image is longer than kShortMax, 128-row tiles of the packed space (several
+    // images per tile); otherwise one image per tile
+    const int T = cu_s[B];
+    const bool short_tiles = lmax <= kShortMax && T > 0;
+    const int total_items = (short_tiles ? (T + BM - 1) / BM : tile_pre[B]) * H;
 
     // decode the block's first items once: every role walks the same list
     Item *items = reinterpret_cast<Item *>(base + kOffItems);
-    {
-        const int total = tile_pre[B] * H;
-        for (int k = tid; k < kItemTable; k += kThreads) {
-            const int item = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
-            if (item < total)
-                items[k] = decode_item(item, H, B, tile_pre, cu_s);
-        }
+    for (int k = tid; k < kItemTable; k += kThreads) {
+        const int item = static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x);
+        if (item < total_items)
+            items[k] = decode_item(item, H, B, short_tiles, T, tile_pre, cu_s);
     }
     auto item_at = [&](int k, int item) {
-        return k < kItemTable ? items[k] : decode_item(item, H, B, tile_pre, cu_s);
+        return k < kItemTable ? items[k] : decode_item(item, H, B, short_tiles, T, tile_pre, cu_s);
     };
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_slot;
-    const int total_items = tile_pre[B] * H;
     // work items of this block, dealt round-robin: a block's items come from unrelated images,
     // which evens out the per-block cost
     const int item_first = static_cast<int>(blockIdx.x);
@@ -594,54 +725,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         // copier is done with a list before that epilogue can run); this warp runs up to four
         // items ahead of the copier.
         uint32_t idx_phase = 0;
-        int cur_b = -1, prev_slot = 0, n = 0;
+        int cur_k0 = -1, cur_nk = -1, prev_slot = 0, n = 0;
         bool ok = true;
+        const int nwords = (p.N + 31) / 32;
         for (int item = item_first; ok && item < item_end; item += item_step, ++n) {
             const Item it = item_at(n, item);
-            const int row_off = it.b * p.N;
             const int islot = n & (kIdxSlots - 1);
-            int16_t *list = idx_list(islot);
-            uint32_t *bits = idx_bits(islot);
-            int32_t *offs = idx_offs(islot);
-            const int nwords = (p.N + 31) / 32;
+            int32_t *list = idx_list(islot);
             ok = warp_wait(&bars->idx_free[islot], ((idx_phase >> islot) & 1u) ^ 1u, bars, p);
             if (!ok)
                 break;
             idx_phase ^= 1u << islot;
-            if (it.b == cur_b) {
-                // same image as the previous item: copy its list
-                const int16_t *pl = idx_list(prev_slot);
-                const int32_t *po = idx_offs(prev_slot);
-                const uint32_t *pb = idx_bits(prev_slot);
-                for (int i = lane; i < it.L; i += 32) {
+            if (it.k0 == cur_k0 && it.nk == cur_nk) {
+                // same key rows as the previous item (another head or q-tile): copy its list
+                const int32_t *pl = idx_list(prev_slot);
+                for (int i = lane; i < it.nk; i += 32)
                     list[i] = pl[i];
-                    offs[i] = po[i];
-                }
-                for (int i = lane; i < nwords; i += 32)
-                    bits[i] = pb[i];
             } else {
-                // kept positions of this image in order: mask bytes fetched 8 words of 32 at a
-                // time (independent loads), then one ballot per word
+                // the padded rows of the kept tokens of every image of the item, in packed order:
+                // per image, mask bytes fetched 8 words of 32 at a time (independent loads), then
+                // one ballot per word
                 int running = 0;
-                for (int w0 = 0; w0 < nwords; w0 += 8) {
-                    bool keep[8];
+                for (int b = it.b0; b < B && cu_s[b] < it.k0 + it.nk; ++b) {
+                    const int row_off = b * p.N;
+                    for (int w0 = 0; w0 < nwords; w0 += 8) {
+                        bool keep[8];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int tok = (w0 + u) * 32 + lane;
-                        keep[u] = tok < p.N && p.mask[row_off + tok] != 0;
-                    }
+                        for (int u = 0; u < 8; ++u) {
+                            const int tok = (w0 + u) * 32 + lane;
+                            keep[u] = tok < p.N && p.mask[row_off + tok] != 0;
+                        }
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const unsigned bal = __ballot_sync(0xffffffffu, keep[u]);
-                        if (w0 + u < nwords) {
+                        for (int u = 0; u < 8; ++u) {
+                            const unsigned bal = __ballot_sync(0xffffffffu, keep[u]);
                             if (keep[u]) {
                                 const int slot_i = running + __popc(bal & ((1u << lane) - 1u));
-                                const int tok = (w0 + u) * 32 + lane;
-                                list[slot_i] = static_cast<int16_t>(tok);
-                                offs[slot_i] = tok * H * kD * 2;  // < 2^31 (checked on the host)
+                                list[slot_i] = row_off + (w0 + u) * 32 + lane;  // < B * N < 2^31
                             }
-                            if (lane == 0)
-                                bits[w0 + u] = bal;
                             running += __popc(bal);
                         }
                     }
@@ -650,7 +770,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&bars->idx_full[islot]);
-            cur_b = it.b;
+            cur_k0 = it.k0;
+            cur_nk = it.nk;
             prev_slot = islot;
         }
     } else if (warp < (kFused ? kCopyWarps : 1)) {
@@ -666,8 +787,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int item = item_first; ok && item < item_end; item += item_step) {
             const Item it = item_at(static_cast<int>(n_items), item);
-            const int nkc = (it.L + BN - 1) / BN;
-            const int row_off = it.b * p.N;  // fused: first padded row of this image
+            const int nkc = (it.nk + BN - 1) / BN;
             const int islot = static_cast<int>(n_items & (kIdxSlots - 1));
             if constexpr (kFused) {
                 // the kept-row list of this item (built by the list warp)
@@ -680,16 +800,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok)
                 break;
             q_phase ^= 1u << qs;
-            // fused: this head's 128 bytes of the image's padded row 0 in Q, K, V
-            const int64_t head0 = (static_cast<int64_t>(row_off) * H + it.h) * kD * 2;
+            // fused: this head's 128 bytes of padded row 0 in Q, K, V; one padded row is H * 128 bytes
+            const int64_t head0 = static_cast<int64_t>(it.h) * kD * 2;
+            const int64_t row_bytes = static_cast<int64_t>(H) * kD * 2;
             if constexpr (kFused) {
-                const int q0 = it.qt * BM;
-                copy_tile_async(base + kOffQ + qs * kTileBytes, p.src[0] + head0, &bars->q_full[qs], idx_offs(islot), q0,
-                                min(BM, it.L - q0), warp, lane);
+                gather_tile(base + kOffQ + qs * kTileBytes, &tm_q, it.h, p.src[0] + head0, row_bytes,
+                            &bars->q_full[qs], idx_list(islot), it.q0 - it.k0, it.nq, warp, lane);
             } else {
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&bars->q_full[qs], kTileBytes);
-                    tma_load_3d(base + kOffQ + qs * kTileBytes, &tm_q, &bars->q_full[qs], 0, it.h, it.seq0 + it.qt * BM);
+                    tma_load_3d(base + kOffQ + qs * kTileBytes, &tm_q, &bars->q_full[qs], 0, it.h, it.q0);
                 }
             }
             __syncwarp();
@@ -702,16 +822,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 kv_phase ^= 1u << ks;
                 uint64_t *full = &bars->kv_full[ks][n_items & 1u];  // the owning group's barrier
                 if constexpr (kFused) {
-                    const int cnt = min(BN, it.L - kc * BN);
-                    copy_tile_async(base + kOffK + ks * kTileBytes, p.src[1] + head0, full, idx_offs(islot), kc * BN,
-                                    cnt, warp, lane);
-                    copy_tile_async(base + kOffV + ks * kTileBytes, p.src[2] + head0, full, idx_offs(islot), kc * BN,
-                                    cnt, warp, lane);
+                    const int cnt = min(BN, it.nk - kc * BN);
+                    gather_tile(base + kOffK + ks * kTileBytes, &tm_k, it.h, p.src[1] + head0, row_bytes, full,
+                                idx_list(islot), kc * BN, cnt, warp, lane);
+                    gather_tile(base + kOffV + ks * kTileBytes, &tm_v, it.h, p.src[2] + head0, row_bytes, full,
+                                idx_list(islot), kc * BN, cnt, warp, lane);
                 } else {
                     if (lane == 0) {
                         mbar_arrive_expect_tx(full, 2 * kTileBytes);
-                        tma_load_3d(base + kOffK + ks * kTileBytes, &tm_k, full, 0, it.h, it.seq0 + kc * BN);
-                        tma_load_3d(base + kOffV + ks * kTileBytes, &tm_v, full, 0, it.h, it.seq0 + kc * BN);
+                        tma_load_3d(base + kOffK + ks * kTileBytes, &tm_k, full, 0, it.h, it.k0 + kc * BN);
+                        tma_load_3d(base + kOffV + ks * kTileBytes, &tm_v, full, 0, it.h, it.k0 + kc * BN);
                     }
                 }
                 __syncwarp();
@@ -742,27 +862,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ================================================================ tcgen05 issuers
         // One issuing thread per softmax group (warp 3: group 0, warp 2: group 1), so the two
         // groups' tensor-core work is issued concurrently.  Group g owns the items n = g, g+2, ...
-        // of the block, S buffer g and O buffer g; for each 128-key chunk of its items its issuer
-        // runs S = Q K^T, waits for the softmax to write P over S, then O += P V.  The Q/K/V rings
-        // are filled in item order for both groups, so each issuer walks every item and, for the
-        // other group's, only advances its ring positions and phase bits.
+        // of the block and TMEM columns [256 g, 256 g + 256).  Per chunk kc of an item: S = Q K^T
+        // into S; once the softmax has turned S(kc) into P(kc) (p_full), S(kc+1) is issued at once
+        // -- S and P are separate, so it overlaps O += P(kc) V(kc) -- then that PV, once the V
+        // warp has prepared V(kc).
+        // The Q/K/V rings are filled in item order for both groups, so each issuer walks every
+        // item and, for the other group's, only advances its ring positions.
         const int g = kMmaWarp0 + 1 - warp;
-        uint32_t q_ph = 0, kv_ph = 0, p_ph = 0, sfree_ph = 0, ofree_ph = 0;
-        const uint32_t idPV = idesc_f16(BM, kPvN, kBF16 ? 1u : 0u, 1u);
+        uint32_t q_ph = 0, kv_ph = 0, p_ph = 0, ofree_ph = 0;
         // shared-memory descriptors of the ring slots: stepping K inside a 128-byte swizzled row
         // adds 32 bytes (2 units) to the start address, stepping 16 key rows adds 2048 bytes (128
-        // units), and a slot is 1024 units further.  V descriptors carry, as leading offset, the
-        // distance to the ones tile that supplies PV columns 64..79.
+        // units), and a slot is 1024 units further
         const uint64_t qdesc0 = smem_desc_sw128(smem_addr(base + kOffQ), 16, 1024);
         const uint64_t kdesc0 = smem_desc_sw128(smem_addr(base + kOffK), 16, 1024);
-        const uint64_t vdesc0 = smem_desc_sw128(smem_addr(base + kOffV), kOffOnes - kOffV, 1024);
+        const uint64_t vdesc0 = smem_desc_sw128(smem_addr(base + kOffV), 16, 1024);
         auto slot_desc = [](uint64_t d0, int slot) { return d0 + static_cast<uint64_t>(slot) * (kTileBytes >> 4); };
-        const uint32_t dS = tmem + kColS0 + 128 * g;
-        const uint32_t dO = tmem + kColO0 + kOCols * g;
+        const uint32_t dS = tmem + kGroupCols * g + kColS;
+        const uint32_t dP = tmem + kGroupCols * g + kColP;
+        const uint32_t dO = tmem + kGroupCols * g + kColO;
+        // S(kc) = Q K(kc)^T into S: one MMA per 16 of the 64 head dims
+        auto issue_qk = [&](int qs, int ks, int nk, bool last) {
+            if (lane == 0) {
+                tc_fence_after();
+                if constexpr (kFused)
+                    fence_proxy_async_smem();  // Q/K/V arrived through cp.async (generic proxy)
+                const uint64_t qd = slot_desc(qdesc0, qs);
+                const uint64_t kd = slot_desc(kdesc0, ks);
+                const uint32_t idS = idesc_f16(BM, (nk + 15) & ~15, kBF16 ? 1u : 0u, 0u);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    mma_ss(dS, qd + 2 * kk, kd + 2 * kk, idS, kk > 0 ? 1u : 0u);
+                mma_commit(&bars->s_full[g]);
+                if (last)
+                    mma_commit(&bars->q_empty[qs]);  // last read of this Q tile
+            }
+            __syncwarp();
+        };
+        uint32_t v_ph = 0;
         int qs = 0, ks = 0, n = 0;
-        bool s_busy = false, ok = true;
+        bool ok = true;
         for (int item = item_first; ok && item < item_end; item += item_step, ++n) {
-            const int nkc = (item_at(n, item).L + BN - 1) / BN;
+            const Item it = item_at(n, item);
+            const int nkc = (it.nk + BN - 1) / BN;
             if ((n & 1) != g) {
                 // the other group's item: its Q slot is never ours (item n uses slot n % 2), and
                 // its K/V chunks pass through the same slots but signal the other group's
@@ -772,83 +913,58 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ks = (ks + nkc) % kKVStages;
                 continue;
             }
-            const int L = item_at(n, item).L;
             ok = warp_wait(&bars->q_full[qs], (q_ph >> qs) & 1u, bars, p);
             if (!ok)
                 break;
             q_ph ^= 1u << qs;
+            ok = warp_wait(&bars->kv_full[ks][g], (kv_ph >> ks) & 1u, bars, p);
+            if (!ok)
+                break;
+            kv_ph ^= 1u << ks;
+            issue_qk(qs, ks, min(BN, it.nk), nkc == 1);
             for (int kc = 0; kc < nkc; ++kc) {
-                const int nk = min(BN, L - kc * BN);
-                const int nk16 = (nk + 15) & ~15;
-                ok = warp_wait(&bars->kv_full[ks][g], (kv_ph >> ks) & 1u, bars, p);
-                if (!ok)
-                    break;
-                kv_ph ^= 1u << ks;
-                uint8_t *sV = base + kOffV + ks * kTileBytes;
-                // zero V rows [nk, nk16): they enter the PV MMA with probability 0
-                if (nk < nk16) {
-                    for (int i = lane; i < (nk16 - nk) * 8; i += 32)
-                        *reinterpret_cast<uint4 *>(sV + (nk + (i >> 3)) * 128 + (i & 7) * 16) = make_uint4(0, 0, 0, 0);
-                    fence_proxy_async_smem();
-                }
-                __syncwarp();
-                // the S buffer holds the previous chunk's P until that chunk's PV has completed
-                if (s_busy) {
-                    ok = warp_wait(&bars->s_free[g], sfree_ph, bars, p);
-                    if (!ok)
-                        break;
-                    sfree_ph ^= 1u;
-                }
-                if (lane == 0) {
-                    tc_fence_after();
-                    if constexpr (kFused)
-                        fence_proxy_async_smem();  // Q/K/V arrived through cp.async (generic proxy)
-                    const uint64_t qd = slot_desc(qdesc0, qs);
-                    const uint64_t kd = slot_desc(kdesc0, ks);
-                    const uint32_t idS = idesc_f16(BM, nk16, kBF16 ? 1u : 0u, 0u);
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk)
-                        mma_ss(dS, qd + 2 * kk, kd + 2 * kk, idS, kk > 0 ? 1u : 0u);
-                    mma_commit(&bars->s_full[g]);
-                    if (kc == nkc - 1)
-                        mma_commit(&bars->q_empty[qs]);  // last read of this Q tile
-                }
-                __syncwarp();
-                // P of this chunk in TMEM; before the first PV of an item, the group's previous
-                // item must have been read out of O
+                const int nk = min(BN, it.nk - kc * BN);
+                const int ks_next = (ks + 1 == kKVStages) ? 0 : ks + 1;
+                // P(kc) written (and S(kc) read) by the softmax
                 ok = warp_wait(&bars->p_full[g], p_ph, bars, p);
                 if (!ok)
                     break;
                 p_ph ^= 1u;
+                if (kc + 1 < nkc) {
+                    ok = warp_wait(&bars->kv_full[ks_next][g], (kv_ph >> ks_next) & 1u, bars, p);
+                    if (!ok)
+                        break;
+                    kv_ph ^= 1u << ks_next;
+                    issue_qk(qs, ks_next, min(BN, it.nk - (kc + 1) * BN), kc + 1 == nkc - 1);
+                }
+                // before the first PV of an item, the group's previous item must have been read out of O
                 if (kc == 0 && n >= 2) {
                     ok = warp_wait(&bars->o_free[g], ofree_ph, bars, p);
                     if (!ok)
                         break;
                     ofree_ph ^= 1u;
                 }
+                // V(kc) prepared by the V warp (zero tail; fp16 unless out of its range)
+                ok = warp_wait(&bars->v_ready[ks][g], (v_ph >> ks) & 1u, bars, p);
+                if (!ok)
+                    break;
+                v_ph ^= 1u << ks;
+                const bool fp16 = !kBF16 || bars->v_fmt[ks] == 0;
                 if (lane == 0) {
                     tc_fence_after();
-                    const uint64_t vd = slot_desc(vdesc0, ks) - (static_cast<uint64_t>(ks) * (kTileBytes >> 4) << 16);
-                    const int nj = nk16 >> 4;
-                    // keys 16j..16j+15 live in slice j/2: head part at column 32(j/2) + 8(j%2),
-                    // remainder (bf16) 16 columns further
+                    const uint64_t vd = slot_desc(vdesc0, ks);
+                    const uint32_t idPV = idesc_f16(BM, kD, fp16 ? 0u : 1u, 1u);
+                    const int nj = ((nk + 15) & ~15) >> 4;
+                    // keys 16j .. 16j+15: P columns 8j .. 8j+7 (two 16-bit values per column)
 #pragma unroll
                     for (int j = 0; j < BN / 16; ++j)
                         if (j < nj)
-                            mma_ts(dO, dS + 32 * (j >> 1) + 8 * (j & 1), vd + 128 * j, idPV, (kc > 0 || j > 0) ? 1u : 0u);
-                    if (kBF16) {
-#pragma unroll
-                        for (int j = 0; j < BN / 16; ++j)
-                            if (j < nj)
-                                mma_ts(dO, dS + 32 * (j >> 1) + 8 * (j & 1) + 16, vd + 128 * j, idPV, 1u);
-                    }
-                    mma_commit(&bars->o_full[g]);
-                    mma_commit(&bars->s_free[g]);
+                            mma_ts(dO, dP + 8 * j, vd + 128 * j, idPV, (kc > 0 || j > 0) ? 1u : 0u);
+                    mma_commit(&bars->pv_done[g]);
                     mma_commit(&bars->kv_empty[ks]);
                 }
                 __syncwarp();
-                s_busy = true;
-                ks = (ks + 1 == kKVStages) ? 0 : ks + 1;
+                ks = ks_next;
             }
             qs = (qs + 1 == kQStages) ? 0 : qs + 1;
         }
@@ -858,66 +974,151 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait_bounded(&bars->drain[g], 0, kDrainNs);
         }
         __syncwarp();
+    } else if (warp >= kVWarp0 && warp < kVWarp0 + kVWarps) {
+        // ================================================================ V tiles
+        // The K/V fills in production order, V warp v preparing fills v, v + 2, ..., each as soon
+        // as it has landed: zero the V rows past the chunk's keys and, for bf16 inputs, convert the
+        // tile to fp16 in place when it fits; then record the slot's format and tell the owning
+        // group (its issuer before the PV, its softmax before writing P).  A slot is refilled only
+        // after that chunk's PV, which follows these reads of v_fmt.
+        const int vw = warp - kVWarp0;
+        uint32_t kv_ph = 0;  // bit 2*slot + group: parity of kv_full[slot][group] waits
+        int ks = 0, n = 0, fill = 0;
+        bool ok = true;
+        for (int item = item_first; ok && item < item_end; item += item_step, ++n) {
+            const Item it = item_at(n, item);
+            const int nkc = (it.nk + BN - 1) / BN;
+            const int gi = n & 1;
+            for (int kc = 0; kc < nkc; ++kc, ++fill) {
+                // every V warp waits for every fill in order (so that no parity wait can run a phase
+                // ahead of a fill still in flight), and prepares only its own
+                const uint32_t bit = 1u << (2 * ks + gi);
+                ok = warp_wait(&bars->kv_full[ks][gi], (kv_ph & bit) ? 1u : 0u, bars, p);
+                if (!ok)
+                    break;
+                kv_ph ^= bit;
+                if (fill % kVWarps == vw) {
+                    // where the tile's rows came from, should it have to be restored as bf16
+                    const uint8_t *vsrc = p.src[2] + static_cast<int64_t>(it.h) * kD * 2;
+                    const int32_t *rows = kFused ? idx_list(n & (kIdxSlots - 1)) : nullptr;
+                    const bool fp16 = prepare_v<kBF16>(base + kOffV + ks * kTileBytes, min(BN, it.nk - kc * BN),
+                                                       lane, vsrc, static_cast<int64_t>(H) * kD * 2, rows, kc * BN,
+                                                       static_cast<int64_t>(it.k0) + kc * BN);
+                    if (lane == 0) {
+                        bars->v_fmt[ks] = fp16 ? 0 : 1;
+                        mbar_arrive(&bars->v_ready[ks][gi]);
+                    }
+                    __syncwarp();
+                }
+                ks = (ks + 1 == kKVStages) ? 0 : ks + 1;
+            }
+        }
+    } else if (kFused && warp == kZeroWarp) {
+        // ================================================================ pruned rows
+        // The block's contiguous share of the B*N padded rows: every pruned one becomes zero bytes
+        // (all heads, 16-byte stores along the row), concurrently with the attention work, which
+        // never writes those rows.
+        const int64_t rows = static_cast<int64_t>(B) * p.N;
+        const int64_t share = (rows + gridDim.x - 1) / gridDim.x;
+        const int64_t r0 = static_cast<int64_t>(blockIdx.x) * share;
+        const int64_t r1 = min(rows, r0 + share);
+        const int row_vecs = H * ((p.out_dt == RRA_F32 ? 4 : 2) * kD / 16);
+        for (int64_t t0 = r0; t0 < r1; t0 += 32) {
+            const bool pruned = t0 + lane < r1 && p.mask[t0 + lane] == 0;
+            unsigned bal = __ballot_sync(0xffffffffu, pruned);
+            while (bal != 0u) {
+                const int64_t t = t0 + __ffs(bal) - 1;
+                bal &= bal - 1u;
+                uint4 *y = reinterpret_cast<uint4 *>(p.out) + t * row_vecs;
+                for (int v = lane; v < row_vecs; v += 32)
+                    y[v] = make_uint4(0, 0, 0, 0);
+            }
+        }
     } else if (warp >= kSoftmaxWarp0 && warp < kSoftmaxWarp0 + kSoftmaxWarps) {
         // ================================================================ softmax + epilogue
-        // Group g (4 warps) takes items n = g, g+2, ...; thread r of the group owns row r of
-        // S buffer g and O buffer g (its TMEM lane), so row max and row sum need no exchange.
+        // Group g (4 warps) takes items n = g, g+2, ...; thread r of the group owns row r of the
+        // group's S, P and O (its TMEM lane), so the row max and row sum need no exchange.  Per
+        // chunk: the row max of S; once the previous chunk's PV has completed, O and the row sum
+        // are rescaled if the max rose; then P = exp2(scale log2(e) (s - max)) goes to P, rounded
+        // to the 16-bit type of the chunk's V tile, and its fp32 values are added to the row sum.
         const int q4 = warp & 3;                     // TMEM lane quarter of this warp
         const int g = (warp - kSoftmaxWarp0) >> 2;   // softmax group
-        const int row = q4 * 32 + lane;              // row of S / O owned by this thread
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-        const uint32_t sbase = lane_base + kColS0 + 128 * g;
-        const uint32_t obase = lane_base + kColO0 + kOCols * g;
-        uint32_t s_ph = 0, o_ph = 0, idxf_ph = 0;
+        const int row = q4 * 32 + lane;              // row of S / P / O owned by this thread
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16) + kGroupCols * g;
+        const uint32_t sbase = lane_base + kColS;
+        const uint32_t pbase = lane_base + kColP;
+        const uint32_t obase = lane_base + kColO;
+        uint32_t s_ph = 0, pv_ph = 0, v_ph = 0, idxf_ph = 0;
         bool ok = true;
-        int n = 0;
+        int n = 0, ks = 0;  // ks: K/V ring slot of the item's first chunk
         for (int item = item_first; ok && item < item_end; item += item_step, ++n) {
-            if ((n & 1) != g)
-                continue;
             const Item it = item_at(n, item);
-            const int nkc = (it.L + BN - 1) / BN;
-            const int q0 = it.qt * BM;
-            const int qrows = min(BM, it.L - q0);
+            const int nkc = (it.nk + BN - 1) / BN;
+            if ((n & 1) != g) {
+                ks = (ks + nkc) % kKVStages;
+                continue;
+            }
+            const int qrows = it.nq;
             const bool warp_active = q4 * 32 < qrows;
-            float m_run = -INFINITY;
+            // this row's keys, relative to k0: every kept token of its own image
+            // (rows past the tile's last query row keep the whole range in per-image tiling: their
+            // output is never stored, and whole-slice ranges keep the unmasked path)
+            int klo = 0, khi = it.nk;
+            if (short_tiles) {
+                if (row < qrows) {
+                    const int b = image_of_row(cu_s, it.b0, B, it.q0 + row);
+                    klo = cu_s[b] - it.k0;
+                    khi = cu_s[b + 1] - it.k0;
+                } else {
+                    khi = 0;
+                }
+            }
+            float m_run = -INFINITY, l_run = 0.f;
             for (int kc = 0; kc < nkc; ++kc) {
-                const int nk = min(BN, it.L - kc * BN);
+                const int nk = min(BN, it.nk - kc * BN);
                 const int nk16 = (nk + 15) & ~15;
+                // the row's keys inside this chunk, [lo, hi), and their union over the warp
+                int lo = max(klo - kc * BN, 0), hi = min(khi - kc * BN, nk);
+                if (hi <= lo)
+                    lo = hi = 0;
+                const int wlo = __reduce_min_sync(0xffffffffu, hi > lo ? lo : BN);
+                const int whi = __reduce_max_sync(0xffffffffu, hi);
                 ok = warp_wait(&bars->s_full[g], s_ph, bars, p);
                 if (!ok)
                     break;
                 s_ph ^= 1u;
                 tc_fence_after();
-                // pass 1, row max: two 32-key slices per TMEM round trip (a rolled loop: every
-                // slice runs the same code, which keeps the kernel's instruction footprint small)
+                // pass 1, row max: two 32-key slices per TMEM round trip
                 float m_new = m_run;
                 if (warp_active) {
                     float mx = -INFINITY;
 #pragma unroll 1
-                    for (int c = 0; c < nk; c += 64) {
+                    for (int c = wlo & ~31; c < whi; c += 64) {
                         uint32_t ra[32], rb[32];
                         tmem_ld32(sbase + c, ra);
                         tmem_ld32(sbase + c + 32, rb);  // columns past the chunk are ignored below
                         tmem_wait_ld_dep(ra);
                         tmem_wait_ld_dep(rb);
-                        mx = slice_max(ra, c, nk, mx);
-                        if (c + 32 < nk)
-                            mx = slice_max(rb, c + 32, nk, mx);
+                        const uint32_t ka = key_bits(c, lo, hi), kb = key_bits(c + 32, lo, hi);
+                        mx = slice_max(ra, ka, __all_sync(0xffffffffu, ka == 0xffffffffu), mx);
+                        if (c + 32 < whi)
+                            mx = slice_max(rb, kb, __all_sync(0xffffffffu, kb == 0xffffffffu), mx);
                     }
                     m_new = fmaxf(m_run, mx);
                 }
-                // later chunks: the previous PV has landed in O; rescale rows whose max rose
-                // (before any P of this chunk is handed over, so no PV of it can start earlier)
+                // later chunks: the previous chunk's PV has completed (P is free again and O holds
+                // every earlier chunk); rescale O and the row sum where the running max rose
                 if (kc > 0) {
-                    ok = warp_wait(&bars->o_full[g], o_ph, bars, p);
+                    ok = warp_wait(&bars->pv_done[g], pv_ph, bars, p);
                     if (!ok)
                         break;
-                    o_ph ^= 1u;
+                    pv_ph ^= 1u;
                     tc_fence_after();
                     if (warp_active && __any_sync(0xffffffffu, m_new > m_run)) {
                         const float alpha = ex2_approx((m_run - m_new) * p.scale_log2);
+                        l_run *= alpha;
 #pragma unroll 1
-                        for (uint32_t c = 0; c < kPvN; c += 16) {
+                        for (uint32_t c = 0; c < kD; c += 16) {
                             uint32_t o[16];
                             tmem_ld16(obase + c, o);
                             tmem_wait_ld();
@@ -930,15 +1131,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 m_run = m_new;
                 const float neg_m = -m_new * p.scale_log2;
-                // pass 2: P = exp2(scale*log2e*(s - m)), one 32-key slice per round trip
+                // the chunk's V format (fp16 unless its bf16 tile exceeds fp16's range)
+                const int kslot = (ks + kc) % kKVStages;
+                ok = warp_wait(&bars->v_ready[kslot][g], (v_ph >> kslot) & 1u, bars, p);
+                if (!ok)
+                    break;
+                v_ph ^= 1u << kslot;
+                const bool p_f16 = !kBF16 || bars->v_fmt[kslot] == 0;
+                // pass 2: P = exp2(scale*log2e*(s - m)), one 32-key slice per round trip, 16 P
+                // columns per slice; slices outside the warp's keys get P = 0 without being read
                 if (warp_active) {
+                    float lsum = 0.f;
 #pragma unroll 1
                     for (int c = 0; c < nk16; c += 32) {
+                        if (c + 32 <= wlo || c >= whi) {
+                            zero_p16(pbase + (c >> 1));
+                            continue;
+                        }
                         uint32_t ra[32];
                         tmem_ld32(sbase + c, ra);
                         tmem_wait_ld_dep(ra);
-                        softmax_slice<kBF16>(ra, c, nk, p.scale_log2, neg_m, sbase + c);
+                        const uint32_t kk = key_bits(c, lo, hi);
+                        lsum += softmax_slice(ra, kk, __all_sync(0xffffffffu, kk == 0xffffffffu), p_f16, p.scale_log2,
+                                              neg_m, pbase + (c >> 1));
                     }
+                    l_run += lsum;
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -948,11 +1165,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok)
                 break;
-            // epilogue: the last PV has landed; normalise by the row sum (O column 64) and store
-            ok = warp_wait(&bars->o_full[g], o_ph, bars, p);
+            ks = (ks + nkc) % kKVStages;
+            // epilogue: the last PV has completed; normalise by the row sum and store
+            ok = warp_wait(&bars->pv_done[g], pv_ph, bars, p);
             if (!ok)
                 break;
-            o_ph ^= 1u;
+            pv_ph ^= 1u;
             const int islot = n & (kIdxSlots - 1);
             if constexpr (kFused) {
                 ok = warp_wait(&bars->idx_full[islot], (idxf_ph >> islot) & 1u, bars, p);
@@ -962,13 +1180,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             if (warp_active) {
-                uint32_t sum[1];
-                tmem_ld1(obase + 64, sum);
-                tmem_wait_ld();
-                const float inv = 1.f / __uint_as_float(sum[0]);
-                int64_t out_row = static_cast<int64_t>(it.seq0) + q0 + row;
-                if constexpr (kFused)
-                    out_row = static_cast<int64_t>(it.b) * p.N + idx_list(islot)[q0 + (row < qrows ? row : 0)];
+                const float inv = 1.f / l_run;
+                int64_t out_row = static_cast<int64_t>(it.q0) + row;
+                if constexpr (kFused)  // the padded row of this packed row
+                    out_row = idx_list(islot)[it.q0 - it.k0 + (row < qrows ? row : 0)];
                 const int64_t off = (out_row * H + it.h) * kD;
 #pragma unroll 1
                 for (int h2 = 0; h2 < 2; ++h2) {
@@ -984,19 +1199,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0)
                 mbar_arrive(&bars->o_free[g]);
             if constexpr (kFused) {
-                if (it.qt == 0) {
-                    // pruned rows of this (image, head) in the padded output become zero: 16-byte
-                    // stores, consecutive threads along a row
-                    const uint32_t *bits = idx_bits(islot);
-                    const int lg = p.out_dt == RRA_F32 ? 4 : 3;  // log2 of 16-byte vectors per head row
-                    const int nvec = p.N << lg;
-                    for (int i = q4 * 32 + lane; i < nvec; i += kGroupWarps * 32) {
-                        const int tok = i >> lg;
-                        if (!((bits[tok >> 5] >> (tok & 31)) & 1u))
-                            reinterpret_cast<uint4 *>(p.out)[(((static_cast<int64_t>(it.b) * p.N + tok) * H + it.h) << lg) +
-                                                             (i & ((1 << lg) - 1))] = make_uint4(0, 0, 0, 0);
-                    }
-                }
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&bars->idx_free[islot]);
@@ -1101,6 +1303,7 @@ cudaError_t launch_attend(const AttendArgs &a, int num_sms, cudaStream_t stream)
         return cudaErrorInvalidValue;
     Params p{};
     p.cu = a.cu;
+    p.src[2] = static_cast<const uint8_t *>(a.v);  // read back only to restore a bf16 V tile
     p.out = a.o;
     p.B = a.B;
     p.H = a.H;
@@ -1121,7 +1324,11 @@ cudaError_t launch_fused(const FusedArgs &a, int num_sms, cudaStream_t stream)
         return cudaSuccess;
     }
     const int64_t rows = static_cast<int64_t>(a.B) * a.N;
-    alignas(64) CUtensorMap unused{};  // the single-launch path copies with cp.async, not TMA
+    // the padded tensors seen as [B*N, H, 64]: the TMA box of a tile whose kept rows are consecutive
+    alignas(64) CUtensorMap tq, tk, tv;
+    if (!make_tmap(&tq, a.q, rows, a.H, a.in_bf16) || !make_tmap(&tk, a.k, rows, a.H, a.in_bf16) ||
+        !make_tmap(&tv, a.v, rows, a.H, a.in_bf16))
+        return cudaErrorInvalidValue;
     Params p{};
     p.src[0] = static_cast<const uint8_t *>(a.q);
     p.src[1] = static_cast<const uint8_t *>(a.k);
@@ -1138,7 +1345,7 @@ cudaError_t launch_fused(const FusedArgs &a, int num_sms, cudaStream_t stream)
     p.err = a.err;
     p.wait_ns = a.wait_ns;
     const int smem = smem_bytes<true>(a.B);
-    return launch_variant<true>(a.in_bf16, unused, unused, unused, p, grid_for(a.B, a.H, a.N, num_sms), smem, stream);
+    return launch_variant<true>(a.in_bf16, tq, tk, tv, p, grid_for(a.B, a.H, a.N, num_sms), smem, stream);
 }
 
 }  // namespace rra

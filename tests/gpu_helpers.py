@@ -110,3 +110,28 @@ def compare_attention(gpu_o: torch.Tensor, oracle_o: np.ndarray, out_dtype: torc
     tol = tolerance(oracle_o, out_dtype)
     bad = err > tol
     return float(err.max()) if err.size else 0.0, int(bad.sum()), np.isfinite(g).all()
+
+
+def oracle_attention_threaded(w, stage: int = 0, threads: int | None = None) -> tuple[np.ndarray, np.ndarray]:
+    """The oracle's float64 attention over every kept row of one stage, one image per task on a
+    thread pool (the oracle's C calls release the GIL), reassembled in packed order: (O [T, H, d],
+    cu_seqlens)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    mask = w.masks[stage]
+    cu = O.cu_seqlens(mask)
+    T = int(cu[-1])
+    out = np.zeros((T, w.H, 64), dtype=np.float64)
+
+    def one(b):
+        m = mask[b:b + 1]
+        qp, c = O.pack(m, w.q[b:b + 1])
+        kp, _ = O.pack(m, w.k[b:b + 1])
+        vp, _ = O.pack(m, w.v[b:b + 1])
+        out[cu[b]:cu[b + 1]] = O.attend(qp, kp, vp, c, w.H, 64, dtype=w.dtype)
+
+    n = threads or max(1, len(os.sched_getaffinity(0)))
+    with ThreadPoolExecutor(max_workers=n) as ex:
+        list(ex.map(one, range(w.B)))
+    return out, cu

@@ -308,3 +308,71 @@ def test_pack_single_tensor_and_f32():
     T = int(cu[-1])
     assert np.array_equal(dcu.cpu().numpy(), cu)
     assert np.array_equal(out[:T].cpu().numpy().view(np.uint32), want[:T].view(np.uint32))
+
+
+@pytest.mark.parametrize("name", ["c4", "c5:1.0:64", "c2"])
+def test_full_size_every_row(name):
+    """Full-size workloads compared with the float64 oracle on EVERY kept row and head (the oracle
+    runs one image per thread), both output types; the single launch is byte-identical to the
+    three calls."""
+    from gpu_helpers import oracle_attention_threaded
+    w = W.by_name(name)
+    want, cu = oracle_attention_threaded(w)
+    T = int(cu[-1])
+    for od in (torch.float32, None):
+        g = GpuRun(w, out_dtype=od).run()
+        assert g.error() == 0
+        assert np.array_equal(g.cu[:-1].cpu().numpy(), cu)
+        err, nbad, finite = compare_attention(g.o[:T], want, g.out_dtype)
+        assert finite and nbad == 0, err
+        if od == torch.float32:
+            assert err <= ATOL
+        y = torch.empty_like(g.y)
+        rra.rra_pack_attend_unpack(g.mask, g.q, g.k, g.v, y)
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.uint8), g.y.view(torch.uint8))
+
+
+@pytest.mark.parametrize("B", [1024, 1025, 3000])
+def test_large_batch_pack_and_path(B):
+    """From 1025 images on, rra_pack writes cu_seqlens in a separate one-block launch and the
+    gather blocks read their image start from it: bit-exact either side of the switch, with the
+    whole path checked against the oracle."""
+    rng = np.random.default_rng(B)
+    lengths = rng.integers(0, 34, size=B)
+    w = W.from_lengths(lengths.tolist(), 33, 1, seed=B)
+    assert check_full(w, out_dtype=torch.float32) <= ATOL
+
+
+@pytest.mark.parametrize("bad", [70000.0, float("inf")])
+@pytest.mark.parametrize("fused", [False, True])
+def test_v_tile_beyond_fp16_range(bad, fused):
+    """A V tile holding a value beyond fp16's range (or an infinity) is not converted to fp16: it is
+    restored to its bf16 bytes and meets a bf16 P.  That (image, head) keeps bf16-P precision
+    (relative 2^-9 of the largest |v| it attends); every other one keeps the usual tolerance, and
+    non-finite outputs sit exactly where the oracle's are."""
+    lengths = [150, 100, 197, 130]  # one image per tile: the fallback stays inside its image
+    w = W.from_lengths(lengths, 197, 2, seed=31)
+    b, h = 2, 1
+    kept = np.nonzero(w.masks[0][b].numpy())[0]
+    w.v[b, kept[57], h, 5] = bad  # in the first 128-key chunk of image 2, head 1
+    ref = oracle_stage(w)
+    T, cu = ref["T"], ref["cu"]
+    if fused:
+        y = torch.empty(w.B, w.N, w.H, 64, dtype=torch.float32, device="cuda")
+        rra.rra_pack_attend_unpack(w.masks[0].cuda(), w.q.cuda(), w.k.cuda(), w.v.cuda(), y)
+        torch.cuda.synchronize()
+        got = y.cpu()[w.masks[0].bool()].double().numpy()
+    else:
+        g = GpuRun(w, out_dtype=torch.float32).run()
+        assert g.error() == 0
+        got = g.o[:T].cpu().double().numpy()
+    want = ref["o"]
+    assert np.array_equal(np.isfinite(got), np.isfinite(want))
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    fin = np.isfinite(want)
+    tol = np.full(want.shape, ATOL)
+    vb = w.v[b][w.masks[0][b].bool(), h].double().abs()
+    vmax = float(torch.where(torch.isfinite(vb), vb, torch.zeros_like(vb)).max())
+    tol[cu[b]:cu[b + 1], h] = ATOL + 2.0 ** -8 * vmax
+    assert np.all(np.abs(got[fin] - want[fin]) <= tol[fin])

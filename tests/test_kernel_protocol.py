@@ -1,16 +1,21 @@
 """A model check of the attention kernel's whole synchronisation protocol (CPU only).
 
 Every role of one block is an actor: the list builder (single-launch path), the producer (Q tile
-and K/V chunk fills), the two tensor-core issuers and the two softmax groups.  Copies and MMAs
-complete asynchronously, in issue order per issuer, through a hardware actor.  Every barrier of
+and K/V chunk fills), the two tensor-core issuers, the two softmax groups and the two V-tile
+warps.  Copies and MMAs complete asynchronously through a hardware actor: MMAs in issue order per
+issuer, copies in issue order per ring slot (fills of different slots may land in any order).  Every barrier of
 the kernel is modelled with mbarrier parity semantics: a waiter keeps one phase bit per barrier,
 exactly as the kernel does, and a wait passes when the barrier's phase parity differs from it.
 Besides that, the model tracks which phase each wait is *meant* to see, and fails when a wait
-passes before that phase completed, or when a schedule can make no progress.
+passes before that phase completed, or when a schedule can make no progress.  It also tracks who
+owns each group's TMEM buffers -- S (written by Q K^T, read by the softmax), P (written by the
+softmax, read by the PV MMA) and O (accumulated by PV, rescaled and read out by the softmax) --
+and fails when a writer or reader touches a buffer another role still owns.
 
 The roles' orders of waits and arrivals restate the kernel's (csrc/attend.cu): item n belongs to
 softmax group n % 2 and uses Q slot n % 2 and kept-row list slot n % 4; K/V chunks go round a
-3-slot ring in production order, with one "full" barrier per slot and group.
+4-slot ring in production order, with one "full" barrier per slot and group (the 3-slot ring of an
+earlier design is checked too).
 """
 import random
 
@@ -27,8 +32,13 @@ class Bar:
 
 
 class Model:
-    def __init__(self, nkc, fused, rng):
+    def __init__(self, nkc, fused, rng, early_qk=False, shared_v_ready=False, v_skip=False, stages=4):
         self.nkc, self.fused, self.rng = nkc, fused, rng
+        self.stages = stages  # K/V ring slots (the kernel's kKVStages)
+        self.early_qk = early_qk  # planted mistake: the next S = Q K^T before the softmax released S
+        self.shared_v_ready = shared_v_ready  # planted mistake: one V-ready barrier per group
+        self.v_skip = v_skip  # planted mistake: a V warp waits only for the fills it prepares
+        self.v_fill = {}  # fill -> "landed" / "ready" (what the V warps may rely on)
         self.items = len(nkc)
         B = {}
 
@@ -38,13 +48,23 @@ class Model:
 
         self.q_full = [bar(f"q_full{s}") for s in range(2)]
         self.q_empty = [bar(f"q_empty{s}") for s in range(2)]
-        self.kv_full = [[bar(f"kv_full{s}.{g}") for g in range(2)] for s in range(3)]
-        self.kv_empty = [bar(f"kv_empty{s}") for s in range(3)]
+        self.kv_full = [[bar(f"kv_full{s}.{g}") for g in range(2)] for s in range(stages)]
+        self.kv_empty = [bar(f"kv_empty{s}") for s in range(stages)]
         self.s_full = [bar(f"s_full{g}") for g in range(2)]
         self.p_full = [bar(f"p_full{g}") for g in range(2)]
-        self.s_free = [bar(f"s_free{g}") for g in range(2)]
-        self.o_full = [bar(f"o_full{g}") for g in range(2)]
+        self.pv_done = [bar(f"pv_done{g}") for g in range(2)]
+        self.v_ready = [[bar(f"v_ready{s}.{g}") for g in range(2)] for s in range(stages)]
+        if shared_v_ready:
+            one = [bar("v_ready0"), bar("v_ready1")]
+            self.v_ready = [[one[0], one[1]] for _ in range(stages)]
         self.o_free = [bar(f"o_free{g}") for g in range(2)]
+        # buffer ownership per group: S "free" / "qk" (MMA writing) / "softmax"; P "free" /
+        # "softmax" (written) / "pv" (MMA reading); O: PVs in flight, and whether the epilogue holds it
+        self.S = ["free", "free"]
+        self.P = ["free", "free"]
+        self.pv_flight = [0, 0]
+        self.o_reading = [False, False]
+        self.error = None
         self.idx_full = [bar(f"idx_full{s}") for s in range(4)]
         self.idx_free = [bar(f"idx_free{s}") for s in range(4)]
         self.hw = []  # pending asynchronous completions: (source, barrier, check) in issue order
@@ -53,10 +73,10 @@ class Model:
         t = 0
         for n, k in enumerate(nkc):
             for c in range(k):
-                self.slot[(n, c)] = t % 3
+                self.slot[(n, c)] = t % stages
                 t += 1
         self.actors = [self.list_builder(), self.producer(), self.issuer(0), self.issuer(1),
-                       self.softmax(0), self.softmax(1)]
+                       self.softmax(0), self.softmax(1), self.v_warp(0), self.v_warp(1)]
         self.finished = [False] * len(self.actors)
 
     # -- helpers: a generator yields ("wait", barrier, bit, expected_phase) or ("step",)
@@ -64,8 +84,12 @@ class Model:
         """Wait for completed phase `phase` (0-based) of `bar` with the waiter's parity `bit`."""
         return ("wait", bar, bit, phase)
 
-    def complete_async(self, source, bar):
-        self.hw.append((source, bar))
+    def complete_async(self, source, bar, effect=None):
+        self.hw.append((source, bar, effect))
+
+    def check(self, cond, what):
+        if not cond and self.error is None:
+            self.error = what
 
     def list_builder(self):
         if not self.fused:
@@ -82,7 +106,7 @@ class Model:
     def producer(self):
         qb = kb = fb = 0
         qfill = [0, 0]
-        kvfill = [0, 0, 0]
+        kvfill = [0] * self.stages
         for n in range(self.items):
             g = n % 2
             if self.fused:
@@ -94,23 +118,81 @@ class Model:
                 yield self.wait(self.q_empty[qs], ((qb >> qs) & 1) ^ 1, qfill[qs] - 1)
             qb ^= 1 << qs
             qfill[qs] += 1
-            self.complete_async("copy", self.q_full[qs])
+            self.complete_async(f"copy_q{qs}", self.q_full[qs], None)
             for c in range(self.nkc[n]):
                 s = self.slot[(n, c)]
                 if kvfill[s] >= 1:
                     yield self.wait(self.kv_empty[s], ((kb >> s) & 1) ^ 1, kvfill[s] - 1)
                 kb ^= 1 << s
                 kvfill[s] += 1
-                self.complete_async("copy", self.kv_full[s][g])
+                # bulk copies into different slots may land in any order
+                self.complete_async(f"copy_kv{s}", self.kv_full[s][g], None)
             yield ("step",)
 
+    def v_warp(self, vw):
+        """V warp vw (of two): waits for every fill in production order as soon as it has landed,
+        and prepares fills vw, vw + 2, ... (the kernel's split)."""
+        kb = 0
+        seen = {}  # fills of kv_full[s][g] seen so far
+        fill = 0
+        for n in range(self.items):
+            g = n % 2
+            for c in range(self.nkc[n]):
+                s = self.slot[(n, c)]
+                k = seen.get((s, g), 0)
+                mine = fill % 2 == vw
+                if mine or not self.v_skip:
+                    yield self.wait(self.kv_full[s][g], (kb >> (2 * s + g)) & 1, k)
+                kb ^= 1 << (2 * s + g)
+                seen[(s, g)] = k + 1
+                if mine:
+                    yield ("step",)
+                    self.v_ready[s][g].done += 1
+                fill += 1
+
+    def v_wait(self, g, s, bits, seen):
+        """A group's wait for the V tile of its next chunk in slot s (per-slot parity bits)."""
+        if self.shared_v_ready:
+            k = sum(seen.values())
+            b = bits.get("all", 0)
+            bits["all"] = b ^ 1
+        else:
+            k = seen.get(s, 0)
+            b = bits.get(s, 0)
+            bits[s] = b ^ 1
+        seen[s] = seen.get(s, 0) + 1
+        return self.wait(self.v_ready[s][g], b, k)
+
     def issuer(self, g):
-        qb = kb = pb = sb = ob = 0
-        own_kv = [0, 0, 0]  # fills of kv_full[s][g] seen so far
+        qb = kb = pb = ob = 0
+        vbits, vseen = {}, {}
+        own_kv = [0] * self.stages  # fills of kv_full[s][g] seen so far
         qseen = 0
-        s_busy = False
-        pv_done = 0
+        p_seen = 0
         items_done = 0
+
+        def qk(qs, last):
+            self.check(self.S[g] == "free", f"QK into S{g} while {self.S[g]} owns it")
+            self.S[g] = "qk"
+
+            def done():
+                self.S[g] = "softmax"
+            self.complete_async(f"mma{g}", self.s_full[g], done)
+            if last:
+                self.complete_async(f"mma{g}", self.q_empty[qs], None)
+
+        def pv(s):
+            self.check(self.P[g] == "softmax", f"PV reads P{g} in state {self.P[g]}")
+            self.check(not self.o_reading[g], f"PV into O{g} while the epilogue reads it")
+            self.P[g] = "pv"
+            self.pv_flight[g] += 1
+
+            def done():
+                self.P[g] = "free"
+                self.pv_flight[g] -= 1
+            self.complete_async(f"mma{g}", self.pv_done[g], done)
+            self.complete_async(f"mma{g}", self.kv_empty[s], None)
+
         for n in range(self.items):
             if n % 2 != g:
                 continue
@@ -118,32 +200,39 @@ class Model:
             yield self.wait(self.q_full[qs], (qb >> qs) & 1, qseen)
             qb ^= 1 << qs
             qseen += 1
+            s0 = self.slot[(n, 0)]
+            yield self.wait(self.kv_full[s0][g], (kb >> s0) & 1, own_kv[s0])
+            kb ^= 1 << s0
+            own_kv[s0] += 1
+            qk(qs, self.nkc[n] == 1)
             for c in range(self.nkc[n]):
                 s = self.slot[(n, c)]
-                yield self.wait(self.kv_full[s][g], (kb >> s) & 1, own_kv[s])
-                kb ^= 1 << s
-                own_kv[s] += 1
-                if s_busy:
-                    yield self.wait(self.s_free[g], sb, pv_done - 1)
-                    sb ^= 1
-                self.complete_async(f"mma{g}", self.s_full[g])
-                if c == self.nkc[n] - 1:
-                    self.complete_async(f"mma{g}", self.q_empty[qs])
-                yield self.wait(self.p_full[g], pb, pv_done)
+                if self.early_qk and c + 1 < self.nkc[n]:
+                    sn = self.slot[(n, c + 1)]
+                    yield self.wait(self.kv_full[sn][g], (kb >> sn) & 1, own_kv[sn])
+                    kb ^= 1 << sn
+                    own_kv[sn] += 1
+                    qk(qs, c + 1 == self.nkc[n] - 1)
+                yield self.wait(self.p_full[g], pb, p_seen)
                 pb ^= 1
+                p_seen += 1
+                if c + 1 < self.nkc[n] and not self.early_qk:
+                    sn = self.slot[(n, c + 1)]
+                    yield self.wait(self.kv_full[sn][g], (kb >> sn) & 1, own_kv[sn])
+                    kb ^= 1 << sn
+                    own_kv[sn] += 1
+                    qk(qs, c + 1 == self.nkc[n] - 1)
                 if c == 0 and items_done >= 1:
                     yield self.wait(self.o_free[g], ob, items_done - 1)
                     ob ^= 1
-                self.complete_async(f"mma{g}", self.o_full[g])
-                self.complete_async(f"mma{g}", self.s_free[g])
-                self.complete_async(f"mma{g}", self.kv_empty[s])
-                pv_done += 1
-                s_busy = True
+                yield self.v_wait(g, s, vbits, vseen)
+                pv(s)
             items_done += 1
 
     def softmax(self, g):
-        sb = ob = fb = 0
-        s_seen = o_seen = 0
+        sb = pvb = fb = 0
+        s_seen = pv_seen = 0
+        vbits, vseen = {}, {}
         for n in range(self.items):
             if n % 2 != g:
                 continue
@@ -151,20 +240,30 @@ class Model:
                 yield self.wait(self.s_full[g], sb, s_seen)
                 sb ^= 1
                 s_seen += 1
+                self.check(self.S[g] == "softmax", f"softmax reads S{g} in state {self.S[g]}")
                 if c > 0:
-                    yield self.wait(self.o_full[g], ob, o_seen)
-                    ob ^= 1
-                    o_seen += 1
+                    yield self.wait(self.pv_done[g], pvb, pv_seen)
+                    pvb ^= 1
+                    pv_seen += 1
+                    self.check(self.pv_flight[g] == 0, f"O{g} rescaled while a PV is in flight")
+                yield self.v_wait(g, self.slot[(n, c)], vbits, vseen)
+                self.check(self.P[g] == "free", f"softmax writes P{g} in state {self.P[g]}")
                 yield ("step",)
+                self.check(self.S[g] == "softmax", f"S{g} overwritten during the softmax")
+                self.S[g] = "free"
+                self.P[g] = "softmax"
                 self.p_full[g].done += 1
-            yield self.wait(self.o_full[g], ob, o_seen)
-            ob ^= 1
-            o_seen += 1
+            yield self.wait(self.pv_done[g], pvb, pv_seen)
+            pvb ^= 1
+            pv_seen += 1
+            self.check(self.pv_flight[g] == 0, f"O{g} read out while a PV is in flight")
             if self.fused:
                 s = n % 4
                 yield self.wait(self.idx_full[s], (fb >> s) & 1, n // 4)
                 fb ^= 1 << s
+            self.o_reading[g] = True
             yield ("step",)
+            self.o_reading[g] = False
             self.o_free[g].done += 1
             if self.fused:
                 self.idx_free[n % 4].done += 1
@@ -179,8 +278,10 @@ class Model:
                 w = pending[i]
                 if w is None or w[1].passes(w[2]):
                     choices.append(("actor", i))
+            if self.error is not None:
+                return f"hazard:{self.error}"
             sources = []
-            for src, _ in self.hw:
+            for src, _, _ in self.hw:
                 if src not in sources:
                     sources.append(src)
             choices += [("hw", src) for src in sources]
@@ -188,8 +289,10 @@ class Model:
                 return "ok" if all(self.finished) and not self.hw else "stuck"
             kind, who = self.rng.choice(choices)
             if kind == "hw":
-                k = next(j for j, (src, _) in enumerate(self.hw) if src == who)  # in order per source
-                _, bar = self.hw.pop(k)
+                k = next(j for j, (src, _, _) in enumerate(self.hw) if src == who)  # in order per source
+                _, bar, effect = self.hw.pop(k)
+                if effect is not None:
+                    effect()
                 bar.done += 1
                 continue
             w = pending[who]
@@ -203,7 +306,7 @@ class Model:
                 continue
             if nxt[0] == "wait":
                 pending[who] = nxt
-        return "stuck"
+        return "stuck" if self.error is None else f"hazard:{self.error}"
 
 
 def random_cases(count, seed):
@@ -213,11 +316,12 @@ def random_cases(count, seed):
         yield nkc, random.Random(rng.random())
 
 
+@pytest.mark.parametrize("stages", [4, 3])
 @pytest.mark.parametrize("fused", [False, True])
-def test_protocol_never_passes_early_or_hangs(fused):
+def test_protocol_never_passes_early_or_hangs(fused, stages):
     bad = []
     for nkc, rng in random_cases(1500, 7 + fused):
-        out = Model(nkc, fused, rng).run()
+        out = Model(nkc, fused, rng, stages=stages).run()
         if out != "ok":
             bad.append((nkc, out))
     assert not bad, bad[:5]
@@ -229,9 +333,44 @@ def test_model_sees_a_shared_kv_barrier_fail():
     bad = 0
     for nkc, rng in random_cases(1500, 11):
         m = Model(nkc, False, rng)
-        shared = [Bar(f"kv_full{s}") for s in range(3)]
-        m.kv_full = [[shared[s], shared[s]] for s in range(3)]
-        m.actors = [m.list_builder(), m.producer(), m.issuer(0), m.issuer(1), m.softmax(0), m.softmax(1)]
+        shared = [Bar(f"kv_full{s}") for s in range(m.stages)]
+        m.kv_full = [[shared[s], shared[s]] for s in range(m.stages)]
+        m.actors = [m.list_builder(), m.producer(), m.issuer(0), m.issuer(1), m.softmax(0), m.softmax(1), m.v_warp(0),
+                    m.v_warp(1)]
+        m.finished = [False] * len(m.actors)
         if m.run() != "ok":
+            bad += 1
+    assert bad > 0
+
+
+def test_model_sees_an_early_qk_fail():
+    """Issuing the next chunk's S = Q K^T before the softmax has released S (p_full) is caught as a
+    buffer hazard in some schedule: the ownership checks have teeth."""
+    bad = 0
+    for nkc, rng in random_cases(800, 13):
+        if max(nkc) < 2:
+            continue
+        if Model(nkc, False, rng, early_qk=True).run() != "ok":
+            bad += 1
+    assert bad > 0
+
+
+def test_model_sees_a_shared_v_ready_fail():
+    """With one V-ready barrier per group (the V warp may prepare two of a group's chunks before
+    that group waits for the first), some schedule sees a phase early or hangs."""
+    bad = 0
+    for nkc, rng in random_cases(800, 17):
+        if Model(nkc, False, rng, shared_v_ready=True).run() != "ok":
+            bad += 1
+    assert bad > 0
+
+
+def test_model_sees_v_warps_skipping_fills_fail():
+    """If each V warp waited only for the fills it prepares, a parity wait could pass on the fill
+    before (still in flight) and some schedule fails: the V warps wait for every fill.  (With the
+    4-slot ring a slot's fills all fall to one V warp, so the mistake shows with a 3-slot ring.)"""
+    bad = 0
+    for nkc, rng in random_cases(800, 19):
+        if Model(nkc, False, rng, v_skip=True, stages=3).run() != "ok":
             bad += 1
     assert bad > 0
