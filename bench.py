@@ -50,6 +50,10 @@ from ragged_varlen_attention_rra_b200 import rra, workloads  # noqa: E402
 METRIC = "packed tokens/s & us per pack-attend-unpack call (1 B200, graph); % roofline"
 UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+# ex2 results per clock per SM of the special-function unit (the documented throughput of the base-2
+# exponential on this architecture; the attention kernel's XU-pipe utilisation under ncu agrees with it)
+EX2_PER_CLK_PER_SM = 16
 L2_FLUSH_BYTES = 256 << 20
 KERNELS = {"three": ("pack", "attend", "unpack"), "fused": ("pack_attend_unpack",)}
 KERNEL_SOURCES = {
@@ -91,6 +95,25 @@ def peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Dense bf16 TFLOP/s: the measured burst figure (a kernel timed alone), else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def attention_bounds_us(bytes_, flops, exps, hbm_gbs, sm_mhz, num_sms):
+    """Lower bounds (us) on one attention launch from each resource: HBM bytes, tensor-core FLOPs
+    at the bf16 peak, and exponentials at the special-function unit's rate."""
+    tf, _ = tensor_peak()
+    ex2_rate = EX2_PER_CLK_PER_SM * num_sms * sm_mhz * 1e6
+    return {"hbm": bytes_ / (hbm_gbs * 1e3), "tensor": flops / (tf * 1e6), "exp": exps / ex2_rate * 1e6}
 
 
 def source_hash(rel):
@@ -632,14 +655,23 @@ def main_gpu(args):
     per_kernel = kernel_table(kern_ms, alg, stages, hbm_peak)
     other_kernels = kernel_table(o_kern_ms, alg, stages, hbm_peak)
     roofline = None
+    flops = attention_flops([(w.H, l) for l in lengths])
+    exps = sum(w.H * int((l.astype(np.int64) ** 2).sum()) for l in lengths)
     if per_kernel:
         dom = max(per_kernel, key=lambda k: per_kernel[k]["us_per_launch"])
         ach = per_kernel[dom]["gbs"]
+        clk_summary = clk.summary()
+        sm_mhz = clk_summary["sm_mhz"] or clk_summary["sm_max_mhz"] or 1965
+        bounds = None
+        if dom in ("attend", "pack_attend_unpack"):
+            bounds = attention_bounds_us(per_kernel[dom]["alg_bytes_per_launch"], flops / stages, exps / stages,
+                                         hbm_peak, sm_mhz, torch.cuda.get_device_properties(dev_index).multi_processor_count)
         roofline = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
                     "frac": ach / hbm_peak, "peak_source": peak_kind, "traffic": ncu_traffic(dom, w.name),
                     "alg_bytes_per_launch": per_kernel[dom]["alg_bytes_per_launch"],
-                    "us_per_launch": per_kernel[dom]["us_per_launch"]}
-    flops = attention_flops([(w.H, l) for l in lengths])
+                    "us_per_launch": per_kernel[dom]["us_per_launch"],
+                    "lower_bounds_us": bounds,
+                    "exps_per_launch": exps / stages, "flops_per_launch": flops / stages}
     attn_key = "pack_attend_unpack" if args.path == "fused" else "attend"
     attn_tflops = (flops / (per_kernel[attn_key]["us_per_launch"] * stages * 1e-6) / 1e12) if per_kernel else None
 
