@@ -976,33 +976,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp >= kVWarp0 && warp < kVWarp0 + kVWarps) {
         // ================================================================ V tiles
-        // The K/V fills in production order, V warp v preparing fills v, v + 2, ..., each as soon
-        // as it has landed: zero the V rows past the chunk's keys and, for bf16 inputs, convert the
-        // tile to fp16 in place when it fits; then record the slot's format and tell the owning
-        // group (its issuer before the PV, its softmax before writing P).  A slot is refilled only
-        // after that chunk's PV, which follows these reads of v_fmt.
+        // V warp v owns the K/V ring slots s = v (mod 2): it waits for every fill of those slots in
+        // production order and prepares each as soon as it has landed -- zero the V rows past the
+        // chunk's keys and, for bf16 inputs, convert the tile to fp16 in place when it fits -- then
+        // records the slot's format and tells the owning group (its issuer before the PV, its
+        // softmax before writing P).  A slot is refilled only after that chunk's PV, which follows
+        // this warp's v_ready, so no fill of its slots can land before it has looked at the last
+        // one (a warp that also watched slots another warp prepares could be lapped there).
+        static_assert(kKVStages % kVWarps == 0, "each V warp owns whole ring slots");
         const int vw = warp - kVWarp0;
         uint32_t kv_ph = 0;  // bit 2*slot + group: parity of kv_full[slot][group] waits
-        int ks = 0, n = 0, fill = 0;
+        int ks = 0, n = 0;
         bool ok = true;
         for (int item = item_first; ok && item < item_end; item += item_step, ++n) {
             const Item it = item_at(n, item);
             const int nkc = (it.nk + BN - 1) / BN;
             const int gi = n & 1;
-            for (int kc = 0; kc < nkc; ++kc, ++fill) {
-                // every V warp waits for every fill in order (so that no parity wait can run a phase
-                // ahead of a fill still in flight), and prepares only its own
-                const uint32_t bit = 1u << (2 * ks + gi);
-                ok = warp_wait(&bars->kv_full[ks][gi], (kv_ph & bit) ? 1u : 0u, bars, p);
-                if (!ok)
-                    break;
-                kv_ph ^= bit;
-                if (fill % kVWarps == vw) {
+            for (int kc = 0; kc < nkc; ++kc) {
+                if (ks % kVWarps == vw) {
+                    const uint32_t bit = 1u << (2 * ks + gi);
+                    ok = warp_wait(&bars->kv_full[ks][gi], (kv_ph & bit) ? 1u : 0u, bars, p);
+                    if (!ok)
+                        break;
+                    kv_ph ^= bit;
                     // where the tile's rows came from, should it have to be restored as bf16
                     const uint8_t *vsrc = p.src[2] + static_cast<int64_t>(it.h) * kD * 2;
                     const int32_t *rows = kFused ? idx_list(n & (kIdxSlots - 1)) : nullptr;
-                    const bool fp16 = prepare_v<kBF16>(base + kOffV + ks * kTileBytes, min(BN, it.nk - kc * BN),
-                                                       lane, vsrc, static_cast<int64_t>(H) * kD * 2, rows, kc * BN,
+                    const bool fp16 = prepare_v<kBF16>(base + kOffV + ks * kTileBytes, min(BN, it.nk - kc * BN), lane,
+                                                       vsrc, static_cast<int64_t>(H) * kD * 2, rows, kc * BN,
                                                        static_cast<int64_t>(it.k0) + kc * BN);
                     if (lane == 0) {
                         bars->v_fmt[ks] = fp16 ? 0 : 1;

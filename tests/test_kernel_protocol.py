@@ -32,12 +32,16 @@ class Bar:
 
 
 class Model:
-    def __init__(self, nkc, fused, rng, early_qk=False, shared_v_ready=False, v_skip=False, stages=4):
+    def __init__(self, nkc, fused, rng, early_qk=False, shared_v_ready=False, v_mode="slot", stages=4, starve=()):
         self.nkc, self.fused, self.rng = nkc, fused, rng
         self.stages = stages  # K/V ring slots (the kernel's kKVStages)
         self.early_qk = early_qk  # planted mistake: the next S = Q K^T before the softmax released S
         self.shared_v_ready = shared_v_ready  # planted mistake: one V-ready barrier per group
-        self.v_skip = v_skip  # planted mistake: a V warp waits only for the fills it prepares
+        # V warps: "slot" -- warp w owns ring slots s = w (mod 2), waits for and prepares every fill of
+        # them (the kernel); planted mistakes: "observe_all" -- warp w prepares fills w, w + 2, ... and
+        # waits for every fill; "alt_skip" -- it prepares fills w, w + 2, ... and waits only for those
+        self.v_mode = v_mode
+        self.starve = set(starve)  # actors scheduled only when nothing else can move
         self.v_fill = {}  # fill -> "landed" / "ready" (what the V warps may rely on)
         self.items = len(nkc)
         B = {}
@@ -130,8 +134,7 @@ class Model:
             yield ("step",)
 
     def v_warp(self, vw):
-        """V warp vw (of two): waits for every fill in production order as soon as it has landed,
-        and prepares fills vw, vw + 2, ... (the kernel's split)."""
+        """V warp vw (of two), in production order, as each fill lands (see v_mode)."""
         kb = 0
         seen = {}  # fills of kv_full[s][g] seen so far
         fill = 0
@@ -140,8 +143,12 @@ class Model:
             for c in range(self.nkc[n]):
                 s = self.slot[(n, c)]
                 k = seen.get((s, g), 0)
-                mine = fill % 2 == vw
-                if mine or not self.v_skip:
+                if self.v_mode == "slot":
+                    mine = watch = s % 2 == vw
+                else:
+                    mine = fill % 2 == vw
+                    watch = mine or self.v_mode == "observe_all"
+                if watch:
                     yield self.wait(self.kv_full[s][g], (kb >> (2 * s + g)) & 1, k)
                 kb ^= 1 << (2 * s + g)
                 seen[(s, g)] = k + 1
@@ -287,7 +294,8 @@ class Model:
             choices += [("hw", src) for src in sources]
             if not choices:
                 return "ok" if all(self.finished) and not self.hw else "stuck"
-            kind, who = self.rng.choice(choices)
+            preferred = [c for c in choices if not (c[0] == "actor" and c[1] in self.starve)]
+            kind, who = self.rng.choice(preferred or choices)
             if kind == "hw":
                 k = next(j for j, (src, _, _) in enumerate(self.hw) if src == who)  # in order per source
                 _, bar, effect = self.hw.pop(k)
@@ -316,14 +324,19 @@ def random_cases(count, seed):
         yield nkc, random.Random(rng.random())
 
 
+ACTORS = ["list", "producer", "issuer0", "issuer1", "softmax0", "softmax1", "v0", "v1"]
+
+
 @pytest.mark.parametrize("stages", [4, 3])
 @pytest.mark.parametrize("fused", [False, True])
 def test_protocol_never_passes_early_or_hangs(fused, stages):
+    """Random schedules, some of them starving one role (it moves only when nothing else can)."""
     bad = []
-    for nkc, rng in random_cases(1500, 7 + fused):
-        out = Model(nkc, fused, rng, stages=stages).run()
+    for i, (nkc, rng) in enumerate(random_cases(1500, 7 + fused)):
+        starve = () if i % 3 == 0 else (i % len(ACTORS),)
+        out = Model(nkc, fused, rng, stages=stages, starve=starve).run()
         if out != "ok":
-            bad.append((nkc, out))
+            bad.append((nkc, starve, out))
     assert not bad, bad[:5]
 
 
@@ -366,11 +379,23 @@ def test_model_sees_a_shared_v_ready_fail():
 
 
 def test_model_sees_v_warps_skipping_fills_fail():
-    """If each V warp waited only for the fills it prepares, a parity wait could pass on the fill
-    before (still in flight) and some schedule fails: the V warps wait for every fill.  (With the
-    4-slot ring a slot's fills all fall to one V warp, so the mistake shows with a 3-slot ring.)"""
+    """V warps that prepare alternate fills and wait only for those: with a 3-slot ring a slot's
+    fills alternate between the warps, so a parity wait can pass on the fill before (still in
+    flight) and some schedule fails."""
     bad = 0
     for nkc, rng in random_cases(800, 19):
-        if Model(nkc, False, rng, v_skip=True, stages=3).run() != "ok":
+        if Model(nkc, False, rng, v_mode="alt_skip", stages=3).run() != "ok":
+            bad += 1
+    assert bad > 0
+
+
+def test_model_sees_observing_v_warps_lapped():
+    """V warps that prepare alternate fills but wait for every fill: a warp that only looks at a fill
+    the other one prepares can be lapped -- the slot is released and refilled for the same group
+    before it looks, and its parity wait then sees two phases at once and never passes.  A schedule
+    that starves one V warp finds it; owning whole slots (the kernel) cannot be lapped."""
+    bad = 0
+    for i, (nkc, rng) in enumerate(random_cases(600, 23)):
+        if Model(nkc, i % 2 == 1, rng, v_mode="observe_all", starve=(6 + i % 2,)).run() != "ok":
             bad += 1
     assert bad > 0
