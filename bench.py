@@ -32,6 +32,7 @@ per image) on the same workload, metric and unit, one bounded sample of images p
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -108,12 +109,40 @@ def tensor_peak():
     return FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def attention_bounds_us(bytes_, flops, exps, hbm_gbs, sm_mhz, num_sms):
+def measure_ex2_rate(stream, num_sms, iters=2048, reps=5):
+    """Exponentials per second of the whole GPU (ex2.approx.ftz.f32): the microbenchmark in
+    libmicrobench.so, 8 blocks of 256 threads per SM, each thread 8 independent chains, timed with
+    CUDA events on `stream` (best of `reps` launches).  None when the library is missing."""
+    path = os.path.join(ROOT, "ragged_varlen_attention_rra_b200", "libmicrobench.so")
+    if not os.path.exists(path):
+        return None
+    mb = ctypes.CDLL(path)
+    mb.rra_mb_ex2_launch.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    mb.rra_mb_ex2_launch.restype = ctypes.c_int
+    per = int(mb.rra_mb_ex2_per_block_iter())
+    blocks = num_sms * 8
+    out = torch.empty(blocks * 256, dtype=torch.float32, device="cuda")
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            if mb.rra_mb_ex2_launch(out.data_ptr(), blocks, iters, ctypes.c_void_p(stream.cuda_stream)) != 0:
+                return None
+        best = None
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            mb.rra_mb_ex2_launch(out.data_ptr(), blocks, iters, ctypes.c_void_p(stream.cuda_stream))
+            e1.record(stream)
+            e1.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+    return blocks * per * iters / (best * 1e-3)
+
+
+def attention_bounds_us(bytes_, flops, exps, hbm_gbs, ex2_per_s):
     """Lower bounds (us) on one attention launch from each resource: HBM bytes, tensor-core FLOPs
-    at the bf16 peak, and exponentials at the special-function unit's rate."""
+    at the bf16 peak, and exponentials at the measured (or nominal) exponential-unit rate."""
     tf, _ = tensor_peak()
-    ex2_rate = EX2_PER_CLK_PER_SM * num_sms * sm_mhz * 1e6
-    return {"hbm": bytes_ / (hbm_gbs * 1e3), "tensor": flops / (tf * 1e6), "exp": exps / ex2_rate * 1e6}
+    return {"hbm": bytes_ / (hbm_gbs * 1e3), "tensor": flops / (tf * 1e6), "exp": exps / ex2_per_s * 1e6}
 
 
 def source_hash(rel):
@@ -437,6 +466,66 @@ def time_mask_producer(B, N, H, seed, flush, stream, steps, warmup, hbm_peak):
             "alg_bytes_per_launch": nbytes, "gbs": gbs, "frac_of_hbm": gbs / hbm_peak}
 
 
+def time_block(w, cu, flush, stream, steps, warmup):
+    """The synthetic-weight DeiT block (NEXT 4) on the packed rows of the workload's first stage:
+    LN1, QKV, the ragged attention, the output projection, LN2, FC1 + GELU, FC2 (rra.DeitBlock),
+    with random N(0, 1) rows and seeded synthetic weights.  Whole-block time from a graph of the
+    seven launches, per-stage time from a second graph with an event between stages (which
+    serialises them), L2 flushed before each replay.  Reports the attention part (LN1, QKV,
+    attention, projection) against the MLP part (LN2, FC1, FC2) and each GEMM's TFLOP/s."""
+    H, B, N = w.H, w.B, w.N
+    C = 64 * H
+    if C % 256 != 0:
+        return {"skipped": f"width C = {C} is not a multiple of 256, the GEMM kernel's output tile"}
+    cap = B * N
+    T = int(w.lengths[0].sum())
+    g = torch.Generator(device="cuda").manual_seed(int(w.seed) + 5)
+    x = torch.randn(cap, C, generator=g, device="cuda").to(torch.bfloat16)
+    blk = rra.DeitBlock({k: v.cuda() for k, v in workloads.block_weights(C, seed=w.seed).items()}, cap, H)
+    names = blk.STAGES
+    with torch.cuda.stream(stream):
+        blk(x, cu, B, N, stream=stream)
+    stream.synchronize()
+    graph, graph_ev = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(names) + 1)]
+    with torch.cuda.graph(graph, stream=stream):
+        blk(x, cu, B, N, stream=stream)
+    with torch.cuda.graph(graph_ev, stream=stream):
+        ev[0].record(stream)
+        for i, name in enumerate(names):
+            blk.stage(name, x, cu, B, N, stream)
+            ev[i + 1].record(stream)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    whole, per = [], {n: [] for n in names}
+    for i in range(warmup + steps):
+        with torch.cuda.stream(stream):
+            flush.fill_((i + 5) & 0xFF)
+            start.record(stream)
+            graph.replay()
+            end.record(stream)
+            flush.fill_((i + 6) & 0xFF)
+            graph_ev.replay()
+        stream.synchronize()
+        if i >= warmup:
+            whole.append(start.elapsed_time(end))
+            for j, n in enumerate(names):
+                per[n].append(ev[j].elapsed_time(ev[j + 1]))
+    assert rra.rra_get_device_error(blk.err, stream) == 0
+    us = {n: 1e3 * statistics.mean(v) for n, v in per.items()}
+    gemm_flops = {"qkv": 2 * T * C * 3 * C, "proj": 2 * T * C * C, "fc1": 2 * T * C * 4 * C, "fc2": 2 * T * 4 * C * C}
+    tf, tf_kind = tensor_peak()
+    gemms = {n: {"us": us[n], "tflops": f / (us[n] * 1e-6) / 1e12, "frac_of_tensor_peak": f / (us[n] * 1e-6) / 1e12 / tf}
+             for n, f in gemm_flops.items()}
+    attn = sum(us[n] for n in ("ln1", "qkv", "attend", "proj"))
+    mlp = sum(us[n] for n in ("ln2", "fc1", "fc2"))
+    del graph, graph_ev
+    return {"model": f"DeiT block, C = {C}, H = {H}, MLP {4 * C}, synthetic weights", "T": T,
+            "us_per_block": 1e3 * statistics.mean(whole), "us_per_stage": us,
+            "attention_part_us": attn, "mlp_part_us": mlp, "attention_share": attn / (attn + mlp),
+            "gemms": gemms, "tensor_peak_tflops": tf, "tensor_peak_source": tf_kind,
+            "note": "per-stage times come from a graph with events between stages (serialised)"}
+
+
 def kernel_table(kms, alg, stages, hbm_peak):
     table = {}
     for k, v in kms.items():
@@ -663,14 +752,22 @@ def main_gpu(args):
         clk_summary = clk.summary()
         sm_mhz = clk_summary["sm_mhz"] or clk_summary["sm_max_mhz"] or 1965
         bounds = None
+        ex2 = None
         if dom in ("attend", "pack_attend_unpack"):
+            n_sms = torch.cuda.get_device_properties(dev_index).multi_processor_count
+            ex2_per_s = None if args.profile else measure_ex2_rate(stream, n_sms)
+            ex2 = {"per_s": ex2_per_s, "source": "microbenchmark (libmicrobench.so, CUDA events)"}
+            if ex2_per_s is None:
+                ex2_per_s = EX2_PER_CLK_PER_SM * n_sms * sm_mhz * 1e6
+                ex2 = {"per_s": ex2_per_s, "source": "nominal 16 per clock per SM"}
+            ex2["per_clk_per_sm"] = ex2_per_s / (n_sms * sm_mhz * 1e6)
             bounds = attention_bounds_us(per_kernel[dom]["alg_bytes_per_launch"], flops / stages, exps / stages,
-                                         hbm_peak, sm_mhz, torch.cuda.get_device_properties(dev_index).multi_processor_count)
+                                         hbm_peak, ex2_per_s)
         roofline = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
                     "frac": ach / hbm_peak, "peak_source": peak_kind, "traffic": ncu_traffic(dom, w.name),
                     "alg_bytes_per_launch": per_kernel[dom]["alg_bytes_per_launch"],
                     "us_per_launch": per_kernel[dom]["us_per_launch"],
-                    "lower_bounds_us": bounds,
+                    "lower_bounds_us": bounds, "ex2_rate": ex2,
                     "exps_per_launch": exps / stages, "flops_per_launch": flops / stages}
     attn_key = "pack_attend_unpack" if args.path == "fused" else "attend"
     attn_tflops = (flops / (per_kernel[attn_key]["us_per_launch"] * stages * 1e-6) / 1e12) if per_kernel else None
@@ -721,6 +818,10 @@ def main_gpu(args):
 
     mask_producer = None if args.profile else time_mask_producer(w.B, w.N, w.H, w.seed, flush, stream, args.steps,
                                                                  args.warmup, hbm_peak)
+    deit_block = None
+    if not args.profile and not args.no_block and ws == 1:
+        cu0 = torch.from_numpy(np.concatenate([[0], np.cumsum(w.lengths[0])]).astype(np.int32)).cuda()
+        deit_block = time_block(w, cu0, flush, stream, args.steps, args.warmup)
     del pipe.graph_ev, other.graph_ev
 
     sweep = None
@@ -760,6 +861,7 @@ def main_gpu(args):
                            "identical_output": bool(same)},
             "attention_tflops": attn_tflops,
             "mask_producer": mask_producer,
+            "deit_block": deit_block,
             "roofline": roofline,
             "e2e": e2e,
             "cpu_baseline": cpu,
@@ -786,9 +888,13 @@ def main(argv=None):
                     help="single launch (default) or the three calls pack, attend, unpack")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-block", action="store_true", help="skip the synthetic-weight DeiT block timing")
     ap.add_argument("--sweep", default="all", help="'all' or a comma-separated list of workload names")
     ap.add_argument("--profile", action="store_true",
                     help="timed steps only (no dispatch loops, e2e, sweep or CPU leg): the command ncu captures")
+    ap.add_argument("--mask-only", action="store_true",
+                    help="time only the token-selection step (rra_l2_mask) on the workload's shape: the "
+                         "command ncu captures for it")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-images", type=int, default=0,
@@ -797,7 +903,20 @@ def main(argv=None):
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
+    if args.mask_only:
+        return main_mask(args)
     return main_gpu(args)
+
+
+def main_mask(args):
+    """One GPU: rra_l2_mask alone on the workload's shape (L2 flushed before each launch)."""
+    w = workloads.by_name(args.workload)
+    stream = torch.cuda.Stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    hbm_peak, _ = peaks()
+    r = time_mask_producer(w.B, w.N, w.H, w.seed, flush, stream, args.steps, args.warmup, hbm_peak)
+    print(json.dumps({"workload": w.name, "mask_producer": r}), flush=True)
+    return 0
 
 
 if __name__ == "__main__":

@@ -24,6 +24,11 @@ FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2", "-shared",
          "--expt-relaxed-constexpr"]
 
 
+# the exponential-unit microbenchmark bench.py uses for the attention kernel's exp bound
+MB_SRC = os.path.join(HERE, "microbench", "ex2_rate.cu")
+MB_LIB = os.path.join(HERE, "libmicrobench.so")
+
+
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
@@ -40,7 +45,17 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in sources() + headers())
 
 
+def build_microbench(force: bool = False) -> str:
+    if not force and os.path.exists(MB_LIB) and os.path.getmtime(MB_SRC) <= os.path.getmtime(MB_LIB):
+        return MB_LIB
+    tmp = MB_LIB + f".tmp{os.getpid()}"
+    subprocess.run([NVCC, *ARCH_FLAGS, *FLAGS, MB_SRC, "-o", tmp], check=True)
+    os.replace(tmp, MB_LIB)
+    return MB_LIB
+
+
 def build(force: bool = False, verbose_ptxas: bool = False, extra=()) -> str:
+    build_microbench(force)
     if not force and not verbose_ptxas and up_to_date():
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"

@@ -282,3 +282,18 @@ def test_binding_checks_shapes_and_dtypes():
                              "o": t.o})()
     _raises(lambda: rra.forward(t.mask[:1], t.q, t.k, t.v, bufs), "mask")
     _raises(lambda: rra.forward(t.mask, t.q[:, :, :1], t.k, t.v, bufs), "q/k/v")
+
+
+def test_microbench_library_exports_and_validates():
+    """The exponential-unit microbenchmark bench.py times builds, exports its two calls, and
+    refuses bad arguments before any CUDA call."""
+    path = rra_build.build_microbench()
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True)
+    exported = set(re.findall(r"\bT (rra_mb_\w+)", out.stdout))
+    assert {"rra_mb_ex2_launch", "rra_mb_ex2_per_block_iter"} <= exported
+    mb = ctypes.CDLL(path)
+    mb.rra_mb_ex2_launch.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    assert mb.rra_mb_ex2_per_block_iter() == 256 * 8
+    assert mb.rra_mb_ex2_launch(None, 4, 16, None) != 0
+    assert mb.rra_mb_ex2_launch(FAKE, 0, 16, None) != 0
+    assert mb.rra_mb_ex2_launch(FAKE, 4, 0, None) != 0
