@@ -199,6 +199,51 @@ rra_status rra_l2_mask(const void *x, int B, int N, int C, rra_dtype dt, const i
                        rra_stream_t stream);
 
 /*
+ * The dense parts of a transformer block, on the same packed token rows the path produces, for
+ * the attention-vs-MLP latency split of a token-pruned ViT block (aissential.tech summary, "In
+ * practice": decompose attention vs. MLP latency contributions).  A block on packed rows x [T, C]:
+ *   h = LayerNorm1(x); [q | k | v] = h Wqkv^T + bqkv (rra_linear, three outputs); a = the
+ *   ragged attention of q, k, v over cu_seqlens (rra_attend); x1 = x + a Wo^T + bo; h2 =
+ *   LayerNorm2(x1); m = GELU(h2 W1^T + b1); y = x1 + m W2^T + b2.
+ */
+typedef enum { RRA_ACT_NONE = 0, RRA_ACT_GELU = 1 } rra_activation;
+
+/*
+ * rra_linear -- Y = act(X W^T + bias) (+ residual): the projection and MLP layers, on tcgen05
+ * tensor cores with fp32 accumulation and one rounding to bf16 per output element.
+ *   x         device bf16 [M, K], row-major
+ *   w         device bf16 [N, K] (an nn.Linear weight: one row per output feature)
+ *   bias      device bf16 [N], or NULL
+ *   residual  device bf16 [M, N], or NULL; added after the activation.  It may be exactly the
+ *             buffer of the single output (n_outs = 1: each element is read, then written, by
+ *             the same thread); otherwise it must not overlap an output
+ *   act       RRA_ACT_NONE or RRA_ACT_GELU (the exact GELU, x (1 + erf(x / sqrt 2)) / 2)
+ *   outs      host array of n_outs (1..4) device bf16 pointers: outs[j] is [M, N / n_outs] and
+ *             receives columns [j N / n_outs, (j + 1) N / n_outs) of Y (n_outs = 3 splits a fused
+ *             QKV projection into packed Q, K and V)
+ *   M >= 0 rows of buffer; K a positive multiple of 64; N / n_outs a positive multiple of 256
+ *   m_dev     device int32 or NULL: when given, only rows [0, min(M, *m_dev)) are computed and
+ *             written -- on packed rows, cu_seqlens[B] of the pack, so the host need not know T
+ *   dev_error device int32 word for a bounded wait that ran out (RRA_ERR_TIMEOUT), or NULL
+ * Outputs must not overlap x, w, bias or each other (RRA_ERR_INVALID_ARG).  Its shapes and
+ * layouts are this library's; the pages define none for the dense layers.
+ */
+rra_status rra_linear(const void *x, const void *w, const void *bias, const void *residual,
+                      void *const *outs, int n_outs, int64_t M, const int32_t *m_dev, int N, int K,
+                      rra_activation act, int32_t *dev_error, rra_stream_t stream);
+
+/*
+ * rra_layernorm -- y = (x - mean) / sqrt(var + eps) * gamma + beta over each row of x, with
+ * the mean and the (biased) variance of the row in fp32 and one rounding to bf16 per output.
+ *   x, y          device bf16 [M, C]; y must not overlap x
+ *   gamma, beta   device bf16 [C]
+ *   C a positive multiple of 8, at most 2048; eps > 0
+ *   M, m_dev      rows of buffer, and an optional device row count as for rra_linear
+ */
+rra_status rra_layernorm(const void *x, const void *gamma, const void *beta, void *y, int64_t M,
+                         const int32_t *m_dev, int C, float eps, rra_stream_t stream);
+
+/*
  * rra_get_device_error -- copy the device error word to *host_out.  This SYNCHRONISES `stream`
  * (it is the only call that does) and so must not be used inside stream capture.
  */
@@ -208,7 +253,7 @@ rra_status rra_get_device_error(const int32_t *dev_error, rra_stream_t stream, i
 const char *rra_status_string(rra_status status);
 
 /*
- * Debugging knob for the bounded waits inside rra_attend: the time, in nanoseconds of the
+ * Debugging knob for the bounded waits inside rra_attend and rra_linear: the time, in nanoseconds of the
  * GPU global timer, after which a wait for an asynchronous copy or tensor-core operation gives
  * up, raises RRA_ERR_TIMEOUT and ends its block after draining the work it issued.  The default
  * is 2e9 (two seconds); 0 makes every wait that is not already complete give up at once.

@@ -233,6 +233,82 @@ rra_status rra_l2_mask(const void *x, int B, int N, int C, rra_dtype dt, const i
     return e == cudaSuccess ? RRA_OK : RRA_ERR_CUDA;
 }
 
+rra_status rra_linear(const void *x, const void *w, const void *bias, const void *residual, void *const *outs,
+                      int n_outs, int64_t M, const int32_t *m_dev, int N, int K, rra_activation act,
+                      int32_t *dev_error, rra_stream_t stream)
+{
+    if (x == nullptr || w == nullptr || outs == nullptr || n_outs < 1 || n_outs > rra::kLinearMaxOuts)
+        return RRA_ERR_INVALID_ARG;
+    if (M < 0 || N < 1 || K < 1 || M > kMaxRows || (act != RRA_ACT_NONE && act != RRA_ACT_GELU))
+        return RRA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(bias) || !aligned16(residual))
+        return RRA_ERR_INVALID_ARG;
+    if (K % 64 != 0 || N % n_outs != 0 || (N / n_outs) % 256 != 0)
+        return RRA_ERR_UNSUPPORTED;
+    const uint64_t out_b = static_cast<uint64_t>(M) * (N / n_outs) * 2;
+    const uint64_t x_b = static_cast<uint64_t>(M) * K * 2, w_b = static_cast<uint64_t>(N) * K * 2;
+    const uint64_t res_b = static_cast<uint64_t>(M) * N * 2;
+    for (int j = 0; j < n_outs; ++j) {
+        if (outs[j] == nullptr || !aligned16(outs[j]))
+            return RRA_ERR_INVALID_ARG;
+        if (!disjoint(outs[j], out_b, x, x_b) || !disjoint(outs[j], out_b, w, w_b) ||
+            !disjoint(outs[j], out_b, bias, 2ull * N))
+            return RRA_ERR_INVALID_ARG;
+        // the residual may be the single output itself, element for element
+        if (!(n_outs == 1 && residual == outs[0]) && !disjoint(outs[j], out_b, residual, res_b))
+            return RRA_ERR_INVALID_ARG;
+        for (int i = 0; i < j; ++i)
+            if (!disjoint(outs[j], out_b, outs[i], out_b))
+                return RRA_ERR_INVALID_ARG;
+    }
+    if (M == 0)
+        return RRA_OK;
+    int sms = 0;
+    if (num_sms_of_current_device(&sms) != 0)
+        return RRA_ERR_CUDA;
+    rra::LinearArgs a{};
+    a.x = x;
+    a.w = w;
+    a.bias = bias;
+    a.residual = residual;
+    for (int j = 0; j < n_outs; ++j)
+        a.outs[j] = outs[j];
+    a.n_outs = n_outs;
+    a.M = M;
+    a.m_dev = m_dev;
+    a.N = N;
+    a.K = K;
+    a.act = static_cast<int>(act);
+    a.err = dev_error;
+    a.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+    const cudaError_t e = rra::launch_linear(a, sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RRA_OK : RRA_ERR_CUDA;
+}
+
+rra_status rra_layernorm(const void *x, const void *gamma, const void *beta, void *y, int64_t M,
+                         const int32_t *m_dev, int C, float eps, rra_stream_t stream)
+{
+    if (x == nullptr || gamma == nullptr || beta == nullptr || y == nullptr)
+        return RRA_ERR_INVALID_ARG;
+    if (M < 0 || M > kMaxRows || C < 1 || !(eps > 0.f))
+        return RRA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gamma) || !aligned16(beta) || !aligned16(y))
+        return RRA_ERR_INVALID_ARG;
+    if (C % 8 != 0 || C > rra::kLayerNormMaxC)
+        return RRA_ERR_UNSUPPORTED;
+    const uint64_t row_b = static_cast<uint64_t>(M) * C * 2;
+    if (!disjoint(y, row_b, x, row_b) || !disjoint(y, row_b, gamma, 2ull * C) || !disjoint(y, row_b, beta, 2ull * C))
+        return RRA_ERR_INVALID_ARG;
+    if (M == 0)
+        return RRA_OK;
+    int sms = 0;
+    if (num_sms_of_current_device(&sms) != 0)
+        return RRA_ERR_CUDA;
+    const cudaError_t e =
+        rra::launch_layernorm(x, gamma, beta, y, M, m_dev, C, eps, sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? RRA_OK : RRA_ERR_CUDA;
+}
+
 size_t rra_attend_workspace_size(int B, int H, int max_seqlen)
 {
     (void)B;

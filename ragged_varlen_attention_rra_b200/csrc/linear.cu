@@ -1,0 +1,494 @@
+// linear.cu -- the dense parts of a transformer block on packed token rows, for the
+// attention-vs-MLP latency split of a token-pruned ViT block ("Dispatch-Aware Ragged Attention
+// for Pruned Vision Transformers", aissential.tech summary, "In practice": decompose attention
+// vs. MLP latency contributions):
+//   * linear_kernel: Y = act(X W^T + b) (+ R), X [M, K] and W [N, K] bf16 (an nn.Linear weight,
+//     [out, in]), fp32 accumulation on tcgen05 tensor cores, bf16 out; act = identity or the
+//     exact (erf) GELU; R an optional residual [M, N]; Y may be split column-wise into several
+//     outputs (the Q, K, V of a fused QKV projection, each [M, N / n_outs]).
+//   * layernorm_kernel: y = (x - mean) / sqrt(var + eps) * gamma + beta per row, fp32 statistics.
+// Both may take their row count from a device word (cu_seqlens[B] of the pack that produced the
+// rows), so that a whole block on packed rows is enqueued without the host knowing T.
+//
+// linear_kernel (B200 design):
+//   * persistent: one block per SM walks 128 x 256 output tiles, tile t of the block = block id +
+//     t * grid; tiles are numbered along N first, so the blocks in flight share their X rows
+//     (read from HBM once, then from L2) and W (a few MiB) stays in L2;
+//   * a 4-stage ring of (X 128 x 64, W 256 x 64) bf16 tiles in 128-byte-swizzled shared memory,
+//     filled by TMA (warp 0); one thread of warp 1 issues 4 tcgen05.mma (M 128, N 256, K 16) per
+//     stage into one of two TMEM accumulators (2 x 256 columns), so the epilogue of a tile
+//     overlaps the MMAs of the next;
+//   * warps 4..19 are the epilogue: warp w reads TMEM lane quarter w % 4 and columns
+//     [64 p, 64 p + 64) with p = (w - 4) / 4, adds the bias, applies the activation and the
+//     residual in fp32, rounds to bf16 and stores 64-byte row segments;
+//   * every wait is bounded in time; on expiry the block records RRA_ERR_TIMEOUT, raises an abort
+//     flag so every role leaves, drains what it issued and frees TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "rra_device.cuh"
+#include "rra_internal.h"
+
+namespace rra {
+
+namespace {
+
+constexpr int GM = 128;  // output rows per tile (TMEM lanes)
+constexpr int GN = 256;  // output columns per tile (TMEM columns of one accumulator)
+constexpr int GK = 64;   // K per ring stage: one 128-byte swizzle atom of bf16
+constexpr int kLinStages = 4;
+constexpr int kLinThreads = 640;  // 20 warps: producer, issuer, TMEM owner, idle, 16 x epilogue
+constexpr int kEpiWarp0 = 4;
+constexpr int kEpiWarps = 16;
+constexpr int kEpiCols = GN / (kEpiWarps / 4);  // columns per epilogue warp (64)
+constexpr uint32_t kXBytes = GM * GK * 2;        // 16 KiB
+constexpr uint32_t kWBytes = GN * GK * 2;        // 32 KiB
+constexpr uint32_t kLinStageBytes = kXBytes + kWBytes;
+constexpr uint32_t kLinTmemCols = 2 * GN;
+constexpr uint32_t kOffLinBar = kLinStages * kLinStageBytes;
+constexpr int kLinSmem = 1024 + static_cast<int>(kOffLinBar) + 256;
+static_assert(kEpiWarp0 + kEpiWarps == kLinThreads / 32, "warp roles");
+static_assert(kLinSmem <= 232448, "linear tiles exceed shared memory");
+constexpr uint64_t kLinDrainNs = 2000000000ull;
+
+struct LinBars {
+    uint64_t full[kLinStages], empty[kLinStages];  // ring stage loaded / consumed by the MMAs
+    uint64_t acc_full[2], acc_empty[2];            // accumulator computed / read out by the epilogue
+    uint64_t drain;
+    uint32_t tmem_slot;
+    int abort;
+};
+static_assert(sizeof(LinBars) <= 256, "barrier block");
+
+struct LinParams {
+    int M, N, K;
+    const int32_t *m_dev;      // device row count (rows [0, min(M, *m_dev)) are computed), or null
+    const uint16_t *bias;      // [N] bf16, or null
+    const uint16_t *residual;  // [M, N] bf16, or null
+    uint16_t *outs[kLinearMaxOuts];
+    int n_outs, out_ld;        // outs[j] holds columns [j out_ld, (j + 1) out_ld), rows out_ld apart
+    int act;                   // 0: identity, 1: GELU (erf)
+    int32_t *err;
+    uint64_t wait_ns;
+};
+
+// Bounded wait of the whole warp: false when the block aborts or the wait runs out (which
+// raises the abort flag and records the timeout).
+__device__ __noinline__ bool lin_wait_slow(uint64_t *bar, uint32_t parity, LinBars *bars, const LinParams &p)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (*reinterpret_cast<volatile int *>(&bars->abort))
+            return false;
+        if (p.wait_ns == 0 ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity))
+            return true;
+        if (global_timer_ns() - t0 >= p.wait_ns) {
+            *reinterpret_cast<volatile int *>(&bars->abort) = 1;
+            raise_error(p.err, RRA_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ bool lin_wait(uint64_t *bar, uint32_t parity, LinBars *bars, const LinParams &p)
+{
+    const bool ok = mbar_test_wait(bar, parity) || lin_wait_slow(bar, parity, bars, p);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t h) { return __uint_as_float(h << 16); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// The exact GELU of the transformer MLP: x Phi(x) = x (1 + erf(x / sqrt 2)) / 2.
+__device__ __forceinline__ float gelu_erf(float x) { return 0.5f * x * (1.f + erff(x * 0.70710678118654752f)); }
+
+__device__ __forceinline__ void lin_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__global__ void __launch_bounds__(kLinThreads, 1)
+    linear_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const LinParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    LinBars *bars = reinterpret_cast<LinBars *>(base + kOffLinBar);
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    pdl_trigger();
+    if (tid == 0) {
+        prefetch_tmap(&tm_x);
+        prefetch_tmap(&tm_w);
+        for (int s = 0; s < kLinStages; ++s) {
+            mbar_init(&bars->full[s], 1);   // the producer's arrival plus the TMA bytes
+            mbar_init(&bars->empty[s], 1);  // the issuer's MMA commit
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&bars->acc_full[a], 1);
+            mbar_init(&bars->acc_empty[a], kEpiWarps);  // one arrival per epilogue warp
+        }
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(&bars->tmem_slot, kLinTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_slot;
+    pdl_wait();  // X, W, bias, residual and the row count may come from the previous kernel
+
+    const int M = p.m_dev != nullptr ? max(0, min(p.M, *p.m_dev)) : p.M;
+    const int tiles_n = p.N / GN;
+    const int tiles = ((M + GM - 1) / GM) * tiles_n;
+    const int nkb = p.K / GK;
+    const int t_first = static_cast<int>(blockIdx.x), t_step = static_cast<int>(gridDim.x);
+
+    if (warp == 0) {
+        // ================================================================ TMA producer
+        // Empty-stage waits use the parity idiom: on a fresh barrier the phase before phase 0
+        // counts as complete, so the first fill of each stage passes at once.
+        int s = 0;
+        uint32_t ph = 0;
+        uint32_t fills = 0;
+        bool ok = true;
+        for (int t = t_first; ok && t < tiles; t += t_step) {
+            const int m0 = (t / tiles_n) * GM, n0 = (t % tiles_n) * GN;
+            for (int kb = 0; kb < nkb; ++kb) {
+                ok = lin_wait(&bars->empty[s], ((ph >> s) & 1u) ^ 1u, bars, p);
+                if (!ok)
+                    break;
+                ph ^= 1u << s;
+                if (lane == 0) {
+                    uint8_t *st = base + s * kLinStageBytes;
+                    mbar_arrive_expect_tx(&bars->full[s], kLinStageBytes);
+                    tma_load_2d(st, &tm_x, &bars->full[s], kb * GK, m0);  // rows past M read as zeros
+                    tma_load_2d(st + kXBytes, &tm_w, &bars->full[s], kb * GK, n0);
+                }
+                __syncwarp();
+                ++fills;
+                s = (s + 1 == kLinStages) ? 0 : s + 1;
+            }
+        }
+        // drain: every issued fill has landed before the block may leave
+        if (lane == 0)
+            for (int st = 0; st < kLinStages; ++st) {
+                const uint32_t n = fills / kLinStages + (static_cast<uint32_t>(st) < fills % kLinStages ? 1u : 0u);
+                if (n > 0)
+                    mbar_wait_bounded(&bars->full[st], (n - 1) & 1u, kLinDrainNs);
+            }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ================================================================ tcgen05 issuer
+        // Tile t of this block accumulates in TMEM buffer t % 2 (columns 256 (t % 2) ...); the
+        // epilogue releases the buffer (acc_empty) once it has read the tile out.
+        const uint32_t idesc = idesc_f16(GM, GN, 1u, 0u);
+        const uint64_t d0 = smem_desc_sw128(smem_addr(base), 16, 1024);
+        int s = 0, tl = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int t = t_first; ok && t < tiles; t += t_step, ++tl) {
+            const int ab = tl & 1;
+            ok = lin_wait(&bars->acc_empty[ab], ((tl >> 1) & 1u) ^ 1u, bars, p);
+            if (!ok)
+                break;
+            tc_fence_after();
+            for (int kb = 0; kb < nkb; ++kb) {
+                ok = lin_wait(&bars->full[s], (ph >> s) & 1u, bars, p);
+                if (!ok)
+                    break;
+                ph ^= 1u << s;
+                if (lane == 0) {
+                    tc_fence_after();
+                    // stepping K by 16 inside the 128-byte swizzled rows adds 32 bytes (2 units)
+                    const uint64_t xd = d0 + ((s * kLinStageBytes) >> 4);
+                    const uint64_t wd = xd + (kXBytes >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < GK / 16; ++kk)
+                        mma_ss(tmem + GN * ab, xd + 2 * kk, wd + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&bars->empty[s]);
+                }
+                __syncwarp();
+                s = (s + 1 == kLinStages) ? 0 : s + 1;
+            }
+            if (!ok)
+                break;
+            if (lane == 0)
+                mma_commit(&bars->acc_full[ab]);
+            __syncwarp();
+        }
+        // drain: every MMA this thread issued has completed
+        if (lane == 0) {
+            mma_commit(&bars->drain);
+            mbar_wait_bounded(&bars->drain, 0, kLinDrainNs);
+        }
+        __syncwarp();
+    } else if (warp >= kEpiWarp0) {
+        // ================================================================ epilogue
+        const int q4 = warp & 3;
+        const int part = (warp - kEpiWarp0) >> 2;
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+        int tl = 0;
+        bool ok = true;
+        for (int t = t_first; ok && t < tiles; t += t_step, ++tl) {
+            const int ab = tl & 1;
+            ok = lin_wait(&bars->acc_full[ab], (tl >> 1) & 1u, bars, p);
+            if (!ok)
+                break;
+            tc_fence_after();
+            const int m0 = (t / tiles_n) * GM, n0 = (t % tiles_n) * GN;
+            const int row = m0 + q4 * 32 + lane;
+#pragma unroll 1
+            for (int c = 0; c < kEpiCols; c += 32) {
+                const int col = part * kEpiCols + c;
+                uint32_t r[32];
+                tmem_ld32(lane_addr + GN * ab + col, r);
+                tmem_wait_ld_dep(r);
+                const int n = n0 + col;
+                float v[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    v[j] = __uint_as_float(r[j]);
+                if (p.bias != nullptr) {
+                    const uint4 *b4 = reinterpret_cast<const uint4 *>(p.bias + n);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 w = __ldg(b4 + q);
+                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            v[8 * q + 2 * e] += bf16_bits_to_float(ws[e] & 0xFFFFu);
+                            v[8 * q + 2 * e + 1] += bf16_bits_to_float(ws[e] >> 16);
+                        }
+                    }
+                }
+                if (p.act == RRA_ACT_GELU) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        v[j] = gelu_erf(v[j]);
+                }
+                if (row < M) {
+                    if (p.residual != nullptr) {
+                        const uint4 *r4 = reinterpret_cast<const uint4 *>(p.residual + static_cast<int64_t>(row) * p.N + n);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint4 w = r4[q];
+                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                v[8 * q + 2 * e] += bf16_bits_to_float(ws[e] & 0xFFFFu);
+                                v[8 * q + 2 * e + 1] += bf16_bits_to_float(ws[e] >> 16);
+                            }
+                        }
+                    }
+                    const int oi = n / p.out_ld;
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.outs[oi] + static_cast<int64_t>(row) * p.out_ld +
+                                                           (n - oi * p.out_ld));
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                            pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                                            pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                lin_arrive(&bars->acc_empty[ab]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kLinTmemCols);
+    }
+}
+
+// ---- layernorm ------------------------------------------------------------------------------
+
+constexpr int kLnThreads = 256;  // 8 rows in flight per block, one warp each
+constexpr int kLnMaxChunks = kLayerNormMaxC / (32 * 8);
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+// One warp per row: the row's 16-byte chunks spread over the lanes (chunk c to lane c % 32), the
+// mean, then the variance of (x - mean) (two passes over registers), each a warp reduction in fp32.
+__global__ void __launch_bounds__(kLnThreads) layernorm_kernel(const uint16_t *x, const uint16_t *gamma,
+                                                               const uint16_t *beta, uint16_t *y, int64_t M_max,
+                                                               const int32_t *m_dev, int C, float eps)
+{
+    pdl_trigger();
+    pdl_wait();
+    const int64_t M = m_dev != nullptr ? max(int64_t{0}, min(M_max, static_cast<int64_t>(*m_dev))) : M_max;
+    const int lane = threadIdx.x & 31;
+    const int nch = C >> 3;
+    const float inv_c = 1.f / static_cast<float>(C);
+    for (int64_t row = static_cast<int64_t>(blockIdx.x) * (kLnThreads / 32) + (threadIdx.x >> 5); row < M;
+         row += static_cast<int64_t>(gridDim.x) * (kLnThreads / 32)) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * C);
+        float v[kLnMaxChunks][8];
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < kLnMaxChunks; ++i) {
+            const int c = lane + 32 * i;
+            const uint4 w = c < nch ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                v[i][2 * e] = bf16_bits_to_float(ws[e] & 0xFFFFu);
+                v[i][2 * e + 1] = bf16_bits_to_float(ws[e] >> 16);
+                s += v[i][2 * e] + v[i][2 * e + 1];
+            }
+        }
+        const float mean = warp_sum(s) * inv_c;
+        float q = 0.f;
+#pragma unroll
+        for (int i = 0; i < kLnMaxChunks; ++i)
+            if (lane + 32 * i < nch) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float d = v[i][e] - mean;
+                    q = fmaf(d, d, q);
+                }
+            }
+        const float rstd = rsqrtf(warp_sum(q) * inv_c + eps);
+#pragma unroll
+        for (int i = 0; i < kLnMaxChunks; ++i) {
+            const int c = lane + 32 * i;
+            if (c < nch) {
+                const uint4 g = __ldg(reinterpret_cast<const uint4 *>(gamma) + c);
+                const uint4 b = __ldg(reinterpret_cast<const uint4 *>(beta) + c);
+                const uint32_t gs[4] = {g.x, g.y, g.z, g.w}, bs[4] = {b.x, b.y, b.z, b.w};
+                uint32_t o[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float y0 = (v[i][2 * e] - mean) * rstd * bf16_bits_to_float(gs[e] & 0xFFFFu) +
+                                     bf16_bits_to_float(bs[e] & 0xFFFFu);
+                    const float y1 = (v[i][2 * e + 1] - mean) * rstd * bf16_bits_to_float(gs[e] >> 16) +
+                                     bf16_bits_to_float(bs[e] >> 16);
+                    o[e] = pack_bf16x2(y0, y1);
+                }
+                reinterpret_cast<uint4 *>(y + row * C)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+        }
+    }
+}
+
+// ---- host side -----------------------------------------------------------------------------
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// A row-major bf16 matrix [rows, K] seen as 2-D (k, row); box = 64 k x box_rows rows, 128-byte
+// swizzle (one box row is one swizzle span).
+bool make_tmap_2d(CUtensorMap *map, const void *ptr, int64_t rows, int K, int box_rows)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (enc == nullptr)
+        return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(GK), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+cudaError_t set_linear_smem()
+{
+    static std::mutex mu;
+    static bool done[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 64 && done[dev])
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem);
+    if (e == cudaSuccess && dev < 64)
+        done[dev] = true;
+    return e;
+}
+
+}  // namespace
+
+cudaError_t launch_linear(const LinearArgs &a, int num_sms, cudaStream_t stream)
+{
+    if (a.M == 0)
+        return cudaSuccess;
+    alignas(64) CUtensorMap tx, tw;
+    if (!make_tmap_2d(&tx, a.x, a.M, a.K, GM) || !make_tmap_2d(&tw, a.w, a.N, a.K, GN))
+        return cudaErrorInvalidValue;
+    LinParams p{};
+    p.M = static_cast<int>(a.M);
+    p.m_dev = a.m_dev;
+    p.N = a.N;
+    p.K = a.K;
+    p.bias = static_cast<const uint16_t *>(a.bias);
+    p.residual = static_cast<const uint16_t *>(a.residual);
+    for (int j = 0; j < a.n_outs; ++j)
+        p.outs[j] = static_cast<uint16_t *>(a.outs[j]);
+    p.n_outs = a.n_outs;
+    p.out_ld = a.N / a.n_outs;
+    p.act = a.act;
+    p.err = a.err;
+    p.wait_ns = a.wait_ns;
+    cudaError_t e = set_linear_smem();
+    if (e != cudaSuccess)
+        return e;
+    const int64_t tiles = ((a.M + GM - 1) / GM) * (a.N / GN);
+    const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+    return launch_pdl(linear_kernel, dim3(grid), dim3(kLinThreads), kLinSmem, stream, tx, tw, p);
+}
+
+cudaError_t launch_layernorm(const void *x, const void *gamma, const void *beta, void *y, int64_t M,
+                             const int32_t *m_dev, int C, float eps, int num_sms, cudaStream_t stream)
+{
+    if (M == 0)
+        return cudaSuccess;
+    const int64_t blocks_needed = (M + kLnThreads / 32 - 1) / (kLnThreads / 32);
+    const int64_t cap = static_cast<int64_t>(num_sms) * 16;
+    const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
+    return launch_pdl(layernorm_kernel, dim3(grid), dim3(kLnThreads), 0, stream, static_cast<const uint16_t *>(x),
+                      static_cast<const uint16_t *>(gamma), static_cast<const uint16_t *>(beta),
+                      static_cast<uint16_t *>(y), M, m_dev, C, eps);
+}
+
+}  // namespace rra

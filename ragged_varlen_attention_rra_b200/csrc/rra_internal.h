@@ -80,4 +80,24 @@ constexpr int kMaskMaxN = 4096;
 cudaError_t launch_l2_mask(const void *x, int B, int N, int C, bool bf16, const int32_t *k_keep, double thr_sq,
                            const uint8_t *prev, uint8_t *mask, int num_sms, cudaStream_t stream);
 
+// Dense parts of a transformer block on packed rows (linear.cu).
+constexpr int kLinearMaxOuts = 4;     // a fused projection's outputs (Q, K, V)
+constexpr int kLayerNormMaxC = 2048;  // row width rra_layernorm accepts (8 16-byte chunks per lane)
+
+struct LinearArgs {
+    const void *x, *w, *bias, *residual;
+    void *outs[kLinearMaxOuts];
+    int n_outs;
+    int64_t M;
+    const int32_t *m_dev;
+    int N, K, act;
+    int32_t *err;
+    uint64_t wait_ns;
+};
+
+cudaError_t launch_linear(const LinearArgs &a, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_layernorm(const void *x, const void *gamma, const void *beta, void *y, int64_t M,
+                             const int32_t *m_dev, int C, float eps, int num_sms, cudaStream_t stream);
+
 }  // namespace rra

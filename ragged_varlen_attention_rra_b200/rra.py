@@ -57,6 +57,11 @@ def _declare(lib):
     lib.rra_pack_attend_unpack.restype = c.c_int
     lib.rra_l2_mask.argtypes = [vp, c.c_int, c.c_int, c.c_int, c.c_int, i32p, c.c_double, vp, vp, vp]
     lib.rra_l2_mask.restype = c.c_int
+    lib.rra_linear.argtypes = [vp, vp, vp, vp, c.POINTER(c.c_void_p), c.c_int, c.c_int64, i32p, c.c_int, c.c_int,
+                               c.c_int, i32p, vp]
+    lib.rra_linear.restype = c.c_int
+    lib.rra_layernorm.argtypes = [vp, vp, vp, vp, c.c_int64, i32p, c.c_int, c.c_float, vp]
+    lib.rra_layernorm.restype = c.c_int
     lib.rra_get_device_error.argtypes = [i32p, vp, c.POINTER(c.c_int32)]
     lib.rra_get_device_error.restype = c.c_int
     lib.rra_status_string.argtypes = [c.c_int]
@@ -293,6 +298,116 @@ def rra_l2_mask(x: torch.Tensor, keep_mask: torch.Tensor, k_keep: Optional[torch
     st = lib().rra_l2_mask(_ptr(x), B, N, C, _DT[x.dtype], _ptr(k_keep), float(threshold_sq), _ptr(prev_mask),
                            _ptr(keep_mask), _stream(stream))
     _check(st, what)
+
+
+RRA_ACT_NONE, RRA_ACT_GELU = 0, 1
+
+
+def rra_linear(x: torch.Tensor, w: torch.Tensor, outs: Sequence[torch.Tensor], bias: Optional[torch.Tensor] = None,
+               residual: Optional[torch.Tensor] = None, act: int = RRA_ACT_NONE, m_dev: Optional[torch.Tensor] = None,
+               dev_error: Optional[torch.Tensor] = None, stream=None) -> None:
+    """outs = split(act(x w^T + bias) + residual): x bf16 [M, K], w bf16 [N, K], bias [N], residual
+    [M, N], outs n_outs tensors bf16 [M, N / n_outs].  With m_dev (int32 device word) only rows
+    [0, min(M, m_dev)) are computed."""
+    what = "rra_linear"
+    bf = torch.bfloat16
+    _expect(x.dim() == 2 and x.dtype == bf and w.dim() == 2 and w.dtype == bf, f"{what}: x, w must be bf16 2-D")
+    M, K = x.shape
+    N = w.shape[0]
+    _expect(w.shape[1] == K, f"{what}: w must be [N, {K}]")
+    outs = list(outs)
+    _expect(1 <= len(outs) <= 4 and N % len(outs) == 0, f"{what}: 1..4 outputs splitting N = {N}")
+    for o in outs:
+        _expect(o.dtype == bf and tuple(o.shape) == (M, N // len(outs)), f"{what}: outs must be bf16 [{M}, {N // len(outs)}]")
+    if bias is not None:
+        _expect(bias.dtype == bf and bias.numel() == N, f"{what}: bias must be bf16 [{N}]")
+    if residual is not None:
+        _expect(residual.dtype == bf and tuple(residual.shape) == (M, N), f"{what}: residual must be bf16 [{M}, {N}]")
+    if m_dev is not None:
+        _expect(m_dev.dtype == torch.int32 and m_dev.numel() >= 1, f"{what}: m_dev must be an int32 word")
+    _check_err(dev_error, what)
+    _disjoint(outs, [x, w, bias], what)
+    if residual is not None and not (len(outs) == 1 and outs[0].data_ptr() == residual.data_ptr()):
+        _disjoint(outs, [residual], what)
+    for i, o in enumerate(outs):
+        _disjoint([o], outs[:i], what)
+    _require_cuda(x, w, bias, residual, m_dev, dev_error, *outs)
+    arr = (ctypes.c_void_p * len(outs))(*[o.data_ptr() for o in outs])
+    st = lib().rra_linear(_ptr(x), _ptr(w), _ptr(bias), _ptr(residual), arr, len(outs), M, _ptr(m_dev), N, K, act,
+                          _ptr(dev_error), _stream(stream))
+    _check(st, what)
+
+
+def rra_layernorm(x: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor, y: torch.Tensor, eps: float = 1e-6,
+                  m_dev: Optional[torch.Tensor] = None, stream=None) -> None:
+    """y = LayerNorm(x) * gamma + beta per row: x, y bf16 [M, C]; with m_dev only rows [0, min(M, m_dev))."""
+    what = "rra_layernorm"
+    bf = torch.bfloat16
+    _expect(x.dim() == 2 and x.dtype == bf, f"{what}: x must be bf16 [M, C]")
+    M, C = x.shape
+    _expect(y.dtype == bf and tuple(y.shape) == (M, C), f"{what}: y must be bf16 [{M}, {C}]")
+    _expect(gamma.dtype == bf and beta.dtype == bf and gamma.numel() == C and beta.numel() == C,
+            f"{what}: gamma, beta must be bf16 [{C}]")
+    if m_dev is not None:
+        _expect(m_dev.dtype == torch.int32 and m_dev.numel() >= 1, f"{what}: m_dev must be an int32 word")
+    _disjoint([y], [x, gamma, beta], what)
+    _require_cuda(x, gamma, beta, y, m_dev)
+    st = lib().rra_layernorm(_ptr(x), _ptr(gamma), _ptr(beta), _ptr(y), M, _ptr(m_dev), C, float(eps), _stream(stream))
+    _check(st, what)
+
+
+class DeitBlock:
+    """A transformer block on packed token rows (weights and activation buffers): LN1, the fused
+    QKV projection split into packed Q, K, V, the ragged attention, the output projection with its
+    residual, LN2, FC1 with GELU and FC2 with its residual.  `weights` maps the nn.Linear /
+    nn.LayerNorm names (qkv_w [3C, C], qkv_b, proj_w [C, C], proj_b, fc1_w [4C, C], fc1_b, fc2_w
+    [C, 4C], fc2_b, ln1_g, ln1_b, ln2_g, ln2_b) to bf16 device tensors."""
+
+    STAGES = ("ln1", "qkv", "attend", "proj", "ln2", "fc1", "fc2")
+
+    def __init__(self, weights, capacity: int, H: int, eps: float = 1e-6, device="cuda"):
+        C = H * 64
+        self.w, self.C, self.H, self.cap, self.eps = weights, C, H, capacity, eps
+        e = lambda n: torch.empty(capacity, n, dtype=torch.bfloat16, device=device)
+        self.h, self.q, self.k, self.v, self.a, self.x1, self.h2 = (e(C) for _ in range(7))
+        self.m = e(4 * C)
+        self.y = e(C)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def stage(self, name: str, x: torch.Tensor, cu: torch.Tensor, B: int, max_seqlen: int, stream=None):
+        """Enqueue one of STAGES on `stream` (rows [0, cu[B]) of the capacity-row buffers)."""
+        w, T = self.w, cu[B:B + 1]
+        if name == "ln1":
+            rra_layernorm(x, w["ln1_g"], w["ln1_b"], self.h, self.eps, m_dev=T, stream=stream)
+        elif name == "qkv":
+            rra_linear(self.h, w["qkv_w"], [self.q, self.k, self.v], bias=w["qkv_b"], m_dev=T, dev_error=self.err,
+                       stream=stream)
+        elif name == "attend":
+            sh = (self.cap, self.H, 64)
+            rra_attend(self.q.view(sh), self.k.view(sh), self.v.view(sh), self.a.view(sh), cu, max_seqlen=max_seqlen,
+                       dev_error=self.err, stream=stream)
+        elif name == "proj":
+            rra_linear(self.a, w["proj_w"], [self.x1], bias=w["proj_b"], residual=x, m_dev=T, dev_error=self.err,
+                       stream=stream)
+        elif name == "ln2":
+            rra_layernorm(self.x1, w["ln2_g"], w["ln2_b"], self.h2, self.eps, m_dev=T, stream=stream)
+        elif name == "fc1":
+            rra_linear(self.h2, w["fc1_w"], [self.m], bias=w["fc1_b"], act=RRA_ACT_GELU, m_dev=T, dev_error=self.err,
+                       stream=stream)
+        elif name == "fc2":
+            rra_linear(self.m, w["fc2_w"], [self.y], bias=w["fc2_b"], residual=self.x1, m_dev=T, dev_error=self.err,
+                       stream=stream)
+        else:
+            raise ValueError(name)
+
+    def __call__(self, x: torch.Tensor, cu: torch.Tensor, B: int, max_seqlen: int, stream=None) -> torch.Tensor:
+        """The block on packed rows x [capacity, C] whose first cu[B] rows are the kept tokens of B
+        images (cu_seqlens of the pack); returns self.y (rows past cu[B] are not written)."""
+        _expect(x.dtype == torch.bfloat16 and tuple(x.shape) == (self.cap, self.C),
+                f"DeitBlock: x must be bf16 [{self.cap}, {self.C}]")
+        for name in self.STAGES:
+            self.stage(name, x, cu, B, max_seqlen, stream)
+        return self.y
 
 
 # ------------------------------------------------------------------------------------ whole call

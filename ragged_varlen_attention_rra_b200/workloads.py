@@ -214,6 +214,27 @@ def embeddings(B: int, N: int, C: int = 384, dtype: str = "bf16", seed: int = 0,
     return torch.from_numpy(x).to(_TORCH_DTYPES[dtype]).contiguous()
 
 
+def block_weights(C: int, seed: int = 0, std: float = 0.02) -> dict:
+    """Synthetic weights of one DeiT block of width C (there are no trained weights): the linear
+    layers N(0, std^2) as a truncated-normal init draws them (nn.Linear layout [out, in]), biases
+    N(0, std^2), LayerNorm gamma 1 + N(0, 0.1^2) and beta N(0, 0.1^2) (so the affine part is
+    exercised); all rounded to bf16, on the CPU."""
+    rng = np.random.default_rng(np.random.SeedSequence([int(seed), 91, int(C)]))
+    shapes = {"qkv_w": (3 * C, C), "qkv_b": (3 * C,), "proj_w": (C, C), "proj_b": (C,), "fc1_w": (4 * C, C),
+              "fc1_b": (4 * C,), "fc2_w": (C, 4 * C), "fc2_b": (C,)}
+    w = {k: np.clip(rng.standard_normal(sh), -2, 2) * std for k, sh in shapes.items()}
+    for ln in ("ln1", "ln2"):
+        w[ln + "_g"] = 1 + 0.1 * rng.standard_normal(C)
+        w[ln + "_b"] = 0.1 * rng.standard_normal(C)
+    return {k: torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16) for k, v in w.items()}
+
+
+def block_input(T: int, C: int, seed: int = 0) -> torch.Tensor:
+    """Packed token rows [T, C] entering a block: N(0, 1) in bf16, on the CPU."""
+    rng = np.random.default_rng(np.random.SeedSequence([int(seed), 92, int(T), int(C)]))
+    return torch.from_numpy(rng.standard_normal((T, C), dtype=np.float32)).to(torch.bfloat16)
+
+
 def keep_counts(B: int, N: int, lo: float = 0.3, hi: float = 0.7, seed: int = 0) -> np.ndarray:
     """Patches kept per image at ratios r_b ~ U[lo, hi] (the configs' recipe), int32 [B]."""
     rng = np.random.default_rng(np.random.SeedSequence([int(seed), 78, int(B), int(N)]))
