@@ -895,6 +895,9 @@ def main(argv=None):
     ap.add_argument("--mask-only", action="store_true",
                     help="time only the token-selection step (rra_l2_mask) on the workload's shape: the "
                          "command ncu captures for it")
+    ap.add_argument("--block-only", action="store_true",
+                    help="time only the synthetic-weight DeiT block on the workload's packed rows: the "
+                         "command ncu captures for its kernels")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-images", type=int, default=0,
@@ -905,7 +908,20 @@ def main(argv=None):
         return run_reference(args)
     if args.mask_only:
         return main_mask(args)
+    if args.block_only:
+        return main_block(args)
     return main_gpu(args)
+
+
+def main_block(args):
+    """One GPU: the synthetic-weight DeiT block alone on the workload's packed rows."""
+    w = workloads.by_name(args.workload)
+    stream = torch.cuda.Stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    cu0 = torch.from_numpy(np.concatenate([[0], np.cumsum(w.lengths[0])]).astype(np.int32)).cuda()
+    print(json.dumps({"workload": w.name, "deit_block": time_block(w, cu0, flush, stream, args.steps, args.warmup)}),
+          flush=True)
+    return 0
 
 
 def main_mask(args):

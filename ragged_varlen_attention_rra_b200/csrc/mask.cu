@@ -196,7 +196,7 @@ __device__ __noinline__ Key slow_key(const uint16_t *xrow, int nchunks, int lane
 }
 
 template <bool kBF16>
-__global__ void __launch_bounds__(kMaskThreads) l2_mask_kernel(const uint16_t *__restrict__ x, int N, int C,
+__global__ void __launch_bounds__(kMaskThreads, 4) l2_mask_kernel(const uint16_t *__restrict__ x, int N, int C,
                                                                 const int32_t *__restrict__ k_keep, double thr_sq,
                                                                 const uint8_t *prev, uint8_t *mask)
 {
@@ -320,12 +320,77 @@ __global__ void __launch_bounds__(kMaskThreads) l2_mask_kernel(const uint16_t *_
 // CTAs per image: enough for about two CTAs per SM over the batch (one CTA per image once the
 // batch alone fills the GPU, where clusters would only limit how many CTAs can be resident), at
 // least 16 tokens per CTA, at most the portable cluster size; a power of two.
-int cluster_for(int B, int N, int num_sms)
+// Clusters of 1, 2, 4 and 8 CTAs that can be resident at once, for this kernel at a given
+// shared-memory size, from the occupancy query (which knows the GPU's actual GPC layout);
+// -1 where a size cannot be used.  Queried once per device and size, then cached.
+static_assert(kMaxCluster == 8, "cluster sizes 1, 2, 4, 8 are queried");
+
+template <bool kBF16>
+struct ClusterFit {
+    int smem = -1;
+    int act[4] = {0, 0, 0, 0};
+};
+
+template <bool kBF16>
+const int *max_active_clusters(int smem)
 {
-    int cs = 1;
-    while (cs < kMaxCluster && static_cast<int64_t>(B) * cs < 2 * num_sms && N >= 32 * cs)
-        cs *= 2;
-    return cs;
+    static std::mutex mu;
+    static ClusterFit<kBF16> cache[64][4];  // per device: the last four shared-memory sizes seen
+    static int next[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64)
+        return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    for (auto &c : cache[dev])
+        if (c.smem == smem)
+            return c.act;
+    ClusterFit<kBF16> &c = cache[dev][next[dev]];
+    next[dev] = (next[dev] + 1) & 3;
+    for (int i = 0; i < 4; ++i) {
+        const int cs = 1 << i;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(cs));
+        cfg.blockDim = dim3(kMaskThreads);
+        cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(cs);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, l2_mask_kernel<kBF16>, &cfg) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = -1;
+        }
+        c.act[i] = n;
+    }
+    c.smem = smem;
+    return c.act;
+}
+
+// Cluster size (CTAs per image): the fewest waves of clusters (one image per cluster), then the
+// largest size (more SMs per image), keeping at least 16 tokens per CTA.
+template <bool kBF16>
+int cluster_for(int B, int N, int smem)
+{
+    const int *act = max_active_clusters<kBF16>(smem);
+    int best = 1;
+    int64_t best_waves = -1;
+    for (int i = 0; i < 4; ++i) {
+        const int cs = 1 << i;
+        if (cs > 1 && N < 16 * cs)
+            break;
+        if (act == nullptr || act[i] <= 0)
+            continue;
+        const int64_t waves = (static_cast<int64_t>(B) + act[i] - 1) / act[i];
+        if (best_waves < 0 || waves <= best_waves) {
+            best_waves = waves;
+            best = cs;
+        }
+    }
+    return best;
 }
 
 template <bool kBF16>
@@ -350,11 +415,12 @@ template <bool kBF16>
 cudaError_t launch_mask_variant(const uint16_t *x, int B, int N, int C, const int32_t *k_keep, double thr_sq,
                                 const uint8_t *prev, uint8_t *mask, int num_sms, cudaStream_t stream)
 {
-    const int cs = cluster_for(B, N, num_sms);
     const int smem = N * static_cast<int>(sizeof(Key));
     cudaError_t e = set_mask_smem<kBF16>(smem);
     if (e != cudaSuccess)
         return e;
+    (void)num_sms;
+    const int cs = cluster_for<kBF16>(B, N, smem);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(B) * cs);
     cfg.blockDim = dim3(kMaskThreads);
