@@ -20,7 +20,9 @@
 //     overlaps the MMAs of the next;
 //   * warps 4..19 are the epilogue: warp w reads TMEM lane quarter w % 4 and columns
 //     [64 p, 64 p + 64) with p = (w - 4) / 4, adds the bias, applies the activation and the
-//     residual in fp32, rounds to bf16 and stores 64-byte row segments;
+//     residual in fp32, rounds to bf16, and passes each 32 x 32 block through its own 2 KiB of
+//     shared memory, so that the global stores go out as whole 64-byte row segments, 8 rows per
+//     instruction;
 //   * every wait is bounded in time; on expiry the block records RRA_ERR_TIMEOUT, raises an abort
 //     flag so every role leaves, drains what it issued and frees TMEM.
 #include <cuda.h>
@@ -48,7 +50,10 @@ constexpr uint32_t kWBytes = GN * GK * 2;        // 32 KiB
 constexpr uint32_t kLinStageBytes = kXBytes + kWBytes;
 constexpr uint32_t kLinTmemCols = 2 * GN;
 constexpr uint32_t kOffLinBar = kLinStages * kLinStageBytes;
-constexpr int kLinSmem = 1024 + static_cast<int>(kOffLinBar) + 256;
+// per epilogue warp, a 32 x 32 bf16 block of the output on its way to global memory (2 KiB)
+constexpr uint32_t kOffLinStage = kOffLinBar + 256;
+constexpr uint32_t kStageWarpBytes = 32 * 32 * 2;
+constexpr int kLinSmem = 1024 + static_cast<int>(kOffLinStage + kEpiWarps * kStageWarpBytes);
 static_assert(kEpiWarp0 + kEpiWarps == kLinThreads / 32, "warp roles");
 static_assert(kLinSmem <= 232448, "linear tiles exceed shared memory");
 constexpr uint64_t kLinDrainNs = 2000000000ull;
@@ -248,7 +253,6 @@ __global__ void __launch_bounds__(kLinThreads, 1)
                 break;
             tc_fence_after();
             const int m0 = (t / tiles_n) * GM, n0 = (t % tiles_n) * GN;
-            const int row = m0 + q4 * 32 + lane;
 #pragma unroll 1
             for (int c = 0; c < kEpiCols; c += 32) {
                 const int col = part * kEpiCols + c;
@@ -278,29 +282,52 @@ __global__ void __launch_bounds__(kLinThreads, 1)
                     for (int j = 0; j < 32; ++j)
                         v[j] = gelu_erf(v[j]);
                 }
-                if (row < M) {
-                    if (p.residual != nullptr) {
-                        const uint4 *r4 = reinterpret_cast<const uint4 *>(p.residual + static_cast<int64_t>(row) * p.N + n);
+                // the warp's 32 x 32 block goes through its own staging buffer: row r at 64 r bytes,
+                // 16-byte piece q at (q ^ ((r >> 1) & 3)) -- an XOR that spreads the 32 rows of a
+                // piece over all the banks; global memory sees whole 64-byte row segments, lane l
+                // taking piece l % 4 of rows l / 4 + 8 i
+                uint8_t *stg = base + kOffLinStage + (warp - kEpiWarp0) * kStageWarpBytes;
+                auto piece = [&](int rr, int q) { return stg + rr * 64 + ((q ^ ((rr >> 1) & 3)) << 4); };
+                if (p.residual != nullptr) {
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint4 w = r4[q];
-                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                    for (int i = 0; i < 4; ++i) {
+                        const int rr = (lane >> 2) + 8 * i, q = lane & 3;
+                        const int grow = m0 + q4 * 32 + rr;
+                        uint4 w = make_uint4(0, 0, 0, 0);
+                        if (grow < M)
+                            w = *reinterpret_cast<const uint4 *>(p.residual + static_cast<int64_t>(grow) * p.N + n + 8 * q);
+                        *reinterpret_cast<uint4 *>(piece(rr, q)) = w;
+                    }
+                    __syncwarp();
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                v[8 * q + 2 * e] += bf16_bits_to_float(ws[e] & 0xFFFFu);
-                                v[8 * q + 2 * e + 1] += bf16_bits_to_float(ws[e] >> 16);
-                            }
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 w = *reinterpret_cast<const uint4 *>(piece(lane, q));
+                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            v[8 * q + 2 * e] += bf16_bits_to_float(ws[e] & 0xFFFFu);
+                            v[8 * q + 2 * e + 1] += bf16_bits_to_float(ws[e] >> 16);
                         }
                     }
-                    const int oi = n / p.out_ld;
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.outs[oi] + static_cast<int64_t>(row) * p.out_ld +
-                                                           (n - oi * p.out_ld));
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                            pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                                            pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+                    __syncwarp();
                 }
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(piece(lane, q)) =
+                        make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                   pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+                __syncwarp();
+                const int oi = n / p.out_ld;
+                uint16_t *obase = p.outs[oi] + (n - oi * p.out_ld);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int rr = (lane >> 2) + 8 * i, q = lane & 3;
+                    const int grow = m0 + q4 * 32 + rr;
+                    if (grow < M)
+                        *reinterpret_cast<uint4 *>(obase + static_cast<int64_t>(grow) * p.out_ld + 8 * q) =
+                            *reinterpret_cast<const uint4 *>(piece(rr, q));
+                }
+                __syncwarp();  // the buffer is reused by the next block
             }
             tc_fence_before();
             __syncwarp();
