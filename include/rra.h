@@ -221,7 +221,7 @@ typedef enum { RRA_ACT_NONE = 0, RRA_ACT_GELU = 1 } rra_activation;
  *   outs      host array of n_outs (1..4) device bf16 pointers: outs[j] is [M, N / n_outs] and
  *             receives columns [j N / n_outs, (j + 1) N / n_outs) of Y (n_outs = 3 splits a fused
  *             QKV projection into packed Q, K and V)
- *   M >= 0 rows of buffer; K a positive multiple of 64; N / n_outs a positive multiple of 256
+ *   M >= 0 rows of buffer; K a positive multiple of 64; N / n_outs a positive multiple of 128
  *   m_dev     device int32 or NULL: when given, only rows [0, min(M, *m_dev)) are computed and
  *             written -- on packed rows, cu_seqlens[B] of the pack, so the host need not know T
  *   dev_error device int32 word for a bounded wait that ran out (RRA_ERR_TIMEOUT), or NULL

@@ -243,7 +243,7 @@ rra_status rra_linear(const void *x, const void *w, const void *bias, const void
         return RRA_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w) || !aligned16(bias) || !aligned16(residual))
         return RRA_ERR_INVALID_ARG;
-    if (K % 64 != 0 || N % n_outs != 0 || (N / n_outs) % 256 != 0)
+    if (K % 64 != 0 || N % n_outs != 0 || (N / n_outs) % 128 != 0)
         return RRA_ERR_UNSUPPORTED;
     const uint64_t out_b = static_cast<uint64_t>(M) * (N / n_outs) * 2;
     const uint64_t x_b = static_cast<uint64_t>(M) * K * 2, w_b = static_cast<uint64_t>(N) * K * 2;

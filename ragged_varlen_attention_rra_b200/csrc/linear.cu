@@ -11,7 +11,8 @@
 // rows), so that a whole block on packed rows is enqueued without the host knowing T.
 //
 // linear_kernel (B200 design):
-//   * persistent: one block per SM walks 128 x 256 output tiles, tile t of the block = block id +
+//   * persistent: one block per SM walks 128 x 256 output tiles (128 x 128 when an output's width
+//     is an odd multiple of 128), tile t of the block = block id +
 //     t * grid; tiles are numbered along N first, so the blocks in flight share their X rows
 //     (read from HBM once, then from L2) and W (a few MiB) stays in L2;
 //   * a 4-stage ring of (X 128 x 64, W 256 x 64) bf16 tiles in 128-byte-swizzled shared memory,
@@ -38,24 +39,29 @@ namespace rra {
 namespace {
 
 constexpr int GM = 128;  // output rows per tile (TMEM lanes)
-constexpr int GN = 256;  // output columns per tile (TMEM columns of one accumulator)
 constexpr int GK = 64;   // K per ring stage: one 128-byte swizzle atom of bf16
 constexpr int kLinStages = 4;
 constexpr int kLinThreads = 640;  // 20 warps: producer, issuer, TMEM owner, idle, 16 x epilogue
 constexpr int kEpiWarp0 = 4;
 constexpr int kEpiWarps = 16;
-constexpr int kEpiCols = GN / (kEpiWarps / 4);  // columns per epilogue warp (64)
-constexpr uint32_t kXBytes = GM * GK * 2;        // 16 KiB
-constexpr uint32_t kWBytes = GN * GK * 2;        // 32 KiB
-constexpr uint32_t kLinStageBytes = kXBytes + kWBytes;
-constexpr uint32_t kLinTmemCols = 2 * GN;
-constexpr uint32_t kOffLinBar = kLinStages * kLinStageBytes;
+constexpr uint32_t kXBytes = GM * GK * 2;  // 16 KiB
 // per epilogue warp, a 32 x 32 bf16 block of the output on its way to global memory (2 KiB)
-constexpr uint32_t kOffLinStage = kOffLinBar + 256;
 constexpr uint32_t kStageWarpBytes = 32 * 32 * 2;
-constexpr int kLinSmem = 1024 + static_cast<int>(kOffLinStage + kEpiWarps * kStageWarpBytes);
 static_assert(kEpiWarp0 + kEpiWarps == kLinThreads / 32, "warp roles");
-static_assert(kLinSmem <= 232448, "linear tiles exceed shared memory");
+
+// The output tile's width GN (TMEM columns of one accumulator): 256, or 128 for outputs whose
+// width is an odd multiple of 128 (DeiT-S's 384, 1152, 1536).
+template <int GN>
+struct LinCfg {
+    static constexpr int kEpiCols = GN / (kEpiWarps / 4);  // columns per epilogue warp (64 or 32)
+    static constexpr uint32_t kWBytes = GN * GK * 2;
+    static constexpr uint32_t kStageBytes = kXBytes + kWBytes;
+    static constexpr uint32_t kTmemCols = 2 * GN;
+    static constexpr uint32_t kOffBar = kLinStages * kStageBytes;
+    static constexpr uint32_t kOffStage = kOffBar + 256;
+    static constexpr int kSmem = 1024 + static_cast<int>(kOffStage + kEpiWarps * kStageWarpBytes);
+    static_assert(kEpiCols % 32 == 0 && kSmem <= 232448, "linear tile configuration");
+};
 constexpr uint64_t kLinDrainNs = 2000000000ull;
 
 struct LinBars {
@@ -119,9 +125,14 @@ __device__ __forceinline__ void lin_arrive(uint64_t *bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+template <int GN>
 __global__ void __launch_bounds__(kLinThreads, 1)
     linear_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const LinParams p)
 {
+    using Cfg = LinCfg<GN>;
+    constexpr int kEpiCols = Cfg::kEpiCols;
+    constexpr uint32_t kLinStageBytes = Cfg::kStageBytes, kLinTmemCols = Cfg::kTmemCols;
+    constexpr uint32_t kOffLinBar = Cfg::kOffBar, kOffLinStage = Cfg::kOffStage;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     LinBars *bars = reinterpret_cast<LinBars *>(base + kOffLinBar);
@@ -457,6 +468,7 @@ bool make_tmap_2d(CUtensorMap *map, const void *ptr, int64_t rows, int K, int bo
     return r == CUDA_SUCCESS;
 }
 
+template <int GN>
 cudaError_t set_linear_smem()
 {
     static std::mutex mu;
@@ -468,18 +480,15 @@ cudaError_t set_linear_smem()
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 64 && done[dev])
         return cudaSuccess;
-    e = cudaFuncSetAttribute(linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kLinSmem);
+    e = cudaFuncSetAttribute(linear_kernel<GN>, cudaFuncAttributeMaxDynamicSharedMemorySize, LinCfg<GN>::kSmem);
     if (e == cudaSuccess && dev < 64)
         done[dev] = true;
     return e;
 }
 
-}  // namespace
-
-cudaError_t launch_linear(const LinearArgs &a, int num_sms, cudaStream_t stream)
+template <int GN>
+cudaError_t launch_linear_gn(const LinearArgs &a, int num_sms, cudaStream_t stream)
 {
-    if (a.M == 0)
-        return cudaSuccess;
     alignas(64) CUtensorMap tx, tw;
     if (!make_tmap_2d(&tx, a.x, a.M, a.K, GM) || !make_tmap_2d(&tw, a.w, a.N, a.K, GN))
         return cudaErrorInvalidValue;
@@ -497,12 +506,23 @@ cudaError_t launch_linear(const LinearArgs &a, int num_sms, cudaStream_t stream)
     p.act = a.act;
     p.err = a.err;
     p.wait_ns = a.wait_ns;
-    cudaError_t e = set_linear_smem();
+    cudaError_t e = set_linear_smem<GN>();
     if (e != cudaSuccess)
         return e;
     const int64_t tiles = ((a.M + GM - 1) / GM) * (a.N / GN);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-    return launch_pdl(linear_kernel, dim3(grid), dim3(kLinThreads), kLinSmem, stream, tx, tw, p);
+    return launch_pdl(linear_kernel<GN>, dim3(grid), dim3(kLinThreads), LinCfg<GN>::kSmem, stream, tx, tw, p);
+}
+
+}  // namespace
+
+cudaError_t launch_linear(const LinearArgs &a, int num_sms, cudaStream_t stream)
+{
+    if (a.M == 0)
+        return cudaSuccess;
+    // the widest tile that does not straddle two outputs
+    return (a.N / a.n_outs) % 256 == 0 ? launch_linear_gn<256>(a, num_sms, stream)
+                                       : launch_linear_gn<128>(a, num_sms, stream);
 }
 
 cudaError_t launch_layernorm(const void *x, const void *gamma, const void *beta, void *y, int64_t M,

@@ -297,3 +297,44 @@ def test_microbench_library_exports_and_validates():
     assert mb.rra_mb_ex2_launch(None, 4, 16, None) != 0
     assert mb.rra_mb_ex2_launch(FAKE, 0, 16, None) != 0
     assert mb.rra_mb_ex2_launch(FAKE, 4, 0, None) != 0
+
+
+def _linear(L, x=FAKE, w=FAKE, bias=None, res=None, outs=(FAKE,), M=256, m_dev=None, N=256, K=64, act=0):
+    arr = (ctypes.c_void_p * len(outs))(*outs) if outs is not None else None
+    return L.rra_linear(x, w, bias, res, arr, len(outs) if outs is not None else 0, M, m_dev, N, K, act, None, None)
+
+
+def test_linear_validation_before_any_launch(L):
+    """rra_linear refuses bad arguments before touching the device (these pointers are never
+    dereferenced): every case below is refused, or has M = 0 and succeeds without a launch."""
+    big = 1 << 30
+    assert _linear(L, M=0) == rra.RRA_OK
+    assert _linear(L, x=None) == rra.RRA_ERR_INVALID_ARG
+    assert _linear(L, outs=None) == rra.RRA_ERR_INVALID_ARG
+    assert _linear(L, act=7) == rra.RRA_ERR_INVALID_ARG
+    assert _linear(L, x=FAKE + 8) == rra.RRA_ERR_INVALID_ARG            # misaligned
+    assert _linear(L, K=96) == rra.RRA_ERR_UNSUPPORTED                  # K not a multiple of 64
+    assert _linear(L, N=192) == rra.RRA_ERR_UNSUPPORTED                 # width not a multiple of 128
+    assert _linear(L, N=192, outs=(FAKE + big, FAKE + 2 * big, FAKE + 3 * big)) == rra.RRA_ERR_UNSUPPORTED
+    # outputs overlapping an input or each other
+    assert _linear(L, outs=(FAKE,)) == rra.RRA_ERR_INVALID_ARG          # out == x
+    assert _linear(L, x=FAKE, w=FAKE + big, outs=(FAKE + 2 * big, FAKE + 2 * big + 4096), N=512, M=64) \
+        == rra.RRA_ERR_INVALID_ARG
+    # the residual may be the single output itself, but must not partly overlap it
+    assert _linear(L, M=0, res=FAKE + 2 * big, outs=(FAKE + 2 * big,)) == rra.RRA_OK
+    assert _linear(L, M=4, x=FAKE, w=FAKE + big, res=FAKE + 2 * big + 16, outs=(FAKE + 2 * big,)) == rra.RRA_ERR_INVALID_ARG
+
+
+def test_layernorm_validation_before_any_launch(L):
+    f = ctypes.c_float
+    big = 1 << 30
+    ok = dict(x=FAKE, g=FAKE + big, b=FAKE + 2 * big, y=FAKE + 3 * big)
+
+    def ln(x=ok["x"], g=ok["g"], b=ok["b"], y=ok["y"], M=8, C=768, eps=1e-6):
+        return L.rra_layernorm(x, g, b, y, M, None, C, f(eps), None)
+    assert ln(M=0) == rra.RRA_OK
+    assert ln(x=None) == rra.RRA_ERR_INVALID_ARG
+    assert ln(eps=0.0) == rra.RRA_ERR_INVALID_ARG
+    assert ln(C=12) == rra.RRA_ERR_UNSUPPORTED
+    assert ln(C=4096) == rra.RRA_ERR_UNSUPPORTED
+    assert ln(y=FAKE) == rra.RRA_ERR_INVALID_ARG                        # y over x

@@ -113,6 +113,10 @@ CASES = [
     (300, 768, 3072, 1, rra.RRA_ACT_NONE, True, True),
     (129, 512, 128, 2, rra.RRA_ACT_GELU, False, True),
     (4097, 1024, 256, 4, rra.RRA_ACT_NONE, True, True),
+    # 128-column tiles: DeiT-S widths (odd multiples of 128)
+    (777, 1152, 384, 3, rra.RRA_ACT_NONE, True, False),
+    (300, 1536, 384, 1, rra.RRA_ACT_GELU, True, False),
+    (300, 384, 1536, 1, rra.RRA_ACT_NONE, True, True),
 ]
 
 
@@ -211,6 +215,29 @@ def test_block_stagewise_and_end_to_end():
     # end to end against the oracle's own chain (bf16 at the same stored points): the stages' one-ulp
     # rounding differences propagate through the layers, so this bound is looser; it catches a
     # wrong wiring (a missing residual or a swapped buffer moves values by O(1))
+    want = OB.block(f64(x[:T]), cu_np, {k: f64(v) for k, v in w.items()}, H)["y"]
+    err = np.abs(f64(g(y)) - want)
+    assert float(err.max()) <= 0.0625 and float(err.mean()) <= 2e-3, (float(err.max()), float(err.mean()))
+
+
+def test_deit_s_block_stagewise():
+    """The DeiT-S width (C = 384, H = 6): every GEMM on 128-column tiles; each stage against the
+    oracle on the GPU's own inputs, and the block end to end."""
+    lengths = [197, 40, 0, 150]
+    B, N, H, C, T, cu_np, x, wts, blk = _block_case(lengths, H=6, seed=3)
+    xd, cu = x.cuda(), torch.from_numpy(cu_np).cuda()
+    y = blk(xd, cu, B, N)
+    torch.cuda.synchronize()
+    assert int(blk.err.item()) == 0
+    w = wts
+    g = lambda t: t[:T].cpu()
+    ref, tol = linear_ref(g(blk.h), w["qkv_w"], w["qkv_b"], None, rra.RRA_ACT_NONE)
+    got = np.concatenate([f64(g(blk.q)), f64(g(blk.k)), f64(g(blk.v))], axis=1)
+    assert (np.abs(got - ref) <= tol).all()
+    ref, tol = linear_ref(g(blk.h2), w["fc1_w"], w["fc1_b"], None, rra.RRA_ACT_GELU)
+    assert (np.abs(f64(g(blk.m)) - ref) <= tol).all()
+    ref, tol = linear_ref(g(blk.m), w["fc2_w"], w["fc2_b"], g(blk.x1), rra.RRA_ACT_NONE)
+    assert (np.abs(f64(g(y)) - ref) <= tol).all()
     want = OB.block(f64(x[:T]), cu_np, {k: f64(v) for k, v in w.items()}, H)["y"]
     err = np.abs(f64(g(y)) - want)
     assert float(err.max()) <= 0.0625 and float(err.mean()) <= 2e-3, (float(err.max()), float(err.mean()))
