@@ -5,8 +5,9 @@
 // Each image is scored by a thread-block cluster of up to eight CTAs, so every SM takes part even
 // at small batches (one CTA per image once the batch alone fills the GPU): CTA r of the cluster
 // owns a contiguous slice of the image's tokens, and a warp computes the squared norms of four
-// tokens at a time from coalesced 16-byte loads of their embedding rows.  The squared norm is first accumulated in plain double, one fused multiply-add per input
-// (each square of a 16-bit input is exact in double: at most 22 significant bits); that sum is
+// tokens at a time from coalesced 16-byte loads of their embedding rows.  The squared norm is
+// first accumulated in plain double, one addition per input of its square (exact in fp32: at most
+// 22 significant bits, and bf16 inputs are range-checked against overflow and underflow); that sum is
 // provably exact, in any order, when every square is a multiple of 2^q and the total stays below
 // 2^(q+52), which a token checks from the smallest exponent among its inputs -- true for almost
 // every token of realistic embeddings.  A token that fails the check (a tiny, subnormal, infinite
@@ -17,11 +18,16 @@
 // equals the exact selection whenever every token's squares lie within 2^96 of one another (any
 // realistic embedding; beyond that, only tokens whose exact scores agree to ~2^-96 relative could
 // be ordered differently).  A token's (hi, lo) becomes a 128-bit key whose unsigned order is the
-// score order (0 = not a candidate, then NaN, then the finite scores, then +infinity); each CTA
-// writes its keys into the shared memory of every CTA of the cluster (distributed shared memory),
-// one cluster barrier publishes them, and each CTA then ranks its own tokens: a candidate's rank
-// is the number of candidates that beat it (a higher key, or an equal key and a lower index), and
-// it is kept when that rank is below k_b -- N comparisons per token, spread over a warp, no sort.
+// score order (0 = not a candidate, then NaN, then the finite scores, then +infinity).  Each CTA
+// writes its keys to its own shared memory; the threads then send them, one (token, CTA) pair
+// each, to the other CTAs of the cluster (distributed shared memory), and one cluster barrier
+// publishes them.  Each CTA then ranks its own tokens: a candidate's rank is the number of
+// candidates that beat it (a higher key, or an equal key and a lower index), and it is kept when
+// that rank is below k_b -- N comparisons per token, no sort.  The comparisons run on the keys
+// rounded to fp32 (a monotone rounding: a higher fp32 key is a higher score), one lane per token
+// against broadcast reads of all N keys, the key range split over the warps when a CTA has few
+// tokens; only a token whose fp32 key another token shares is settled on the full keys.  In
+// threshold mode a token's own key decides, and no keys are exchanged.
 #include <cuda_fp16.h>
 
 #include <mutex>
@@ -88,6 +94,19 @@ __device__ __forceinline__ bool key_greater(const Key &a, const Key &b)
     return a.hi > b.hi || (a.hi == b.hi && a.lo > b.lo);
 }
 
+// A key rounded to fp32, in the same (non-strict) order: -2 not a candidate, -1 NaN, else RN(S)
+// rounded to fp32 (a monotone map of RN(S), so a higher fp32 key means a higher exact score).
+__device__ __forceinline__ float key_float(const Key &k)
+{
+    if (k.hi == 0ull)
+        return -2.0f;
+    if (k.hi == 1ull)
+        return -1.0f;
+    return __double2float_rn(__longlong_as_double(static_cast<long long>(k.hi - 2ull)));
+}
+
+constexpr float kPadKeyF = -3.0f;  // fp32 key of the padding past N: below every token's
+
 __device__ __forceinline__ uint32_t cluster_rank()
 {
     uint32_t r;
@@ -109,6 +128,13 @@ __device__ __forceinline__ void st_cluster_key(const Key *local, uint32_t rank, 
     uint32_t remote;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
     asm volatile("st.shared::cluster.v2.u64 [%0], {%1, %2};" ::"r"(remote), "l"(k.hi), "l"(k.lo) : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_f32(const float *local, uint32_t rank, float v)
+{
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
 }
 
 __device__ __forceinline__ void cluster_sync_all()
@@ -201,23 +227,34 @@ __global__ void __launch_bounds__(kMaskThreads, 4) l2_mask_kernel(const uint16_t
                                                                 const uint8_t *prev, uint8_t *mask)
 {
     extern __shared__ __align__(16) uint8_t sm[];
-    Key *keys = reinterpret_cast<Key *>(sm);  // [N]: the keys of every token of the image
+    const int N4 = (N + 3) & ~3;
+    Key *keys = reinterpret_cast<Key *>(sm);                  // [N]: the keys of every token of the image
+    float *keyf = reinterpret_cast<float *>(keys + N);        // [N4]: the same keys rounded to fp32, padded
+    uint32_t *cnt = reinterpret_cast<uint32_t *>(keyf + N4);  // [n1 - n0]: rank counts of this CTA's tokens
     const uint32_t cs = cluster_size();
     const uint32_t rank = cluster_rank();
     const int b = static_cast<int>(blockIdx.x / cs);
     const int per_cta = (N + static_cast<int>(cs) - 1) / static_cast<int>(cs);
     const int n0 = static_cast<int>(rank) * per_cta;
     const int n1 = min(N, n0 + per_cta);
+    const int T = max(0, n1 - n0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row0 = static_cast<int64_t>(b) * N;
     const int nchunks = C / 8;
+    for (int i = threadIdx.x; i < T; i += kMaskThreads)
+        cnt[i] = 0u;
+    if (threadIdx.x < N4 - N)
+        keyf[N + threadIdx.x] = kPadKeyF;
     pdl_trigger();
     pdl_wait();  // the embeddings and the previous stage's mask may come from the previous kernel
 
     // ---- scores of this CTA's tokens: a warp takes kTokPerWarp tokens at a time (n, n + 8, ...,
-    // all their loads of a pass in flight together), then writes their keys to every CTA of the
-    // cluster
+    // all their loads of a pass in flight together) and writes their keys to this CTA's shared
+    // memory
     for (int nb = n0 + warp; nb < n1; nb += kTokPerWarp * kMaskWarps) {
+        // candidacy of the group's tokens (lane t: token t), loaded alongside the embeddings
+        const int nl = nb + lane * kMaskWarps;
+        const bool cand_l = lane < kTokPerWarp && nl < n1 && nl >= 1 && (prev == nullptr || prev[row0 + nl] != 0);
         double acc[kTokPerWarp];
         uint32_t tmin[kTokPerWarp], tmax[kTokPerWarp];  // 16x2 magnitude bounds
 #pragma unroll
@@ -262,6 +299,7 @@ __global__ void __launch_bounds__(kMaskThreads, 4) l2_mask_kernel(const uint16_t
                 }
             }
         }
+        const uint32_t cand_bits = __ballot_sync(0xffffffffu, cand_l);
 #pragma unroll
         for (int t = 0; t < kTokPerWarp; ++t) {
             const int n = nb + t * kMaskWarps;
@@ -277,43 +315,99 @@ __global__ void __launch_bounds__(kMaskThreads, 4) l2_mask_kernel(const uint16_t
             else
                 k = {static_cast<unsigned long long>(__double_as_longlong(acc[t])) + 2ull, ordered_bits(0.0)};
             if (lane == 0 && n < n1) {
-                const bool cand = n >= 1 && (prev == nullptr || prev[row0 + n] != 0);
-                if (!cand)
+                if (((cand_bits >> t) & 1u) == 0u)
                     k = {0ull, 0ull};
-                for (uint32_t r = 0; r < cs; ++r)
-                    st_cluster_key(keys + n, r, k);
+                keys[n] = k;
+                keyf[n] = key_float(k);
             }
         }
     }
+    __syncthreads();  // this CTA's keys are complete
+
+    if (k_keep == nullptr) {
+        // ---- threshold mode: each token's own key decides (exact S >= t: RN(S) > t, or
+        // RN(S) == t and S - RN(S) >= 0); NaN and non-candidates never pass
+        for (int n = n0 + static_cast<int>(threadIdx.x); n < n1; n += kMaskThreads) {
+            const Key kn = keys[n];
+            uint8_t keep = 0;
+            if (n == 0) {
+                keep = 1;  // CLS
+            } else if (kn.hi > 1ull) {
+                const double h = __longlong_as_double(static_cast<long long>(kn.hi - 2ull));
+                keep = (h > thr_sq || (h == thr_sq && kn.lo >= 0x8000000000000000ull)) ? 1 : 0;
+            }
+            mask[row0 + n] = keep;
+        }
+        return;  // no shared memory of another CTA was touched
+    }
+
+    // ---- the other CTAs of the cluster receive this CTA's keys (one store per thread and item)
+    for (int i = static_cast<int>(threadIdx.x); i < T * static_cast<int>(cs - 1); i += kMaskThreads) {
+        const int n = n0 + i % T;
+        uint32_t r = static_cast<uint32_t>(i / T);
+        r += r >= rank ? 1u : 0u;
+        st_cluster_key(keys + n, r, keys[n]);
+        st_cluster_f32(keyf + n, r, keyf[n]);
+    }
     cluster_sync_all();  // every key of the image is now in this CTA's shared memory
 
-    // ---- selection of this CTA's tokens
-    const int kb = k_keep != nullptr ? k_keep[b] : 0;
-    for (int n = n0 + warp; n < n1; n += kMaskWarps) {
-        const Key kn = keys[n];
-        uint8_t keep;
-        if (n == 0) {
-            keep = 1;  // CLS
-        } else if (kn.hi == 0) {
-            keep = 0;  // not a candidate
-        } else if (k_keep != nullptr) {
-            // non-candidates have key 0 and never beat a candidate
-            int r = 0;
-            for (int m = 1 + lane; m < N; m += 32) {
-                const Key km = keys[m];
-                r += (key_greater(km, kn) || (km.hi == kn.hi && km.lo == kn.lo && m < n)) ? 1 : 0;
-            }
-            r = __reduce_add_sync(0xffffffffu, r);
-            keep = r < kb ? 1 : 0;
-        } else if (kn.hi == 1) {
-            keep = 0;  // NaN never reaches a threshold
-        } else {
-            // exact S >= t:  RN(S) > t, or RN(S) == t and S - RN(S) >= 0
-            const double h = __longlong_as_double(static_cast<long long>(kn.hi - 2ull));
-            keep = (h > thr_sq || (h == thr_sq && kn.lo >= 0x8000000000000000ull)) ? 1 : 0;
+    // ---- ranks of this CTA's tokens: lane = token (32 per group), the N keys split into S slices
+    // across warps when the CTA has few groups; fp32 keys first (gt | eq << 16 per token), the
+    // 128-bit keys only for tokens whose fp32 key is shared
+    const int G = (T + 31) / 32;
+    const int S = G >= kMaskWarps ? 1 : kMaskWarps / max(G, 1);
+    const int Q = N4 / 4;
+    const float4 *kf4 = reinterpret_cast<const float4 *>(keyf);
+    for (int it = warp; it < G * S; it += kMaskWarps) {
+        const int g = it / S, s = it % S;
+        const int n = n0 + g * 32 + lane;
+        const float fn = n < n1 ? keyf[n] : 0.0f;
+        uint32_t c = 0u;
+        const int qe = (s + 1) * Q / S;
+#pragma unroll 4
+        for (int q = s * Q / S; q < qe; ++q) {
+            const float4 f = kf4[q];  // the same address across the warp: a broadcast
+            c += (f.x > fn ? 1u : 0u) + (f.x == fn ? 0x10000u : 0u);
+            c += (f.y > fn ? 1u : 0u) + (f.y == fn ? 0x10000u : 0u);
+            c += (f.z > fn ? 1u : 0u) + (f.z == fn ? 0x10000u : 0u);
+            c += (f.w > fn ? 1u : 0u) + (f.w == fn ? 0x10000u : 0u);
         }
-        if (lane == 0)
-            mask[row0 + n] = keep;
+        if (n < n1)
+            atomicAdd(cnt + (n - n0), c);
+    }
+    __syncthreads();
+
+    const int kb = k_keep[b];
+    for (int g = warp; g < G; g += kMaskWarps) {
+        const int n = n0 + g * 32 + lane;
+        const bool valid = n < n1;
+        const Key kn = valid ? keys[n] : Key{0ull, 0ull};
+        const uint32_t c = valid ? cnt[n - n0] : 0u;
+        const bool cand = valid && n != 0 && kn.hi != 0ull;
+        // rank = candidates with a higher key or an equal key and a lower index; with no other
+        // token at the same fp32 key that is the count of higher fp32 keys (the rounding is
+        // monotone), otherwise the tied tokens are compared on their full keys
+        int r = static_cast<int>(c & 0xFFFFu);
+        uint32_t tied = __ballot_sync(0xffffffffu, cand && (c >> 16) > 1u);
+        while (tied != 0u) {
+            const int src = __ffs(tied) - 1;
+            tied &= tied - 1u;
+            const int nt = n0 + g * 32 + src;
+            const Key kt = keys[nt];
+            const float ft = keyf[nt];
+            int e = 0;
+            for (int m = lane; m < N; m += 32) {
+                if (m != nt && keyf[m] == ft) {
+                    const Key km = keys[m];
+                    e += (key_greater(km, kt) || (km.hi == kt.hi && km.lo == kt.lo && m < nt)) ? 1 : 0;
+                }
+            }
+            e = __reduce_add_sync(0xffffffffu, e);
+            if (lane == src)
+                r += e;
+        }
+        if (valid)
+            mask[row0 + n] = (n == 0 || (cand && r < kb)) ? 1 : 0;
     }
 }
 
@@ -324,6 +418,13 @@ __global__ void __launch_bounds__(kMaskThreads, 4) l2_mask_kernel(const uint16_t
 // shared-memory size, from the occupancy query (which knows the GPU's actual GPC layout);
 // -1 where a size cannot be used.  Queried once per device and size, then cached.
 static_assert(kMaxCluster == 8, "cluster sizes 1, 2, 4, 8 are queried");
+
+// Shared memory of the kernel: the 128-bit keys [N], the fp32 keys [N rounded up to 4] and the
+// rank counts of one CTA's tokens (at most N).
+constexpr int mask_smem_bytes(int N)
+{
+    return N * static_cast<int>(sizeof(Key)) + ((N + 3) & ~3) * 4 + N * 4;
+}
 
 template <bool kBF16>
 struct ClusterFit {
@@ -415,7 +516,7 @@ template <bool kBF16>
 cudaError_t launch_mask_variant(const uint16_t *x, int B, int N, int C, const int32_t *k_keep, double thr_sq,
                                 const uint8_t *prev, uint8_t *mask, int num_sms, cudaStream_t stream)
 {
-    const int smem = N * static_cast<int>(sizeof(Key));
+    const int smem = mask_smem_bytes(N);
     cudaError_t e = set_mask_smem<kBF16>(smem);
     if (e != cudaSuccess)
         return e;
@@ -440,7 +541,7 @@ cudaError_t launch_mask_variant(const uint16_t *x, int B, int N, int C, const in
 
 }  // namespace
 
-static_assert(kMaskMaxN * sizeof(Key) <= 227 * 1024, "keys exceed shared memory at the largest N");
+static_assert(mask_smem_bytes(kMaskMaxN) <= 227 * 1024, "keys exceed shared memory at the largest N");
 
 cudaError_t launch_l2_mask(const void *x, int B, int N, int C, bool bf16, const int32_t *k_keep, double thr_sq,
                            const uint8_t *prev, uint8_t *mask, int num_sms, cudaStream_t stream)
