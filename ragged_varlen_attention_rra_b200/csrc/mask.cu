@@ -45,12 +45,6 @@ constexpr int kMaxCluster = 8;  // portable cluster size
 constexpr int kChunksPerPass = 2;  // 16-byte loads in flight per lane and token
 constexpr int kTokPerWarp = 4;     // tokens a warp scores at once
 
-// Two copies of the value 1.0 in the 16-bit type.
-template <bool kBF16>
-struct One2 {
-    static constexpr uint32_t value = kBF16 ? 0x3F803F80u : 0x3C003C00u;
-};
-
 struct Key {
     unsigned long long hi, lo;
 };
@@ -153,30 +147,27 @@ __device__ __forceinline__ float2 widen2(uint32_t w)
         return __half22float2(*reinterpret_cast<const __half2 *>(&w));
 }
 
-// True when the plain double accumulation of the squares was exact, so `acc` is the exact sum.
-// tmin2 / tmax2 hold, per 16-bit half, the minimum / maximum magnitude bits (sign cleared) seen.
-// Required: no zero input (a zero goes to the slow path, which is exact for it too), no
-// infinite or NaN input, and for bf16 every |x| in [2^-63, 2^64), so that each square x * x is
-// exact in fp32 (at most 16 significant bits, exponent in range; fp16 squares always are); and
-// every square is a multiple of 2^q (q = twice the last-bit exponent of the smallest-exponent
-// input) while the sum stays below 2^(q+52) -- then every partial sum, in any order, is an
-// integer multiple of 2^q below 2^(q+53), representable exactly, so no addition rounded (the
-// factor-2 margin covers the rounding of `acc` itself when the condition fails).
+// True when the plain double accumulation of the squares was exact, so `acc` is the exact sum;
+// sqmin is the smallest fp32 square seen.  Required: every square exact in fp32 -- it has at most
+// 16 (bf16) or 22 (fp16) significant bits, so it is exact unless it overflows (an input of 2^64
+// or more, or an infinite or NaN one: `acc` is then infinite or NaN and the final test fails) or
+// leaves fp32's normal range at the bottom (a zero or subnormal sqmin: refused; a zero input goes
+// to the slow path, which is exact for it too); and every square a multiple of 2^q, q = twice
+// the last-bit exponent of the smallest input, while the sum stays below 2^(q+52) -- then every
+// partial sum, in any order, is an integer multiple of 2^q below 2^(q+53), representable exactly,
+// so no addition rounded (the factor-2 margin covers the rounding of `acc` itself when the
+// condition fails).  The smallest input has the smallest square; its exponent e is half the
+// square's exponent, rounded down, and its last bit is 2^(e-7) for bf16 and at least 2^(e-10) for
+// fp16 (a subnormal fp16's is 2^-24, coarser, which only makes the test stricter).
 template <bool kBF16>
-__device__ __forceinline__ bool fast_sum_exact(double acc, uint32_t tmin2, uint32_t tmax2)
+__device__ __forceinline__ bool fast_sum_exact(double acc, float sqmin)
 {
-    const uint32_t tmin = min(tmin2 & 0xFFFFu, tmin2 >> 16), tmax = max(tmax2 & 0xFFFFu, tmax2 >> 16);
-    int emin;
-    if constexpr (kBF16) {
-        if (tmin < (64u << 7) || tmax >= (191u << 7))
-            return false;
-        emin = static_cast<int>(tmin >> 7) - 127 - 7;  // last-bit exponent of the smallest input
-    } else {
-        if (tmin == 0u || tmax >= 0x7C00u)
-            return false;
-        emin = max(static_cast<int>(tmin >> 10), 1) - 15 - 10;
-    }
-    return acc < __hiloint2double((2 * emin + 52 + 1023) << 20, 0);  // 2^(q+52), a normal double here
+    const int e2 = static_cast<int>(__float_as_uint(sqmin) >> 23);  // biased exponent, sign 0
+    if (e2 == 0)
+        return false;
+    const int e = (e2 - 127) >> 1;  // arithmetic shift: rounds down for negative exponents
+    const int q = 2 * (e - (kBF16 ? 7 : 10));
+    return acc < __hiloint2double((q + 52 + 1023) << 20, 0);  // 2^(q+52), a normal double here
 }
 
 // Key of a token that the fast path cannot settle: the squared norm in double-double arithmetic
@@ -256,12 +247,11 @@ __global__ void __launch_bounds__(kMaskThreads, 4) l2_mask_kernel(const uint16_t
         const int nl = nb + lane * kMaskWarps;
         const bool cand_l = lane < kTokPerWarp && nl < n1 && nl >= 1 && (prev == nullptr || prev[row0 + nl] != 0);
         double acc[kTokPerWarp];
-        uint32_t tmin[kTokPerWarp], tmax[kTokPerWarp];  // 16x2 magnitude bounds
+        float sqmin[kTokPerWarp];  // smallest square
 #pragma unroll
         for (int t = 0; t < kTokPerWarp; ++t) {
             acc[t] = 0.0;
-            tmin[t] = 0xFFFFFFFFu;
-            tmax[t] = 0u;
+            sqmin[t] = __uint_as_float(0x7F800000u);
         }
         for (int j0 = 0; j0 < nchunks; j0 += 32 * kChunksPerPass) {
             uint4 v[kTokPerWarp][kChunksPerPass];
@@ -272,8 +262,7 @@ __global__ void __launch_bounds__(kMaskThreads, 4) l2_mask_kernel(const uint16_t
 #pragma unroll
                 for (int u = 0; u < kChunksPerPass; ++u) {
                     const int j = j0 + lane + 32 * u;
-                    // padding lanes read the value 1.0 (in range, not zero): no effect on the bounds
-                    v[t][u] = (n < n1 && j < nchunks) ? __ldg(row + j) : make_uint4(One2<kBF16>::value, One2<kBF16>::value, One2<kBF16>::value, One2<kBF16>::value);
+                    v[t][u] = (n < n1 && j < nchunks) ? __ldg(row + j) : make_uint4(0u, 0u, 0u, 0u);  // padding: not accumulated
                 }
             }
 #pragma unroll
@@ -282,18 +271,16 @@ __global__ void __launch_bounds__(kMaskThreads, 4) l2_mask_kernel(const uint16_t
                 for (int u = 0; u < kChunksPerPass; ++u) {
                     const int j = j0 + lane + 32 * u;
                     const uint32_t w[4] = {v[t][u].x, v[t][u].y, v[t][u].z, v[t][u].w};
-                    const uint32_t m0 = w[0] & 0x7FFF7FFFu, m1 = w[1] & 0x7FFF7FFFu, m2 = w[2] & 0x7FFF7FFFu,
-                                   m3 = w[3] & 0x7FFF7FFFu;
-                    tmin[t] = __vimin3_u16x2(tmin[t], __vimin3_u16x2(m0, m1, m2), m3);
-                    tmax[t] = __vimax3_u16x2(tmax[t], __vimax3_u16x2(m0, m1, m2), m3);
                     if (j < nchunks) {
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const float2 f = widen2<kBF16>(w[i]);
                             // exact fp32 squares (checked by fast_sum_exact), exact widening, one
                             // rounded-to-nearest double addition each
-                            acc[t] = __dadd_rn(acc[t], static_cast<double>(__fmul_rn(f.x, f.x)));
-                            acc[t] = __dadd_rn(acc[t], static_cast<double>(__fmul_rn(f.y, f.y)));
+                            const float sx = __fmul_rn(f.x, f.x), sy = __fmul_rn(f.y, f.y);
+                            sqmin[t] = fminf(sqmin[t], fminf(sx, sy));
+                            acc[t] = __dadd_rn(acc[t], static_cast<double>(sx));
+                            acc[t] = __dadd_rn(acc[t], static_cast<double>(sy));
                         }
                     }
                 }
@@ -306,11 +293,10 @@ __global__ void __launch_bounds__(kMaskThreads, 4) l2_mask_kernel(const uint16_t
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) {
                 acc[t] = __dadd_rn(acc[t], __shfl_xor_sync(0xffffffffu, acc[t], off));
-                { const uint32_t o = __shfl_xor_sync(0xffffffffu, tmin[t], off); tmin[t] = __vimin3_u16x2(tmin[t], o, o); }
-                { const uint32_t o = __shfl_xor_sync(0xffffffffu, tmax[t], off); tmax[t] = __vimax3_u16x2(tmax[t], o, o); }
+                sqmin[t] = fminf(sqmin[t], __shfl_xor_sync(0xffffffffu, sqmin[t], off));
             }
             Key k;
-            if (!fast_sum_exact<kBF16>(acc[t], tmin[t], tmax[t]) && n < n1)
+            if (!fast_sum_exact<kBF16>(acc[t], sqmin[t]) && n < n1)
                 k = slow_key<kBF16>(x + (row0 + n) * C, nchunks, lane);  // warp-uniform, rare
             else
                 k = {static_cast<unsigned long long>(__double_as_longlong(acc[t])) + 2ull, ordered_bits(0.0)};
