@@ -139,6 +139,35 @@ def test_linear_matches_oracle(case):
     assert not bad.any(), (int(bad.sum()), float(np.abs(got - ref).max()))
 
 
+def test_gelu_epilogue_across_its_range():
+    """The GELU epilogue alone: an identity weight makes each output GELU of one bf16 input
+    (the single-term dot product is exact in fp32).  Every bf16 value in [-16, 16] -- the far
+    negative tail, where the output is tiny and 1 + erf cancels, included -- must round to the
+    bf16 value of the exact GELU, up to one unit in the last place and the approximation's own
+    error (below 5e-6 |x|; Abramowitz and Stegun 7.1.28 for erfc)."""
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    with np.errstate(invalid="ignore"):
+        vals = (bits << 16).view(np.float32)
+    vals = vals[np.isfinite(vals) & (np.abs(vals) <= 16.0)]
+    K = N = 128
+    M = -(-vals.size // K)
+    flat = np.zeros(M * K, np.float32)
+    flat[:vals.size] = vals
+    x = torch.from_numpy(flat.reshape(M, K)).to(bf)
+    w = torch.eye(N, K, dtype=bf)
+    y = torch.empty(M, N, dtype=bf, device="cuda")
+    rra.rra_linear(x.cuda(), w.cuda(), [y], act=rra.RRA_ACT_GELU)
+    torch.cuda.synchronize()
+    z = f64(x)
+    ref = OB.bf16_round(OB.gelu(z))
+    err = np.abs(f64(y) - ref)
+    tol = ulp_bf16(ref) + 5e-6 * np.abs(z)
+    assert (err <= tol).all(), (float(err.max()), float(z.ravel()[np.argmax((err - tol).ravel())]))
+    # the tail is really formed: large negative inputs give tiny negative outputs, not zero
+    tail = (z < -4) & (z > -8)
+    assert (f64(y)[tail] < 0).all()
+
+
 def test_linear_residual_in_place_and_row_count_from_device():
     M, N, K = 600, 768, 768
     x = rand_bf16((M, K), seed=11).cuda()
