@@ -109,11 +109,15 @@ constexpr int kItemTable = 56;
 constexpr uint32_t kBarBytes = 640;
 constexpr uint32_t kOffItems = kOffBar + kBarBytes;
 constexpr uint32_t kOffIdx = kOffItems + kItemTable * 24;
-// tile_pre[B+1], then cu[B+1]: after the list slots on the fused path, in their place otherwise
+// fused: a block of zero bytes, the source of the bulk stores that clear pruned output rows
+constexpr uint32_t kZeroBytes = 4096;
+constexpr uint32_t kOffZero = kOffIdx + kIdxSlots * kIdxSlotBytes;
+// tile_pre[B+1], then cu[B+1]: after the list slots and the zero block on the fused path, in
+// their place otherwise
 template <bool kFused>
 constexpr uint32_t off_tile()
 {
-    return kFused ? kOffIdx + kIdxSlots * kIdxSlotBytes : kOffIdx;
+    return kFused ? kOffZero + kZeroBytes : kOffIdx;
 }
 template <bool kFused>
 constexpr int smem_bytes(int B)
@@ -583,43 +587,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- work list: tile_pre[b] = number of 128-row query tiles of images < b; cu staged too.
     if constexpr (kFused) {
-        // kept tokens per image, counted from 16-byte chunks of the flat mask into cu_s[b+1]
+        // kept tokens per image, counted from 16-byte chunks of the flat mask into cu_s[b+1]: a
+        // thread per image, all of its chunks (up to kCntBatch at a time) loaded before any is
+        // counted, so one memory round trip serves kThreads images (the whole batch at B <= 512)
         const uintptr_t addr = reinterpret_cast<uintptr_t>(p.mask);
         const int off = static_cast<int>(addr & 15u);
         const uint4 *m16 = reinterpret_cast<const uint4 *>(addr - off);
-        // a warp per image, six images per warp at a time: lane l loads 16-byte chunks l,
-        // l + 32, ... of each image's byte range (coalesced), all loads of a round issued before
-        // any is used; the counts are summed with one warp reduction per image
-        constexpr int kImg = 6;
-        for (int bw = warp * kImg; bw < B; bw += (kThreads / 32) * kImg) {
-            int64_t lo[kImg], c0[kImg], c1[kImg];
-            int cnt[kImg];
+        constexpr int kCntBatch = 16;
+        for (int b = tid; b < B; b += kThreads) {
+            const int64_t lo = static_cast<int64_t>(b) * p.N, hi = lo + p.N;
+            const int64_t c0 = (off + lo) >> 4, c1 = (off + hi + 15) >> 4;
+            int cnt = 0;
+            for (int64_t j0 = c0; j0 < c1; j0 += kCntBatch) {
+                uint4 w[kCntBatch];
 #pragma unroll
-            for (int i = 0; i < kImg; ++i) {
-                const int b = min(bw + i, B - 1);
-                lo[i] = static_cast<int64_t>(b) * p.N;
-                c0[i] = (off + lo[i]) >> 4;
-                c1[i] = (off + lo[i] + p.N + 15) >> 4;
-                cnt[i] = 0;
+                for (int i = 0; i < kCntBatch; ++i)
+                    w[i] = j0 + i < c1 ? __ldg(m16 + j0 + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int i = 0; i < kCntBatch; ++i)
+                    cnt += __popc(kept_bits16_(w[i]) & range16_((j0 + i) * 16 - off, lo, hi));
             }
-            for (int k = 0; k * 32 < p.N / 16 + 2; ++k) {
-                uint4 w[kImg];
-#pragma unroll
-                for (int i = 0; i < kImg; ++i) {
-                    const int64_t j = c0[i] + lane + 32 * k;
-                    w[i] = j < c1[i] ? __ldg(m16 + j) : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int i = 0; i < kImg; ++i)
-                    cnt[i] += __popc(kept_bits16_(w[i]) &
-                                     range16_((c0[i] + lane + 32 * k) * 16 - off, lo[i], lo[i] + p.N));
-            }
-#pragma unroll
-            for (int i = 0; i < kImg; ++i) {
-                const int sum = __reduce_add_sync(0xffffffffu, cnt[i]);
-                if (lane == 0 && bw + i < B)
-                    cu_s[bw + i + 1] = sum;
-            }
+            cu_s[b + 1] = cnt;
         }
         __syncthreads();
     }
@@ -1019,24 +1007,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (kFused && warp == kZeroWarp) {
         // ================================================================ pruned rows
         // The block's contiguous share of the B*N padded rows: every pruned one becomes zero bytes
-        // (all heads, 16-byte stores along the row), concurrently with the attention work, which
-        // never writes those rows.
+        // (all heads), concurrently with the attention work, which never writes those rows.  Each
+        // lane clears its own pruned rows with bulk copies from a zeroed block of shared memory
+        // (the copy engine moves the bytes; the warp only issues), then waits for them to land.
+        uint8_t *zero = base + kOffZero;
+        for (uint32_t i = 16u * lane; i < kZeroBytes; i += 16u * 32u)
+            *reinterpret_cast<uint4 *>(zero + i) = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();  // the zeros are visible to the copy engine
+        __syncwarp();
         const int64_t rows = static_cast<int64_t>(B) * p.N;
         const int64_t share = (rows + gridDim.x - 1) / gridDim.x;
         const int64_t r0 = static_cast<int64_t>(blockIdx.x) * share;
         const int64_t r1 = min(rows, r0 + share);
-        const int row_vecs = H * ((p.out_dt == RRA_F32 ? 4 : 2) * kD / 16);
-        for (int64_t t0 = r0; t0 < r1; t0 += 32) {
-            const bool pruned = t0 + lane < r1 && p.mask[t0 + lane] == 0;
-            unsigned bal = __ballot_sync(0xffffffffu, pruned);
-            while (bal != 0u) {
-                const int64_t t = t0 + __ffs(bal) - 1;
-                bal &= bal - 1u;
-                uint4 *y = reinterpret_cast<uint4 *>(p.out) + t * row_vecs;
-                for (int v = lane; v < row_vecs; v += 32)
-                    y[v] = make_uint4(0, 0, 0, 0);
-            }
+        const uint32_t row_bytes = static_cast<uint32_t>(H) * (p.out_dt == RRA_F32 ? 4u : 2u) * kD;
+        for (int64_t t = r0 + lane; t < r1; t += 32) {
+            if (p.mask[t] != 0)
+                continue;
+            uint8_t *y = static_cast<uint8_t *>(p.out) + t * row_bytes;
+            for (uint32_t o = 0; o < row_bytes; o += kZeroBytes)
+                bulk_store(y + o, zero, min(kZeroBytes, row_bytes - o));
         }
+        bulk_commit();
+        bulk_wait_all();
     } else if (warp >= kSoftmaxWarp0 && warp < kSoftmaxWarp0 + kSoftmaxWarps) {
         // ================================================================ softmax + epilogue
         // Group g (4 warps) takes items n = g, g+2, ...; thread r of the group owns row r of the
