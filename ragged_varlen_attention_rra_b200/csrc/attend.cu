@@ -587,27 +587,65 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- work list: tile_pre[b] = number of 128-row query tiles of images < b; cu staged too.
     if constexpr (kFused) {
-        // kept tokens per image, counted from 16-byte chunks of the flat mask into cu_s[b+1]: a
-        // thread per image, all of its chunks (up to kCntBatch at a time) loaded before any is
-        // counted, so one memory round trip serves kThreads images (the whole batch at B <= 512)
+        // kept tokens per image, counted from 16-byte chunks of the flat mask into cu_s[b+1], by
+        // whichever of two layouts takes fewer dependent memory round trips (a block-uniform
+        // choice): a warp per image (lanes over the image's chunks, coalesced, six images per warp
+        // at a time, one warp reduction each) for few or long images; a thread per image (all of
+        // its chunks, up to kCntBatch, loaded before any is counted) for many short ones
         const uintptr_t addr = reinterpret_cast<uintptr_t>(p.mask);
         const int off = static_cast<int>(addr & 15u);
         const uint4 *m16 = reinterpret_cast<const uint4 *>(addr - off);
-        constexpr int kCntBatch = 16;
-        for (int b = tid; b < B; b += kThreads) {
-            const int64_t lo = static_cast<int64_t>(b) * p.N, hi = lo + p.N;
-            const int64_t c0 = (off + lo) >> 4, c1 = (off + hi + 15) >> 4;
-            int cnt = 0;
-            for (int64_t j0 = c0; j0 < c1; j0 += kCntBatch) {
-                uint4 w[kCntBatch];
+        constexpr int kImg = 6, kCntBatch = 16;
+        const int chunks = p.N / 16 + 2;  // 16-byte chunks an image's bytes can touch, at most
+        const int rounds_warp = (B + (kThreads / 32) * kImg - 1) / ((kThreads / 32) * kImg) * ((chunks + 31) / 32);
+        const int rounds_thread = (B + kThreads - 1) / kThreads * ((chunks + kCntBatch - 1) / kCntBatch);
+        if (rounds_thread < rounds_warp) {
+            for (int b = tid; b < B; b += kThreads) {
+                const int64_t lo = static_cast<int64_t>(b) * p.N, hi = lo + p.N;
+                const int64_t c0 = (off + lo) >> 4, c1 = (off + hi + 15) >> 4;
+                int cnt = 0;
+                for (int64_t j0 = c0; j0 < c1; j0 += kCntBatch) {
+                    uint4 w[kCntBatch];
 #pragma unroll
-                for (int i = 0; i < kCntBatch; ++i)
-                    w[i] = j0 + i < c1 ? __ldg(m16 + j0 + i) : make_uint4(0, 0, 0, 0);
+                    for (int i = 0; i < kCntBatch; ++i)
+                        w[i] = j0 + i < c1 ? __ldg(m16 + j0 + i) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-                for (int i = 0; i < kCntBatch; ++i)
-                    cnt += __popc(kept_bits16_(w[i]) & range16_((j0 + i) * 16 - off, lo, hi));
+                    for (int i = 0; i < kCntBatch; ++i)
+                        cnt += __popc(kept_bits16_(w[i]) & range16_((j0 + i) * 16 - off, lo, hi));
+                }
+                cu_s[b + 1] = cnt;
             }
-            cu_s[b + 1] = cnt;
+        } else {
+            for (int bw = warp * kImg; bw < B; bw += (kThreads / 32) * kImg) {
+                int64_t lo[kImg], c0[kImg], c1[kImg];
+                int cnt[kImg];
+#pragma unroll
+                for (int i = 0; i < kImg; ++i) {
+                    const int b = min(bw + i, B - 1);
+                    lo[i] = static_cast<int64_t>(b) * p.N;
+                    c0[i] = (off + lo[i]) >> 4;
+                    c1[i] = (off + lo[i] + p.N + 15) >> 4;
+                    cnt[i] = 0;
+                }
+                for (int k = 0; k * 32 < chunks; ++k) {
+                    uint4 w[kImg];
+#pragma unroll
+                    for (int i = 0; i < kImg; ++i) {
+                        const int64_t j = c0[i] + lane + 32 * k;
+                        w[i] = j < c1[i] ? __ldg(m16 + j) : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int i = 0; i < kImg; ++i)
+                        cnt[i] += __popc(kept_bits16_(w[i]) &
+                                         range16_((c0[i] + lane + 32 * k) * 16 - off, lo[i], lo[i] + p.N));
+                }
+#pragma unroll
+                for (int i = 0; i < kImg; ++i) {
+                    const int sum = __reduce_add_sync(0xffffffffu, cnt[i]);
+                    if (lane == 0 && bw + i < B)
+                        cu_s[bw + i + 1] = sum;
+                }
+            }
         }
         __syncthreads();
     }
