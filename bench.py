@@ -150,6 +150,9 @@ def source_hash(rel):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
+E2E_CHUNK = 64  # images per chunk of the end-to-end (host memory in and out) measurement
+
+
 def ncu_traffic(kernel, workload):
     """DRAM bytes per launch from a committed ncu summary, if the kernel source still matches."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
@@ -775,23 +778,15 @@ def main_gpu(args):
     # ---- end to end through the public API: pinned host inputs in, padded result out
     e2e = None
     if not args.no_e2e and not args.profile:
-        host_in = [t.pin_memory() for t in (w.q, w.k, w.v)]
-        host_masks = [m.pin_memory() for m in w.masks]
+        host_in = [t.contiguous().pin_memory() for t in (w.q, w.k, w.v)]
+        host_masks = [m.contiguous().pin_memory() for m in w.masks]
         host_out = [torch.empty(pipe.ys[0].shape, dtype=pipe.ys[0].dtype).pin_memory() for _ in w.masks]
-        eq, ek, ev = (torch.empty(w.q.shape, dtype=w.q.dtype, device="cuda") for _ in range(3))
-        emasks = [torch.empty(m.shape, dtype=m.dtype, device="cuda") for m in w.masks]
-        bufs = rra.Buffers(w.B, w.N, w.H, w.q.dtype, out_dtype=out_dtype)
+        hs = rra.HostStream(w.B, w.N, w.H, w.q.dtype, stages=len(w.masks), chunk=E2E_CHUNK, out_dtype=out_dtype,
+                            fused=args.path == "fused")
         e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
         def e2e_step():
-            with torch.cuda.stream(stream):
-                for d, h in zip((eq, ek, ev), host_in):
-                    d.copy_(h, non_blocking=True)
-                for d, h in zip(emasks, host_masks):
-                    d.copy_(h, non_blocking=True)
-                for i, m in enumerate(emasks):
-                    y = rra.forward(m, eq, ek, ev, bufs, stream=stream, fused=args.path == "fused")
-                    host_out[i].copy_(y, non_blocking=True)
+            hs(host_masks, *host_in, host_out, stream=stream)
         for _ in range(max(3, args.warmup)):
             e2e_step()
         torch.cuda.synchronize()
@@ -810,11 +805,12 @@ def main_gpu(args):
         d2h = sum(t.numel() * t.element_size() for t in host_out)
         e2e = {"value": job_throughput(ws, args.steps, T_call, tot), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": tot / args.steps,
-               "api": f"rra.forward (eager, {args.path} path)"}
-        err2 = rra.rra_get_device_error(bufs.err, stream)
+               "api": f"rra.HostStream ({args.path} path, chunks of {min(E2E_CHUNK, w.B)} images: host-to-device copies, "
+                      "kernels and device-to-host copies of successive chunks overlap)"}
+        err2 = rra.rra_get_device_error(hs.err, stream)
         if err2 != 0:
             raise RuntimeError(f"device error {rra.rra_status_string(err2)} in the e2e region")
-        del bufs, eq, ek, ev
+        del hs
 
     mask_producer = None if args.profile else time_mask_producer(w.B, w.N, w.H, w.seed, flush, stream, args.steps,
                                                                  args.warmup, hbm_peak)

@@ -447,3 +447,100 @@ def forward(mask: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tenso
                softmax_scale=softmax_scale, dev_error=bufs.err, stream=stream)
     rra_unpack(bufs.o, bufs.cu, mask, bufs.y, fill_mode=0, dev_error=bufs.err, stream=stream)
     return bufs.y
+
+
+class HostStream:
+    """Pack-attend-unpack of a batch held in pinned host memory, streamed through the GPU in chunks
+    of images (images are independent, so a chunk is a complete call of its own).
+
+    Per chunk: its Q, K, V and masks go host -> device on one stream, the chunk's calls (one per
+    pruning stage, through the same kernels as `forward`) run on a second, and each stage's padded
+    output goes device -> host on a third.  Two sets of device buffers alternate, so the copies of
+    chunk j+1 in, chunk j's kernels and chunk j-1's results out overlap: PCIe carries both
+    directions at once and the kernels hide behind the copies.  Only copies, events and stream
+    waits are issued here; every step of the path runs in the library's kernels.
+    """
+
+    def __init__(self, B: int, N: int, H: int, dtype: torch.dtype, stages: int = 1, chunk: int = 128,
+                 out_dtype: Optional[torch.dtype] = None, fused: bool = True, device="cuda"):
+        _expect(B >= 1 and N >= 1 and H >= 1 and stages >= 1 and chunk >= 1, "HostStream: sizes must be positive")
+        self.B, self.N, self.H, self.stages, self.fused = B, N, H, stages, fused
+        self.chunk = min(chunk, B)
+        od = out_dtype or dtype
+        self.dtype, self.out_dtype = dtype, od
+        c = self.chunk
+        self.sets = []
+        for _ in range(2):
+            st = {"qkv": [torch.empty(c, N, H, 64, dtype=dtype, device=device) for _ in range(3)],
+                  "masks": [torch.empty(c, N, dtype=torch.uint8, device=device) for _ in range(stages)],
+                  "ys": [torch.empty(c, N, H, 64, dtype=od, device=device) for _ in range(stages)],
+                  "cu": torch.empty(c + 1, dtype=torch.int32, device=device),
+                  "in_done": torch.cuda.Event(), "run_done": torch.cuda.Event(), "out_done": torch.cuda.Event()}
+            if not fused:
+                cap = c * N
+                st["packed"] = [torch.empty(cap, H, 64, dtype=dtype, device=device) for _ in range(3)]
+                st["o"] = torch.empty(cap, H, 64, dtype=od, device=device)
+            self.sets.append(st)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.s_in, self.s_run, self.s_out = (torch.cuda.Stream(device=device) for _ in range(3))
+        self.start = torch.cuda.Event()
+
+    def __call__(self, masks: Sequence[torch.Tensor], q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                 outs: Sequence[torch.Tensor], softmax_scale: float = 0.0, stream=None) -> None:
+        """masks: `stages` uint8 [B', N]; q, k, v: [B', N, H, 64]; outs: `stages` [B', N, H, 64] in the
+        output dtype (all pinned host tensors, B' <= B).  The work starts after what is already on
+        `stream`, and `stream` waits for the last copy back, so an event or a synchronisation on
+        `stream` covers the whole call.  Device errors land in self.err."""
+        stream = stream or torch.cuda.current_stream()
+        Bp = q.shape[0]
+        _expect(len(masks) == self.stages and len(outs) == self.stages, f"HostStream: {self.stages} masks and outputs expected")
+        _expect(1 <= Bp <= self.B, f"HostStream: batch {Bp} outside [1, {self.B}]")
+        for t in (q, k, v):
+            _expect(t.device.type == "cpu" and t.is_pinned() and t.is_contiguous() and t.dtype == self.dtype
+                    and tuple(t.shape) == (Bp, self.N, self.H, 64), "HostStream: q/k/v must be pinned host [B', N, H, 64]")
+        for m in masks:
+            _expect(m.device.type == "cpu" and m.is_pinned() and m.is_contiguous() and m.dtype == torch.uint8
+                    and tuple(m.shape) == (Bp, self.N), "HostStream: masks must be pinned host uint8 [B', N]")
+        for o in outs:
+            _expect(o.device.type == "cpu" and o.is_pinned() and o.is_contiguous() and o.dtype == self.out_dtype
+                    and tuple(o.shape) == (Bp, self.N, self.H, 64), "HostStream: outputs must be pinned host [B', N, H, 64]")
+        self.start.record(stream)
+        for s in (self.s_in, self.s_run, self.s_out):
+            s.wait_event(self.start)
+        chunks = list(range(0, Bp, self.chunk))
+        for j, b0 in enumerate(chunks):
+            st = self.sets[j % 2]
+            b1 = min(Bp, b0 + self.chunk)
+            n = b1 - b0
+            if j >= 2:
+                self.s_in.wait_event(st["run_done"])   # chunk j-2's kernels are done with these inputs
+            with torch.cuda.stream(self.s_in):
+                for d, h in zip(st["qkv"], (q, k, v)):
+                    d[:n].copy_(h[b0:b1], non_blocking=True)
+                for d, h in zip(st["masks"], masks):
+                    d[:n].copy_(h[b0:b1], non_blocking=True)
+                st["in_done"].record(self.s_in)
+            self.s_run.wait_event(st["in_done"])
+            if j >= 2:
+                self.s_run.wait_event(st["out_done"])  # chunk j-2's results have left these outputs
+            qd, kd, vd = (t[:n] for t in st["qkv"])
+            for s in range(self.stages):
+                m, y = st["masks"][s][:n], st["ys"][s][:n]
+                if self.fused:
+                    rra_pack_attend_unpack(m, qd, kd, vd, y, st["cu"][:n + 1], softmax_scale=softmax_scale,
+                                           dev_error=self.err, stream=self.s_run)
+                else:
+                    pk = [t[:n * self.N] for t in st["packed"]]
+                    o = st["o"][:n * self.N]
+                    rra_pack(m, [qd, kd, vd], pk, st["cu"][:n + 1], dev_error=self.err, stream=self.s_run)
+                    rra_attend(pk[0], pk[1], pk[2], o, st["cu"][:n + 1], max_seqlen=self.N,
+                               softmax_scale=softmax_scale, dev_error=self.err, stream=self.s_run)
+                    rra_unpack(o, st["cu"][:n + 1], m, y, fill_mode=0, dev_error=self.err, stream=self.s_run)
+            st["run_done"].record(self.s_run)
+            self.s_out.wait_event(st["run_done"])
+            with torch.cuda.stream(self.s_out):
+                for s in range(self.stages):
+                    outs[s][b0:b1].copy_(st["ys"][s][:n], non_blocking=True)
+                st["out_done"].record(self.s_out)
+        for st in self.sets[:min(2, len(chunks))]:
+            stream.wait_event(st["out_done"])
