@@ -399,9 +399,13 @@ __device__ __forceinline__ float warp_sum(float v)
 
 // One warp per row: the row's 16-byte chunks spread over the lanes (chunk c to lane c % 32), the
 // mean, then the variance of (x - mean) (two passes over registers), each a warp reduction in fp32.
-__global__ void __launch_bounds__(kLnThreads) layernorm_kernel(const uint16_t *x, const uint16_t *gamma,
-                                                               const uint16_t *beta, uint16_t *y, int64_t M_max,
-                                                               const int32_t *m_dev, int C, float eps)
+// kChunks = chunks per lane (C / 256 rounded up): a narrow row needs few registers, so more blocks
+// fit on an SM and more rows are in flight -- the kernel streams each row once, so rows in flight
+// set its bandwidth.
+template <int kChunks>
+__global__ void __launch_bounds__(kLnThreads, kChunks <= 4 ? 4 : 2)
+    layernorm_kernel(const uint16_t *x, const uint16_t *gamma, const uint16_t *beta, uint16_t *y, int64_t M_max,
+                     const int32_t *m_dev, int C, float eps)
 {
     pdl_trigger();
     pdl_wait();
@@ -412,10 +416,10 @@ __global__ void __launch_bounds__(kLnThreads) layernorm_kernel(const uint16_t *x
     for (int64_t row = static_cast<int64_t>(blockIdx.x) * (kLnThreads / 32) + (threadIdx.x >> 5); row < M;
          row += static_cast<int64_t>(gridDim.x) * (kLnThreads / 32)) {
         const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * C);
-        float v[kLnMaxChunks][8];
+        float v[kChunks][8];
         float s = 0.f;
 #pragma unroll
-        for (int i = 0; i < kLnMaxChunks; ++i) {
+        for (int i = 0; i < kChunks; ++i) {
             const int c = lane + 32 * i;
             const uint4 w = c < nch ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -429,7 +433,7 @@ __global__ void __launch_bounds__(kLnThreads) layernorm_kernel(const uint16_t *x
         const float mean = warp_sum(s) * inv_c;
         float q = 0.f;
 #pragma unroll
-        for (int i = 0; i < kLnMaxChunks; ++i)
+        for (int i = 0; i < kChunks; ++i)
             if (lane + 32 * i < nch) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -439,7 +443,7 @@ __global__ void __launch_bounds__(kLnThreads) layernorm_kernel(const uint16_t *x
             }
         const float rstd = rsqrtf(warp_sum(q) * inv_c + eps);
 #pragma unroll
-        for (int i = 0; i < kLnMaxChunks; ++i) {
+        for (int i = 0; i < kChunks; ++i) {
             const int c = lane + 32 * i;
             if (c < nch) {
                 const uint4 g = __ldg(reinterpret_cast<const uint4 *>(gamma) + c);
@@ -562,9 +566,21 @@ cudaError_t launch_layernorm(const void *x, const void *gamma, const void *beta,
     const int64_t blocks_needed = (M + kLnThreads / 32 - 1) / (kLnThreads / 32);
     const int64_t cap = static_cast<int64_t>(num_sms) * 16;
     const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
-    return launch_pdl(layernorm_kernel, dim3(grid), dim3(kLnThreads), 0, stream, static_cast<const uint16_t *>(x),
-                      static_cast<const uint16_t *>(gamma), static_cast<const uint16_t *>(beta),
-                      static_cast<uint16_t *>(y), M, m_dev, C, eps);
+    const int chunks = (C / 8 + 31) / 32;
+    auto go = [&](auto kernel) {
+        return launch_pdl(kernel, dim3(grid), dim3(kLnThreads), 0, stream, static_cast<const uint16_t *>(x),
+                          static_cast<const uint16_t *>(gamma), static_cast<const uint16_t *>(beta),
+                          static_cast<uint16_t *>(y), M, m_dev, C, eps);
+    };
+    if (chunks <= 1)
+        return go(layernorm_kernel<1>);
+    if (chunks == 2)
+        return go(layernorm_kernel<2>);
+    if (chunks == 3)
+        return go(layernorm_kernel<3>);
+    if (chunks == 4)
+        return go(layernorm_kernel<4>);
+    return go(layernorm_kernel<kLnMaxChunks>);
 }
 
 }  // namespace rra
