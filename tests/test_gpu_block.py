@@ -61,7 +61,7 @@ def rand_bf16(shape, scale=1.0, shift=0.0, seed=0):
 
 # ------------------------------------------------------------------------------ LayerNorm
 
-@pytest.mark.parametrize("M,C", [(1, 768), (37, 384), (1000, 768), (300, 2048)])
+@pytest.mark.parametrize("M,C", [(1, 768), (37, 384), (1000, 768), (300, 2048), (5, 8), (7, 256), (9, 1024), (11, 1280)])
 def test_layernorm_matches_oracle(M, C):
     x = rand_bf16((M, C), 2.0, 0.5, seed=M)
     g = rand_bf16((C,), 0.1, 1.0, seed=1)
