@@ -23,16 +23,17 @@
 //                   the single-launch path warps 0 and 1 gather them with cp.async;
 //       warps 2..3  tensor-core issuers, one per softmax group: S = Q K^T (smem x smem) and
 //                   O += P V (P from TMEM as the A operand), fp32 accumulation, completion
-//                   signalled through mbarriers; between bursts each prepares its group's next
-//                   V tile (zero tail; for bf16 inputs an in-place conversion to fp16);
+//                   signalled through mbarriers;
 //       warps 4..11 softmax: two groups of four warps take alternate items; in a group, thread
 //                   r owns row r of its S, P and O (TMEM lane r), so the row max and row sum
 //                   need no exchange (the row sum is kept in a register); it rescales its row of O
 //                   in TMEM when the running max rises, and finally normalises and stores the row;
 //       warp 12     (single-launch path) builds each item's kept-row list ahead of the gathers;
-//       warps 13-14 prepare each V tile as soon as it lands (alternate fills);
-//       warp 15     (single-launch path) zero-fills the block's share of pruned padded rows while
-//                   the rest of the block computes;
+//       warps 13-14 prepare each V tile as soon as it lands (zero tail; for bf16 inputs an
+//                   in-place conversion to fp16), each owning two of the four K/V slots;
+//       warp 15     (single-launch path) clears the block's share of pruned padded rows while
+//                   the rest of the block computes, one bulk copy per row from zeroed shared
+//                   memory;
 //   * P is rounded to fp16 (11 significant bits) and meets an fp16 V: for bf16 inputs every V
 //     tile is converted in shared memory, exactly for |v| in [2^-14, 65504] and with an
 //     absolute error below 2^-25 under it; a tile holding a finite |v| >= 65536 keeps bf16 and
@@ -45,7 +46,8 @@
 //
 // The same kernel body, instantiated with kFused, runs the whole pack -> attend -> unpack call
 // in one launch (the pages' pipeline without its two copies through HBM): the block derives
-// the kept counts of every image from the keep mask itself, the producer gathers the kept rows
+// the kept counts of every image from the keep mask itself (a warp or a thread per image,
+// whichever needs fewer memory round trips), the producer gathers the kept rows
 // of the padded Q/K/V straight into the swizzled tiles with 16-byte cp.async (32 lanes, one
 // coalesced 128-byte row segment per 8 lanes), and the epilogue writes each output row back to
 // its padded position.
