@@ -894,6 +894,9 @@ def main(argv=None):
     ap.add_argument("--block-only", action="store_true",
                     help="time only the synthetic-weight DeiT block on the workload's packed rows: the "
                          "command ncu captures for its kernels")
+    ap.add_argument("--comparators", action="store_true",
+                    help="time only torch's padded and NestedTensor SDPA against the single launch on "
+                         "the workload's inputs (measurement context; library code)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-images", type=int, default=0,
@@ -904,6 +907,8 @@ def main(argv=None):
         return run_reference(args)
     if args.mask_only:
         return main_mask(args)
+    if args.comparators:
+        return main_comparators(args)
     if args.block_only:
         return main_block(args)
     return main_gpu(args)
@@ -917,6 +922,69 @@ def main_block(args):
     cu0 = torch.from_numpy(np.concatenate([[0], np.cumsum(w.lengths[0])]).astype(np.int32)).cuda()
     print(json.dumps({"workload": w.name, "deit_block": time_block(w, cu0, flush, stream, args.steps, args.warmup)}),
           flush=True)
+    return 0
+
+
+def main_comparators(args):
+    """One GPU: the same-box comparators on identical inputs, against the single launch --
+    torch's padded SDPA (scaled_dot_product_attention over [B, H, N, 64] with a key-padding mask)
+    and SDPA over a jagged NestedTensor of the kept tokens (values [T, H, 64] built once, outside
+    the timed call).  Both are library code, called as they are.  Reports µs per call (events, L2
+    flushed before each call) and the largest difference from the single launch's output on the
+    kept rows."""
+    import torch.nn.functional as F
+    B, N, H, dt, std = workloads.shape_of(args.workload)
+    q, k, v = workloads.device_values(B, N, H, dt, std=std)
+    mask = torch.from_numpy(workloads.sweep_masks(args.workload)[0]).cuda()
+    keep = mask.bool()
+    stream = torch.cuda.Stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(q)
+    cu = torch.empty(B + 1, dtype=torch.int32, device="cuda")
+    qt, kt, vt = (t.transpose(1, 2) for t in (q, k, v))
+    am = keep[:, None, None, :]
+    with torch.cuda.stream(stream):
+        rra.rra_pack_attend_unpack(mask, q, k, v, y, cu, stream=stream)
+        offsets = cu.long()
+        nq, nk, nv = (torch.nested.nested_tensor_from_jagged(t[keep], offsets).transpose(1, 2) for t in (q, k, v))
+    stream.synchronize()
+
+    def ours():
+        rra.rra_pack_attend_unpack(mask, q, k, v, y, cu, stream=stream)
+
+    out = {}
+
+    def padded():
+        out["padded"] = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=am)
+
+    def nested():
+        out["nested"] = F.scaled_dot_product_attention(nq, nk, nv)
+
+    def timed(fn):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ms = []
+        for i in range(args.warmup + args.steps):
+            with torch.cuda.stream(stream):
+                flush.fill_((i + 1) & 0xFF)
+                start.record(stream)
+                fn()
+                end.record(stream)
+            stream.synchronize()
+            if i >= args.warmup:
+                ms.append(start.elapsed_time(end))
+        return 1e3 * statistics.mean(ms)
+
+    res = {"workload": args.workload, "B": B, "N": N, "H": H, "T": int(keep.sum()), "ours_us": timed(ours)}
+    ref = y[keep].float()
+    for name, fn in (("padded_sdpa", padded), ("nested_sdpa", nested)):
+        try:
+            res[name + "_us"] = timed(fn)
+            o = out["padded"].transpose(1, 2)[keep] if name == "padded_sdpa" else out["nested"].transpose(1, 2).values()
+            res[name + "_max_abs_diff"] = float((o.float() - ref).abs().max())
+            res[name + "_over_ours"] = res[name + "_us"] / res["ours_us"]
+        except Exception as e:  # a library path this torch build does not offer
+            res[name + "_unavailable"] = f"{type(e).__name__}: {e}"[:200]
+    print(json.dumps({"comparators": res}), flush=True)
     return 0
 
 
