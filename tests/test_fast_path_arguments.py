@@ -3,6 +3,9 @@
 * the Threshold-l2 fast path: when the smallest fp32 square of a row's (exactly squared) 16-bit
   inputs gives q = twice the last-bit exponent of the smallest input, and the double sum of the
   squares stays below 2^(q+52), the sum is exact -- whatever the order of the additions;
+* the Threshold-l2 ranking: counting on fp32-rounded keys, with the tokens whose fp32 key is
+  shared settled on the full keys, gives every token the rank of the full-key order (index
+  breaking ties);
 * the GEMM epilogue's GELU: erfc from Abramowitz and Stegun 7.1.28, evaluated in fp32 as the
   kernel does, stays within 5e-6 |x| of the exact GELU over every bf16 input in [-16, 16].
 
@@ -126,3 +129,39 @@ def test_fast_path_bound_needs_the_last_bit_term():
     acc = float(sq[0]) + float(sq[1])
     assert acc < 2.0 ** (2 * e + 52)           # the mistaken bound passes ...
     assert Fraction(acc) != _exact(sq)         # ... an inexact sum
+
+
+def _rank_by_fp32_counts(hi, lo):
+    """The kernel's ranking, restated: fp32-rounded keys counted (greater, equal); a token whose
+    fp32 key another token shares is settled on the full (hi, lo) keys, index breaking ties."""
+    f = hi.astype(np.float32)  # a monotone rounding of the high part
+    n = len(hi)
+    ranks = np.zeros(n, np.int64)
+    for i in range(n):
+        gt = int((f > f[i]).sum())
+        eq = int((f == f[i]).sum())
+        r = gt
+        if eq > 1:
+            for m in np.nonzero(f == f[i])[0]:
+                if m == i:
+                    continue
+                if hi[m] > hi[i] or (hi[m] == hi[i] and (lo[m] > lo[i] or (lo[m] == lo[i] and m < i))):
+                    r += 1
+        ranks[i] = r
+    return ranks
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_fp32_key_ranking_equals_the_full_key_order(seed):
+    rng = np.random.default_rng(seed)
+    n = 197
+    # scores with many near-ties: equal in fp32, different in double, some fully equal
+    base = rng.choice([1.0, 3.0, 768.0, 1e6], size=n)
+    hi = base * (1.0 + rng.integers(0, 5, n) * 2.0 ** -40)
+    lo = rng.integers(-2, 3, n) * 2.0 ** -80
+    lo[rng.random(n) < 0.3] = 0.0
+    ranks = _rank_by_fp32_counts(hi, lo)
+    order = sorted(range(n), key=lambda i: (-hi[i], -lo[i], i))
+    want = np.empty(n, np.int64)
+    want[order] = np.arange(n)
+    assert np.array_equal(ranks, want)
