@@ -12,6 +12,10 @@ owns each group's TMEM buffers -- S (written by Q K^T, read by the softmax), P (
 softmax, read by the PV MMA) and O (accumulated by PV, rescaled and read out by the softmax) --
 and fails when a writer or reader touches a buffer another role still owns.
 
+On the single-launch path each copier warp is an actor of its own running the producer loop; the
+Q and K/V full barriers complete a phase after one arrival per copier, and an arrival must land in
+the phase of the fill it belongs to (checked for two copiers, the kernel, and three).
+
 The roles' orders of waits and arrivals restate the kernel's (csrc/attend.cu): item n belongs to
 softmax group n % 2 and uses Q slot n % 2 and kept-row list slot n % 4; K/V chunks go round a
 4-slot ring in production order, with one "full" barrier per slot and group (the 3-slot ring of an
@@ -23,17 +27,32 @@ import pytest
 
 
 class Bar:
-    def __init__(self, name):
+    def __init__(self, name, count=1):
         self.name = name
         self.done = 0  # completed phases
+        self.count = count  # arrivals that complete a phase
+        self.pending = 0
 
     def passes(self, bit):
         return self.done % 2 != bit
 
+    def arrive(self):
+        self.pending += 1
+        if self.pending == self.count:
+            self.pending = 0
+            self.done += 1
+
 
 class Model:
-    def __init__(self, nkc, fused, rng, early_qk=False, shared_v_ready=False, v_mode="slot", stages=4, starve=()):
+    def __init__(self, nkc, fused, rng, early_qk=False, shared_v_ready=False, v_mode="slot", stages=4, starve=(),
+                 copiers=1, full_count=None):
         self.nkc, self.fused, self.rng = nkc, fused, rng
+        # single-launch path: `copiers` warps each run the producer loop and each arrives once per
+        # fill on the Q / K/V full barriers, whose phases complete after `full_count` arrivals (the
+        # kernel: 32 * kCopyWarps lanes, modelled as one arrival per warp); planted mistake: a count
+        # that assumes fewer copiers than run
+        self.copiers = copiers if fused else 1
+        full_count = self.copiers if full_count is None else full_count
         self.stages = stages  # K/V ring slots (the kernel's kKVStages)
         self.early_qk = early_qk  # planted mistake: the next S = Q K^T before the softmax released S
         self.shared_v_ready = shared_v_ready  # planted mistake: one V-ready barrier per group
@@ -46,13 +65,13 @@ class Model:
         self.items = len(nkc)
         B = {}
 
-        def bar(name):
-            B[name] = Bar(name)
+        def bar(name, count=1):
+            B[name] = Bar(name, count)
             return B[name]
 
-        self.q_full = [bar(f"q_full{s}") for s in range(2)]
+        self.q_full = [bar(f"q_full{s}", full_count) for s in range(2)]
         self.q_empty = [bar(f"q_empty{s}") for s in range(2)]
-        self.kv_full = [[bar(f"kv_full{s}.{g}") for g in range(2)] for s in range(stages)]
+        self.kv_full = [[bar(f"kv_full{s}.{g}", full_count) for g in range(2)] for s in range(stages)]
         self.kv_empty = [bar(f"kv_empty{s}") for s in range(stages)]
         self.s_full = [bar(f"s_full{g}") for g in range(2)]
         self.p_full = [bar(f"p_full{g}") for g in range(2)]
@@ -79,8 +98,8 @@ class Model:
             for c in range(k):
                 self.slot[(n, c)] = t % stages
                 t += 1
-        self.actors = [self.list_builder(), self.producer(), self.issuer(0), self.issuer(1),
-                       self.softmax(0), self.softmax(1), self.v_warp(0), self.v_warp(1)]
+        self.actors = [self.list_builder()] + [self.producer(j) for j in range(self.copiers)] + [
+            self.issuer(0), self.issuer(1), self.softmax(0), self.softmax(1), self.v_warp(0), self.v_warp(1)]
         self.finished = [False] * len(self.actors)
 
     # -- helpers: a generator yields ("wait", barrier, bit, expected_phase) or ("step",)
@@ -107,10 +126,17 @@ class Model:
             yield ("step",)
             self.idx_full[s].done += 1
 
-    def producer(self):
+    def arrival(self, bar, fill):
+        """An arrival for fill `fill` (0-based) of a full barrier: it must land in that phase."""
+        def effect():
+            self.check(bar.done == fill, f"an arrival for fill {fill} of {bar.name} landed in phase {bar.done}")
+        return effect
+
+    def producer(self, j=0):
         qb = kb = fb = 0
         qfill = [0, 0]
         kvfill = [0] * self.stages
+        kvseen = {}  # fills of kv_full[s][g] issued so far
         for n in range(self.items):
             g = n % 2
             if self.fused:
@@ -122,15 +148,17 @@ class Model:
                 yield self.wait(self.q_empty[qs], ((qb >> qs) & 1) ^ 1, qfill[qs] - 1)
             qb ^= 1 << qs
             qfill[qs] += 1
-            self.complete_async(f"copy_q{qs}", self.q_full[qs], None)
+            self.complete_async(f"copy{j}_q{qs}", self.q_full[qs], self.arrival(self.q_full[qs], qfill[qs] - 1))
             for c in range(self.nkc[n]):
                 s = self.slot[(n, c)]
                 if kvfill[s] >= 1:
                     yield self.wait(self.kv_empty[s], ((kb >> s) & 1) ^ 1, kvfill[s] - 1)
                 kb ^= 1 << s
                 kvfill[s] += 1
+                f = kvseen.get((s, g), 0)
+                kvseen[(s, g)] = f + 1
                 # bulk copies into different slots may land in any order
-                self.complete_async(f"copy_kv{s}", self.kv_full[s][g], None)
+                self.complete_async(f"copy{j}_kv{s}", self.kv_full[s][g], self.arrival(self.kv_full[s][g], f))
             yield ("step",)
 
     def v_warp(self, vw):
@@ -301,7 +329,7 @@ class Model:
                 _, bar, effect = self.hw.pop(k)
                 if effect is not None:
                     effect()
-                bar.done += 1
+                bar.arrive()
                 continue
             w = pending[who]
             if w is not None and w[1].done <= w[3]:
@@ -397,5 +425,32 @@ def test_model_sees_observing_v_warps_lapped():
     bad = 0
     for i, (nkc, rng) in enumerate(random_cases(600, 23)):
         if Model(nkc, i % 2 == 1, rng, v_mode="observe_all", starve=(6 + i % 2,)).run() != "ok":
+            bad += 1
+    assert bad > 0
+
+
+@pytest.mark.parametrize("copiers", [2, 3])
+def test_protocol_with_several_copier_warps(copiers):
+    """The single-launch path with two copier warps (the kernel) and three (a tried variant):
+    every copier runs the producer loop and arrives once per fill; random schedules, some
+    starving one role or one copier, never pass a wait early, never land an arrival in the wrong
+    phase, and never hang -- nothing in the protocol assumes two copiers."""
+    bad = []
+    for i, (nkc, rng) in enumerate(random_cases(1200, 29 + copiers)):
+        n_actors = 1 + copiers + 6
+        starve = () if i % 3 == 0 else (i % n_actors,)
+        out = Model(nkc, True, rng, copiers=copiers, starve=starve).run()
+        if out != "ok":
+            bad.append((nkc, starve, out))
+    assert not bad, bad[:5]
+
+
+def test_model_sees_a_copier_count_mistake():
+    """Three copiers against full barriers that complete after two arrivals (a constant that
+    assumes two copiers): some schedule lands an arrival in the wrong phase, passes a wait early
+    or hangs -- the check has teeth for the mistake it is meant to rule out."""
+    bad = 0
+    for nkc, rng in random_cases(600, 31):
+        if Model(nkc, True, rng, copiers=3, full_count=2).run() != "ok":
             bad += 1
     assert bad > 0
