@@ -836,6 +836,16 @@ def main_gpu(args):
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and not args.profile:
         cpu = cpu_baseline(w, args.cpu_seconds)
 
+    comparators = None
+    if rank == 0 and ws == 1 and not args.profile and not args.no_comparators:
+        comparators = {}
+        for wl in dict.fromkeys(("c5:0.2:512", args.workload)):
+            try:
+                comparators[wl] = run_comparators(wl, min(args.steps, 10), 3)
+                torch.cuda.empty_cache()
+            except Exception as e:  # measurement context only: never lose the line for it
+                comparators[wl] = {"error": f"{type(e).__name__}: {e}"[:200]}
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
@@ -864,6 +874,7 @@ def main_gpu(args):
             "clocks": clk.summary(),
             "gpu_launches": args.steps * len(pipe.kernels) * stages,
             "sweep": sweep,
+            "comparators": comparators,
         }
         print(json.dumps(line), flush=True)
     del pipe
@@ -894,6 +905,8 @@ def main(argv=None):
     ap.add_argument("--block-only", action="store_true",
                     help="time only the synthetic-weight DeiT block on the workload's packed rows: the "
                          "command ncu captures for its kernels")
+    ap.add_argument("--no-comparators", action="store_true",
+                    help="skip the same-box comparator timing (torch's padded and NestedTensor SDPA)")
     ap.add_argument("--comparators", action="store_true",
                     help="time only torch's padded and NestedTensor SDPA against the single launch on "
                          "the workload's inputs (measurement context; library code)")
@@ -926,16 +939,22 @@ def main_block(args):
 
 
 def main_comparators(args):
-    """One GPU: the same-box comparators on identical inputs, against the single launch --
+    """One GPU: `run_comparators` on the workload, printed as one JSON line."""
+    print(json.dumps({"comparators": run_comparators(args.workload, args.steps, args.warmup)}), flush=True)
+    return 0
+
+
+def run_comparators(workload, steps, warmup):
+    """The same-box comparators on identical inputs, against the single launch --
     torch's padded SDPA (scaled_dot_product_attention over [B, H, N, 64] with a key-padding mask)
     and SDPA over a jagged NestedTensor of the kept tokens (values [T, H, 64] built once, outside
     the timed call).  Both are library code, called as they are.  Reports µs per call (events, L2
     flushed before each call) and the largest difference from the single launch's output on the
     kept rows."""
     import torch.nn.functional as F
-    B, N, H, dt, std = workloads.shape_of(args.workload)
+    B, N, H, dt, std = workloads.shape_of(workload)
     q, k, v = workloads.device_values(B, N, H, dt, std=std)
-    mask = torch.from_numpy(workloads.sweep_masks(args.workload)[0]).cuda()
+    mask = torch.from_numpy(workloads.sweep_masks(workload)[0]).cuda()
     keep = mask.bool()
     stream = torch.cuda.Stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
@@ -963,18 +982,18 @@ def main_comparators(args):
     def timed(fn):
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ms = []
-        for i in range(args.warmup + args.steps):
+        for i in range(warmup + steps):
             with torch.cuda.stream(stream):
                 flush.fill_((i + 1) & 0xFF)
                 start.record(stream)
                 fn()
                 end.record(stream)
             stream.synchronize()
-            if i >= args.warmup:
+            if i >= warmup:
                 ms.append(start.elapsed_time(end))
         return 1e3 * statistics.mean(ms)
 
-    res = {"workload": args.workload, "B": B, "N": N, "H": H, "T": int(keep.sum()), "ours_us": timed(ours)}
+    res = {"workload": workload, "B": B, "N": N, "H": H, "T": int(keep.sum()), "ours_us": timed(ours)}
     ref = y[keep].float()
     for name, fn in (("padded_sdpa", padded), ("nested_sdpa", nested)):
         try:
@@ -984,8 +1003,7 @@ def main_comparators(args):
             res[name + "_over_ours"] = res[name + "_us"] / res["ours_us"]
         except Exception as e:  # a library path this torch build does not offer
             res[name + "_unavailable"] = f"{type(e).__name__}: {e}"[:200]
-    print(json.dumps({"comparators": res}), flush=True)
-    return 0
+    return res
 
 
 def main_mask(args):
